@@ -1,0 +1,230 @@
+"""fp64 CPU oracle for SANA's multi-head ReLU linear attention.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this module.  It shares no code with
+the CUDA library (``relu_linear_attention_attn_b200``) and imports nothing from
+it; both sides are fed the same seeded inputs by the tests.
+
+The arithmetic lives in ``sana_oracle.c`` (plain fp64 loops written from
+Eq. (1) of "Sana: Efficient High-Resolution Image Synthesis with Linear
+Diffusion Transformers", section 2.1, and the QK-Norm bullet of "SANA 1.5:
+Efficient Scaling of Training-Time and Inference-Time Compute in Linear
+Diffusion Transformer", section "Model architecture").  This file marshals
+arrays to fp64 and adds one library step: the QKV projection ``x @ Wqkv`` of
+the fused variant (section 7, on-device deployment, of the Sana notes: the
+ReLU(K)^T V reduction fused with the QKV projection), done as an fp64 numpy
+matmul.
+
+Pins (checked by ``tests/test_oracle_pins.py``): the quadratic form of Eq. (1)
+brute-forced on tiny inputs, hand-derived worked examples in
+``tests/golden/``, closed forms (N = 1, one-hot keys, constant values),
+invariants (linearity in V, token permutation, scale invariance), and
+torch's own ``rms_norm`` for the feature map.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sana_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_sana_oracle.so")
+
+NORM_OFF = 0
+NORM_PER_HEAD = 1
+NORM_FULL_C = 2
+
+_lib = None
+_lock = threading.Lock()
+
+
+def build(force: bool = False) -> str:
+    """Compile sana_oracle.c into oracle/_sana_oracle.so with gcc (no fast-math,
+    no FMA contraction, so fp64 operations happen in the written order)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + ".tmp.%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off",
+           "-fno-fast-math", "-o", tmp, _SRC, "-lpthread", "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _bind(lib):
+    """Declare the C signatures on a loaded oracle library."""
+    dp = ctypes.POINTER(ctypes.c_double)
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    i64, ci, cd = ctypes.c_int64, ctypes.c_int, ctypes.c_double
+    lib.oracle_phi_f64.argtypes = [dp, dp, dp, i64, ci, ci, cd, ci, ci]
+    lib.oracle_kv_state_f64.argtypes = [dp, dp, dp, dp, i64, i64, ci, ci, cd, ci, ci]
+    lib.oracle_apply_f64.argtypes = [dp, dp, dp, dp, i64p, i64, i64, i64, ci, ci, cd, ci, ci]
+    lib.oracle_forward_f64.argtypes = [dp, dp, dp, dp, dp, dp, i64, i64, ci, ci, cd, ci, ci]
+    for f in (lib.oracle_phi_f64, lib.oracle_kv_state_f64, lib.oracle_apply_f64,
+              lib.oracle_forward_f64):
+        f.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            _lib = _bind(ctypes.CDLL(_LIB_PATH))
+    return _lib
+
+
+def host_threads() -> int:
+    """Threads the oracle uses by default: the cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _f64(a) -> np.ndarray:
+    """Any array-like (numpy, torch CPU tensor of any float dtype) -> C-contiguous fp64.
+    bf16 and fp32 values are exactly representable in fp64, so nothing is rounded."""
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor, converted without importing torch here
+        a = a.detach().cpu()
+        if str(a.dtype) in ("torch.bfloat16", "torch.float16"):
+            a = a.float()
+        a = a.double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _norm_mode(gq, gk, scope: str) -> int:
+    if gq is None and gk is None:
+        return NORM_OFF
+    if gq is None or gk is None:
+        raise ValueError("gq and gk must both be given (norm on) or both be None (norm off)")
+    if scope == "head":
+        return NORM_PER_HEAD
+    if scope == "full":
+        return NORM_FULL_C
+    raise ValueError("scope must be 'head' or 'full'")
+
+
+def phi(x, g, H: int, eps: float, scope: str = "head", nthreads: int = 0) -> np.ndarray:
+    """phi(x) = ReLU(RMSNorm(x) * g) per token; g None = norm off (plain ReLU).
+    x: (..., C).  Returns fp64 of the same shape."""
+    x = _f64(x)
+    g = _f64(g)
+    C = x.shape[-1]
+    mode = NORM_OFF if g is None else (NORM_PER_HEAD if scope == "head" else NORM_FULL_C)
+    out = np.empty_like(x)
+    T = x.size // C if C else 0
+    rc = _load().oracle_phi_f64(_ptr(x), _ptr(g), _ptr(out), T, C, H, float(eps), mode,
+                                nthreads or host_threads())
+    if rc != 0:
+        raise ValueError("oracle_phi_f64 rejected its arguments")
+    return out
+
+
+def kv_state(k, v, gk, H: int, eps: float, scope: str = "head", nthreads: int = 0,
+             norm: bool | None = None) -> np.ndarray:
+    """S[b,h] = sum_n phi(K_n)^T [V_n | 1], shape (B, H, D, D+1), fp64.
+    Norm is on iff gk is given (pass norm=False to force it off)."""
+    k = _f64(k)
+    v = _f64(v)
+    gk = _f64(gk)
+    B, N, C = k.shape
+    if v.shape != k.shape:
+        raise ValueError("k and v must have the same shape")
+    D = C // H
+    mode = NORM_OFF if (gk is None or norm is False) else (
+        NORM_PER_HEAD if scope == "head" else NORM_FULL_C)
+    S = np.empty((B, H, D, D + 1), dtype=np.float64)
+    rc = _load().oracle_kv_state_f64(_ptr(k), _ptr(v), _ptr(gk), _ptr(S), B, N, C, H,
+                                     float(eps), mode, nthreads or host_threads())
+    if rc != 0:
+        raise ValueError("oracle_kv_state_f64 rejected its arguments")
+    return S
+
+
+def apply(q, gq, S, H: int, eps: float, tokens=None, scope: str = "head",
+          nthreads: int = 0) -> np.ndarray:
+    """O = phi(Q) S[:, :D] / (phi(Q) S[:, D] + eps).
+    q: (B, N, C); S: (B, H, D, D+1).  tokens: optional flat indices b*N+n; then the
+    result is (len(tokens), C), otherwise (B, N, C)."""
+    q = _f64(q)
+    gq = _f64(gq)
+    S = _f64(S)
+    B, N, C = q.shape
+    mode = NORM_OFF if gq is None else (NORM_PER_HEAD if scope == "head" else NORM_FULL_C)
+    if tokens is None:
+        out = np.empty((B, N, C), dtype=np.float64)
+        tp, T = None, 0
+    else:
+        tok = np.ascontiguousarray(np.asarray(tokens, dtype=np.int64))
+        T = tok.size
+        out = np.empty((T, C), dtype=np.float64)
+        tp = tok.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+    rc = _load().oracle_apply_f64(_ptr(q), _ptr(gq), _ptr(S), _ptr(out), tp, T, B, N, C, H,
+                                  float(eps), mode, nthreads or host_threads())
+    if rc != 0:
+        raise ValueError("oracle_apply_f64 rejected its arguments")
+    return out
+
+
+def forward(q, k, v, gq, gk, H: int, eps: float, scope: str = "head",
+            nthreads: int = 0) -> np.ndarray:
+    """Eq. (1) with QK-RMSNorm: (B, N, C) fp64 output.  gq = gk = None: norm off."""
+    mode = _norm_mode(gq, gk, scope)
+    q, k, v, gq, gk = (_f64(a) for a in (q, k, v, gq, gk))
+    B, N, C = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same (B, N, C) shape")
+    out = np.empty((B, N, C), dtype=np.float64)
+    rc = _load().oracle_forward_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(gq), _ptr(gk), _ptr(out),
+                                    B, N, C, H, float(eps), mode, nthreads or host_threads())
+    if rc != 0:
+        raise ValueError("oracle_forward_f64 rejected its arguments")
+    return out
+
+
+def qkv_project(x, W, rows=None) -> np.ndarray:
+    """[Q | K | V] = x @ Wqkv in fp64 (a library matmul step).
+    x: (B, N, C); W: (C, 3C) with columns [0,C) = Q, [C,2C) = K, [2C,3C) = V.
+    rows: optional column range (lo, hi) of W to project onto."""
+    x = _f64(x)
+    W = _f64(W)
+    if rows is not None:
+        W = W[:, rows[0]:rows[1]]
+    return np.matmul(x, W)
+
+
+def fused_forward(x, W, gq, gk, H: int, eps: float, tokens=None, nthreads: int = 0):
+    """The fused variant end to end: projection, then Eq. (1) with QK-RMSNorm.
+    The projected Q, K, V stay in fp64 (no intermediate rounding).
+    tokens: optional flat token indices; then only those rows of O are formed
+    (K and V are still projected for every token, since the state needs them)."""
+    x = _f64(x)
+    B, N, C = x.shape
+    kvp = qkv_project(x, W, rows=(C, 3 * C))
+    k, v = kvp[..., :C], kvp[..., C:]
+    S = kv_state(np.ascontiguousarray(k), np.ascontiguousarray(v), gk, H, eps,
+                 nthreads=nthreads, norm=gk is not None)
+    if tokens is None:
+        q = qkv_project(x, W, rows=(0, C))
+        return apply(q, gq, S, H, eps, nthreads=nthreads)
+    tok = np.asarray(tokens, dtype=np.int64)
+    xs = x.reshape(B * N, C)[tok]
+    q = qkv_project(xs, W, rows=(0, C))
+    # apply() indexes q by flat token; give it a (B, N, C) view with only the
+    # sampled rows filled, which it never reads past.
+    qfull = np.zeros((B * N, C), dtype=np.float64)
+    qfull[tok] = q
+    return apply(qfull.reshape(B, N, C), gq, S, H, eps, tokens=tok, nthreads=nthreads)
