@@ -1,0 +1,460 @@
+"""Throughput benchmark of the SANA ReLU-linear-attention library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload sweep|fused|1024px|2048px|4096px] [--no-fused] [--no-cpu]
+
+One step (default workload "sweep") is one pass of the linear-attention op over
+each of the SANA latent sizes the metric names (C = 2240, H = 70, D = 32, bf16):
+1024px B=1 N=1024, 2048px B=8 N=4096 (per-token LogNormal scales), 4096px B=2
+N=16384 (keys x100, norm off).  Each pass runs the op's two halves through the
+C ABI (sana_linattn_kv_state: pass 1 + combine, then sana_linattn_apply: pass 2,
+exactly the kernels sana_linattn_forward launches) so each half is timed with
+CUDA events on its stream.  The fused-QKV variant (2048px B=4, x @ Wqkv first) is
+timed in the same run and reported under "fused".
+
+value: tokens of all ranks / device time of the K timed steps (max over ranks).
+e2e: the same metric through sana_linattn_forward with host (pinned) buffers,
+host->device copies of q, k, v and the device->host copy of the output inside the
+timed region.  cpu_baseline: the fp64 CPU oracle, as it stands, on a bounded
+sample of the same workload (rank 0, N=1 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "linear-attn Mtokens/s at C=2240, N=1K–16K; % of B200 HBM roofline"
+HBM_FALLBACK_GBS = 6650.0
+BF16_FALLBACK_TFLOPS = 1590.0
+# algorithmic bytes per token of each pass (bf16, C = 2240): pass 1 reads k and v,
+# pass 2 reads q and writes out; 17,920 B/token for the whole op
+PASS_BYTES_PER_TOKEN = 2 * 2240 * 2
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return (float(j["hbm_gbs"]), float(j["bf16_tflops"]),
+                float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured")
+    except Exception:
+        return HBM_FALLBACK_GBS, BF16_FALLBACK_TFLOPS, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- workloads
+def sweep_workloads():
+    from relu_linear_attention_attn_b200.synthetic import CONFIGS
+    return {"1024px": CONFIGS[1], "2048px": CONFIGS[2], "4096px": CONFIGS[3]}
+
+
+def select(workload: str):
+    sw = sweep_workloads()
+    if workload == "sweep":
+        return list(sw.values())
+    if workload in sw:
+        return [sw[workload]]
+    raise SystemExit(f"unknown workload {workload}")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sana_bench_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        except Exception:
+            return None
+        if not rows:
+            return None
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1])]
+        mx = [num(r[2]) for r in rows if num(r[2])]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        top = max(sm) if sm else 0
+        loaded = [s for s in sm if s >= 0.5 * top] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def cpu_oracle_sample(pairs, budget_s: float = 12.0):
+    """Time the fp64 oracle as it stands on a bounded sample of the workload: whole
+    batch items taken in order until about budget_s of CPU work is done.
+    pairs: [(workload, CPU input tensors)]."""
+    from oracle import oracle as O
+    tokens, t_total, parts = 0, 0.0, []
+    for w, x in pairs:
+        for b in range(w.B):
+            q, k, v = (x[n][b:b + 1] for n in ("q", "k", "v"))
+            t0 = time.perf_counter()
+            O.forward(q, k, v, x["gq"], x["gk"], w.H, w.eps)
+            t_total += time.perf_counter() - t0
+            tokens += w.N
+            parts.append(f"{w.name}[b={b}]")
+            if t_total >= budget_s:
+                break
+        if t_total >= budget_s:
+            break
+    return {"value": tokens / t_total / 1e6, "unit": "Mtokens/s", "cores": O.host_threads(),
+            "kind": "oracle", "sample": f"{tokens} tokens ({', '.join(parts)}), fp64 C oracle, "
+                                        f"{t_total:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle on the host cores, same metric and config."""
+    if rank != 0:
+        return
+    from oracle import oracle as O
+    from relu_linear_attention_attn_b200.synthetic import make_inputs
+    wl = select(args.workload)
+    # each step: one whole batch item of every workload in the sweep, bounded so
+    # the --steps/--warmup run stays within a few minutes
+    data = []
+    for w in wl:
+        x = make_inputs(w)
+        data.append((w, x["q"][:1], x["k"][:1], x["v"][:1], x["gq"], x["gk"]))
+    per_step_tokens = sum(w.N for w, *_ in data)
+
+    def step():
+        for w, q, k, v, gq, gk in data:
+            O.forward(q, k, v, gq, gk, w.H, w.eps)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = per_step_tokens * args.steps / dt / 1e6
+    sample = (f"one batch item of each workload per step ({per_step_tokens} tokens): "
+              + ", ".join(f"{w.name} N={w.N}" for w, *_ in data))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "Mtokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block(args, wl),
+            "cpu_baseline": {"value": value, "unit": "Mtokens/s", "cores": O.host_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "Mtokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def config_block(args, wl):
+    return {"workload": "sana-latent-sweep-N1K-16K" if args.workload == "sweep" else
+            args.workload,
+            "parts": [{"name": w.name, "B": w.B, "N": w.N, "C": w.C, "H": w.H, "D": w.D,
+                       "recipe": w.recipe, "gains": w.gains, "eps": w.eps} for w in wl],
+            "global_batch_tokens": sum(w.tokens for w in wl),
+            "l2": "inputs larger than L2: one step streams >1.1 GB, so each workload's "
+                  "inputs are evicted before they are used again",
+            "parallelism": f"dp{args.gpus} (batch-sharded, no collective)"}
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local):
+    import torch
+
+    import relu_linear_attention_attn_b200 as sla
+    from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
+
+    sla.load()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = measured_peaks()
+    wl = select(args.workload) if args.workload != "fused" else []
+
+    # inputs resident in HBM; each rank works on its own batch (weak scaling)
+    sets = []
+    for w in wl:
+        w_r = w.scaled(seed=w.seed + 1000 * rank) if rank else w
+        x = make_inputs(w_r)
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+        D = w.D
+        d["kv"] = torch.empty((w.B, w.H, D, D + 1), dtype=torch.float32, device=dev)
+        d["out"] = torch.empty_like(d["q"])
+        nb = sla.workspace_bytes(w.B, w.N, w.C, w.H)
+        d["ws"] = torch.empty(nb, dtype=torch.uint8, device=dev)
+        sets.append((w, d, x))
+    tokens_per_step = sum(w.tokens for w in wl)
+
+    def step(events=None):
+        for i, (w, d, _) in enumerate(sets):
+            if events is not None:
+                events[i][0].record(stream)
+            sla.kv_state(d["k"], d["v"], d["gk"], w.H, w.eps, kv=d["kv"], workspace=d["ws"])
+            if events is not None:
+                events[i][1].record(stream)
+            sla.apply(d["q"], d["gq"], d["kv"], w.H, w.eps, out=d["out"])
+            if events is not None:
+                events[i][2].record(stream)
+
+    line = {"metric": METRIC, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_block(args, wl)}
+
+    if sets:
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in sets]
+              for _ in range(args.steps)]
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local) as clk:
+            barrier(world)
+            torch.cuda.synchronize()
+            t_start.record(stream)
+            for s in range(args.steps):
+                step(ev[s])
+            t_end.record(stream)
+            torch.cuda.synchronize()
+            barrier(world)
+        elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+        ms_per_step = elapsed_ms / args.steps
+        value = tokens_per_step * world / (ms_per_step * 1e-3) / 1e6
+        # per-pass durations (average per launch) and algorithmic bytes
+        parts = []
+        p1_ms = p2_ms = 0.0
+        p1_b = p2_b = 0
+        for i, (w, d, _) in enumerate(sets):
+            a = statistics.fmean(ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps))
+            b = statistics.fmean(ev[s][i][1].elapsed_time(ev[s][i][2]) for s in range(args.steps))
+            by = w.tokens * PASS_BYTES_PER_TOKEN
+            p1_ms += a
+            p2_ms += b
+            p1_b += by
+            p2_b += by
+            parts.append({"workload": w.name, "tokens": w.tokens, "ms": a + b,
+                          "Mtokens_per_s": w.tokens / ((a + b) * 1e-3) / 1e6,
+                          "pass1_ms": a, "pass2_ms": b,
+                          "hbm_frac_of_measured": 2 * by / ((a + b) * 1e-3) / 1e9 / hbm_gbs})
+        dom = ("pass1 kv_state (kv_partial + kv_combine)", p1_ms, p1_b) if p1_ms >= p2_ms else \
+            ("pass2 apply", p2_ms, p2_b)
+        achieved = dom[2] / (dom[1] * 1e-3) / 1e9
+        line.update({"value": value, "ms_per_step": ms_per_step,
+                     "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs,
+                                  "unit": "GB/s", "frac": achieved / hbm_gbs,
+                                  "traffic": None, "kernel": dom[0],
+                                  "peak_kind": f"{peak_kind} copy bandwidth (hbm_gbs)",
+                                  "algorithmic_bytes_per_token": PASS_BYTES_PER_TOKEN,
+                                  "whole_op_frac": 2 * p1_b / ((p1_ms + p2_ms) * 1e-3) / 1e9
+                                  / hbm_gbs},
+                     "parts": parts,
+                     "gpu_launches": args.steps * len(sets) * 3,
+                     "clocks": clk.summary()})
+
+        # e2e: the public call with host buffers, copies inside the timed region
+        if not args.no_e2e:
+            line["e2e"] = e2e_measure(args, sla, sets, stream, world)
+
+    if args.workload == "fused" or (args.workload == "sweep" and not args.no_fused):
+        line["fused"] = fused_measure(args, sla, CONFIGS[4], rank, dev, stream, world, bf16_tf,
+                                      peak_kind)
+        if not sets:
+            f = line["fused"]
+            line.update({"value": f["value"], "ms_per_step": f["ms_per_step"],
+                         "roofline": f["roofline"], "gpu_launches": f["gpu_launches"],
+                         "clocks": f.get("clocks"), "e2e": f.get("e2e")})
+            line["config"] = {"workload": CONFIGS[4].name, "B": 4, "N": 4096, "C": 2240, "H": 70,
+                              "parallelism": f"dp{args.gpus}"}
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        pairs = [(w, x) for w, _, x in sets]
+        if not pairs:
+            w = CONFIGS[1]
+            pairs = [(w, make_inputs(w))]
+        line["cpu_baseline"] = cpu_oracle_sample(pairs)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def e2e_measure(args, sla, sets, stream, world):
+    import torch
+    host = []
+    for w, d, x in sets:
+        h = {n: x[n].pin_memory() for n in ("q", "k", "v")}
+        h["out"] = torch.empty_like(x["q"]).pin_memory()
+        host.append(h)
+    h2d = sum(3 * w.tokens * w.C * 2 for w, *_ in sets)
+    d2h = sum(w.tokens * w.C * 2 for w, *_ in sets)
+    tokens = sum(w.tokens for w, *_ in sets)
+
+    def step():
+        for (w, d, _), h in zip(sets, host):
+            for n in ("q", "k", "v"):
+                d[n].copy_(h[n], non_blocking=True)
+            sla.forward(d["q"], d["k"], d["v"], d["gq"], d["gk"], w.H, w.eps, out=d["out"],
+                        workspace=d["ws"])
+            h["out"].copy_(d["out"], non_blocking=True)
+    steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), world) / steps
+    return {"value": tokens * world / (ms * 1e-3) / 1e6, "unit": "Mtokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "steps": steps, "api": "sana_linattn_forward"}
+
+
+def fused_measure(args, sla, w, rank, dev, stream, world, bf16_tf, peak_kind):
+    import torch
+    from relu_linear_attention_attn_b200.synthetic import make_inputs
+    x = make_inputs(w.scaled(seed=w.seed + 1000 * rank) if rank else w)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    out = torch.empty_like(d["x"])
+    ws = torch.empty(sla.workspace_bytes(w.B, w.N, w.C, w.H, fused=True), dtype=torch.uint8,
+                     device=dev)
+    steps = max(3, min(args.steps, 20))
+
+    def call():
+        sla.qkv_fused(d["x"], d["W"], d["gq"], d["gk"], w.H, w.eps, out=out, workspace=ws)
+    for _ in range(max(args.warmup, 3)):
+        call()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    with ClockSampler(dev.index) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        for a, b in evs:
+            a.record(stream)
+            call()
+            b.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = max_over_ranks(statistics.fmean(a.elapsed_time(b) for a, b in evs), world)
+    flops = 2.0 * w.tokens * w.C * 3 * w.C
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": w.name, "value": w.tokens * world / (ms * 1e-3) / 1e6,
+            "unit": "Mtokens/s", "ms_per_step": ms, "steps": steps,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16_tf, "unit": "TFLOP/s",
+                         "frac": tf / bf16_tf, "traffic": None,
+                         "kernel": "whole fused op (QKV projection + attention)",
+                         "peak_kind": f"{peak_kind} bf16 burst (bf16_tflops)"},
+            "gpu_launches": steps * 4, "clocks": clk.summary()}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="sweep",
+                    choices=["sweep", "fused", "1024px", "2048px", "4096px"])
+    ap.add_argument("--no-fused", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        run_reference(args, rank, world)
+        return
+    rank, world, local = dist_setup(args)
+    try:
+        run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

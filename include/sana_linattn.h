@@ -1,0 +1,124 @@
+/*
+ * sana_linattn.h -- C ABI of the B200 (sm_100a) library for SANA's multi-head
+ * ReLU linear attention with QK-RMSNorm.
+ *
+ * The operation (Eq. (1) of "Sana: Efficient High-Resolution Image Synthesis
+ * with Linear Diffusion Transformers", section 2.1, with the QK-Norm of "SANA
+ * 1.5: Efficient Scaling of Training-Time and Inference-Time Compute in Linear
+ * Diffusion Transformer", section "Model architecture"):
+ *
+ *   phi(x)  = ReLU(g * x / sqrt(mean_d(x_d^2) + eps))  per token and head
+ *             (the mean over the head's D channels; with the norm off,
+ *             phi(x) = ReLU(x))
+ *   S_{b,h} = sum_n phi(K_{b,n,h})^T [V_{b,n,h} | 1]    (D x (D+1), fp32)
+ *   O_{b,n,h} = phi(Q_{b,n,h}) S[:, :D] / (phi(Q_{b,n,h}) S[:, D] + eps)
+ *
+ * The sums run over all N tokens (non-causal).  The same eps is the RMSNorm
+ * epsilon and the denominator's.  Accumulation is fp32 throughout, so sums far
+ * beyond the fp16 range (the overflow the SANA-1.5 page attributes to growing
+ * attention sums) stay finite.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are row-major (B, N, C) with C = H * D and channel c = h*D + d.
+ *     D = C / H must be 32 (anything else returns SANA_EUNSUPPORTED).
+ *   - Every pointer is DEVICE memory owned by the caller (the library never
+ *     allocates, frees or keeps a pointer after the call returns).
+ *   - q, k, v, x, Wqkv and out must be 16-byte aligned; the workspace 256-byte
+ *     aligned; gains 4-byte aligned.  out must not overlap any input.
+ *   - gq == NULL && gk == NULL switches the RMSNorm off (phi = ReLU); gains are
+ *     fp32 vectors of length C.  Passing exactly one of them is SANA_EINVAL.
+ *   - Work is enqueued on `stream` asynchronously; the call never synchronises.
+ *     Argument errors are returned before anything is enqueued.  A failed
+ *     launch returns SANA_ECUDA; faults during execution surface at the
+ *     caller's next synchronisation, as for any CUDA kernel.
+ *   - B == 0 or N == 0 is an empty problem: nothing is launched and SANA_OK is
+ *     returned (sana_linattn_kv_state then zero-fills its state output).
+ *   - For a given shape, dtype and device two calls give bitwise-identical
+ *     results: split counts are a fixed function of the shape and partial sums
+ *     are combined in a fixed order.
+ */
+#ifndef SANA_LINATTN_H
+#define SANA_LINATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define SANA_API __attribute__((visibility("default")))
+#else
+#define SANA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SANA_OK = 0,
+    SANA_EINVAL = -1,        /* bad shape, NULL pointer, eps < 0, overlap, dtype   */
+    SANA_EALIGN = -2,        /* a pointer violates its alignment requirement       */
+    SANA_EUNSUPPORTED = -3,  /* well-formed but not supported (D != 32, too large) */
+    SANA_EWORKSPACE = -4,    /* workspace NULL or smaller than the queried size    */
+    SANA_ECUDA = -5          /* a CUDA launch or runtime call failed               */
+} sana_status;
+
+typedef enum {
+    SANA_BF16 = 0,           /* bf16 inputs and output, fp32 arithmetic            */
+    SANA_F32 = 1             /* fp32 inputs and output, fp32 arithmetic            */
+} sana_dtype;
+
+/* Bytes of device workspace that sana_linattn_forward (fused == 0),
+ * sana_linattn_kv_state (fused == 0) or sana_linattn_qkv_fused (fused != 0)
+ * needs for this shape.  Returns 0 for an invalid or empty shape. */
+SANA_API size_t sana_linattn_workspace_bytes(int64_t B, int64_t N, int C, int H, int fused);
+
+/* Eq. (1) end to end on projected q, k, v.
+ * q, k, v, out: (B, N, C) in `dtype`.  gq, gk: fp32 [C] or both NULL.
+ * workspace: at least sana_linattn_workspace_bytes(B, N, C, H, 0) bytes; its
+ * contents on entry do not matter and are garbage on exit. */
+SANA_API int sana_linattn_forward(const void* q, const void* k, const void* v,
+                         const float* gq, const float* gk, void* out,
+                         int64_t B, int64_t N, int C, int H, float eps,
+                         sana_dtype dtype, void* workspace, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/* The state half of Eq. (1) (the sums formed once and reused by every query,
+ * section 2.1 of the Sana notes): kv (B, H, D, D+1) fp32 receives
+ * S_{b,h}[d][e] = sum_n phi(K)[d] V[e] for e < D and S_{b,h}[d][D] =
+ * sum_n phi(K)[d].  Because S is a plain sum over tokens, states of disjoint
+ * token ranges add up to the state of their union (sequence sharding reduces
+ * them with one sum all-reduce).  workspace as for sana_linattn_forward. */
+SANA_API int sana_linattn_kv_state(const void* k, const void* v, const float* gk, float* kv,
+                          int64_t B, int64_t N, int C, int H, float eps,
+                          sana_dtype dtype, void* workspace, size_t ws_bytes,
+                          cudaStream_t stream);
+
+/* The query half of Eq. (1) with a given state:
+ * out = phi(Q) kv[:, :D] / (phi(Q) kv[:, D] + eps).
+ * q, out: (B, N, C) in `dtype`; kv: (B, H, D, D+1) fp32; gq: fp32 [C] or NULL
+ * (norm off).  Needs no workspace. */
+SANA_API int sana_linattn_apply(const void* q, const float* gq, const float* kv, void* out,
+                       int64_t B, int64_t N, int C, int H, float eps,
+                       sana_dtype dtype, cudaStream_t stream);
+
+/* The variant fused with the QKV projection (section 7 of the Sana notes,
+ * on-device deployment: ReLU(K)^T V fused with the QKV projection).
+ * x: (B, N, C) bf16; Wqkv: (C, 3C) bf16 row-major, columns [0,C) project to Q,
+ * [C,2C) to K and [2C,3C) to V, no bias.  The projected Q, K, V are kept in
+ * fp32 until the norm (no intermediate rounding).  out: (B, N, C) bf16.
+ * gq, gk: fp32 [C] or both NULL.  workspace: at least
+ * sana_linattn_workspace_bytes(B, N, C, H, 1) bytes. */
+SANA_API int sana_linattn_qkv_fused(const void* x, const void* Wqkv,
+                           const float* gq, const float* gk, void* out,
+                           int64_t B, int64_t N, int C, int H, float eps,
+                           void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Static description of a status code (never NULL). */
+SANA_API const char* sana_linattn_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SANA_LINATTN_H */

@@ -50,35 +50,40 @@
 /* Feature map phi: RMSNorm (optional) -> gain -> ReLU, one token.         */
 /* ---------------------------------------------------------------------- */
 
-/* x, g, out: C values of one token.  norm selects the RMSNorm scope. */
+/* phi of head h of one token: x and g hold the token's C values and gains,
+ * out receives the head's D values.  norm selects the RMSNorm scope: the mean
+ * square is taken over the head's D channels, or over all C channels of the
+ * token for the full-channel comparison scope. */
+static void phi_head(const double* x, const double* g, double* out,
+                     int C, int H, int h, double eps, int norm)
+{
+    const int D = C / H;
+    const double* xh = x + (size_t)h * D;
+    if (norm == ORACLE_NORM_OFF) {
+        for (int d = 0; d < D; ++d) out[d] = xh[d] > 0.0 ? xh[d] : 0.0;
+        return;
+    }
+    double ss = 0.0;
+    double r;
+    if (norm == ORACLE_NORM_FULL_C) {
+        for (int c = 0; c < C; ++c) ss += x[c] * x[c];
+        r = 1.0 / sqrt(ss / (double)C + eps);
+    } else {
+        for (int d = 0; d < D; ++d) ss += xh[d] * xh[d];
+        r = 1.0 / sqrt(ss / (double)D + eps);
+    }
+    for (int d = 0; d < D; ++d) {
+        const double y = g[h * D + d] * (xh[d] * r);
+        out[d] = y > 0.0 ? y : 0.0;
+    }
+}
+
+/* phi of every head of one token (C values in, C values out). */
 static void phi_token(const double* x, const double* g, double* out,
                       int C, int H, double eps, int norm)
 {
     const int D = C / H;
-    if (norm == ORACLE_NORM_OFF) {
-        for (int c = 0; c < C; ++c) out[c] = x[c] > 0.0 ? x[c] : 0.0;
-        return;
-    }
-    if (norm == ORACLE_NORM_FULL_C) {
-        double ss = 0.0;
-        for (int c = 0; c < C; ++c) ss += x[c] * x[c];
-        const double r = 1.0 / sqrt(ss / (double)C + eps);
-        for (int c = 0; c < C; ++c) {
-            const double y = g[c] * (x[c] * r);
-            out[c] = y > 0.0 ? y : 0.0;
-        }
-        return;
-    }
-    for (int h = 0; h < H; ++h) {
-        const double* xh = x + (size_t)h * D;
-        double ss = 0.0;
-        for (int d = 0; d < D; ++d) ss += xh[d] * xh[d];
-        const double r = 1.0 / sqrt(ss / (double)D + eps);
-        for (int d = 0; d < D; ++d) {
-            const double y = g[h * D + d] * (xh[d] * r);
-            out[h * D + d] = y > 0.0 ? y : 0.0;
-        }
-    }
+    for (int h = 0; h < H; ++h) phi_head(x, g, out + (size_t)h * D, C, H, h, eps, norm);
 }
 
 /* ---------------------------------------------------------------------- */
@@ -174,21 +179,18 @@ static void kv_one(int64_t bh, void* vctx)
     const int64_t b = bh / c->H;
     const int h = (int)(bh % c->H);
     double* S = c->S + (size_t)bh * D * (D + 1);
-    double* phik = (double*)malloc(sizeof(double) * (size_t)c->C);
+    double* kk = (double*)malloc(sizeof(double) * (size_t)D);
     memset(S, 0, sizeof(double) * (size_t)D * (D + 1));
     for (int64_t n = 0; n < c->N; ++n) {
         const size_t row = ((size_t)b * c->N + n) * c->C;
-        /* phi is computed for the whole token so that the full-C norm scope
-         * sees every channel; only head h is used below. */
-        phi_token(c->k + row, c->gk, phik, c->C, c->H, c->eps, c->norm);
-        const double* kk = phik + (size_t)h * D;
+        phi_head(c->k + row, c->gk, kk, c->C, c->H, h, c->eps, c->norm);
         const double* vv = c->v + row + (size_t)h * D;
         for (int d = 0; d < D; ++d) {
             for (int e = 0; e < D; ++e) S[d * (D + 1) + e] += kk[d] * vv[e];
             S[d * (D + 1) + D] += kk[d];
         }
     }
-    free(phik);
+    free(kk);
 }
 
 int oracle_kv_state_f64(const double* k, const double* v, const double* gk,

@@ -1,0 +1,195 @@
+"""Python binding of the B200 SANA ReLU-linear-attention library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libsana_linattn.so`` (declared in ``include/sana_linattn.h``).
+PyTorch provides device memory and the current stream.  There is no CPU or
+PyTorch fallback: if the shared library is missing, ``load()`` raises.
+
+    import relu_linear_attention_attn_b200 as sla
+    out = sla.forward(q, k, v, gq, gk, H=70, eps=1e-6)     # (B, N, C) bf16/fp32
+    out = sla.qkv_fused(x, Wqkv, gq, gk, H=70, eps=1e-6)   # bf16
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = ["load", "lib_path", "workspace_bytes", "forward", "kv_state", "apply", "qkv_fused",
+           "SanaError", "STATUS", "BF16", "F32"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libsana_linattn.so"
+
+BF16, F32 = 0, 1
+STATUS = {0: "SANA_OK", -1: "SANA_EINVAL", -2: "SANA_EALIGN", -3: "SANA_EUNSUPPORTED",
+          -4: "SANA_EWORKSPACE", -5: "SANA_ECUDA"}
+
+_lib = None
+_lock = threading.Lock()
+
+
+class SanaError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} -> {STATUS.get(status, status)} ({status}): {msg}")
+        self.status = status
+
+
+def lib_path() -> str:
+    return os.path.join(_PKG, _LIB_NAME)
+
+
+def _declare(lib):
+    vp, fp = ctypes.c_void_p, ctypes.c_void_p
+    i64, ci, cf, sz = ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.sana_linattn_workspace_bytes.argtypes = [i64, i64, ci, ci, ci]
+    lib.sana_linattn_workspace_bytes.restype = sz
+    lib.sana_linattn_forward.argtypes = [vp, vp, vp, fp, fp, vp, i64, i64, ci, ci, cf, ci, vp, sz,
+                                         vp]
+    lib.sana_linattn_kv_state.argtypes = [vp, vp, fp, fp, i64, i64, ci, ci, cf, ci, vp, sz, vp]
+    lib.sana_linattn_apply.argtypes = [vp, fp, fp, vp, i64, i64, ci, ci, cf, ci, vp]
+    lib.sana_linattn_qkv_fused.argtypes = [vp, vp, fp, fp, vp, i64, i64, ci, ci, cf, vp, sz, vp]
+    for f in (lib.sana_linattn_forward, lib.sana_linattn_kv_state, lib.sana_linattn_apply,
+              lib.sana_linattn_qkv_fused):
+        f.restype = ctypes.c_int
+    lib.sana_linattn_strerror.argtypes = [ci]
+    lib.sana_linattn_strerror.restype = ctypes.c_char_p
+    return lib
+
+
+def load():
+    """Load the in-tree CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = lib_path()
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    f"{path} is missing: build it with `python -m relu_linear_attention_attn_b200"
+                    ".build` (there is no fallback implementation)")
+            _lib = _declare(ctypes.CDLL(path))
+    return _lib
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        raise SanaError(fn, rc, load().sana_linattn_strerror(rc).decode())
+
+
+def workspace_bytes(B: int, N: int, C: int, H: int, fused: bool = False) -> int:
+    return int(load().sana_linattn_workspace_bytes(B, N, C, H, 1 if fused else 0))
+
+
+# --------------------------------------------------------------------------- torch marshalling
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _dev(t, name: str):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _gain(g, name: str):
+    if g is None:
+        return None
+    torch = _torch()
+    if g.dtype != torch.float32:
+        raise TypeError(f"{name} must be float32")
+    return _dev(g, name)
+
+
+def _stream(stream) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _workspace(nbytes: int, device, workspace):
+    torch = _torch()
+    if nbytes == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    if workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace needs {nbytes} bytes")
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def forward(q, k, v, gq, gk, H: int, eps: float, out=None, workspace=None, stream=None):
+    """Eq. (1) with QK-RMSNorm on projected q, k, v of shape (B, N, C).
+    gq, gk: float32 [C] tensors, or both None to switch the norm off."""
+    B, N, C = q.shape
+    if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share shape and dtype")
+    dt = _dtype_code(q)
+    if out is None:
+        out = _torch().empty_like(q)
+    ws, wsb = _workspace(workspace_bytes(B, N, C, H), q.device, workspace)
+    rc = load().sana_linattn_forward(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _gain(gq, "gq"),
+                                     _gain(gk, "gk"), _dev(out, "out"), B, N, C, H, float(eps), dt,
+                                     None if ws is None else ws.data_ptr(), wsb, _stream(stream))
+    _check("sana_linattn_forward", rc)
+    return out
+
+
+def kv_state(k, v, gk, H: int, eps: float, kv=None, workspace=None, stream=None):
+    """State S (B, H, D, D+1) fp32 of Eq. (1): sum_n phi(K_n)^T [V_n | 1]."""
+    torch = _torch()
+    B, N, C = k.shape
+    D = C // H
+    dt = _dtype_code(k)
+    if kv is None:
+        kv = torch.empty((B, H, D, D + 1), dtype=torch.float32, device=k.device)
+    ws, wsb = _workspace(workspace_bytes(B, N, C, H), k.device, workspace)
+    rc = load().sana_linattn_kv_state(_dev(k, "k"), _dev(v, "v"), _gain(gk, "gk"), _dev(kv, "kv"),
+                                      B, N, C, H, float(eps), dt,
+                                      None if ws is None else ws.data_ptr(), wsb, _stream(stream))
+    _check("sana_linattn_kv_state", rc)
+    return kv
+
+
+def apply(q, gq, kv, H: int, eps: float, out=None, stream=None):
+    """O = phi(Q) S[:, :D] / (phi(Q) S[:, D] + eps) with a given state kv."""
+    B, N, C = q.shape
+    dt = _dtype_code(q)
+    if out is None:
+        out = _torch().empty_like(q)
+    rc = load().sana_linattn_apply(_dev(q, "q"), _gain(gq, "gq"), _dev(kv, "kv"), _dev(out, "out"),
+                                   B, N, C, H, float(eps), dt, _stream(stream))
+    _check("sana_linattn_apply", rc)
+    return out
+
+
+def qkv_fused(x, W, gq, gk, H: int, eps: float, out=None, workspace=None, stream=None):
+    """The fused variant: [Q|K|V] = x @ Wqkv, QK-RMSNorm, ReLU, Eq. (1).  bf16 in and out."""
+    torch = _torch()
+    B, N, C = x.shape
+    if x.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
+        raise TypeError("the fused path takes bf16 x and Wqkv")
+    if tuple(W.shape) != (C, 3 * C):
+        raise ValueError("Wqkv must be (C, 3C)")
+    if out is None:
+        out = torch.empty_like(x)
+    ws, wsb = _workspace(workspace_bytes(B, N, C, H, fused=True), x.device, workspace)
+    rc = load().sana_linattn_qkv_fused(_dev(x, "x"), _dev(W, "Wqkv"), _gain(gq, "gq"),
+                                       _gain(gk, "gk"), _dev(out, "out"), B, N, C, H, float(eps),
+                                       None if ws is None else ws.data_ptr(), wsb,
+                                       _stream(stream))
+    _check("sana_linattn_qkv_fused", rc)
+    return out

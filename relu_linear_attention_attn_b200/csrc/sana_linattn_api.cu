@@ -1,0 +1,275 @@
+// C ABI of the SANA linear-attention library: argument validation, workspace
+// planning and kernel launches.  No allocation, no host synchronisation.
+#include "../../include/sana_linattn.h"
+
+#include <math.h>
+#include <stdint.h>
+
+#include "sana_common.cuh"
+#include "simt_kernels.cuh"
+
+namespace sana {
+namespace {
+
+constexpr int64_t kSplitTile = 128;     // tokens per split are a multiple of this
+constexpr int kTargetCtas = 4 * 148;    // pass-1 CTAs to aim for (4 per SM on 148 SMs)
+constexpr int kMaxSplits = 64;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Split-N plan for pass 1: a fixed function of (B, N, H), so results are
+// reproducible bit for bit.
+struct Plan {
+    int S;            // splits per (b, h)
+    int64_t tps;      // tokens per split
+};
+
+Plan make_plan(int64_t B, int64_t N, int H) {
+    const int64_t bh = B * (int64_t)H;
+    const int64_t max_by_tokens = (N + kSplitTile - 1) / kSplitTile;
+    int64_t S = (kTargetCtas + bh - 1) / bh;
+    if (S > max_by_tokens) S = max_by_tokens;
+    if (S > kMaxSplits) S = kMaxSplits;
+    if (S < 1) S = 1;
+    int64_t tps = (N + S - 1) / S;
+    tps = (tps + kSplitTile - 1) / kSplitTile * kSplitTile;
+    S = (N + tps - 1) / tps;   // drop splits that would be empty
+    if (S < 1) S = 1;
+    return Plan{(int)S, tps};
+}
+
+// Workspace layout of the unfused path: [partials B*H*S*1056 fp32][state B*H*1056 fp32].
+struct WsLayout {
+    size_t part_off, kv_off, fused_qkv_off, total;
+};
+
+WsLayout ws_layout(int64_t B, int64_t N, int C, int H, bool fused) {
+    const Plan p = make_plan(B, N, H);
+    WsLayout w{};
+    size_t off = 0;
+    if (fused) {
+        w.fused_qkv_off = off;
+        off = align_up(off + (size_t)B * N * 3 * C * sizeof(float), 256);
+    }
+    w.part_off = off;
+    off = align_up(off + (size_t)B * H * p.S * kStateFloats * sizeof(float), 256);
+    w.kv_off = off;
+    off = align_up(off + (size_t)B * H * kStateFloats * sizeof(float), 256);
+    w.total = off;
+    return w;
+}
+
+bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t a0 = (uintptr_t)a, b0 = (uintptr_t)b;
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+int check_dims(int64_t B, int64_t N, int C, int H) {
+    if (B < 0 || N < 0 || C <= 0 || H <= 0 || C % H != 0) return SANA_EINVAL;
+    if (C / H != kD) return SANA_EUNSUPPORTED;
+    if (B > 65535 || H > 65535) return SANA_EUNSUPPORTED;     // grid z / y limits
+    if (N > ((int64_t)1 << 40) || B * N > ((int64_t)1 << 40)) return SANA_EUNSUPPORTED;
+    return SANA_OK;
+}
+
+int check_eps(float eps) { return (eps >= 0.f && isfinite(eps)) ? SANA_OK : SANA_EINVAL; }
+
+int check_gains(const float* gq, const float* gk) {
+    if ((gq == nullptr) != (gk == nullptr)) return SANA_EINVAL;
+    if (gq && (!aligned(gq, 4) || !aligned(gk, 4))) return SANA_EALIGN;
+    return SANA_OK;
+}
+
+size_t elem_size(sana_dtype dt) { return dt == SANA_BF16 ? 2 : 4; }
+
+int launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SANA_OK : SANA_ECUDA;
+}
+
+// Pass 1 + combine on inputs of element type T with row strides ldk, ldv.
+template <typename T>
+void launch_state(const T* k, const T* v, const float* gk, float* part, float* kv,
+                  int64_t B, int64_t N, int H, int64_t ldk, int64_t ldv, float eps,
+                  const Plan& p, cudaStream_t st) {
+    const dim3 g1(p.S, H, (unsigned)B);
+    kv_partial_simt<T><<<g1, 128, 0, st>>>(k, v, gk, part, N, H, ldk, ldv, p.S, p.tps, eps,
+                                           gk != nullptr);
+    kv_combine<<<(unsigned)(B * H), 256, 0, st>>>(part, kv, p.S);
+}
+
+template <typename TI, typename TO>
+void launch_apply(const TI* q, const float* gq, const float* kv, TO* out, int64_t B, int64_t N,
+                  int H, int64_t ldq, int64_t ldo, float eps, cudaStream_t st) {
+    const dim3 g((unsigned)((N + 127) / 128), H, (unsigned)B);
+    apply_simt<TI, TO><<<g, 128, 0, st>>>(q, gq, kv, out, N, H, ldq, ldo, eps, gq != nullptr);
+}
+
+int validate_qkv(const void* q, const void* k, const void* v, const void* out, int64_t B,
+                 int64_t N, int C, sana_dtype dtype) {
+    if (dtype != SANA_BF16 && dtype != SANA_F32) return SANA_EINVAL;
+    if (!q || !k || !v || !out) return SANA_EINVAL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+        return SANA_EALIGN;
+    const size_t bytes = (size_t)B * N * C * elem_size(dtype);
+    if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) ||
+        overlaps(out, bytes, v, bytes))
+        return SANA_EINVAL;
+    return SANA_OK;
+}
+
+int validate_ws(void* ws, size_t ws_bytes, size_t need) {
+    if (need == 0) return SANA_OK;
+    if (!ws || ws_bytes < need) return SANA_EWORKSPACE;
+    if (!aligned(ws, 256)) return SANA_EALIGN;
+    return SANA_OK;
+}
+
+}  // namespace
+}  // namespace sana
+
+using namespace sana;
+
+extern "C" {
+
+size_t sana_linattn_workspace_bytes(int64_t B, int64_t N, int C, int H, int fused) {
+    if (check_dims(B, N, C, H) != SANA_OK || B == 0 || N == 0) return 0;
+    return ws_layout(B, N, C, H, fused != 0).total;
+}
+
+const char* sana_linattn_strerror(int status) {
+    switch (status) {
+        case SANA_OK: return "success";
+        case SANA_EINVAL: return "invalid argument (shape, NULL pointer, eps, dtype or overlap)";
+        case SANA_EALIGN: return "pointer misaligned (16 B tensors, 256 B workspace, 4 B gains)";
+        case SANA_EUNSUPPORTED: return "unsupported configuration (head dim must be 32)";
+        case SANA_EWORKSPACE: return "workspace missing or smaller than required";
+        case SANA_ECUDA: return "CUDA launch or runtime error";
+        default: return "unknown status";
+    }
+}
+
+int sana_linattn_kv_state(const void* k, const void* v, const float* gk, float* kv, int64_t B,
+                          int64_t N, int C, int H, float eps, sana_dtype dtype, void* workspace,
+                          size_t ws_bytes, cudaStream_t stream) {
+    int rc;
+    if ((rc = check_dims(B, N, C, H)) != SANA_OK) return rc;
+    if ((rc = check_eps(eps)) != SANA_OK) return rc;
+    if (dtype != SANA_BF16 && dtype != SANA_F32) return SANA_EINVAL;
+    if (gk && !aligned(gk, 4)) return SANA_EALIGN;
+    if (B == 0) return SANA_OK;
+    if (!kv) return SANA_EINVAL;
+    if (!aligned(kv, 16)) return SANA_EALIGN;
+    if (N == 0) {
+        return cudaMemsetAsync(kv, 0, (size_t)B * H * kStateFloats * sizeof(float), stream) ==
+                       cudaSuccess ? SANA_OK : SANA_ECUDA;
+    }
+    if (!k || !v) return SANA_EINVAL;
+    if (!aligned(k, 16) || !aligned(v, 16)) return SANA_EALIGN;
+    const WsLayout L = ws_layout(B, N, C, H, false);
+    if ((rc = validate_ws(workspace, ws_bytes, L.total)) != SANA_OK) return rc;
+    const size_t in_bytes = (size_t)B * N * C * elem_size(dtype);
+    const size_t kv_bytes = (size_t)B * H * kStateFloats * sizeof(float);
+    if (overlaps(kv, kv_bytes, k, in_bytes) || overlaps(kv, kv_bytes, v, in_bytes))
+        return SANA_EINVAL;
+    const Plan p = make_plan(B, N, H);
+    float* part = (float*)((char*)workspace + L.part_off);
+    if (dtype == SANA_BF16)
+        launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, kv, B, N, H, C, C, eps, p,
+                           stream);
+    else
+        launch_state<float>((const float*)k, (const float*)v, gk, part, kv, B, N, H, C, C, eps, p,
+                            stream);
+    return launch_status();
+}
+
+int sana_linattn_apply(const void* q, const float* gq, const float* kv, void* out, int64_t B,
+                       int64_t N, int C, int H, float eps, sana_dtype dtype,
+                       cudaStream_t stream) {
+    int rc;
+    if ((rc = check_dims(B, N, C, H)) != SANA_OK) return rc;
+    if ((rc = check_eps(eps)) != SANA_OK) return rc;
+    if (dtype != SANA_BF16 && dtype != SANA_F32) return SANA_EINVAL;
+    if (gq && !aligned(gq, 4)) return SANA_EALIGN;
+    if (B == 0 || N == 0) return SANA_OK;
+    if (!q || !kv || !out) return SANA_EINVAL;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(kv, 16)) return SANA_EALIGN;
+    const size_t bytes = (size_t)B * N * C * elem_size(dtype);
+    if (overlaps(out, bytes, q, bytes) ||
+        overlaps(out, bytes, kv, (size_t)B * H * kStateFloats * sizeof(float)))
+        return SANA_EINVAL;
+    if (dtype == SANA_BF16)
+        launch_apply<bf16, bf16>((const bf16*)q, gq, kv, (bf16*)out, B, N, H, C, C, eps, stream);
+    else
+        launch_apply<float, float>((const float*)q, gq, kv, (float*)out, B, N, H, C, C, eps,
+                                   stream);
+    return launch_status();
+}
+
+int sana_linattn_forward(const void* q, const void* k, const void* v, const float* gq,
+                         const float* gk, void* out, int64_t B, int64_t N, int C, int H,
+                         float eps, sana_dtype dtype, void* workspace, size_t ws_bytes,
+                         cudaStream_t stream) {
+    int rc;
+    if ((rc = check_dims(B, N, C, H)) != SANA_OK) return rc;
+    if ((rc = check_eps(eps)) != SANA_OK) return rc;
+    if ((rc = check_gains(gq, gk)) != SANA_OK) return rc;
+    if (dtype != SANA_BF16 && dtype != SANA_F32) return SANA_EINVAL;
+    if (B == 0 || N == 0) return SANA_OK;
+    if ((rc = validate_qkv(q, k, v, out, B, N, C, dtype)) != SANA_OK) return rc;
+    const WsLayout L = ws_layout(B, N, C, H, false);
+    if ((rc = validate_ws(workspace, ws_bytes, L.total)) != SANA_OK) return rc;
+    const size_t bytes = (size_t)B * N * C * elem_size(dtype);
+    if (overlaps(workspace, L.total, out, bytes) || overlaps(workspace, L.total, q, bytes) ||
+        overlaps(workspace, L.total, k, bytes) || overlaps(workspace, L.total, v, bytes))
+        return SANA_EINVAL;
+    const Plan p = make_plan(B, N, H);
+    float* part = (float*)((char*)workspace + L.part_off);
+    float* kv = (float*)((char*)workspace + L.kv_off);
+    if (dtype == SANA_BF16) {
+        launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, kv, B, N, H, C, C, eps, p,
+                           stream);
+        launch_apply<bf16, bf16>((const bf16*)q, gq, kv, (bf16*)out, B, N, H, C, C, eps, stream);
+    } else {
+        launch_state<float>((const float*)k, (const float*)v, gk, part, kv, B, N, H, C, C, eps, p,
+                            stream);
+        launch_apply<float, float>((const float*)q, gq, kv, (float*)out, B, N, H, C, C, eps,
+                                   stream);
+    }
+    return launch_status();
+}
+
+int sana_linattn_qkv_fused(const void* x, const void* Wqkv, const float* gq, const float* gk,
+                           void* out, int64_t B, int64_t N, int C, int H, float eps,
+                           void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    int rc;
+    if ((rc = check_dims(B, N, C, H)) != SANA_OK) return rc;
+    if ((rc = check_eps(eps)) != SANA_OK) return rc;
+    if ((rc = check_gains(gq, gk)) != SANA_OK) return rc;
+    if (B == 0 || N == 0) return SANA_OK;
+    if (!x || !Wqkv || !out) return SANA_EINVAL;
+    if (!aligned(x, 16) || !aligned(Wqkv, 16) || !aligned(out, 16)) return SANA_EALIGN;
+    const size_t xb = (size_t)B * N * C * 2, wb = (size_t)C * 3 * C * 2;
+    if (overlaps(out, xb, x, xb) || overlaps(out, xb, Wqkv, wb)) return SANA_EINVAL;
+    const WsLayout L = ws_layout(B, N, C, H, true);
+    if ((rc = validate_ws(workspace, ws_bytes, L.total)) != SANA_OK) return rc;
+    if (overlaps(workspace, L.total, out, xb) || overlaps(workspace, L.total, x, xb) ||
+        overlaps(workspace, L.total, Wqkv, wb))
+        return SANA_EINVAL;
+    const int64_t M = B * N;
+    if ((M + 63) / 64 > 65535) return SANA_EUNSUPPORTED;
+    const Plan p = make_plan(B, N, H);
+    float* qkv = (float*)((char*)workspace + L.fused_qkv_off);
+    float* part = (float*)((char*)workspace + L.part_off);
+    float* kv = (float*)((char*)workspace + L.kv_off);
+    const dim3 gg((unsigned)((3 * C + 63) / 64), (unsigned)((M + 63) / 64));
+    gemm_simt_bf16<<<gg, 256, 0, stream>>>((const bf16*)x, (const bf16*)Wqkv, qkv, M, 3 * C, C);
+    launch_state<float>(qkv + C, qkv + 2 * C, gk, part, kv, B, N, H, 3 * C, 3 * C, eps, p, stream);
+    launch_apply<float, bf16>(qkv, gq, kv, (bf16*)out, B, N, H, 3 * C, C, eps, stream);
+    return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,140 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load, export every symbol that include/*.h declares, size its
+workspace, and reject bad arguments with the documented status before touching
+the device.  The rejection tests pass fake device addresses; every call below
+carries at least one violation, so nothing is launched.  They are skipped on a
+machine with a GPU (the GPU suite repeats them with real buffers)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+import torch
+
+import relu_linear_attention_attn_b200 as sla
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, EINVAL, EALIGN, EUNSUP, EWS, ECUDA = 0, -1, -2, -3, -4, -5
+
+
+def declared_symbols():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        names += re.findall(r"SANA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_library_builds_for_sm100a_and_loads():
+    lib = sla.load()
+    assert os.path.exists(sla.lib_path())
+    assert lib is not None
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert "sana_linattn_forward" in names and "sana_linattn_qkv_fused" in names
+    lib = ctypes.CDLL(sla.lib_path())
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_strerror_covers_every_status():
+    lib = sla.load()
+    for code in (OK, EINVAL, EALIGN, EUNSUP, EWS, ECUDA, 12345):
+        s = lib.sana_linattn_strerror(code)
+        assert s and len(s) > 3
+
+
+def test_workspace_bytes():
+    ws = sla.workspace_bytes
+    assert ws(0, 1024, 2240, 70) == 0 and ws(1, 0, 2240, 70) == 0
+    assert ws(1, 1024, 2240, 71) == 0            # C % H != 0
+    assert ws(1, 1024, 2240, 35) == 0            # D = 64 unsupported
+    a = ws(1, 1024, 2240, 70)
+    b = ws(8, 4096, 2240, 70)
+    assert 0 < a < b and a % 256 == 0 and b % 256 == 0
+    assert ws(4, 4096, 2240, 70, fused=True) > ws(4, 4096, 2240, 70)
+    # the state alone: B*H*D*(D+1) fp32, the partials at least as much again
+    assert a >= 2 * 1 * 70 * 32 * 33 * 4
+
+
+FAKE = 1 << 36   # a 256-byte-aligned address that is never dereferenced
+
+
+@pytest.fixture()
+def lib():
+    if torch.cuda.is_available():
+        pytest.skip("fake-pointer rejection tests run on CPU-only machines")
+    return sla.load()
+
+
+def _fwd(lib, q=FAKE, k=FAKE + (1 << 30), v=FAKE + (2 << 30), gq=FAKE + (3 << 30),
+         gk=FAKE + (3 << 30) + 65536, out=FAKE + (4 << 30), B=1, N=1024, C=2240, H=70,
+         eps=1e-6, dtype=0, ws=FAKE + (6 << 30), wsb=1 << 30):
+    return lib.sana_linattn_forward(q, k, v, gq, gk, out, B, N, C, H, eps, dtype, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(H=35), EUNSUP),                      # D = 64
+    (dict(H=71), EINVAL),                      # C % H != 0
+    (dict(C=0), EINVAL),
+    (dict(B=-1), EINVAL),
+    (dict(N=-5), EINVAL),
+    (dict(eps=-1e-6), EINVAL),
+    (dict(eps=float("nan")), EINVAL),
+    (dict(eps=float("inf")), EINVAL),
+    (dict(gq=None), EINVAL),                   # only one gain given
+    (dict(gk=None), EINVAL),
+    (dict(q=None), EINVAL),
+    (dict(out=None), EINVAL),
+    (dict(dtype=7), EINVAL),
+    (dict(q=FAKE + 2), EALIGN),
+    (dict(out=FAKE + (4 << 30) + 8), EALIGN),
+    (dict(gq=FAKE + (3 << 30) + 2), EALIGN),
+    (dict(ws=None), EWS),
+    (dict(wsb=1024), EWS),
+    (dict(ws=FAKE + (6 << 30) + 16), EALIGN),
+    (dict(out=FAKE + 4096), EINVAL),           # out overlaps q
+    (dict(ws=FAKE + (1 << 30) + 256), EINVAL),  # workspace overlaps k
+    (dict(B=1 << 20), EUNSUP),                  # beyond the grid's batch limit
+])
+def test_forward_rejects_bad_arguments(lib, kw, status):
+    assert _fwd(lib, **kw) == status
+
+
+def test_empty_problem_is_a_no_op(lib):
+    assert _fwd(lib, B=0) == OK
+    assert _fwd(lib, N=0) == OK
+    assert lib.sana_linattn_apply(FAKE, None, FAKE + (1 << 30), FAKE + (2 << 30), 3, 0, 2240, 70,
+                                  1e-6, 0, None) == OK
+
+
+def test_other_entry_points_reject_bad_arguments(lib):
+    # kv_state: misaligned k, workspace too small, bad dtype
+    assert lib.sana_linattn_kv_state(FAKE + 4, FAKE + (1 << 30), None, FAKE + (2 << 30), 1, 64,
+                                     2240, 70, 1e-6, 0, FAKE + (3 << 30), 1 << 30, None) == EALIGN
+    assert lib.sana_linattn_kv_state(FAKE, FAKE + (1 << 30), None, FAKE + (2 << 30), 1, 64,
+                                     2240, 70, 1e-6, 0, FAKE + (3 << 30), 16, None) == EWS
+    assert lib.sana_linattn_kv_state(FAKE, FAKE + (1 << 30), None, FAKE + (2 << 30), 1, 64,
+                                     2240, 70, 1e-6, 9, FAKE + (3 << 30), 1 << 30, None) == EINVAL
+    # apply: D = 16, out overlapping the state
+    assert lib.sana_linattn_apply(FAKE, None, FAKE + (1 << 30), FAKE + (2 << 30), 1, 64, 2240, 140,
+                                  1e-6, 0, None) == EUNSUP
+    assert lib.sana_linattn_apply(FAKE, None, FAKE + (1 << 30), FAKE + (1 << 30) + 256, 1, 64,
+                                  2240, 70, 1e-6, 0, None) == EINVAL
+    # fused: misaligned W, too-small workspace, one gain
+    args = [FAKE, FAKE + (1 << 30), None, None, FAKE + (2 << 30), 4, 4096, 2240, 70, 1e-6,
+            FAKE + (4 << 30), 1 << 34, None]
+    a = list(args)
+    a[1] += 2
+    assert lib.sana_linattn_qkv_fused(*a) == EALIGN
+    a = list(args)
+    a[11] = 4096
+    assert lib.sana_linattn_qkv_fused(*a) == EWS
+    a = list(args)
+    a[2] = FAKE + (3 << 30)
+    assert lib.sana_linattn_qkv_fused(*a) == EINVAL

@@ -17,12 +17,12 @@ MUTATIONS = {
                          "S[d * (D + 1) + e] += kk[e] * vv[d];"),
     "normaliser_dropped": ("S[d * (D + 1) + D] += kk[d];", "S[d * (D + 1) + D] += 1.0;"),
     "eps_dropped_from_denominator": ("num / (den + c->eps)", "num / den"),
-    "mean_square_not_divided": ("1.0 / sqrt(ss / (double)D + eps)", "1.0 / sqrt(ss + eps)"),
-    "sqrt_missing": ("1.0 / sqrt(ss / (double)D + eps)", "1.0 / (ss / (double)D + eps)"),
-    "relu_missing_after_norm": ("out[h * D + d] = y > 0.0 ? y : 0.0;", "out[h * D + d] = y;"),
-    "relu_flipped": ("out[h * D + d] = y > 0.0 ? y : 0.0;",
-                     "out[h * D + d] = y < 0.0 ? -y : 0.0;"),
-    "relu_missing_norm_off": ("out[c] = x[c] > 0.0 ? x[c] : 0.0;", "out[c] = x[c];"),
+    "mean_square_not_divided": ("r = 1.0 / sqrt(ss / (double)D + eps)", "r = 1.0 / sqrt(ss + eps)"),
+    "sqrt_missing": ("r = 1.0 / sqrt(ss / (double)D + eps)", "r = 1.0 / (ss / (double)D + eps)"),
+    "relu_missing_after_norm": ("out[d] = y > 0.0 ? y : 0.0;", "out[d] = y;"),
+    "relu_flipped": ("out[d] = y > 0.0 ? y : 0.0;",
+                     "out[d] = y < 0.0 ? -y : 0.0;"),
+    "relu_missing_norm_off": ("out[d] = xh[d] > 0.0 ? xh[d] : 0.0;", "out[d] = xh[d];"),
     "gain_index_ignores_head": ("g[h * D + d] * (xh[d] * r)", "g[d] * (xh[d] * r)"),
     "apply_reads_state_transposed": ("num += qq[d] * S[d * (D + 1) + e];",
                                      "num += qq[d] * S[e * (D + 1) + d];"),
