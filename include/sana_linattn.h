@@ -114,6 +114,21 @@ SANA_API int sana_linattn_qkv_fused(const void* x, const void* Wqkv,
                            int64_t B, int64_t N, int C, int H, float eps,
                            void* workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* Device-side error word of the current device.  The tensor-core kernels bound
+ * every wait (about 2 s); a wait that gives up records an error code (1 = wait
+ * timeout) and the place it gave up (`site`), and the kernel winds down instead
+ * of hanging.  Reads the word into *code and *site (either may be NULL) and
+ * clears it when `clear` is non-zero.  Synchronous: call it after the work of
+ * interest has been synchronised.  Returns SANA_OK or SANA_ECUDA. */
+SANA_API int sana_linattn_device_error(int* code, int* site, int clear);
+
+/* Self-test of the bounded waits: enqueues one kernel whose single thread waits
+ * on an mbarrier that nothing arrives on.  After `limit_us` microseconds (at most
+ * 10 s) the wait gives up and records code 1 (wait timeout) at site 999 in the
+ * device error word (see sana_linattn_device_error); the kernel then exits and
+ * the context stays usable.  Returns SANA_EINVAL for a limit out of range. */
+SANA_API int sana_linattn_selftest_wait_timeout(int64_t limit_us, cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 SANA_API const char* sana_linattn_strerror(int status);
 

@@ -16,7 +16,7 @@ import os
 import threading
 
 __all__ = ["load", "lib_path", "workspace_bytes", "forward", "kv_state", "apply", "qkv_fused",
-           "SanaError", "STATUS", "BF16", "F32"]
+           "device_error", "selftest_wait_timeout", "SanaError", "STATUS", "BF16", "F32"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libsana_linattn.so"
@@ -52,6 +52,10 @@ def _declare(lib):
     for f in (lib.sana_linattn_forward, lib.sana_linattn_kv_state, lib.sana_linattn_apply,
               lib.sana_linattn_qkv_fused):
         f.restype = ctypes.c_int
+    lib.sana_linattn_device_error.argtypes = [ctypes.POINTER(ci), ctypes.POINTER(ci), ci]
+    lib.sana_linattn_device_error.restype = ctypes.c_int
+    lib.sana_linattn_selftest_wait_timeout.argtypes = [i64, vp]
+    lib.sana_linattn_selftest_wait_timeout.restype = ctypes.c_int
     lib.sana_linattn_strerror.argtypes = [ci]
     lib.sana_linattn_strerror.restype = ctypes.c_char_p
     return lib
@@ -174,6 +178,22 @@ def apply(q, gq, kv, H: int, eps: float, out=None, stream=None):
                                    B, N, C, H, float(eps), dt, _stream(stream))
     _check("sana_linattn_apply", rc)
     return out
+
+
+def device_error(clear: bool = True):
+    """(code, site) of the device-side error word (0, 0 when no bounded wait gave up).
+    Synchronous; call after synchronising the work of interest."""
+    code, site = ctypes.c_int(0), ctypes.c_int(0)
+    _check("sana_linattn_device_error",
+           load().sana_linattn_device_error(ctypes.byref(code), ctypes.byref(site),
+                                            1 if clear else 0))
+    return code.value, site.value
+
+
+def selftest_wait_timeout(limit_us: int = 20000, stream=None):
+    """Enqueue the bounded-wait self-test (see include/sana_linattn.h)."""
+    _check("sana_linattn_selftest_wait_timeout",
+           load().sana_linattn_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
 def qkv_fused(x, W, gq, gk, H: int, eps: float, out=None, workspace=None, stream=None):

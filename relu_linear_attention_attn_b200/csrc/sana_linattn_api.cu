@@ -7,6 +7,8 @@
 
 #include "sana_common.cuh"
 #include "simt_kernels.cuh"
+#include "sm100_primitives.cuh"
+#include "tc_kernels.cuh"
 
 namespace sana {
 namespace {
@@ -38,13 +40,44 @@ Plan make_plan(int64_t B, int64_t N, int H) {
     return Plan{(int)S, tps};
 }
 
+// Split plan of the tensor-core pass 1: CTAs of 4 heads x tps tokens (tps a
+// multiple of the 64-token stage), about two waves of 2 CTAs per SM.
+Plan make_plan_tc(int64_t B, int64_t N, int H) {
+    const int64_t groups = B * ((H + tc1::kGroupHeads - 1) / tc1::kGroupHeads);
+    const int64_t max_by_tokens = (N + tc1::kStageTok - 1) / tc1::kStageTok;
+    int64_t S = (kTargetCtas + groups - 1) / groups;
+    if (S > max_by_tokens) S = max_by_tokens;
+    if (S > kMaxSplits) S = kMaxSplits;
+    if (S < 1) S = 1;
+    int64_t tps = (N + S - 1) / S;
+    tps = (tps + tc1::kStageTok - 1) / tc1::kStageTok * tc1::kStageTok;
+    S = (N + tps - 1) / tps;
+    if (S < 1) S = 1;
+    return Plan{(int)S, tps};
+}
+
+// Tiles of 128 tokens per pass-2 CTA: enough CTAs for about two waves.
+int apply_tiles_per_cta(int64_t B, int64_t N, int H) {
+    const int64_t tiles = (N + tc2::kTileTok - 1) / tc2::kTileTok;
+    const int64_t pairs = B * ((H + tc2::kPairHeads - 1) / tc2::kPairHeads);
+    int64_t chunks = (kTargetCtas + pairs - 1) / pairs;
+    if (chunks > tiles) chunks = tiles;
+    if (chunks < 1) chunks = 1;
+    return (int)((tiles + chunks - 1) / chunks);
+}
+
+int max_splits(int64_t B, int64_t N, int H) {
+    const int a = make_plan(B, N, H).S, b = make_plan_tc(B, N, H).S;
+    return a > b ? a : b;
+}
+
 // Workspace layout of the unfused path: [partials B*H*S*1056 fp32][state B*H*1056 fp32].
 struct WsLayout {
     size_t part_off, kv_off, fused_qkv_off, total;
 };
 
 WsLayout ws_layout(int64_t B, int64_t N, int C, int H, bool fused) {
-    const Plan p = make_plan(B, N, H);
+    const int S = max_splits(B, N, H);
     WsLayout w{};
     size_t off = 0;
     if (fused) {
@@ -52,7 +85,7 @@ WsLayout ws_layout(int64_t B, int64_t N, int C, int H, bool fused) {
         off = align_up(off + (size_t)B * N * 3 * C * sizeof(float), 256);
     }
     w.part_off = off;
-    off = align_up(off + (size_t)B * H * p.S * kStateFloats * sizeof(float), 256);
+    off = align_up(off + (size_t)B * H * S * kStateFloats * sizeof(float), 256);
     w.kv_off = off;
     off = align_up(off + (size_t)B * H * kStateFloats * sizeof(float), 256);
     w.total = off;
@@ -106,6 +139,91 @@ void launch_apply(const TI* q, const float* gq, const float* kv, TO* out, int64_
                   int H, int64_t ldq, int64_t ldo, float eps, cudaStream_t st) {
     const dim3 g((unsigned)((N + 127) / 128), H, (unsigned)B);
     apply_simt<TI, TO><<<g, 128, 0, st>>>(q, gq, kv, out, N, H, ldq, ldo, eps, gq != nullptr);
+}
+
+// ---------------------------------------------------------------- TMA tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    }
+    return fn;
+}
+
+// A (B, N, C) bf16 tensor seen by TMA as 3-D (C, N, B), boxes of 64 channels x
+// `rows` tokens x 1 batch, 128-byte swizzle.  Rows past N read as zeros and are
+// not written by stores, so a tile never crosses into the next batch item.
+bool make_tmap_bnc(CUtensorMap* m, const void* base, int64_t B, int64_t N, int C, int rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)N, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {(cuuint64_t)C * 2, (cuuint64_t)N * C * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// Opt the tensor-core kernels into their dynamic shared memory, once per device.
+bool ensure_smem_attrs() {
+    static bool done[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    if (done[dev]) return true;
+    if (cudaFuncSetAttribute(kv_partial_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc1::kSmemBytes) != cudaSuccess)
+        return false;
+    if (cudaFuncSetAttribute(apply_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc2::kSmemBytes) != cudaSuccess)
+        return false;
+    done[dev] = true;
+    return true;
+}
+
+// bf16 pass 1 + combine on the tensor cores.
+int launch_state_tc(const void* k, const void* v, const float* gk, float* part, float* kv,
+                    int64_t B, int64_t N, int C, int H, float eps, cudaStream_t st) {
+    if (!ensure_smem_attrs()) return SANA_ECUDA;
+    CUtensorMap tk, tv;
+    if (!make_tmap_bnc(&tk, k, B, N, C, tc1::kStageTok) ||
+        !make_tmap_bnc(&tv, v, B, N, C, tc1::kStageTok))
+        return SANA_ECUDA;
+    const Plan p = make_plan_tc(B, N, H);
+    const dim3 g1(p.S, (H + tc1::kGroupHeads - 1) / tc1::kGroupHeads, (unsigned)B);
+    kv_partial_tc<<<g1, tc1::kThreads, tc1::kSmemBytes, st>>>(tk, tv, gk, part, (int)N, H, p.S,
+                                                               (int)p.tps, eps, gk != nullptr);
+    kv_combine<<<(unsigned)(B * H), 256, 0, st>>>(part, kv, p.S);
+    return SANA_OK;
+}
+
+// bf16 pass 2 on the tensor cores.
+int launch_apply_tc(const void* q, const float* gq, const float* kv, void* out, int64_t B,
+                    int64_t N, int C, int H, float eps, cudaStream_t st) {
+    if (!ensure_smem_attrs()) return SANA_ECUDA;
+    CUtensorMap tq, to;
+    if (!make_tmap_bnc(&tq, q, B, N, C, tc2::kTileTok) ||
+        !make_tmap_bnc(&to, out, B, N, C, tc2::kTileTok))
+        return SANA_ECUDA;
+    const int tpc = apply_tiles_per_cta(B, N, H);
+    const int64_t tiles = (N + tc2::kTileTok - 1) / tc2::kTileTok;
+    const dim3 g((unsigned)((tiles + tpc - 1) / tpc), (H + tc2::kPairHeads - 1) / tc2::kPairHeads,
+                 (unsigned)B);
+    apply_tc<<<g, tc2::kThreads, tc2::kSmemBytes, st>>>(tq, to, kv, gq, (int)N, H, tpc, eps,
+                                                         gq != nullptr);
+    return SANA_OK;
 }
 
 int validate_qkv(const void* q, const void* k, const void* v, const void* out, int64_t B,
@@ -175,14 +293,14 @@ int sana_linattn_kv_state(const void* k, const void* v, const float* gk, float* 
     const size_t kv_bytes = (size_t)B * H * kStateFloats * sizeof(float);
     if (overlaps(kv, kv_bytes, k, in_bytes) || overlaps(kv, kv_bytes, v, in_bytes))
         return SANA_EINVAL;
-    const Plan p = make_plan(B, N, H);
     float* part = (float*)((char*)workspace + L.part_off);
-    if (dtype == SANA_BF16)
-        launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, kv, B, N, H, C, C, eps, p,
-                           stream);
-    else
-        launch_state<float>((const float*)k, (const float*)v, gk, part, kv, B, N, H, C, C, eps, p,
-                            stream);
+    if (dtype == SANA_BF16) {
+        if ((rc = launch_state_tc(k, v, gk, part, kv, B, N, C, H, eps, stream)) != SANA_OK)
+            return rc;
+    } else {
+        launch_state<float>((const float*)k, (const float*)v, gk, part, kv, B, N, H, C, C, eps,
+                            make_plan(B, N, H), stream);
+    }
     return launch_status();
 }
 
@@ -201,11 +319,12 @@ int sana_linattn_apply(const void* q, const float* gq, const float* kv, void* ou
     if (overlaps(out, bytes, q, bytes) ||
         overlaps(out, bytes, kv, (size_t)B * H * kStateFloats * sizeof(float)))
         return SANA_EINVAL;
-    if (dtype == SANA_BF16)
-        launch_apply<bf16, bf16>((const bf16*)q, gq, kv, (bf16*)out, B, N, H, C, C, eps, stream);
-    else
+    if (dtype == SANA_BF16) {
+        if ((rc = launch_apply_tc(q, gq, kv, out, B, N, C, H, eps, stream)) != SANA_OK) return rc;
+    } else {
         launch_apply<float, float>((const float*)q, gq, kv, (float*)out, B, N, H, C, C, eps,
                                    stream);
+    }
     return launch_status();
 }
 
@@ -230,9 +349,9 @@ int sana_linattn_forward(const void* q, const void* k, const void* v, const floa
     float* part = (float*)((char*)workspace + L.part_off);
     float* kv = (float*)((char*)workspace + L.kv_off);
     if (dtype == SANA_BF16) {
-        launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, kv, B, N, H, C, C, eps, p,
-                           stream);
-        launch_apply<bf16, bf16>((const bf16*)q, gq, kv, (bf16*)out, B, N, H, C, C, eps, stream);
+        if ((rc = launch_state_tc(k, v, gk, part, kv, B, N, C, H, eps, stream)) != SANA_OK)
+            return rc;
+        if ((rc = launch_apply_tc(q, gq, kv, out, B, N, C, H, eps, stream)) != SANA_OK) return rc;
     } else {
         launch_state<float>((const float*)k, (const float*)v, gk, part, kv, B, N, H, C, C, eps, p,
                             stream);
@@ -270,6 +389,28 @@ int sana_linattn_qkv_fused(const void* x, const void* Wqkv, const float* gq, con
     launch_state<float>(qkv + C, qkv + 2 * C, gk, part, kv, B, N, H, 3 * C, 3 * C, eps, p, stream);
     launch_apply<float, bf16>(qkv, gq, kv, (bf16*)out, B, N, H, 3 * C, C, eps, stream);
     return launch_status();
+}
+
+int sana_linattn_selftest_wait_timeout(int64_t limit_us, cudaStream_t stream) {
+    if (limit_us < 0 || limit_us > 10000000) return SANA_EINVAL;
+    wait_timeout_selftest<<<1, 32, 0, stream>>>((uint64_t)limit_us * 1000ull, 999);
+    return launch_status();
+}
+
+int sana_linattn_device_error(int* code, int* site, int clear) {
+    int c = 0, where = 0;
+    if (cudaMemcpyFromSymbol(&c, g_device_error, sizeof(int)) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&where, g_device_error_site, sizeof(int)) != cudaSuccess)
+        return SANA_ECUDA;
+    if (code) *code = c;
+    if (site) *site = where;
+    if (clear) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess ||
+            cudaMemcpyToSymbol(g_device_error_site, &zero, sizeof(int)) != cudaSuccess)
+            return SANA_ECUDA;
+    }
+    return SANA_OK;
 }
 
 }  // extern "C"

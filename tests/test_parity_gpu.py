@@ -197,3 +197,23 @@ def test_validation_with_real_buffers(cuda_lib):
     kv = cuda_lib.kv_state(d["k"], d["v"], d["gk"], w.H, w.eps)
     with pytest.raises(ValueError):
         cuda_lib.apply(q[:, ::2], d["gq"], kv, w.H, w.eps)      # non-contiguous
+
+
+def test_no_device_error_after_the_suite_so_far(cuda_lib):
+    torch.cuda.synchronize()
+    assert cuda_lib.device_error(clear=True) == (0, 0)
+
+
+def test_bounded_wait_gives_up_and_reports(cuda_lib):
+    """A wait that nothing satisfies gives up after its limit, records the error,
+    and leaves the context usable (no trap, no hang)."""
+    cuda_lib.device_error(clear=True)
+    cuda_lib.selftest_wait_timeout(limit_us=20000)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_error(clear=True) == (1, 999)
+    w = CONFIGS[1].scaled(N=200, seed=31)
+    x = make_inputs(w)
+    out = run_forward(cuda_lib, to_dev(x), w)
+    torch.cuda.synchronize()
+    assert_close(out, O.forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps), "bf16")
+    assert cuda_lib.device_error(clear=True) == (0, 0)
