@@ -60,7 +60,8 @@ typedef enum {
     SANA_EALIGN = -2,        /* a pointer violates its alignment requirement       */
     SANA_EUNSUPPORTED = -3,  /* well-formed but not supported (D != 32, too large) */
     SANA_EWORKSPACE = -4,    /* workspace NULL or smaller than the queried size    */
-    SANA_ECUDA = -5          /* a CUDA launch or runtime call failed               */
+    SANA_ECUDA = -5,         /* a CUDA launch or runtime call failed               */
+    SANA_ESCRATCH = -6       /* too large for sana_linattn_forward_noalloc's scratch */
 } sana_status;
 
 typedef enum {
@@ -113,6 +114,31 @@ SANA_API int sana_linattn_qkv_fused(const void* x, const void* Wqkv,
                            const float* gq, const float* gk, void* out,
                            int64_t B, int64_t N, int C, int H, float eps,
                            void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* sana_linattn_forward without a caller-provided workspace, for callers that
+ * cannot allocate device memory: code running inside a CUDA-graph capture or a
+ * framework hook where cudaMalloc is forbidden, allocators that must not be
+ * re-entered, or hosts whose memory budget is fixed up front.  The paper has no
+ * counterpart; this is a library convenience.
+ *
+ * Same arguments, kernels, plan and results as sana_linattn_forward, minus the
+ * workspace.  Its scratch is a 16 MiB array in the library's own device memory,
+ * which every GPU that loads the library holds until the process exits.  The
+ * call allocates nothing and frees nothing.
+ *   - Problems whose workspace (sana_linattn_workspace_bytes(B, N, C, H, 0))
+ *     exceeds 16 MiB return SANA_ESCRATCH; 2048px B=8 and 4096px B=2 at
+ *     C = 2240 fit.
+ *   - The first call on a device looks up the array's device address with the
+ *     device current (cudaGetSymbolAddress); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array and leaves its contents behind; the
+ *     forward path writes every scratch byte before reading it, so stale
+ *     contents never matter.  Calls that overlap on the GPU (different streams,
+ *     no ordering between them) race on the array: serialise them. */
+SANA_API int sana_linattn_forward_noalloc(const void* q, const void* k, const void* v,
+                                          const float* gq, const float* gk, void* out,
+                                          int64_t B, int64_t N, int C, int H, float eps,
+                                          sana_dtype dtype, cudaStream_t stream);
 
 /* Device-side error word of the current device.  The tensor-core kernels bound
  * every wait (about 2 s); a wait that gives up records an error code (1 = wait

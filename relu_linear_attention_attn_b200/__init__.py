@@ -15,7 +15,7 @@ import ctypes
 import os
 import threading
 
-__all__ = ["load", "lib_path", "workspace_bytes", "forward", "kv_state", "apply", "qkv_fused",
+__all__ = ["load", "lib_path", "workspace_bytes", "forward", "forward_noalloc", "kv_state", "apply", "qkv_fused",
            "device_error", "selftest_wait_timeout", "SanaError", "STATUS", "BF16", "F32"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -23,7 +23,7 @@ _LIB_NAME = "libsana_linattn.so"
 
 BF16, F32 = 0, 1
 STATUS = {0: "SANA_OK", -1: "SANA_EINVAL", -2: "SANA_EALIGN", -3: "SANA_EUNSUPPORTED",
-          -4: "SANA_EWORKSPACE", -5: "SANA_ECUDA"}
+          -4: "SANA_EWORKSPACE", -5: "SANA_ECUDA", -6: "SANA_ESCRATCH"}
 
 _lib = None
 _lock = threading.Lock()
@@ -52,6 +52,9 @@ def _declare(lib):
     for f in (lib.sana_linattn_forward, lib.sana_linattn_kv_state, lib.sana_linattn_apply,
               lib.sana_linattn_qkv_fused):
         f.restype = ctypes.c_int
+    lib.sana_linattn_forward_noalloc.argtypes = [vp, vp, vp, fp, fp, vp, i64, i64, ci, ci, cf, ci,
+                                                 vp]
+    lib.sana_linattn_forward_noalloc.restype = ctypes.c_int
     lib.sana_linattn_device_error.argtypes = [ctypes.POINTER(ci), ctypes.POINTER(ci), ci]
     lib.sana_linattn_device_error.restype = ctypes.c_int
     lib.sana_linattn_selftest_wait_timeout.argtypes = [i64, vp]
@@ -149,6 +152,24 @@ def forward(q, k, v, gq, gk, H: int, eps: float, out=None, workspace=None, strea
                                      _gain(gk, "gk"), _dev(out, "out"), B, N, C, H, float(eps), dt,
                                      None if ws is None else ws.data_ptr(), wsb, _stream(stream))
     _check("sana_linattn_forward", rc)
+    return out
+
+
+def forward_noalloc(q, k, v, gq, gk, H: int, eps: float, out=None, stream=None):
+    """forward() without a workspace: the library's static 16 MiB device scratch is
+    used instead, for callers that cannot allocate device memory (see
+    sana_linattn_forward_noalloc in include/sana_linattn.h).  Only `out` is
+    allocated here when not given."""
+    B, N, C = q.shape
+    if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share shape and dtype")
+    dt = _dtype_code(q)
+    if out is None:
+        out = _torch().empty_like(q)
+    rc = load().sana_linattn_forward_noalloc(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
+                                             _gain(gq, "gq"), _gain(gk, "gk"), _dev(out, "out"),
+                                             B, N, C, H, float(eps), dt, _stream(stream))
+    _check("sana_linattn_forward_noalloc", rc)
     return out
 
 

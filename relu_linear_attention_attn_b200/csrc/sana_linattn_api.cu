@@ -5,6 +5,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "sana_common.cuh"
 #include "simt_kernels.cuh"
 #include "sm100_primitives.cuh"
@@ -247,6 +249,36 @@ int validate_ws(void* ws, size_t ws_bytes, size_t need) {
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------- static scratch
+// Scratch for sana_linattn_forward_noalloc: a fixed array in the module's device
+// memory, created when the library's module is loaded on a device and held by
+// every device that loads it until the process exits.
+constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// array's name only stands in for the symbol; its device address has to be
+// looked up once per device, with that device current.
+int noalloc_scratch(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SANA_ECUDA;
+    if (dev < 0 || dev >= 64) return SANA_EUNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return SANA_ECUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SANA_OK;
+}
+}  // namespace
 }  // namespace sana
 
 using namespace sana;
@@ -266,6 +298,9 @@ const char* sana_linattn_strerror(int status) {
         case SANA_EUNSUPPORTED: return "unsupported configuration (head dim must be 32)";
         case SANA_EWORKSPACE: return "workspace missing or smaller than required";
         case SANA_ECUDA: return "CUDA launch or runtime error";
+        case SANA_ESCRATCH:
+            return "problem needs more scratch than the static 16 MiB array of "
+                   "sana_linattn_forward_noalloc (use sana_linattn_forward with a workspace)";
         default: return "unknown status";
     }
 }
@@ -389,6 +424,22 @@ int sana_linattn_qkv_fused(const void* x, const void* Wqkv, const float* gq, con
     launch_state<float>(qkv + C, qkv + 2 * C, gk, part, kv, B, N, H, 3 * C, 3 * C, eps, p, stream);
     launch_apply<float, bf16>(qkv, gq, kv, (bf16*)out, B, N, H, 3 * C, C, eps, stream);
     return launch_status();
+}
+
+int sana_linattn_forward_noalloc(const void* q, const void* k, const void* v, const float* gq,
+                                 const float* gk, void* out, int64_t B, int64_t N, int C, int H,
+                                 float eps, sana_dtype dtype, cudaStream_t stream) {
+    int rc;
+    if ((rc = check_dims(B, N, C, H)) != SANA_OK) return rc;
+    if (B > 0 && N > 0 && ws_layout(B, N, C, H, false).total > kNoAllocScratchBytes)
+        return SANA_ESCRATCH;
+    void* scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch)) != SANA_OK) return rc;
+    // Same kernels and plan as sana_linattn_forward; the scratch takes the place
+    // of the caller's workspace.  Every scratch byte the forward path reads it
+    // has written earlier in the same call, so nothing needs clearing.
+    return sana_linattn_forward(q, k, v, gq, gk, out, B, N, C, H, eps, dtype, scratch,
+                                kNoAllocScratchBytes, stream);
 }
 
 int sana_linattn_selftest_wait_timeout(int64_t limit_us, cudaStream_t stream) {
