@@ -42,40 +42,63 @@ Plan make_plan(int64_t B, int64_t N, int H) {
     return Plan{(int)S, tps};
 }
 
-// Split plan of the tensor-core pass 1: CTAs of 4 heads x tps tokens (tps a
-// multiple of the 64-token stage), about two waves of 2 CTAs per SM.
-Plan make_plan_tc(int64_t B, int64_t N, int H) {
-    const int64_t groups = B * ((H + tc1::kGroupHeads - 1) / tc1::kGroupHeads);
-    const int64_t max_by_tokens = (N + tc1::kStageTok - 1) / tc1::kStageTok;
-    int64_t S = (kTargetCtas + groups - 1) / groups;
-    if (S > max_by_tokens) S = max_by_tokens;
-    if (S > kMaxSplits) S = kMaxSplits;
-    if (S < 1) S = 1;
-    int64_t tps = (N + S - 1) / S;
-    tps = (tps + tc1::kStageTok - 1) / tc1::kStageTok * tc1::kStageTok;
-    S = (N + tps - 1) / tps;
-    if (S < 1) S = 1;
-    return Plan{(int)S, tps};
+// Plans of the persistent tensor-core passes.  The CTA count is the device's SM
+// count capped at kMaxPersistentCtas; workspace sizes use the cap, which bounds
+// every smaller count.
+constexpr int kMaxPersistentCtas = 160;
+constexpr int kMinItemsPerCta = 4;
+
+struct PersistPlan1 {
+    int G, R, Smax, P;   // head groups, stages per row, partial slots per row, CTAs
+    int64_t T;           // work items
+};
+
+PersistPlan1 make_plan_p1(int64_t B, int64_t N, int H, int P) {
+    PersistPlan1 p{};
+    p.G = (H + p1::kGroupHeads - 1) / p1::kGroupHeads;
+    p.R = (int)((N + p1::kStageTok - 1) / p1::kStageTok);
+    p.T = B * p.G * (int64_t)p.R;
+    // At least kMinItemsPerCta stages per CTA (small problems use fewer SMs, and
+    // a row is split among fewer partial states); never an empty range, since the
+    // slot count of a row counts every CTA between the owners of its first and
+    // last items.
+    const int64_t cap = (p.T + kMinItemsPerCta - 1) / kMinItemsPerCta;
+    p.P = (int)(cap < P ? cap : P);
+    P = p.P;
+    // A row's R consecutive items meet at most 1 + ceil((R-1)/L) ranges of length
+    // >= L = floor(T/P), and never more than R of them.
+    const int64_t L = p.T / P;
+    int64_t smax = p.R;
+    if (L >= 1) {
+        const int64_t bound = 1 + (p.R - 1 + L - 1) / L;
+        if (bound < smax) smax = bound;
+    }
+    p.Smax = (int)smax;
+    return p;
 }
 
-// Tiles of 128 tokens per pass-2 CTA: enough CTAs for about two waves.
-int apply_tiles_per_cta(int64_t B, int64_t N, int H) {
-    const int64_t tiles = (N + tc2::kTileTok - 1) / tc2::kTileTok;
-    const int64_t pairs = B * ((H + tc2::kPairHeads - 1) / tc2::kPairHeads);
-    int64_t chunks = (kTargetCtas + pairs - 1) / pairs;
-    if (chunks > tiles) chunks = tiles;
-    if (chunks < 1) chunks = 1;
-    return (int)((tiles + chunks - 1) / chunks);
+struct PersistPlan2 {
+    int Pp, R, P;        // head pairs, tiles per row, CTAs
+    int64_t T;
+};
+
+PersistPlan2 make_plan_p2(int64_t B, int64_t N, int H, int P) {
+    PersistPlan2 p{};
+    p.Pp = (H + p2::kPairHeads - 1) / p2::kPairHeads;
+    p.R = (int)((N + p2::kTileTok - 1) / p2::kTileTok);
+    p.T = B * p.Pp * (int64_t)p.R;
+    p.P = (int)(p.T < P ? p.T : P);
+    return p;
 }
 
 int max_splits(int64_t B, int64_t N, int H) {
-    const int a = make_plan(B, N, H).S, b = make_plan_tc(B, N, H).S;
+    const int a = make_plan(B, N, H).S, b = make_plan_p1(B, N, H, kMaxPersistentCtas).Smax;
     return a > b ? a : b;
 }
 
 // Workspace layout of the unfused path: [partials B*H*S*1056 fp32][state B*H*1056 fp32].
 struct WsLayout {
-    size_t part_off, kv_off, fused_qkv_off, total;
+    size_t part_off, kv_off, fused_qkv_off, counters_off, total;
 };
 
 WsLayout ws_layout(int64_t B, int64_t N, int C, int H, bool fused) {
@@ -86,6 +109,8 @@ WsLayout ws_layout(int64_t B, int64_t N, int C, int H, bool fused) {
         w.fused_qkv_off = off;
         off = align_up(off + (size_t)B * N * 3 * C * sizeof(float), 256);
     }
+    w.counters_off = off;
+    off = align_up(off + (size_t)B * ((H + 3) / 4) * sizeof(int), 256);
     w.part_off = off;
     off = align_up(off + (size_t)B * H * S * kStateFloats * sizeof(float), 256);
     w.kv_off = off;
@@ -175,56 +200,81 @@ bool make_tmap_bnc(CUtensorMap* m, const void* base, int64_t B, int64_t N, int C
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }
 
-// Opt the tensor-core kernels into their dynamic shared memory, once per device.
-bool ensure_smem_attrs() {
-    static bool done[64] = {};
+// The tensor-core kernels keep the gains of every channel in shared memory, so they
+// take C <= 4096 (H <= 128); wider problems run the CUDA-core kernels.
+bool tc_path(sana_dtype dt, int C) { return dt == SANA_BF16 && C <= p1::kGainCache; }
+
+// Per-device setup of the persistent kernels: dynamic shared memory opt-in and
+// the CTA count (SM count, capped).  Returns 0 on failure.
+int persistent_ctas() {
+    static int ctas[64] = {};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-    if (done[dev]) return true;
-    if (cudaFuncSetAttribute(kv_partial_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             tc1::kSmemBytes) != cudaSuccess)
-        return false;
-    if (cudaFuncSetAttribute(apply_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             tc2::kSmemBytes) != cudaSuccess)
-        return false;
-    done[dev] = true;
-    return true;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (ctas[dev]) return ctas[dev];
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms <= 0)
+        return 0;
+    if (cudaFuncSetAttribute(kv_reduce_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             p1::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(apply_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             p2::kSmemBytes) != cudaSuccess)
+        return 0;
+    ctas[dev] = sms < kMaxPersistentCtas ? sms : kMaxPersistentCtas;
+    return ctas[dev];
 }
 
-// bf16 pass 1 + combine on the tensor cores.
-int launch_state_tc(const void* k, const void* v, const float* gk, float* part, float* kv,
-                    int64_t B, int64_t N, int C, int H, float eps, cudaStream_t st) {
-    if (!ensure_smem_attrs()) return SANA_ECUDA;
+// bf16 pass 1 (reduction and last-CTA combine) on the tensor cores.  The row
+// counters in the workspace are zeroed first; the final state lands in kv.
+int launch_state_tc(const void* k, const void* v, const float* gk, int* counters, float* part,
+                    float* kv, int64_t B, int64_t N, int C, int H, float eps, cudaStream_t st) {
+    const int P = persistent_ctas();
+    if (P == 0) return SANA_ECUDA;
     CUtensorMap tk, tv;
-    if (!make_tmap_bnc(&tk, k, B, N, C, tc1::kStageTok) ||
-        !make_tmap_bnc(&tv, v, B, N, C, tc1::kStageTok))
+    if (!make_tmap_bnc(&tk, k, B, N, C, p1::kStageTok) ||
+        !make_tmap_bnc(&tv, v, B, N, C, p1::kStageTok))
         return SANA_ECUDA;
-    const Plan p = make_plan_tc(B, N, H);
-    const dim3 g1(p.S, (H + tc1::kGroupHeads - 1) / tc1::kGroupHeads, (unsigned)B);
-    kv_partial_tc<<<g1, tc1::kThreads, tc1::kSmemBytes, st>>>(tk, tv, gk, part, (int)N, H, p.S,
-                                                               (int)p.tps, eps, gk != nullptr);
-    kv_combine<<<(unsigned)(B * H), 256, 0, st>>>(part, kv, p.S);
+    const PersistPlan1 pl = make_plan_p1(B, N, H, P);
+    if (cudaMemsetAsync(counters, 0, (size_t)B * pl.G * sizeof(int), st) != cudaSuccess)
+        return SANA_ECUDA;
+    P1Args a{};
+    a.gk = gk; a.part = part; a.kv = kv; a.counters = counters; a.T = pl.T;
+    a.N = (int)N; a.H = H; a.G = pl.G; a.R = pl.R; a.Smax = pl.Smax; a.P = pl.P;
+    a.eps = eps; a.norm = gk != nullptr;
+    kv_reduce_persistent<<<pl.P, p1::kThreads, p1::kSmemBytes, st>>>(tk, tv, a);
     return SANA_OK;
 }
 
-// bf16 pass 2 on the tensor cores.
+// bf16 pass 2 on the tensor cores.  chained: launched right behind pass 1 of the
+// same call, as a programmatic dependent launch (its Q stream starts while pass 1
+// finishes; only the state read waits for pass 1).
 int launch_apply_tc(const void* q, const float* gq, const float* kv, void* out, int64_t B,
-                    int64_t N, int C, int H, float eps, cudaStream_t st) {
-    if (!ensure_smem_attrs()) return SANA_ECUDA;
+                    int64_t N, int C, int H, float eps, cudaStream_t st, bool chained) {
+    const int P = persistent_ctas();
+    if (P == 0) return SANA_ECUDA;
     CUtensorMap tq, to;
-    if (!make_tmap_bnc(&tq, q, B, N, C, tc2::kTileTok) ||
-        !make_tmap_bnc(&to, out, B, N, C, tc2::kTileTok))
+    if (!make_tmap_bnc(&tq, q, B, N, C, p2::kTileTok) ||
+        !make_tmap_bnc(&to, out, B, N, C, p2::kTileTok))
         return SANA_ECUDA;
-    const int tpc = apply_tiles_per_cta(B, N, H);
-    const int64_t tiles = (N + tc2::kTileTok - 1) / tc2::kTileTok;
-    const dim3 g((unsigned)((tiles + tpc - 1) / tpc), (H + tc2::kPairHeads - 1) / tc2::kPairHeads,
-                 (unsigned)B);
-    apply_tc<<<g, tc2::kThreads, tc2::kSmemBytes, st>>>(tq, to, kv, gq, (int)N, H, tpc, eps,
-                                                         gq != nullptr);
+    const PersistPlan2 pl = make_plan_p2(B, N, H, P);
+    P2Args a{};
+    a.kv = kv; a.gq = gq; a.T = pl.T; a.N = (int)N; a.H = H; a.Pp = pl.Pp; a.R = pl.R;
+    a.P = pl.P; a.eps = eps; a.norm = gq != nullptr;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.P);
+    cfg.blockDim = dim3(p2::kThreads);
+    cfg.dynamicSmemBytes = p2::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = chained ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, apply_persistent, tq, to, a) != cudaSuccess) return SANA_ECUDA;
     return SANA_OK;
 }
 
@@ -329,9 +379,14 @@ int sana_linattn_kv_state(const void* k, const void* v, const float* gk, float* 
     if (overlaps(kv, kv_bytes, k, in_bytes) || overlaps(kv, kv_bytes, v, in_bytes))
         return SANA_EINVAL;
     float* part = (float*)((char*)workspace + L.part_off);
-    if (dtype == SANA_BF16) {
-        if ((rc = launch_state_tc(k, v, gk, part, kv, B, N, C, H, eps, stream)) != SANA_OK)
+    if (tc_path(dtype, C)) {
+        int* counters = (int*)((char*)workspace + L.counters_off);
+        if ((rc = launch_state_tc(k, v, gk, counters, part, kv, B, N, C, H, eps, stream)) !=
+            SANA_OK)
             return rc;
+    } else if (dtype == SANA_BF16) {
+        launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, kv, B, N, H, C, C, eps,
+                           make_plan(B, N, H), stream);
     } else {
         launch_state<float>((const float*)k, (const float*)v, gk, part, kv, B, N, H, C, C, eps,
                             make_plan(B, N, H), stream);
@@ -354,8 +409,11 @@ int sana_linattn_apply(const void* q, const float* gq, const float* kv, void* ou
     if (overlaps(out, bytes, q, bytes) ||
         overlaps(out, bytes, kv, (size_t)B * H * kStateFloats * sizeof(float)))
         return SANA_EINVAL;
-    if (dtype == SANA_BF16) {
-        if ((rc = launch_apply_tc(q, gq, kv, out, B, N, C, H, eps, stream)) != SANA_OK) return rc;
+    if (tc_path(dtype, C)) {
+        if ((rc = launch_apply_tc(q, gq, kv, out, B, N, C, H, eps, stream, false)) != SANA_OK)
+            return rc;
+    } else if (dtype == SANA_BF16) {
+        launch_apply<bf16, bf16>((const bf16*)q, gq, kv, (bf16*)out, B, N, H, C, C, eps, stream);
     } else {
         launch_apply<float, float>((const float*)q, gq, kv, (float*)out, B, N, H, C, C, eps,
                                    stream);
@@ -383,10 +441,17 @@ int sana_linattn_forward(const void* q, const void* k, const void* v, const floa
     const Plan p = make_plan(B, N, H);
     float* part = (float*)((char*)workspace + L.part_off);
     float* kv = (float*)((char*)workspace + L.kv_off);
-    if (dtype == SANA_BF16) {
-        if ((rc = launch_state_tc(k, v, gk, part, kv, B, N, C, H, eps, stream)) != SANA_OK)
+    if (tc_path(dtype, C)) {
+        int* counters = (int*)((char*)workspace + L.counters_off);
+        if ((rc = launch_state_tc(k, v, gk, counters, part, kv, B, N, C, H, eps, stream)) !=
+            SANA_OK)
             return rc;
-        if ((rc = launch_apply_tc(q, gq, kv, out, B, N, C, H, eps, stream)) != SANA_OK) return rc;
+        if ((rc = launch_apply_tc(q, gq, kv, out, B, N, C, H, eps, stream, true)) != SANA_OK)
+            return rc;
+    } else if (dtype == SANA_BF16) {
+        launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, kv, B, N, H, C, C, eps, p,
+                           stream);
+        launch_apply<bf16, bf16>((const bf16*)q, gq, kv, (bf16*)out, B, N, H, C, C, eps, stream);
     } else {
         launch_state<float>((const float*)k, (const float*)v, gk, part, kv, B, N, H, C, C, eps, p,
                             stream);

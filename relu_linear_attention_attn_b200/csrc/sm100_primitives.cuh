@@ -54,27 +54,33 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// One bounded try: the thread may be suspended (not spinning) until the phase
+// completes or about `suspend_ns` pass; returns whether the phase completed.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity,
+                                              uint32_t suspend_ns) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.b32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
         : "memory");
     return done != 0;
 }
 
-// Wait for the phase with the given parity to complete.  Gives up after
+// Wait for the phase with the given parity to complete.  The waiting thread
+// sleeps in try_wait (woken when the phase completes) rather than polling, so
+// idle roles leave the issue slots to the working warps.  Gives up after
 // `limit_ns` of wall time (default 2 s, far beyond any legitimate wait here),
 // records kErrWaitTimeout with `site`, and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site,
                                           uint64_t limit_ns = 2000000000ull) {
-    if (mbar_try_wait(bar, parity)) return true;
+    const uint32_t hint = limit_ns < 1000000ull ? (uint32_t)limit_ns : 1000000u;
+    if (mbar_try_wait(bar, parity, hint)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait(bar, parity, hint)) return true;
         if (global_timer_ns() - t0 > limit_ns) {
             record_error(kErrWaitTimeout, site);
             return false;
@@ -91,6 +97,17 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ------------------------------------------------------------------ dependent launch
+// Programmatic dependent launch: the primary grid allows its dependent grid to be
+// scheduled; the dependent grid waits for the primary grid's completion (and the
+// visibility of its memory writes) before touching what the primary produced.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_primary() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ TMA
@@ -113,6 +130,17 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(m), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Plain bulk copy global -> shared (no tensor map); 16-byte aligned, size a
+// multiple of 16; completes `bytes` transactions on the mbarrier.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -243,6 +271,17 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool a_mn_m
 // 1024-byte boundary.
 __host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+// ------------------------------------------------------------------ work split
+// A flat list of T work items split over P CTAs in contiguous, balanced ranges:
+// CTA c owns [range_begin(c), range_begin(c + 1)).
+__host__ __device__ __forceinline__ int64_t range_begin(int64_t c, int64_t T, int64_t P) {
+    return c * T / P;
+}
+// The CTA whose range holds item i (the largest c with range_begin(c) <= i).
+__host__ __device__ __forceinline__ int64_t owner_cta(int64_t i, int64_t T, int64_t P) {
+    return ((i + 1) * P + T - 1) / T - 1;
 }
 
 }  // namespace sana

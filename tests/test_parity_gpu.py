@@ -217,3 +217,14 @@ def test_bounded_wait_gives_up_and_reports(cuda_lib):
     torch.cuda.synchronize()
     assert_close(out, O.forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps), "bf16")
     assert cuda_lib.device_error(clear=True) == (0, 0)
+
+
+def test_wide_head_count_runs_the_cuda_core_path(cuda_lib):
+    """H = 130 (C = 4160) is past the tensor-core kernels' gain cache; the library
+    runs its CUDA-core kernels for bf16 there, with the same results."""
+    w = Workload("wide", B=1, N=300, C=32 * 130, H=130, dtype="bf16", recipe="gaussian",
+                 gains="random", eps=1e-6, seed=77)
+    x = make_inputs(w)
+    out = run_forward(cuda_lib, to_dev(x), w)
+    torch.cuda.synchronize()
+    assert_close(out, O.forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps), "bf16")
