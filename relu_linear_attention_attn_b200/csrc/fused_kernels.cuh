@@ -1,0 +1,639 @@
+// The variant fused with the QKV projection ("Sana: Efficient High-Resolution
+// Image Synthesis with Linear Diffusion Transformers", section 7, on-device
+// deployment: the ReLU(K)^T V reduction fused with the QKV projection), on the
+// sm_100a tensor cores.  The projected Q, K and V never leave the SM: they are
+// accumulated in TMEM (fp32), normalised in fp32, and only their bf16 feature
+// maps reach shared memory as operands of the attention contractions.
+//
+//   fused_kv (F1)  CTA (s, g, b): token tiles [s*tps, (s+1)*tps) of batch b,
+//                  head group g (4 heads).  Per tile of 128 tokens:
+//                    [K | V] = x_tile * Wqkv[:, K and V columns of g]   (UMMA 128x256, K=2240)
+//                    phi(K), V -> bf16 operands in smem
+//                    S += phi(K)^T [V | 1]                              (UMMA 128x128 + 128x64)
+//                  then the CTA's partial state, and the last CTA of (b, g)
+//                  sums the partials in split order.
+//   fused_qo (F2)  CTA (s, g, b), same tiles:
+//                    Q = x_tile * Wqkv[:, Q columns of g]               (UMMA 128x128)
+//                    A' = ReLU(gq * q) (bf16), r = rsqrt(mean(q^2) + eps) kept in registers
+//                    D = A' [S_hi | S_lo]                               (UMMA 128x48 per head)
+//                    O = r D[:, :32] / (r D[:, 32] + eps)  -> TMA store
+//                  Only the B-operand build reads the states F1 wrote, so under
+//                  programmatic dependent launch the Q projection overlaps F1's tail.
+//
+// Operand layouts (all 128-byte swizzle, 1024-byte aligned):
+//   x tile        K-major: [128 tokens][64 k] per stage (TMA 3-D map over (C, N, B))
+//   W blocks      MN-major: [64 k][64 n] boxes (TMA 3-D map over (n, section, k)),
+//                 consecutive boxes 8 KB apart form one N = 64 * boxes operand
+//   phi(K), V     MN-major: [128 tokens][64 ch] blocks, 16 KB apart
+//   A' / O        K-major:  [128 tokens][64 ch] blocks (2 heads each), 16 KB apart
+#pragma once
+
+#include "sana_common.cuh"
+#include "sm100_primitives.cuh"
+#include "tc_kernels.cuh"
+
+namespace sana {
+
+namespace fz {
+constexpr int kTileTok = 128;                      // UMMA M
+constexpr int kGroupHeads = 4;                     // heads per CTA
+constexpr int kKStep = 64;                         // k elements per pipeline stage
+constexpr int kXBytes = kTileTok * 128;            // x box: 128 tokens x 64 k = 16 KB
+constexpr int kWBox = kKStep * 128;                // W box: 64 k x 64 n = 8 KB
+constexpr int kBlock = kTileTok * 128;             // 128 tokens x 64 channels = 16 KB
+}  // namespace fz
+
+// ============================================================================ F1
+namespace f1 {
+constexpr int kStageBytes = fz::kXBytes + 4 * fz::kWBox;   // x + K (2 boxes) + V (2 boxes)
+constexpr int kStages = 3;
+constexpr int kOpBytes = 2 * fz::kBlock;                   // phi(K) or V: 128 tokens x 128 ch
+constexpr int kOnesBytes = 16 * 128;
+constexpr int kAccCols = 256;                              // [K | V] accumulator
+constexpr int kKvCol = 256;                                // state accumulator at column 256
+constexpr int kTmemCols = 512;
+constexpr int kThreads = 192;                              // TMA, UMMA, 4 epilogue warps
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 2 * kOpBytes + kOnesBytes + 2048;
+}  // namespace f1
+
+struct F1Args {
+    const float* gk;     // [C] or nullptr (norm off)
+    float* part;         // [B][H][S][D][D+1]
+    float* kv;           // [B][H][D][D+1]
+    int* counters;       // [B * G], zero on entry
+    int N, H, C, S, tps; // tokens per batch, heads, channels, splits, tiles per split
+    float eps;
+    int norm;
+};
+
+__global__ void __launch_bounds__(f1::kThreads, 1)
+fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+         const F1Args a)
+{
+    using namespace f1;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align_1024(smem_raw);
+    uint8_t* stages = smem;
+    uint8_t* opk = stages + kStages * kStageBytes;          // phi(K): A operand of the state MMA
+    uint8_t* opv = opk + kOpBytes;                          // V: B operand
+    uint8_t* ones = opv + kOpBytes;
+    float* sg = (float*)(ones + kOnesBytes);                // 128 gains of the group
+    uint64_t* full = (uint64_t*)(sg + 128);
+    uint64_t* empty = full + kStages;
+    uint64_t* accfull = empty + kStages;
+    uint64_t* accempty = accfull + 1;
+    uint64_t* opready = accempty + 1;
+    uint64_t* opfree = opready + 1;
+    uint64_t* kvdone = opfree + 1;
+    uint32_t* tmem_slot = (uint32_t*)(kvdone + 1);
+    int* last_flag = (int*)(tmem_slot + 1);
+
+    pdl_launch_dependents();
+
+    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles = (a.N + fz::kTileTok - 1) / fz::kTileTok;
+    const int t0 = s * a.tps;
+    const int nt = min(a.tps, tiles - t0);
+    const int ksteps = (a.C + fz::kKStep - 1) / fz::kKStep;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(accfull, 1);
+        mbar_init(accempty, 128);
+        mbar_init(opready, 128);
+        mbar_init(opfree, 1);
+        mbar_init(kvdone, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmap_x);
+        prefetch_tmap(&tmap_w);
+    }
+    for (int i = threadIdx.x; i < kOnesBytes / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(ones)[i] = make_uint4(0, 0, 0, 0);
+    for (int i = threadIdx.x; i < 128; i += blockDim.x) {
+        const int h = g * fz::kGroupHeads + i / kD;
+        sg[i] = (a.norm && h < a.H) ? a.gk[(size_t)h * kD + (i % kD)] : 1.f;
+    }
+    __syncthreads();
+    if (threadIdx.x < 16)
+        *reinterpret_cast<uint16_t*>(ones + sw128_offset(threadIdx.x, 0)) = 0x3F80;   // bf16 1.0
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = nt > 0;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0 && ok) {
+            int64_t step = 0, last = -1;
+            for (int ti = 0; ti < nt && ok; ++ti) {
+                const int y = (t0 + ti) * fz::kTileTok;
+                for (int kk = 0; kk < ksteps; ++kk, ++step) {
+                    const int st = (int)(step % kStages);
+                    if (step >= kStages)
+                        ok = mbar_wait(&empty[st], (uint32_t)((step / kStages) - 1) & 1, 501);
+                    if (!ok) break;
+                    uint8_t* sb = stages + st * kStageBytes;
+                    mbar_arrive_expect_tx(&full[st], kStageBytes);
+                    tma_load_3d(sb, &tmap_x, &full[st], kk * fz::kKStep, y, b);
+                    const int n0 = g * 128;
+                    tma_load_3d(sb + fz::kXBytes, &tmap_w, &full[st], n0, 1, kk * fz::kKStep);
+                    tma_load_3d(sb + fz::kXBytes + fz::kWBox, &tmap_w, &full[st], n0 + 64, 1,
+                                kk * fz::kKStep);
+                    tma_load_3d(sb + fz::kXBytes + 2 * fz::kWBox, &tmap_w, &full[st], n0, 2,
+                                kk * fz::kKStep);
+                    tma_load_3d(sb + fz::kXBytes + 3 * fz::kWBox, &tmap_w, &full[st], n0 + 64, 2,
+                                kk * fz::kKStep);
+                    last = step;
+                }
+            }
+            if (!ok) {
+                for (int st = 0; st < kStages; ++st) {
+                    const int64_t li = last - ((last - st) % kStages + kStages) % kStages;
+                    if (last >= 0 && li >= 0)
+                        mbar_wait(&full[st], (uint32_t)(li / kStages) & 1, 502);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ UMMA issuer
+        if (lane == 0 && ok) {
+            const uint32_t idesc_g = make_idesc_bf16(128, 256, false, true);   // x K-major, W MN-major
+            const uint32_t idesc_v = make_idesc_bf16(128, 128, true, true);    // phi(K), V MN-major
+            const uint32_t idesc_1 = make_idesc_bf16(128, 64, true, true);
+            const uint64_t ones_desc = make_smem_desc(smem_u32(ones), fz::kBlock, 1024, kSwizzle128B);
+            int64_t step = 0;
+            for (int ti = 0; ti < nt && ok; ++ti) {
+                if (ti > 0) ok = mbar_wait(accempty, (uint32_t)(ti - 1) & 1, 503);
+                if (!ok) break;
+                tc_fence_after_sync();
+                for (int kk = 0; kk < ksteps && ok; ++kk, ++step) {
+                    const int st = (int)(step % kStages);
+                    ok = mbar_wait(&full[st], (uint32_t)(step / kStages) & 1, 504);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    const uint32_t xb = smem_u32(stages + st * kStageBytes);
+                    const uint32_t wb = xb + fz::kXBytes;
+#pragma unroll
+                    for (int k4 = 0; k4 < fz::kKStep / 16; ++k4) {
+                        const uint64_t ad = make_smem_desc(xb + k4 * 32, 16, 1024, kSwizzle128B);
+                        const uint64_t bd = make_smem_desc(wb + k4 * 2048, fz::kWBox, 1024, kSwizzle128B);
+                        umma_bf16(tmem, ad, bd, idesc_g, kk > 0 || k4 > 0);
+                    }
+                    umma_commit(&empty[st]);
+                }
+                if (!ok) break;
+                umma_commit(accfull);
+                // the state contraction of this tile, once the epilogue has written its operands
+                ok = mbar_wait(opready, (uint32_t)ti & 1, 505);
+                if (!ok) break;
+                tc_fence_after_sync();
+                const uint32_t kb = smem_u32(opk), vb = smem_u32(opv);
+#pragma unroll
+                for (int k4 = 0; k4 < fz::kTileTok / 16; ++k4) {
+                    const uint64_t ad = make_smem_desc(kb + k4 * 2048, fz::kBlock, 1024, kSwizzle128B);
+                    const uint64_t bd = make_smem_desc(vb + k4 * 2048, fz::kBlock, 1024, kSwizzle128B);
+                    const bool acc = ti > 0 || k4 > 0;
+                    umma_bf16(tmem + kKvCol, ad, bd, idesc_v, acc);
+                    umma_bf16(tmem + kKvCol + 128, ad, ones_desc, idesc_1, acc);
+                }
+                umma_commit(opfree);
+            }
+            umma_commit(kvdone);
+            mbar_wait(kvdone, 0, 506);
+        }
+    } else {
+        // ------------------------------------------------ epilogue: phi(K), V, then the state
+        const int et = threadIdx.x - 64;                  // 0..127
+        const int q = warp & 3;                           // TMEM lane quadrant
+        const int row = 32 * q + lane;                    // token row of the tile
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        for (int ti = 0; ti < nt && ok; ++ti) {
+            ok = mbar_wait(accfull, (uint32_t)ti & 1, 507);
+            if (ok && ti > 0) ok = mbar_wait(opfree, (uint32_t)(ti - 1) & 1, 508);
+            if (!ok) break;
+            tc_fence_after_sync();
+            const bool row_live = (t0 + ti) * fz::kTileTok + row < a.N;
+#pragma unroll 1
+            for (int j = 0; j < fz::kGroupHeads; ++j) {
+                float kx[32], vx[32];
+                tmem_ld16(lane_base + 32 * j, kx);
+                tmem_ld16(lane_base + 32 * j + 16, kx + 16);
+                tmem_ld16(lane_base + 128 + 32 * j, vx);
+                tmem_ld16(lane_base + 128 + 32 * j + 16, vx + 16);
+                tmem_wait_ld();
+                const bool live = row_live && (g * fz::kGroupHeads + j < a.H);
+                if (a.norm) {
+                    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        s0 = fmaf(kx[i], kx[i], s0);
+                        s1 = fmaf(kx[i + 1], kx[i + 1], s1);
+                        s2 = fmaf(kx[i + 2], kx[i + 2], s2);
+                        s3 = fmaf(kx[i + 3], kx[i + 3], s3);
+                    }
+                    const float r = rsqrtf(((s0 + s1) + (s2 + s3)) * (1.f / kD) + a.eps);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) kx[i] = fmaxf(sg[j * kD + i] * (kx[i] * r), 0.f);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) kx[i] = fmaxf(kx[i], 0.f);
+                }
+                uint8_t* kblk = opk + (j >> 1) * fz::kBlock;
+                uint8_t* vblk = opv + (j >> 1) * fz::kBlock;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint4 wk, wv;
+                    if (live) {
+                        wk.x = pack_bf16x2(kx[8 * c + 0], kx[8 * c + 1]);
+                        wk.y = pack_bf16x2(kx[8 * c + 2], kx[8 * c + 3]);
+                        wk.z = pack_bf16x2(kx[8 * c + 4], kx[8 * c + 5]);
+                        wk.w = pack_bf16x2(kx[8 * c + 6], kx[8 * c + 7]);
+                        wv.x = pack_bf16x2(vx[8 * c + 0], vx[8 * c + 1]);
+                        wv.y = pack_bf16x2(vx[8 * c + 2], vx[8 * c + 3]);
+                        wv.z = pack_bf16x2(vx[8 * c + 4], vx[8 * c + 5]);
+                        wv.w = pack_bf16x2(vx[8 * c + 6], vx[8 * c + 7]);
+                    } else {
+                        wk = make_uint4(0, 0, 0, 0);
+                        wv = make_uint4(0, 0, 0, 0);
+                    }
+                    const uint32_t off = sw128_offset(row, (j & 1) * 4 + c);
+                    *reinterpret_cast<uint4*>(kblk + off) = wk;
+                    *reinterpret_cast<uint4*>(vblk + off) = wv;
+                }
+            }
+            tc_fence_before_sync();
+            mbar_arrive(accempty);
+            fence_proxy_async_smem();
+            mbar_arrive(opready);
+        }
+        if (ok) ok = mbar_wait(kvdone, 0, 509);
+        if (ok) {
+            // the CTA's partial state: diagonal blocks of the state accumulator
+            tc_fence_after_sync();
+            const int h = g * fz::kGroupHeads + q;
+            float v[32], ks;
+            tmem_ld16(lane_base + kKvCol + 32 * q, v);
+            tmem_ld16(lane_base + kKvCol + 32 * q + 16, v + 16);
+            tmem_ld1(lane_base + kKvCol + 128, &ks);
+            tmem_wait_ld();
+            if (h < a.H) {
+                float* o = a.part + (((size_t)b * a.H + h) * a.S + s) * kStateFloats + lane * kDP;
+#pragma unroll
+                for (int e = 0; e < kD; ++e) o[e] = v[e];
+                o[kD] = ks;
+            }
+            __threadfence();
+            named_barrier_sync(1, 128);
+            const int row_id = b * gridDim.y + g;
+            const int nsplits = (tiles + a.tps - 1) / a.tps;
+            if (et == 0) *last_flag = (atomicAdd(&a.counters[row_id], 1) == nsplits - 1);
+            named_barrier_sync(1, 128);
+            if (*last_flag) {
+                __threadfence();
+                for (int idx = et; idx < fz::kGroupHeads * (kStateFloats / 4); idx += 128) {
+                    const int hh = g * fz::kGroupHeads + idx / (kStateFloats / 4);
+                    const int e4 = idx % (kStateFloats / 4);
+                    if (hh >= a.H) continue;
+                    const float4* pp = reinterpret_cast<const float4*>(
+                        a.part + ((size_t)b * a.H + hh) * a.S * kStateFloats) + e4;
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int sp = 0; sp < nsplits; ++sp) {
+                        const float4 x = __ldcg(pp + (size_t)sp * (kStateFloats / 4));
+                        acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+                    }
+                    reinterpret_cast<float4*>(a.kv + ((size_t)b * a.H + hh) * kStateFloats)[e4] = acc;
+                }
+            }
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ============================================================================ F2
+namespace f2 {
+constexpr int kStageBytes = fz::kXBytes + 2 * fz::kWBox;   // x + Q (2 boxes)
+constexpr int kStages = 4;
+constexpr int kN = 48;                                     // 32 value columns, normaliser, padding
+constexpr int kBopBytes = kN * 128;                        // per head
+constexpr int kQoBytes = 2 * fz::kBlock;                   // A' operand, then O staging
+constexpr int kStateBytes = fz::kGroupHeads * kStateFloats * 4;
+constexpr int kAccCols = 128;                              // Q accumulator (two buffers)
+constexpr int kDCol = 256;                                 // apply accumulators at column 256
+constexpr int kTmemCols = 512;
+constexpr int kThreads = 192;
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + fz::kGroupHeads * kBopBytes +
+                           kQoBytes + kStateBytes + 2048;
+}  // namespace f2
+
+struct F2Args {
+    const float* kv;     // states [B][H][D][D+1] (F1's output)
+    const float* gq;     // [C] or nullptr
+    int N, H, C, tps;
+    float eps;
+    int norm;
+};
+
+__global__ void __launch_bounds__(f2::kThreads, 1)
+fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+         const __grid_constant__ CUtensorMap tmap_o, const F2Args a)
+{
+    using namespace f2;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align_1024(smem_raw);
+    uint8_t* stages = smem;
+    uint8_t* bop = stages + kStages * kStageBytes;
+    uint8_t* qo = bop + fz::kGroupHeads * kBopBytes;
+    float* sstate = (float*)(qo + kQoBytes);
+    float* sg = sstate + fz::kGroupHeads * kStateFloats;    // 128 gains
+    uint64_t* full = (uint64_t*)(sg + 128);
+    uint64_t* empty = full + kStages;
+    uint64_t* accfull = empty + kStages;                    // [2]
+    uint64_t* accempty = accfull + 2;                       // [2]
+    uint64_t* opready = accempty + 2;
+    uint64_t* ddone = opready + 1;
+    uint64_t* bready = ddone + 1;
+    uint64_t* sready = bready + 1;
+    uint64_t* drain = sready + 1;
+    uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+
+    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles = (a.N + fz::kTileTok - 1) / fz::kTileTok;
+    const int t0 = s * a.tps;
+    const int nt = min(a.tps, tiles - t0);
+    const int ksteps = (a.C + fz::kKStep - 1) / fz::kKStep;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&accfull[i], 1);
+            mbar_init(&accempty[i], 128);
+        }
+        mbar_init(opready, 128);
+        mbar_init(ddone, 1);
+        mbar_init(bready, 128);
+        mbar_init(sready, 1);
+        mbar_init(drain, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmap_x);
+        prefetch_tmap(&tmap_w);
+        prefetch_tmap(&tmap_o);
+    }
+    for (int i = threadIdx.x; i < 128; i += blockDim.x) {
+        const int h = g * fz::kGroupHeads + i / kD;
+        sg[i] = (a.norm && h < a.H) ? a.gq[(size_t)h * kD + (i % kD)] : 1.f;
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = nt > 0;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0 && ok) {
+            int64_t step = 0, last = -1;
+            for (int ti = 0; ti < nt && ok; ++ti) {
+                const int y = (t0 + ti) * fz::kTileTok;
+                for (int kk = 0; kk < ksteps; ++kk, ++step) {
+                    const int st = (int)(step % kStages);
+                    if (step >= kStages)
+                        ok = mbar_wait(&empty[st], (uint32_t)((step / kStages) - 1) & 1, 601);
+                    if (!ok) break;
+                    uint8_t* sb = stages + st * kStageBytes;
+                    mbar_arrive_expect_tx(&full[st], kStageBytes);
+                    tma_load_3d(sb, &tmap_x, &full[st], kk * fz::kKStep, y, b);
+                    tma_load_3d(sb + fz::kXBytes, &tmap_w, &full[st], g * 128, 0, kk * fz::kKStep);
+                    tma_load_3d(sb + fz::kXBytes + fz::kWBox, &tmap_w, &full[st], g * 128 + 64, 0,
+                                kk * fz::kKStep);
+                    last = step;
+                }
+            }
+            if (!ok) {
+                for (int st = 0; st < kStages; ++st) {
+                    const int64_t li = last - ((last - st) % kStages + kStages) % kStages;
+                    if (last >= 0 && li >= 0)
+                        mbar_wait(&full[st], (uint32_t)(li / kStages) & 1, 602);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ UMMA issuer
+        // Order: GEMM(0), GEMM(1), apply(0), GEMM(2), apply(1), ...  The apply of a
+        // tile is issued after the next tile's projection, so the tensor pipe keeps
+        // busy while the epilogue turns the tile's Q into the A' operand.
+        if (lane == 0 && ok) {
+            const uint32_t idesc_g = make_idesc_bf16(128, 128, false, true);
+            const uint32_t idesc_a = make_idesc_bf16(128, kN, false, false);
+            int64_t step = 0;
+            auto gemm = [&](int ti) -> bool {
+                const int ab = ti & 1;
+                if (ti >= 2 && !mbar_wait(&accempty[ab], (uint32_t)((ti >> 1) - 1) & 1, 603))
+                    return false;
+                tc_fence_after_sync();
+                for (int kk = 0; kk < ksteps; ++kk, ++step) {
+                    const int st = (int)(step % kStages);
+                    if (!mbar_wait(&full[st], (uint32_t)(step / kStages) & 1, 604)) return false;
+                    tc_fence_after_sync();
+                    const uint32_t xb = smem_u32(stages + st * kStageBytes);
+                    const uint32_t wb = xb + fz::kXBytes;
+#pragma unroll
+                    for (int k4 = 0; k4 < fz::kKStep / 16; ++k4) {
+                        const uint64_t ad = make_smem_desc(xb + k4 * 32, 16, 1024, kSwizzle128B);
+                        const uint64_t bd = make_smem_desc(wb + k4 * 2048, fz::kWBox, 1024, kSwizzle128B);
+                        umma_bf16(tmem + ab * kAccCols, ad, bd, idesc_g, kk > 0 || k4 > 0);
+                    }
+                    umma_commit(&empty[st]);
+                }
+                umma_commit(&accfull[ab]);
+                return true;
+            };
+            auto apply = [&](int ti) -> bool {
+                if (ti == 0 && !mbar_wait(bready, 0, 605)) return false;
+                if (!mbar_wait(opready, (uint32_t)ti & 1, 606)) return false;
+                tc_fence_after_sync();
+                const uint32_t qb = smem_u32(qo), bb0 = smem_u32(bop);
+#pragma unroll
+                for (int j = 0; j < fz::kGroupHeads; ++j) {
+                    const uint32_t d = tmem + kDCol + j * kN;
+                    const uint32_t ab = qb + (j >> 1) * fz::kBlock + (j & 1) * 64;
+                    const uint32_t bb = bb0 + j * kBopBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk) {
+                        const uint64_t ad = make_smem_desc(ab + kk * 32, 16, 1024, kSwizzle128B);
+                        const uint64_t hi = make_smem_desc(bb + kk * 32, 16, 1024, kSwizzle128B);
+                        const uint64_t lo = make_smem_desc(bb + 64 + kk * 32, 16, 1024, kSwizzle128B);
+                        umma_bf16(d, ad, hi, idesc_a, kk > 0);
+                        umma_bf16(d, ad, lo, idesc_a, true);
+                    }
+                }
+                umma_commit(ddone);
+                return true;
+            };
+            for (int ti = 0; ti <= nt && ok; ++ti) {
+                if (ti < nt) ok = gemm(ti);
+                if (ok && ti >= 1) ok = apply(ti - 1);
+            }
+            umma_commit(drain);
+            mbar_wait(drain, 0, 607);
+        }
+    } else {
+        // ------------------------------------------------ epilogue
+        const int et = threadIdx.x - 64;
+        const int q = warp & 3;
+        const int row = 32 * q + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        // B operand of the apply contraction from the group's fp32 states (F1's output)
+        pdl_wait_primary();
+        const int nh = min(fz::kGroupHeads, a.H - g * fz::kGroupHeads);
+        if (et == 0) {
+            const uint32_t bytes = (uint32_t)(nh * kStateFloats * 4);
+            mbar_arrive_expect_tx(sready, bytes);
+            bulk_load(sstate, a.kv + ((size_t)b * a.H + g * fz::kGroupHeads) * kStateFloats, bytes,
+                      sready);
+        }
+        ok = ok && mbar_wait(sready, 0, 608);
+        for (int idx = et; idx < fz::kGroupHeads * kN * 8; idx += 128) {
+            const int j = idx / (kN * 8), rem = idx % (kN * 8), n = rem >> 3, ch = rem & 7;
+            const float* src = sstate + j * kStateFloats;
+            float vals[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int dd = (ch & 3) * 8 + u;
+                const float x = (ok && j < nh && n <= kD) ? src[dd * kDP + n] : 0.f;
+                const float hi = __bfloat162float(__float2bfloat16_rn(x));
+                vals[u] = (ch < 4) ? hi : (x - hi);
+            }
+            uint4 w;
+            w.x = pack_bf16x2(vals[0], vals[1]);
+            w.y = pack_bf16x2(vals[2], vals[3]);
+            w.z = pack_bf16x2(vals[4], vals[5]);
+            w.w = pack_bf16x2(vals[6], vals[7]);
+            *reinterpret_cast<uint4*>(bop + j * kBopBytes + sw128_offset(n, ch)) = w;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bready);
+
+        for (int ti = 0; ti < nt && ok; ++ti) {
+            const int ab = ti & 1;
+            ok = mbar_wait(&accfull[ab], (uint32_t)(ti >> 1) & 1, 609);
+            if (!ok) break;
+            tc_fence_after_sync();
+            // the previous tile's O store must have read the staging buffer
+            if (et == 0) bulk_wait_group_read<0>();
+            named_barrier_sync(1, 128);
+            const bool row_live = (t0 + ti) * fz::kTileTok + row < a.N;
+            float rq[fz::kGroupHeads];
+#pragma unroll 1
+            for (int j = 0; j < fz::kGroupHeads; ++j) {
+                float x[32];
+                tmem_ld16(lane_base + ab * kAccCols + 32 * j, x);
+                tmem_ld16(lane_base + ab * kAccCols + 32 * j + 16, x + 16);
+                tmem_wait_ld();
+                const bool live = row_live && (g * fz::kGroupHeads + j < a.H);
+                float r = 1.f;
+                if (a.norm) {
+                    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        s0 = fmaf(x[i], x[i], s0);
+                        s1 = fmaf(x[i + 1], x[i + 1], s1);
+                        s2 = fmaf(x[i + 2], x[i + 2], s2);
+                        s3 = fmaf(x[i + 3], x[i + 3], s3);
+                    }
+                    r = rsqrtf(((s0 + s1) + (s2 + s3)) * (1.f / kD) + a.eps);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] = fmaxf(sg[j * kD + i] * x[i], 0.f);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] = fmaxf(x[i], 0.f);
+                }
+                rq[j] = r;
+                uint8_t* blk = qo + (j >> 1) * fz::kBlock;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint4 w = make_uint4(0, 0, 0, 0);
+                    if (live) {
+                        w.x = pack_bf16x2(x[8 * c + 0], x[8 * c + 1]);
+                        w.y = pack_bf16x2(x[8 * c + 2], x[8 * c + 3]);
+                        w.z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
+                        w.w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
+                    }
+                    *reinterpret_cast<uint4*>(blk + sw128_offset(row, (j & 1) * 4 + c)) = w;
+                }
+            }
+            tc_fence_before_sync();
+            mbar_arrive(&accempty[ab]);
+            fence_proxy_async_smem();
+            mbar_arrive(opready);
+            // O = r D[:, :32] / (r D[:, 32] + eps), written over the A' operand
+            ok = mbar_wait(ddone, (uint32_t)ti & 1, 610);
+            if (!ok) break;
+            tc_fence_after_sync();
+#pragma unroll 1
+            for (int j = 0; j < fz::kGroupHeads; ++j) {
+                float v[kD + 1];
+                tmem_ld16(lane_base + kDCol + j * kN, v);
+                tmem_ld16(lane_base + kDCol + j * kN + 16, v + 16);
+                tmem_ld1(lane_base + kDCol + j * kN + kD, v + kD);
+                tmem_wait_ld();
+                const float scale = rq[j] * __frcp_rn(fmaf(rq[j], v[kD], a.eps));
+                uint8_t* blk = qo + (j >> 1) * fz::kBlock;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint4 w;
+                    w.x = pack_bf16x2(v[8 * c + 0] * scale, v[8 * c + 1] * scale);
+                    w.y = pack_bf16x2(v[8 * c + 2] * scale, v[8 * c + 3] * scale);
+                    w.z = pack_bf16x2(v[8 * c + 4] * scale, v[8 * c + 5] * scale);
+                    w.w = pack_bf16x2(v[8 * c + 6] * scale, v[8 * c + 7] * scale);
+                    *reinterpret_cast<uint4*>(blk + sw128_offset(row, (j & 1) * 4 + c)) = w;
+                }
+            }
+            tc_fence_before_sync();
+            fence_proxy_async_smem();
+            named_barrier_sync(1, 128);
+            if (et == 0) {
+                const int y = (t0 + ti) * fz::kTileTok;
+                tma_store_3d(&tmap_o, qo, g * 128, y, b);
+                if (g * 128 + 64 < a.C)                       // no store that starts past C
+                    tma_store_3d(&tmap_o, qo + fz::kBlock, g * 128 + 64, y, b);
+                bulk_commit_group();
+            }
+        }
+        if (et == 0) bulk_wait_group<0>();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace sana

@@ -11,6 +11,7 @@
 #include "simt_kernels.cuh"
 #include "sm100_primitives.cuh"
 #include "tc_kernels.cuh"
+#include "fused_kernels.cuh"
 
 namespace sana {
 namespace {
@@ -91,6 +92,24 @@ PersistPlan2 make_plan_p2(int64_t B, int64_t N, int H, int P) {
     return p;
 }
 
+// Plan of the fused kernels: CTA (s, g, b) takes tiles [s*tps, (s+1)*tps) of batch
+// b for head group g; about one wave of one CTA per SM.
+struct FusedPlan {
+    int G, tiles, S, tps;
+};
+
+FusedPlan make_plan_fused(int64_t B, int64_t N, int H, int P) {
+    FusedPlan f{};
+    f.G = (H + fz::kGroupHeads - 1) / fz::kGroupHeads;
+    f.tiles = (int)((N + fz::kTileTok - 1) / fz::kTileTok);
+    int64_t S = P / (B * f.G);
+    if (S < 1) S = 1;
+    if (S > f.tiles) S = f.tiles;
+    f.tps = (int)((f.tiles + S - 1) / S);
+    f.S = (f.tiles + f.tps - 1) / f.tps;
+    return f;
+}
+
 int max_splits(int64_t B, int64_t N, int H) {
     const int a = make_plan(B, N, H).S, b = make_plan_p1(B, N, H, kMaxPersistentCtas).Smax;
     return a > b ? a : b;
@@ -98,17 +117,13 @@ int max_splits(int64_t B, int64_t N, int H) {
 
 // Workspace layout of the unfused path: [partials B*H*S*1056 fp32][state B*H*1056 fp32].
 struct WsLayout {
-    size_t part_off, kv_off, fused_qkv_off, counters_off, total;
+    size_t part_off, kv_off, counters_off, total;
 };
 
 WsLayout ws_layout(int64_t B, int64_t N, int C, int H, bool fused) {
-    const int S = max_splits(B, N, H);
+    const int S = fused ? make_plan_fused(B, N, H, kMaxPersistentCtas).S : max_splits(B, N, H);
     WsLayout w{};
     size_t off = 0;
-    if (fused) {
-        w.fused_qkv_off = off;
-        off = align_up(off + (size_t)B * N * 3 * C * sizeof(float), 256);
-    }
     w.counters_off = off;
     off = align_up(off + (size_t)B * ((H + 3) / 4) * sizeof(int), 256);
     w.part_off = off;
@@ -204,6 +219,22 @@ bool make_tmap_bnc(CUtensorMap* m, const void* base, int64_t B, int64_t N, int C
            CUDA_SUCCESS;
 }
 
+// Wqkv (C, 3C) row-major seen by TMA as 3-D (n within a section, section, k) =
+// (C, 3, C): boxes of 64 n x 1 section x 64 k, 128-byte swizzle.  Columns past a
+// section's C read as zeros, so head groups past H never pick up the next section.
+bool make_tmap_w(CUtensorMap* m, const void* W, int C) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)C, 3, (cuuint64_t)C};
+    const cuuint64_t strides[2] = {(cuuint64_t)C * 2, (cuuint64_t)C * 3 * 2};
+    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(W), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 // The tensor-core kernels keep the gains of every channel in shared memory, so they
 // take C <= 4096 (H <= 128); wider problems run the CUDA-core kernels.
 bool tc_path(sana_dtype dt, int C) { return dt == SANA_BF16 && C <= p1::kGainCache; }
@@ -222,7 +253,11 @@ int persistent_ctas() {
     if (cudaFuncSetAttribute(kv_reduce_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              p1::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(apply_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             p2::kSmemBytes) != cudaSuccess)
+                             p2::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(fused_kv, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             f1::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(fused_qo, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             f2::kSmemBytes) != cudaSuccess)
         return 0;
     ctas[dev] = sms < kMaxPersistentCtas ? sms : kMaxPersistentCtas;
     return ctas[dev];
@@ -275,6 +310,43 @@ int launch_apply_tc(const void* q, const float* gq, const float* kv, void* out, 
     cfg.attrs = attr;
     cfg.numAttrs = chained ? 1 : 0;
     if (cudaLaunchKernelEx(&cfg, apply_persistent, tq, to, a) != cudaSuccess) return SANA_ECUDA;
+    return SANA_OK;
+}
+
+// The fused variant: F1 (K, V projection + state), then F2 (Q projection + apply)
+// as a programmatic dependent launch.
+int launch_fused(const void* x, const void* W, const float* gq, const float* gk, void* out,
+                 int* counters, float* part, float* kv, int64_t B, int64_t N, int C, int H,
+                 float eps, cudaStream_t st) {
+    const int P = persistent_ctas();
+    if (P == 0) return SANA_ECUDA;
+    CUtensorMap tx, tw, to;
+    if (!make_tmap_bnc(&tx, x, B, N, C, fz::kTileTok) || !make_tmap_w(&tw, W, C) ||
+        !make_tmap_bnc(&to, out, B, N, C, fz::kTileTok))
+        return SANA_ECUDA;
+    const FusedPlan pl = make_plan_fused(B, N, H, P);
+    if (cudaMemsetAsync(counters, 0, (size_t)B * pl.G * sizeof(int), st) != cudaSuccess)
+        return SANA_ECUDA;
+    F1Args a1{};
+    a1.gk = gk; a1.part = part; a1.kv = kv; a1.counters = counters;
+    a1.N = (int)N; a1.H = H; a1.C = C; a1.S = pl.S; a1.tps = pl.tps; a1.eps = eps;
+    a1.norm = gk != nullptr;
+    const dim3 grid(pl.S, pl.G, (unsigned)B);
+    fused_kv<<<grid, f1::kThreads, f1::kSmemBytes, st>>>(tx, tw, a1);
+    F2Args a2{};
+    a2.kv = kv; a2.gq = gq; a2.N = (int)N; a2.H = H; a2.C = C; a2.tps = pl.tps; a2.eps = eps;
+    a2.norm = gq != nullptr;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(f2::kThreads);
+    cfg.dynamicSmemBytes = f2::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, fused_qo, tx, tw, to, a2) != cudaSuccess) return SANA_ECUDA;
     return SANA_OK;
 }
 
@@ -478,16 +550,13 @@ int sana_linattn_qkv_fused(const void* x, const void* Wqkv, const float* gq, con
     if (overlaps(workspace, L.total, out, xb) || overlaps(workspace, L.total, x, xb) ||
         overlaps(workspace, L.total, Wqkv, wb))
         return SANA_EINVAL;
-    const int64_t M = B * N;
-    if ((M + 63) / 64 > 65535) return SANA_EUNSUPPORTED;
-    const Plan p = make_plan(B, N, H);
-    float* qkv = (float*)((char*)workspace + L.fused_qkv_off);
+    if (B * (int64_t)((H + 3) / 4) > 65535 * 65535LL) return SANA_EUNSUPPORTED;
     float* part = (float*)((char*)workspace + L.part_off);
     float* kv = (float*)((char*)workspace + L.kv_off);
-    const dim3 gg((unsigned)((3 * C + 63) / 64), (unsigned)((M + 63) / 64));
-    gemm_simt_bf16<<<gg, 256, 0, stream>>>((const bf16*)x, (const bf16*)Wqkv, qkv, M, 3 * C, C);
-    launch_state<float>(qkv + C, qkv + 2 * C, gk, part, kv, B, N, H, 3 * C, 3 * C, eps, p, stream);
-    launch_apply<float, bf16>(qkv, gq, kv, (bf16*)out, B, N, H, 3 * C, C, eps, stream);
+    int* counters = (int*)((char*)workspace + L.counters_off);
+    if ((rc = launch_fused(x, Wqkv, gq, gk, out, counters, part, kv, B, N, C, H, eps, stream)) !=
+        SANA_OK)
+        return rc;
     return launch_status();
 }
 

@@ -1,8 +1,8 @@
 // CUDA-core (FFMA) kernels for the two passes of Eq. (1) ("Sana: Efficient
 // High-Resolution Image Synthesis with Linear Diffusion Transformers",
 // section 2.1) with the per-head QK-RMSNorm of SANA-1.5 ("Model architecture",
-// QK Norm bullet).  They serve the fp32 dtype and the fp32 intermediates of the
-// fused path; the bf16 path runs the tensor-core kernels.
+// QK Norm bullet).  They serve the fp32 dtype and bf16 problems with more than
+// 128 heads; bf16 up to 128 heads runs the tensor-core kernels.
 //
 //   pass 1  kv_partial_simt : split-N partial states  phi(K)^T [V | 1]
 //   combine kv_combine      : fixed-order sum of the split partials
@@ -151,60 +151,6 @@ apply_simt(const TI* __restrict__ q, const float* __restrict__ gq,
     TO* op = out + ((int64_t)b * N + n) * ldo + h * kD;
 #pragma unroll
     for (int j = 0; j < kD; j += 8) store8(op + j, o + j);
-}
-
-// Plain tiled FFMA GEMM, Y[M, Nc] = X[M, K] * W[K, Nc] (bf16 in, fp32 out),
-// 64x64 tiles, 256 threads, 4x4 outputs per thread.  Used only by the fused
-// path's reference-grade projection.
-__global__ void __launch_bounds__(256)
-gemm_simt_bf16(const bf16* __restrict__ X, const bf16* __restrict__ W, float* __restrict__ Y,
-               int64_t M, int Nc, int K)
-{
-    __shared__ float sA[32][64 + 1];
-    __shared__ float sB[32][64];
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    const int64_t m0 = (int64_t)blockIdx.y * 64;
-    const int n0 = blockIdx.x * 64;
-    float acc[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-    for (int k0 = 0; k0 < K; k0 += 32) {
-        for (int i = threadIdx.x; i < 2048; i += 256) {
-            const int mm = i >> 5, kk = i & 31;
-            const int64_t gm = m0 + mm;
-            const int gkk = k0 + kk;
-            sA[kk][mm] = (gm < M && gkk < K) ? __bfloat162float(X[gm * K + gkk]) : 0.f;
-        }
-        for (int i = threadIdx.x; i < 2048; i += 256) {
-            const int kk = i >> 6, nn = i & 63;
-            const int gkk = k0 + kk, gn = n0 + nn;
-            sB[kk][nn] = (gkk < K && gn < Nc) ? __bfloat162float(W[(int64_t)gkk * Nc + gn]) : 0.f;
-        }
-        __syncthreads();
-#pragma unroll 8
-        for (int kk = 0; kk < 32; ++kk) {
-            float a[4], bb[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) { a[i] = sA[kk][ty * 4 + i]; bb[i] = sB[kk][tx * 4 + i]; }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t gm = m0 + ty * 4 + i;
-        if (gm >= M) continue;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int gn = n0 + tx * 4 + j;
-            if (gn < Nc) Y[gm * Nc + gn] = acc[i][j];
-        }
-    }
 }
 
 }  // namespace sana

@@ -57,7 +57,9 @@ def test_workspace_bytes():
     a = ws(1, 1024, 2240, 70)
     b = ws(8, 4096, 2240, 70)
     assert 0 < a < b and a % 256 == 0 and b % 256 == 0
-    assert ws(4, 4096, 2240, 70, fused=True) > ws(4, 4096, 2240, 70)
+    # the fused path keeps Q, K, V on chip: its workspace is states and partials only
+    f = ws(4, 4096, 2240, 70, fused=True)
+    assert 2 * 4 * 70 * 32 * 33 * 4 <= f < 64 << 20
     # the state alone: B*H*D*(D+1) fp32, the partials at least as much again
     assert a >= 2 * 1 * 70 * 32 * 33 * 4
 
