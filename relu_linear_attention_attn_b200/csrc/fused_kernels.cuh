@@ -52,7 +52,8 @@ constexpr int kOnesBytes = 16 * 128;
 constexpr int kAccCols = 256;                              // [K | V] accumulator
 constexpr int kKvCol = 256;                                // state accumulator at column 256
 constexpr int kTmemCols = 512;
-constexpr int kThreads = 192;                              // TMA, UMMA, 4 epilogue warps
+constexpr int kEpiWarps = 8;                               // two per TMEM lane quadrant
+constexpr int kThreads = 32 * (2 + kEpiWarps);             // TMA, UMMA, epilogue
 constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 2 * kOpBytes + kOnesBytes + 2048;
 }  // namespace f1
 
@@ -103,8 +104,8 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             mbar_init(&empty[i], 1);
         }
         mbar_init(accfull, 1);
-        mbar_init(accempty, 128);
-        mbar_init(opready, 128);
+        mbar_init(accempty, 32 * kEpiWarps);
+        mbar_init(opready, 32 * kEpiWarps);
         mbar_init(opfree, 1);
         mbar_init(kvdone, 1);
         fence_barrier_init();
@@ -215,7 +216,10 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
         }
     } else {
         // ------------------------------------------------ epilogue: phi(K), V, then the state
-        const int et = threadIdx.x - 64;                  // 0..127
+        // Two warps per TMEM lane quadrant: warp half 0 takes heads 0, 1 of the
+        // group, half 1 heads 2, 3.
+        const int et = threadIdx.x - 64;                  // 0..255
+        const int half = et >> 7;
         const int q = warp & 3;                           // TMEM lane quadrant
         const int row = 32 * q + lane;                    // token row of the tile
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
@@ -226,7 +230,7 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             tc_fence_after_sync();
             const bool row_live = (t0 + ti) * fz::kTileTok + row < a.N;
 #pragma unroll 1
-            for (int j = 0; j < fz::kGroupHeads; ++j) {
+            for (int j = 2 * half; j < 2 * half + 2; ++j) {
                 float kx[32], vx[32];
                 tmem_ld16(lane_base + 32 * j, kx);
                 tmem_ld16(lane_base + 32 * j + 16, kx + 16);
@@ -279,7 +283,7 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             mbar_arrive(opready);
         }
         if (ok) ok = mbar_wait(kvdone, 0, 509);
-        if (ok) {
+        if (ok && half == 0) {
             // the CTA's partial state: diagonal blocks of the state accumulator
             tc_fence_after_sync();
             const int h = g * fz::kGroupHeads + q;
@@ -329,17 +333,19 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
 // ============================================================================ F2
 namespace f2 {
 constexpr int kStageBytes = fz::kXBytes + 2 * fz::kWBox;   // x + Q (2 boxes)
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr int kN = 48;                                     // 32 value columns, normaliser, padding
 constexpr int kBopBytes = kN * 128;                        // per head
-constexpr int kQoBytes = 2 * fz::kBlock;                   // A' operand, then O staging
-constexpr int kStateBytes = fz::kGroupHeads * kStateFloats * 4;
+constexpr int kQoBytes = 2 * fz::kBlock;                   // states, then A' / O staging
+constexpr int kStateBytes = fz::kGroupHeads * kStateFloats * 4;   // staged in the qo buffer
 constexpr int kAccCols = 128;                              // Q accumulator (two buffers)
 constexpr int kDCol = 256;                                 // apply accumulators at column 256
 constexpr int kTmemCols = 512;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kSmemBytes = 1024 + kStages * kStageBytes + fz::kGroupHeads * kBopBytes +
-                           kQoBytes + kStateBytes + 2048;
+                           kQoBytes + 2048;
+static_assert(kStateBytes <= kQoBytes, "states must fit the staging buffer");
 }  // namespace f2
 
 struct F2Args {
@@ -360,8 +366,8 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
     uint8_t* stages = smem;
     uint8_t* bop = stages + kStages * kStageBytes;
     uint8_t* qo = bop + fz::kGroupHeads * kBopBytes;
-    float* sstate = (float*)(qo + kQoBytes);
-    float* sg = sstate + fz::kGroupHeads * kStateFloats;    // 128 gains
+    float* sstate = (float*)qo;                             // states before the first tile
+    float* sg = (float*)(qo + kQoBytes);                    // 128 gains
     uint64_t* full = (uint64_t*)(sg + 128);
     uint64_t* empty = full + kStages;
     uint64_t* accfull = empty + kStages;                    // [2]
@@ -387,11 +393,11 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&accfull[i], 1);
-            mbar_init(&accempty[i], 128);
+            mbar_init(&accempty[i], 32 * kEpiWarps);
         }
-        mbar_init(opready, 128);
+        mbar_init(opready, 32 * kEpiWarps);
         mbar_init(ddone, 1);
-        mbar_init(bready, 128);
+        mbar_init(bready, 32 * kEpiWarps);
         mbar_init(sready, 1);
         mbar_init(drain, 1);
         fence_barrier_init();
@@ -504,8 +510,10 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             mbar_wait(drain, 0, 607);
         }
     } else {
-        // ------------------------------------------------ epilogue
-        const int et = threadIdx.x - 64;
+        // ------------------------------------------------ epilogue (two warps per quadrant:
+        // half 0 takes heads 0, 1 of the group, half 1 heads 2, 3)
+        const int et = threadIdx.x - 64;                  // 0..255
+        const int half = et >> 7;
         const int q = warp & 3;
         const int row = 32 * q + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
@@ -519,7 +527,7 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
                       sready);
         }
         ok = ok && mbar_wait(sready, 0, 608);
-        for (int idx = et; idx < fz::kGroupHeads * kN * 8; idx += 128) {
+        for (int idx = et; idx < fz::kGroupHeads * kN * 8; idx += 32 * kEpiWarps) {
             const int j = idx / (kN * 8), rem = idx % (kN * 8), n = rem >> 3, ch = rem & 7;
             const float* src = sstate + j * kStateFloats;
             float vals[8];
@@ -538,6 +546,7 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             *reinterpret_cast<uint4*>(bop + j * kBopBytes + sw128_offset(n, ch)) = w;
         }
         fence_proxy_async_smem();
+        named_barrier_sync(1, 32 * kEpiWarps);             // the states in qo have been read
         mbar_arrive(bready);
 
         for (int ti = 0; ti < nt && ok; ++ti) {
@@ -547,11 +556,11 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             tc_fence_after_sync();
             // the previous tile's O store must have read the staging buffer
             if (et == 0) bulk_wait_group_read<0>();
-            named_barrier_sync(1, 128);
+            named_barrier_sync(1, 32 * kEpiWarps);
             const bool row_live = (t0 + ti) * fz::kTileTok + row < a.N;
-            float rq[fz::kGroupHeads];
+            float rq[2];
 #pragma unroll 1
-            for (int j = 0; j < fz::kGroupHeads; ++j) {
+            for (int j = 2 * half; j < 2 * half + 2; ++j) {
                 float x[32];
                 tmem_ld16(lane_base + ab * kAccCols + 32 * j, x);
                 tmem_ld16(lane_base + ab * kAccCols + 32 * j + 16, x + 16);
@@ -574,7 +583,7 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
 #pragma unroll
                     for (int i = 0; i < 32; ++i) x[i] = fmaxf(x[i], 0.f);
                 }
-                rq[j] = r;
+                rq[j & 1] = r;
                 uint8_t* blk = qo + (j >> 1) * fz::kBlock;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -597,13 +606,13 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             if (!ok) break;
             tc_fence_after_sync();
 #pragma unroll 1
-            for (int j = 0; j < fz::kGroupHeads; ++j) {
+            for (int j = 2 * half; j < 2 * half + 2; ++j) {
                 float v[kD + 1];
                 tmem_ld16(lane_base + kDCol + j * kN, v);
                 tmem_ld16(lane_base + kDCol + j * kN + 16, v + 16);
                 tmem_ld1(lane_base + kDCol + j * kN + kD, v + kD);
                 tmem_wait_ld();
-                const float scale = rq[j] * __frcp_rn(fmaf(rq[j], v[kD], a.eps));
+                const float scale = rq[j & 1] * __frcp_rn(fmaf(rq[j & 1], v[kD], a.eps));
                 uint8_t* blk = qo + (j >> 1) * fz::kBlock;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -617,7 +626,7 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             }
             tc_fence_before_sync();
             fence_proxy_async_smem();
-            named_barrier_sync(1, 128);
+            named_barrier_sync(1, 32 * kEpiWarps);
             if (et == 0) {
                 const int y = (t0 + ti) * fz::kTileTok;
                 tma_store_3d(&tmap_o, qo, g * 128, y, b);

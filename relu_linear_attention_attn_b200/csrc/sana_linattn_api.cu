@@ -338,7 +338,7 @@ int launch_fused(const void* x, const void* W, const float* gq, const float* gk,
     a2.norm = gq != nullptr;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(f2::kThreads);
+    cfg.blockDim = dim3(f2::kThreads);   // fused_qo
     cfg.dynamicSmemBytes = f2::kSmemBytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
