@@ -47,6 +47,7 @@ Plan make_plan(int64_t B, int64_t N, int H) {
 // count capped at kMaxPersistentCtas; workspace sizes use the cap, which bounds
 // every smaller count.
 constexpr int kMaxPersistentCtas = 160;
+constexpr int kP1StageTok = 64;         // tokens per pass-1 pipeline stage (6 ring slots)
 constexpr int kMinItemsPerCta = 4;
 
 struct PersistPlan1 {
@@ -57,7 +58,7 @@ struct PersistPlan1 {
 PersistPlan1 make_plan_p1(int64_t B, int64_t N, int H, int P) {
     PersistPlan1 p{};
     p.G = (H + p1::kGroupHeads - 1) / p1::kGroupHeads;
-    p.R = (int)((N + p1::kStageTok - 1) / p1::kStageTok);
+    p.R = (int)((N + kP1StageTok - 1) / kP1StageTok);
     p.T = B * p.G * (int64_t)p.R;
     // At least kMinItemsPerCta stages per CTA (small problems use fewer SMs, and
     // a row is split among fewer partial states); never an empty range, since the
@@ -250,7 +251,8 @@ int persistent_ctas() {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         sms <= 0)
         return 0;
-    if (cudaFuncSetAttribute(kv_reduce_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(kv_reduce_persistent<kP1StageTok>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              p1::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(apply_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              p2::kSmemBytes) != cudaSuccess ||
@@ -270,8 +272,8 @@ int launch_state_tc(const void* k, const void* v, const float* gk, int* counters
     const int P = persistent_ctas();
     if (P == 0) return SANA_ECUDA;
     CUtensorMap tk, tv;
-    if (!make_tmap_bnc(&tk, k, B, N, C, p1::kStageTok) ||
-        !make_tmap_bnc(&tv, v, B, N, C, p1::kStageTok))
+    if (!make_tmap_bnc(&tk, k, B, N, C, kP1StageTok) ||
+        !make_tmap_bnc(&tv, v, B, N, C, kP1StageTok))
         return SANA_ECUDA;
     const PersistPlan1 pl = make_plan_p1(B, N, H, P);
     if (cudaMemsetAsync(counters, 0, (size_t)B * pl.G * sizeof(int), st) != cudaSuccess)
@@ -280,7 +282,7 @@ int launch_state_tc(const void* k, const void* v, const float* gk, int* counters
     a.gk = gk; a.part = part; a.kv = kv; a.counters = counters; a.T = pl.T;
     a.N = (int)N; a.H = H; a.G = pl.G; a.R = pl.R; a.Smax = pl.Smax; a.P = pl.P;
     a.eps = eps; a.norm = gk != nullptr;
-    kv_reduce_persistent<<<pl.P, p1::kThreads, p1::kSmemBytes, st>>>(tk, tv, a);
+    kv_reduce_persistent<kP1StageTok><<<pl.P, p1::kThreads, p1::kSmemBytes, st>>>(tk, tv, a);
     return SANA_OK;
 }
 

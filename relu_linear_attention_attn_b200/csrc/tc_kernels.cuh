@@ -102,19 +102,32 @@ __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
 
 // ============================================================================ pass 1
 namespace p1 {
-constexpr int kStageTok = 64;                      // tokens per stage
 constexpr int kGroupHeads = 4;                     // heads per row (UMMA M = 128)
-constexpr int kBoxBytes = kStageTok * 128;         // one TMA box: 64 tokens x 64 channels
-constexpr int kStageBytes = 4 * kBoxBytes;         // K box 0, K box 1, V box 0, V box 1
-constexpr int kStages = 6;
+constexpr int kRingBytes = 192 * 1024;             // TMA ring: K and V stages
 constexpr int kOnesBytes = 16 * 128;               // 16 token rows x 64 columns
 constexpr int kAccStride = 256;                    // TMEM columns between the two accumulators
 constexpr int kTmemCols = 512;
-constexpr int kTransformWarps = 8;
+constexpr int kTransformWarps = 8;                 // two groups of 4, alternating stages
 constexpr int kEpilogueWarps = 4;
 constexpr int kThreads = 32 * (2 + kTransformWarps + kEpilogueWarps);
 constexpr int kGainCache = 4096;                   // channels whose gains live in smem
-constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kOnesBytes + kGainCache * 4 + 1024;
+constexpr int kSmemBytes = 1024 + kRingBytes + kOnesBytes + kGainCache * 4 + 1024;
+
+// Stage geometry for kStageTok tokens per stage: boxes of kStageTok tokens x 64
+// channels, [K box 0 | K box 1 | V box 0 | V box 1], as many stages as fit the ring.
+template <int kStageTok>
+struct Stage {
+    static constexpr int kBoxBytes = kStageTok * 128;
+    static constexpr int kBytes = 4 * kBoxBytes;
+    static constexpr int kCount = kRingBytes / kBytes;
+    static constexpr int kItemsPerThread = kStageTok * kGroupHeads / 128;
+    static_assert(kStageTok % 16 == 0 && kStageTok <= 256, "stage rows");
+    // The two transform groups take alternate stages; with an even slot count
+    // every slot belongs to one group, so each mbarrier phase is awaited in order
+    // (an odd count would let a group test a slot's next phase before the current
+    // one completed).
+    static_assert(kCount >= 2 && kCount % 2 == 0, "ring slots must be even");
+};
 }  // namespace p1
 
 struct P1Args {
@@ -128,15 +141,19 @@ struct P1Args {
     int norm;
 };
 
+template <int kStageTok>
 __global__ void __launch_bounds__(p1::kThreads, 1)
 kv_reduce_persistent(const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const P1Args a)
 {
     using namespace p1;
+    constexpr int kBoxBytes = Stage<kStageTok>::kBoxBytes;
+    constexpr int kStageBytes = Stage<kStageTok>::kBytes;
+    constexpr int kStages = Stage<kStageTok>::kCount;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_1024(smem_raw);
     uint8_t* stages = smem;
-    uint8_t* ones = stages + kStages * kStageBytes;
+    uint8_t* ones = stages + kRingBytes;
     float* sgain = (float*)(ones + kOnesBytes);
     uint64_t* full = (uint64_t*)(sgain + kGainCache);
     uint64_t* aready = full + kStages;
@@ -258,24 +275,25 @@ kv_reduce_persistent(const __grid_constant__ CUtensorMap tmap_k,
     } else if (warp < 2 + kTransformWarps) {
         // ------------------------------------------------ phi(K) in place
         // Two groups of 4 warps take alternate stages, so two stages are in the
-        // transform at once; a thread rewrites both heads of one 128-byte box row.
+        // transform at once.  Within a stage, item idx = (head, token row) with the
+        // row fastest, so each quarter warp touches 8 consecutive swizzled rows.
         const int wt = threadIdx.x - 64;                 // 0..255
         const int grp = wt >> 7;                         // stages with li % 2 == grp
         const int gt = wt & 127;
-        const int row = gt & 63, box = gt >> 6;          // token row, channel box (2 heads)
         for (int64_t li = grp; i0 + li < i1 && ok; li += 2) {
             const int st = (int)(li % kStages);
             ok = mbar_wait(&full[st], (uint32_t)(li / kStages) & 1, 306);
             if (!ok) break;
             const int64_t i = i0 + li, r = i / a.R;
             const int t = (int)(i % a.R), g = (int)(r % a.G);
-            const bool row_live = t * kStageTok + row < a.N;
-            uint8_t* kt = stages + st * kStageBytes + box * kBoxBytes;
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int h = g * kGroupHeads + box * 2 + jj;
-                const bool live = row_live && (h < a.H);
-                phi_inplace_sw128<true>(kt, row, jj * 4, sgain + (live ? h : 0) * kD, a.eps,
+            for (int it = 0; it < Stage<kStageTok>::kItemsPerThread; ++it) {
+                const int idx = gt + it * 128;
+                const int row = idx % kStageTok, hl = idx / kStageTok;
+                const int h = g * kGroupHeads + hl;
+                const bool live = (t * kStageTok + row < a.N) && (h < a.H);
+                phi_inplace_sw128<true>(stages + st * kStageBytes + (hl >> 1) * kBoxBytes, row,
+                                        (hl & 1) * 4, sgain + (live ? h : 0) * kD, a.eps,
                                         a.norm != 0, !live);
             }
             fence_proxy_async_smem();
@@ -387,6 +405,7 @@ constexpr int kBufCols = kPairHeads * kN;          // 96 TMEM columns per tile
 constexpr int kTmemBufs = 4;
 constexpr int kTmemCols = 512;
 constexpr int kWorkerWarps = 8;                    // two groups of 4, alternating tiles
+static_assert(kStages % 2 == 0, "each ring slot must belong to one worker group");
 constexpr int kThreads = 32 * (3 + kWorkerWarps);
 constexpr int kGainCache = 4096;
 constexpr int kStateStageBytes = kPairHeads * kStateFloats * 4;   // fp32 states of a pair

@@ -228,3 +228,15 @@ def test_wide_head_count_runs_the_cuda_core_path(cuda_lib):
     out = run_forward(cuda_lib, to_dev(x), w)
     torch.cuda.synchronize()
     assert_close(out, O.forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps), "bf16")
+
+
+@pytest.mark.parametrize("idx", [2, 3])
+def test_state_reduction_is_reproducible_at_full_size(cuda_lib, idx):
+    """Pass 1 at full size, twice: the combine order is fixed, so the states are
+    bitwise equal (a race in the ring or the combine would show up here)."""
+    w = CONFIGS[idx]
+    d = to_dev(make_inputs(w))
+    a = cuda_lib.kv_state(d["k"], d["v"], d["gk"], w.H, w.eps)
+    b = cuda_lib.kv_state(d["k"], d["v"], d["gk"], w.H, w.eps)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
