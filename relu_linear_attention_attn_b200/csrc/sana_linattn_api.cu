@@ -47,7 +47,7 @@ Plan make_plan(int64_t B, int64_t N, int H) {
 // count capped at kMaxPersistentCtas; workspace sizes use the cap, which bounds
 // every smaller count.
 constexpr int kMaxPersistentCtas = 160;
-constexpr int kP1StageTok = 64;         // tokens per pass-1 pipeline stage (6 ring slots)
+constexpr int kP1StageTok = p1::kStageTok;
 constexpr int kMinItemsPerCta = 4;
 
 struct PersistPlan1 {
@@ -251,8 +251,7 @@ int persistent_ctas() {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         sms <= 0)
         return 0;
-    if (cudaFuncSetAttribute(kv_reduce_persistent<kP1StageTok>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(kv_partials_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              p1::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(apply_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              p2::kSmemBytes) != cudaSuccess ||
@@ -261,14 +260,46 @@ int persistent_ctas() {
         cudaFuncSetAttribute(fused_qo, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              f2::kSmemBytes) != cudaSuccess)
         return 0;
+    // each persistent kernel must fit one CTA on an SM (registers, threads, smem)
+    int n1 = 0, n2 = 0, n3 = 0, n4 = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, kv_partials_persistent, p1::kThreads,
+                                                      p1::kSmemBytes) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n2, apply_persistent, p2::kThreads,
+                                                      p2::kSmemBytes) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n3, fused_kv, f1::kThreads,
+                                                      f1::kSmemBytes) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n4, fused_qo, f2::kThreads,
+                                                      f2::kSmemBytes) != cudaSuccess ||
+        n1 < 1 || n2 < 1 || n3 < 1 || n4 < 1)
+        return 0;
     ctas[dev] = sms < kMaxPersistentCtas ? sms : kMaxPersistentCtas;
     return ctas[dev];
 }
 
-// bf16 pass 1 (reduction and last-CTA combine) on the tensor cores.  The row
-// counters in the workspace are zeroed first; the final state lands in kv.
-int launch_state_tc(const void* k, const void* v, const float* gk, int* counters, float* part,
-                    float* kv, int64_t B, int64_t N, int C, int H, float eps, cudaStream_t st) {
+// Launch with programmatic stream serialization: the kernel may start while the
+// previous grid in the stream finishes, and waits for it (griddepcontrol.wait)
+// before it touches global memory.
+template <typename... Args>
+int launch_pdl(void (*kernel)(Args...), dim3 grid, int threads, int smem, cudaStream_t st,
+               bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? SANA_OK : SANA_ECUDA;
+}
+
+// bf16 pass 1 on the tensor cores: per-row-segment partial states into `part`
+// ([B][H][Smax][D+1][D]); nothing else is written.
+int launch_partials_tc(const void* k, const void* v, const float* gk, float* part, int64_t B,
+                       int64_t N, int C, int H, float eps, cudaStream_t st,
+                       PersistPlan1* plan_out) {
     const int P = persistent_ctas();
     if (P == 0) return SANA_ECUDA;
     CUtensorMap tk, tv;
@@ -276,21 +307,29 @@ int launch_state_tc(const void* k, const void* v, const float* gk, int* counters
         !make_tmap_bnc(&tv, v, B, N, C, kP1StageTok))
         return SANA_ECUDA;
     const PersistPlan1 pl = make_plan_p1(B, N, H, P);
-    if (cudaMemsetAsync(counters, 0, (size_t)B * pl.G * sizeof(int), st) != cudaSuccess)
-        return SANA_ECUDA;
     P1Args a{};
-    a.gk = gk; a.part = part; a.kv = kv; a.counters = counters; a.T = pl.T;
+    a.gk = gk; a.part = part; a.T = pl.T;
     a.N = (int)N; a.H = H; a.G = pl.G; a.R = pl.R; a.Smax = pl.Smax; a.P = pl.P;
     a.eps = eps; a.norm = gk != nullptr;
-    kv_reduce_persistent<kP1StageTok><<<pl.P, p1::kThreads, p1::kSmemBytes, st>>>(tk, tv, a);
-    return SANA_OK;
+    if (plan_out) *plan_out = pl;
+    return launch_pdl(kv_partials_persistent, dim3(pl.P), p1::kThreads, p1::kSmemBytes, st, true,
+                      tk, tv, a);
 }
 
-// bf16 pass 2 on the tensor cores.  chained: launched right behind pass 1 of the
-// same call, as a programmatic dependent launch (its Q stream starts while pass 1
-// finishes; only the state read waits for pass 1).
-int launch_apply_tc(const void* q, const float* gq, const float* kv, void* out, int64_t B,
-                    int64_t N, int C, int H, float eps, cudaStream_t st, bool chained) {
+// The final states kv [B][H][D][D+1] from pass-1 partials (right behind pass 1).
+int launch_combine_tc(const float* part, float* kv, int64_t B, int H, const PersistPlan1& pl,
+                      cudaStream_t st) {
+    return launch_pdl(kv_combine_partials, dim3((unsigned)(B * H)), 256, 0, st, true,
+                      (const float*)part, kv, H, pl.G, (int64_t)pl.R, pl.T, (int64_t)pl.P,
+                      pl.Smax);
+}
+
+// bf16 pass 2 on the tensor cores.  With kv == nullptr it sums the pass-1 partials
+// of plan p1 itself and is launched right behind pass 1 (its Q stream starts while
+// pass 1 finishes; only the partial reads wait for pass 1).
+int launch_apply_tc(const void* q, const float* gq, const float* kv, const float* part,
+                    const PersistPlan1* p1pl, void* out, int64_t B, int64_t N, int C, int H,
+                    float eps, cudaStream_t st) {
     const int P = persistent_ctas();
     if (P == 0) return SANA_ECUDA;
     CUtensorMap tq, to;
@@ -299,20 +338,14 @@ int launch_apply_tc(const void* q, const float* gq, const float* kv, void* out, 
         return SANA_ECUDA;
     const PersistPlan2 pl = make_plan_p2(B, N, H, P);
     P2Args a{};
-    a.kv = kv; a.gq = gq; a.T = pl.T; a.N = (int)N; a.H = H; a.Pp = pl.Pp; a.R = pl.R;
-    a.P = pl.P; a.eps = eps; a.norm = gq != nullptr;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(pl.P);
-    cfg.blockDim = dim3(p2::kThreads);
-    cfg.dynamicSmemBytes = p2::kSmemBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = chained ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, apply_persistent, tq, to, a) != cudaSuccess) return SANA_ECUDA;
-    return SANA_OK;
+    a.kv = kv; a.part = part; a.gq = gq; a.T = pl.T; a.N = (int)N; a.H = H; a.Pp = pl.Pp;
+    a.R = pl.R; a.P = pl.P; a.eps = eps; a.norm = gq != nullptr;
+    if (kv == nullptr) {
+        if (!p1pl || !part) return SANA_EINVAL;
+        a.T1 = p1pl->T; a.P1 = p1pl->P; a.R1 = p1pl->R; a.G1 = p1pl->G; a.Smax1 = p1pl->Smax;
+    }
+    return launch_pdl(apply_persistent, dim3(pl.P), p2::kThreads, p2::kSmemBytes, st,
+                      kv == nullptr, tq, to, a);
 }
 
 // The fused variant: F1 (K, V projection + state), then F2 (Q projection + apply)
@@ -454,9 +487,9 @@ int sana_linattn_kv_state(const void* k, const void* v, const float* gk, float* 
         return SANA_EINVAL;
     float* part = (float*)((char*)workspace + L.part_off);
     if (tc_path(dtype, C)) {
-        int* counters = (int*)((char*)workspace + L.counters_off);
-        if ((rc = launch_state_tc(k, v, gk, counters, part, kv, B, N, C, H, eps, stream)) !=
-            SANA_OK)
+        PersistPlan1 pl{};
+        if ((rc = launch_partials_tc(k, v, gk, part, B, N, C, H, eps, stream, &pl)) != SANA_OK ||
+            (rc = launch_combine_tc(part, kv, B, H, pl, stream)) != SANA_OK)
             return rc;
     } else if (dtype == SANA_BF16) {
         launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, kv, B, N, H, C, C, eps,
@@ -484,7 +517,8 @@ int sana_linattn_apply(const void* q, const float* gq, const float* kv, void* ou
         overlaps(out, bytes, kv, (size_t)B * H * kStateFloats * sizeof(float)))
         return SANA_EINVAL;
     if (tc_path(dtype, C)) {
-        if ((rc = launch_apply_tc(q, gq, kv, out, B, N, C, H, eps, stream, false)) != SANA_OK)
+        if ((rc = launch_apply_tc(q, gq, kv, nullptr, nullptr, out, B, N, C, H, eps, stream)) !=
+            SANA_OK)
             return rc;
     } else if (dtype == SANA_BF16) {
         launch_apply<bf16, bf16>((const bf16*)q, gq, kv, (bf16*)out, B, N, H, C, C, eps, stream);
@@ -516,11 +550,10 @@ int sana_linattn_forward(const void* q, const void* k, const void* v, const floa
     float* part = (float*)((char*)workspace + L.part_off);
     float* kv = (float*)((char*)workspace + L.kv_off);
     if (tc_path(dtype, C)) {
-        int* counters = (int*)((char*)workspace + L.counters_off);
-        if ((rc = launch_state_tc(k, v, gk, counters, part, kv, B, N, C, H, eps, stream)) !=
-            SANA_OK)
-            return rc;
-        if ((rc = launch_apply_tc(q, gq, kv, out, B, N, C, H, eps, stream, true)) != SANA_OK)
+        PersistPlan1 pl{};
+        if ((rc = launch_partials_tc(k, v, gk, part, B, N, C, H, eps, stream, &pl)) != SANA_OK ||
+            (rc = launch_apply_tc(q, gq, nullptr, part, &pl, out, B, N, C, H, eps, stream)) !=
+                SANA_OK)
             return rc;
     } else if (dtype == SANA_BF16) {
         launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, kv, B, N, H, C, C, eps, p,

@@ -7,28 +7,40 @@
 // to the tensor cores only because CUDA-core FMAs cannot keep up with HBM here.
 // Both kernels are persistent: one CTA per SM walks a contiguous, balanced range
 // of a flat work list, so there is no tail wave and setup is paid once per SM.
+// Small UMMAs cost about the same issue time whatever their N, so both passes
+// are laid out to issue as few of them per byte as the operand shapes allow.
 //
-// Pass 1, kv_reduce_persistent.  Work item = one 64-token stage of one row
-// (b, g), g a group of 4 heads (128 channels).  Per stage:
-//     D[(h,d), (h',e)] += sum_t phi(K)[t,(h,d)] V[t,(h',e)]       (UMMA M=128, N=128)
-//     D[(h,d), 128]    += sum_t phi(K)[t,(h,d)]                   (UMMA N=64, ones)
-// and the diagonal blocks h == h' are the state.  TMA brings K and V tiles with the
-// 128-byte swizzle, [token][channel]; the transform warps rewrite K in place as
-// phi(K) = ReLU(g * k / rms(k)), which makes it the MN-major A operand; V already
-// is the MN-major B operand.  At the end of each row segment the epilogue warps
-// store the segment's partial state; the last CTA to finish a row (global
-// counter) sums that row's partials in CTA order into the final state, so the
-// result is bitwise reproducible.
+// Pass 1, kv_partials_persistent.  Work item = one 64-token stage of one row
+// (b, g), g a group of 4 heads (128 channels).  Per stage one UMMA chain
+//     D[(h,d), (h',e)] += sum_t phi(K)[t,(h,d)] V[t,(h',e)]       (M=128, N=128, K=64)
+// whose diagonal blocks h == h' are the state's value columns.  The normaliser
+// column sum_t phi(K)[t,(h,d)] is summed on the CUDA cores by the warps that
+// compute phi(K) (from the same bf16-rounded values the UMMA reads).  TMA brings
+// K and V tiles with the 128-byte swizzle, [token][channel]; the transform warps
+// rewrite K in place as phi(K) = ReLU(g * k / rms(k)), which makes it the
+// MN-major A operand; V already is the MN-major B operand.  At the end of each
+// row segment the epilogue warps store the segment's partial state, transposed
+// ([e][d], coalesced); a row's partials are summed in CTA order by the consumer
+// (pass 2's operand builder, or the combine kernel), so results are bitwise
+// reproducible and pass 1 needs no counters or atomics.
 //
 // Pass 2, apply_persistent.  Work item = one 128-token tile of one row (b, p), p a
-// pair of heads (64 channels).  A builder warp turns the fp32 state of the row into
-// the B operand per head (n = value column e or the normaliser, k = d; bf16 hi and
-// lo parts, so the state keeps ~16 mantissa bits); the workers rewrite the Q tile
-// in place as phi(Q) (K-major A operand); UMMA M=128 N=48 (K=16 x 2 x {hi, lo})
-//     D[t, e] = sum_d phi(Q)[t,d] S[d,e],  e < 32;   D[t, 32] = sum_d phi(Q)[t,d] S[d,32]
-// and the workers form O = D[:, :32] * (1 / (D[:, 32] + eps)), write it over the
-// tile and TMA-store it.  Only the builder warp reads what pass 1 wrote, so under
-// programmatic dependent launch the Q stream starts while pass 1 finishes.
+// pair of heads (64 channels).  A builder warp sums the row's partial states (or
+// reads a given state) and writes the B operand of both heads, K-major, one
+// 128-byte row per output column n: rows 0..31 the bf16 "hi" part of the value
+// columns, row 32 / 33 the hi / lo parts of the normaliser column, rows 48..79 the
+// "lo" parts (x - bf16(x)) of the value columns, so the state keeps ~16 mantissa
+// bits.  The workers rewrite the Q tile in place as phi(Q) (K-major A operand);
+// per head two UMMAs (M=128, N=80, K=16 each) give
+//     D[t, n] = sum_d phi(Q)[t,d] Bop[n, d]
+// and the workers form num_e = D[e] + D[48+e], den = D[32] + D[33],
+// O = num * (1 / (den + eps)), write O over the tile; a store warp TMA-stores it
+// and hands the slot back to the producer as soon as the store has read it.
+//
+// Launch chaining (programmatic dependent launch): pass 1 waits for the previous
+// grid before touching memory and only then lets pass 2 launch, so pass 2 may
+// read Q and the gains early; pass 2 reads what pass 1 wrote only after its own
+// wait.  Pass 2 lets the next grid launch at once; whatever follows waits for it.
 //
 // TMEM: warp w reads lanes 32 * (w % 4) .. + 31; D row i is lane i.
 #pragma once
@@ -46,10 +58,11 @@ namespace sana {
 //                 apply later (it is a positive per-token factor).
 //   norm off    : ReLU(x); returns 1.
 //   zero        : writes zeros (rows past N, heads past H); returns 1.
+// sum (optional): the 32 bf16-rounded results are added to sum[0..31].
 template <bool kScaleByRms>
 __device__ __forceinline__ float phi_inplace_sw128(uint8_t* tile, int row, int chunk0,
                                                    const float* g, float eps, bool norm,
-                                                   bool zero) {
+                                                   bool zero, float* sum = nullptr) {
     uint4 u[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c)
@@ -92,6 +105,12 @@ __device__ __forceinline__ float phi_inplace_sw128(uint8_t* tile, int row, int c
         w.z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
         w.w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
         *reinterpret_cast<uint4*>(tile + sw128_offset(row, chunk0 + c)) = w;
+        if (sum) {
+            sum[8 * c + 0] += bf16lo(w.x); sum[8 * c + 1] += bf16hi(w.x);
+            sum[8 * c + 2] += bf16lo(w.y); sum[8 * c + 3] += bf16hi(w.y);
+            sum[8 * c + 4] += bf16lo(w.z); sum[8 * c + 5] += bf16hi(w.z);
+            sum[8 * c + 6] += bf16lo(w.w); sum[8 * c + 7] += bf16hi(w.w);
+        }
     }
     return kScaleByRms ? 1.f : r;
 }
@@ -100,71 +119,76 @@ __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
     return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
 }
 
+// Sum of 32 per-lane values over the 32 lanes of a warp (butterfly
+// reduce-scatter): on return lane l holds the total of entry l in v[0].  The
+// order of the additions is fixed, so the result is reproducible.
+__device__ __forceinline__ void warp_reduce_scatter32(float* v, int lane) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < off; ++i) {
+            const float send = upper ? v[i] : v[i + off];
+            const float keep = upper ? v[i + off] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+}
+
 // ============================================================================ pass 1
 namespace p1 {
 constexpr int kGroupHeads = 4;                     // heads per row (UMMA M = 128)
-constexpr int kRingBytes = 192 * 1024;             // TMA ring: K and V stages
-constexpr int kOnesBytes = 16 * 128;               // 16 token rows x 64 columns
-constexpr int kAccStride = 256;                    // TMEM columns between the two accumulators
-constexpr int kTmemCols = 512;
+constexpr int kStageTok = 64;                      // tokens per stage
+constexpr int kBoxBytes = kStageTok * 128;         // kStageTok tokens x 64 channels
+constexpr int kStageBytes = 4 * kBoxBytes;         // [K box 0 | K box 1 | V box 0 | V box 1]
+constexpr int kRingBytes = 192 * 1024;
+constexpr int kStages = kRingBytes / kStageBytes;  // 6
+constexpr int kAccCols = 128;                      // one accumulator (4 heads x 32 columns)
+constexpr int kTmemCols = 2 * kAccCols;            // double-buffered across row segments
 constexpr int kTransformWarps = 8;                 // two groups of 4, alternating stages
 constexpr int kEpilogueWarps = 4;
 constexpr int kThreads = 32 * (2 + kTransformWarps + kEpilogueWarps);
 constexpr int kGainCache = 4096;                   // channels whose gains live in smem
-constexpr int kSmemBytes = 1024 + kRingBytes + kOnesBytes + kGainCache * 4 + 1024;
-
-// Stage geometry for kStageTok tokens per stage: boxes of kStageTok tokens x 64
-// channels, [K box 0 | K box 1 | V box 0 | V box 1], as many stages as fit the ring.
-template <int kStageTok>
-struct Stage {
-    static constexpr int kBoxBytes = kStageTok * 128;
-    static constexpr int kBytes = 4 * kBoxBytes;
-    static constexpr int kCount = kRingBytes / kBytes;
-    static constexpr int kItemsPerThread = kStageTok * kGroupHeads / 128;
-    static_assert(kStageTok % 16 == 0 && kStageTok <= 256, "stage rows");
-    // The two transform groups take alternate stages; with an even slot count
-    // every slot belongs to one group, so each mbarrier phase is awaited in order
-    // (an odd count would let a group test a slot's next phase before the current
-    // one completed).
-    static_assert(kCount >= 2 && kCount % 2 == 0, "ring slots must be even");
-};
+constexpr int kKsumFloats = kTransformWarps * 32;  // each transform warp's 32 column sums
+constexpr int kSmemBytes = 1024 + kRingBytes + kGainCache * 4 + 2 * kKsumFloats * 4 + 512;
+// Warp w of a transform group handles head w of the row, thread l of the warp
+// token rows l and l + 32, in every stage of its group.
+static_assert(kStageTok == 64 && kGroupHeads == 4, "two items per transform thread");
+// The two transform groups take alternate stages; with an even slot count every
+// slot belongs to one group, so each mbarrier phase is awaited in order (an odd
+// count would let a group test a slot's next phase before the current one
+// completed).
+static_assert(kStages >= 2 && kStages % 2 == 0, "ring slots must be even");
 }  // namespace p1
 
 struct P1Args {
     const float* gk;     // gains [C], or nullptr with the norm off
-    float* part;         // partial states [B][H][Smax][D][D+1]
-    float* kv;           // final states [B][H][D][D+1]
-    int* counters;       // [B * G], zero on entry
+    float* part;         // partial states [B][H][Smax][D+1][D]  (column e major)
     int64_t T;           // work items: B * G rows x R stages
     int N, H, G, R, Smax, P;
     float eps;
     int norm;
 };
 
-template <int kStageTok>
 __global__ void __launch_bounds__(p1::kThreads, 1)
-kv_reduce_persistent(const __grid_constant__ CUtensorMap tmap_k,
-                     const __grid_constant__ CUtensorMap tmap_v, const P1Args a)
+kv_partials_persistent(const __grid_constant__ CUtensorMap tmap_k,
+                       const __grid_constant__ CUtensorMap tmap_v, const P1Args a)
 {
     using namespace p1;
-    constexpr int kBoxBytes = Stage<kStageTok>::kBoxBytes;
-    constexpr int kStageBytes = Stage<kStageTok>::kBytes;
-    constexpr int kStages = Stage<kStageTok>::kCount;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_1024(smem_raw);
     uint8_t* stages = smem;
-    uint8_t* ones = stages + kRingBytes;
-    float* sgain = (float*)(ones + kOnesBytes);
-    uint64_t* full = (uint64_t*)(sgain + kGainCache);
+    float* sgain = (float*)(stages + kRingBytes);
+    float* ksbuf = sgain + kGainCache;                  // [2][kTransformWarps][64]
+    uint64_t* full = (uint64_t*)(ksbuf + 2 * kKsumFloats);
     uint64_t* aready = full + kStages;
     uint64_t* empty = aready + kStages;
     uint64_t* accfull = empty + kStages;
     uint64_t* accempty = accfull + 2;
-    uint64_t* drain = accempty + 2;
+    uint64_t* ksfull = accempty + 2;
+    uint64_t* ksempty = ksfull + 2;
+    uint64_t* drain = ksempty + 2;
     uint32_t* tmem_slot = (uint32_t*)(drain + 1);
-    int* last_flag = (int*)(tmem_slot + 1);
-
-    pdl_launch_dependents();   // the apply pass may take each SM as soon as this CTA leaves
 
     const int64_t c = blockIdx.x;
     const int64_t i0 = range_begin(c, a.T, a.P), i1 = range_begin(c + 1, a.T, a.P);
@@ -180,6 +204,8 @@ kv_reduce_persistent(const __grid_constant__ CUtensorMap tmap_k,
         for (int i = 0; i < 2; ++i) {
             mbar_init(&accfull[i], 1);
             mbar_init(&accempty[i], 32 * kEpilogueWarps);
+            mbar_init(&ksfull[i], 32 * kTransformWarps);
+            mbar_init(&ksempty[i], 32 * kEpilogueWarps);
         }
         mbar_init(drain, 1);
         fence_barrier_init();
@@ -188,22 +214,18 @@ kv_reduce_persistent(const __grid_constant__ CUtensorMap tmap_k,
         prefetch_tmap(&tmap_k);
         prefetch_tmap(&tmap_v);
     }
-    for (int i = threadIdx.x; i < kOnesBytes / 16; i += blockDim.x)
-        reinterpret_cast<uint4*>(ones)[i] = make_uint4(0, 0, 0, 0);
-    if (a.norm)
-        for (int i = threadIdx.x; i < C; i += blockDim.x) sgain[i] = a.gk[i];
-    __syncthreads();
-    if (threadIdx.x < 16)   // the normaliser operand: column 0 of every row is 1.0
-        *reinterpret_cast<uint16_t*>(ones + sw128_offset(threadIdx.x, 0)) = 0x3F80;
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // Nothing above touched global memory.  Wait for the previous grid, then let
+    // the apply pass launch: it may read Q and its gains before its own wait.
+    pdl_wait_primary();
+    pdl_launch_dependents();
     bool ok = i1 > i0;
 
     if (warp == 0) {
@@ -234,12 +256,10 @@ kv_reduce_persistent(const __grid_constant__ CUtensorMap tmap_k,
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ UMMA issuer
-        if (lane == 0 && ok) {
-            const uint32_t idesc_v = make_idesc_bf16(128, 128, true, true);
-            const uint32_t idesc_1 = make_idesc_bf16(128, 64, true, true);
-            const uint64_t ones_desc =
-                make_smem_desc(smem_u32(ones), kBoxBytes, 1024, kSwizzle128B);
+        // ------------------------------------------------ UMMA issuer (whole warp,
+        // one elected lane issues)
+        if (ok) {
+            const uint32_t idesc = make_idesc_bf16(128, 128, true, true);
             int seg = 0;
             for (int64_t li = 0; i0 + li < i1 && ok; ++li) {
                 const int64_t i = i0 + li;
@@ -247,61 +267,86 @@ kv_reduce_persistent(const __grid_constant__ CUtensorMap tmap_k,
                 const bool first = (li == 0) || (t == 0);
                 const bool lastst = (i + 1 == i1) || (t == a.R - 1);
                 const int abuf = seg & 1;
-                if (first && seg >= 2)
-                    ok = mbar_wait(&accempty[abuf], (uint32_t)((seg >> 1) - 1) & 1, 303);
-                if (ok) ok = mbar_wait(&aready[st], (uint32_t)(li / kStages) & 1, 304);
+                if (lane == 0) {
+                    if (first && seg >= 2)
+                        ok = mbar_wait(&accempty[abuf], (uint32_t)((seg >> 1) - 1) & 1, 303);
+                    if (ok) ok = mbar_wait(&aready[st], (uint32_t)(li / kStages) & 1, 304);
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 tc_fence_after_sync();
-                const uint32_t d = tmem + abuf * kAccStride;
+                const uint32_t d = tmem + abuf * kAccCols;
                 const uint32_t kb = smem_u32(stages + st * kStageBytes);
                 const uint32_t vb = kb + 2 * kBoxBytes;
 #pragma unroll
                 for (int kk = 0; kk < kStageTok / 16; ++kk) {
                     const uint64_t ad = make_smem_desc(kb + kk * 2048, kBoxBytes, 1024, kSwizzle128B);
                     const uint64_t bd = make_smem_desc(vb + kk * 2048, kBoxBytes, 1024, kSwizzle128B);
-                    const bool acc = !(first && kk == 0);
-                    umma_bf16(d, ad, bd, idesc_v, acc);
-                    umma_bf16(d + 128, ad, ones_desc, idesc_1, acc);
+                    umma_bf16_elect(d, ad, bd, idesc, !(first && kk == 0));
                 }
-                umma_commit(&empty[st]);
+                umma_commit_elect(&empty[st]);
                 if (lastst) {
-                    umma_commit(&accfull[abuf]);
+                    umma_commit_elect(&accfull[abuf]);
                     ++seg;
                 }
             }
-            umma_commit(drain);
-            mbar_wait(drain, 0, 305);
+            umma_commit_elect(drain);
+            if (lane == 0) mbar_wait(drain, 0, 305);
+            __syncwarp();
         }
     } else if (warp < 2 + kTransformWarps) {
-        // ------------------------------------------------ phi(K) in place
+        // ------------------------------------------------ phi(K) in place + column sums
         // Two groups of 4 warps take alternate stages, so two stages are in the
-        // transform at once.  Within a stage, item idx = (head, token row) with the
-        // row fastest, so each quarter warp touches 8 consecutive swizzled rows.
+        // transform at once.  Within a stage, warp hl of a group takes head hl and
+        // lane l token rows l and l + 32, so each quarter warp touches 8
+        // consecutive swizzled rows; the warp's column sums are one head's.
         const int wt = threadIdx.x - 64;                 // 0..255
+        const int wi = wt >> 5;                          // transform warp 0..7
         const int grp = wt >> 7;                         // stages with li % 2 == grp
-        const int gt = wt & 127;
-        for (int64_t li = grp; i0 + li < i1 && ok; li += 2) {
-            const int st = (int)(li % kStages);
-            ok = mbar_wait(&full[st], (uint32_t)(li / kStages) & 1, 306);
-            if (!ok) break;
-            const int64_t i = i0 + li, r = i / a.R;
-            const int t = (int)(i % a.R), g = (int)(r % a.G);
+        const int hl = wi & 3;                           // head within the row
+        if (a.norm)
+            for (int i = wt; i < C; i += 32 * kTransformWarps) sgain[i] = a.gk[i];
+        named_barrier_sync(2, 32 * kTransformWarps);
+        int seg = 0;
+        for (int64_t sb = i0; sb < i1 && ok; ++seg) {
+            // one row segment [sb, se): this group's stages are those with li % 2 == grp
+            const int64_t r = sb / a.R;
+            const int64_t se = (r + 1) * a.R < i1 ? (r + 1) * a.R : i1;
+            const int g = (int)(r % a.G);
+            const int h = g * kGroupHeads + hl;
+            float ks[kD];
 #pragma unroll
-            for (int it = 0; it < Stage<kStageTok>::kItemsPerThread; ++it) {
-                const int idx = gt + it * 128;
-                const int row = idx % kStageTok, hl = idx / kStageTok;
-                const int h = g * kGroupHeads + hl;
-                const bool live = (t * kStageTok + row < a.N) && (h < a.H);
-                phi_inplace_sw128<true>(stages + st * kStageBytes + (hl >> 1) * kBoxBytes, row,
-                                        (hl & 1) * 4, sgain + (live ? h : 0) * kD, a.eps,
-                                        a.norm != 0, !live);
+            for (int e = 0; e < kD; ++e) ks[e] = 0.f;
+            int64_t li = sb - i0;
+            if ((li & 1) != grp) ++li;
+            for (; i0 + li < se && ok; li += 2) {
+                const int st = (int)(li % kStages);
+                ok = mbar_wait(&full[st], (uint32_t)(li / kStages) & 1, 306);
+                if (!ok) break;
+                const int t = (int)((i0 + li) % a.R);
+#pragma unroll
+                for (int it = 0; it < 2; ++it) {
+                    const int row = lane + 32 * it;
+                    const bool live = (t * kStageTok + row < a.N) && (h < a.H);
+                    phi_inplace_sw128<true>(stages + st * kStageBytes + (hl >> 1) * kBoxBytes, row,
+                                            (hl & 1) * 4, sgain + (live ? h : 0) * kD, a.eps,
+                                            a.norm != 0, !live, ks);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&aready[st]);
             }
-            fence_proxy_async_smem();
-            mbar_arrive(&aready[st]);
+            if (!ok) break;
+            // the warp's 32 column sums (head hl, channel = lane) -> shared memory
+            warp_reduce_scatter32(ks, lane);
+            const int buf = seg & 1;
+            if (seg >= 2) ok = mbar_wait(&ksempty[buf], (uint32_t)((seg >> 1) - 1) & 1, 308);
+            if (!ok) break;
+            ksbuf[buf * kKsumFloats + wi * 32 + lane] = ks[0];
+            mbar_arrive(&ksfull[buf]);
+            sb = se;
         }
     } else {
-        // ------------------------------------------------ segment epilogue + combine
-        const int et = threadIdx.x - 32 * (2 + kTransformWarps);   // 0..127
+        // ------------------------------------------------ segment epilogue
         const int q = warp & 3;                                     // head within the row
         int seg = 0;
         for (int64_t li = 0; i0 + li < i1 && ok; ++li) {
@@ -312,75 +357,32 @@ kv_reduce_persistent(const __grid_constant__ CUtensorMap tmap_k,
             ok = mbar_wait(&accfull[abuf], (uint32_t)(seg >> 1) & 1, 307);
             if (!ok) break;
             tc_fence_after_sync();
-            const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + abuf * kAccStride;
-            float v[32], ks;
+            const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + abuf * kAccCols;
+            float v[kD];
             tmem_ld16(ta + 32 * q, v);
             tmem_ld16(ta + 32 * q + 16, v + 16);
-            tmem_ld1(ta + 128, &ks);
             tmem_wait_ld();
             tc_fence_before_sync();
             mbar_arrive(&accempty[abuf]);
+            ok = mbar_wait(&ksfull[abuf], (uint32_t)(seg >> 1) & 1, 309);
+            if (!ok) break;
+            // head q's column sums from transform warp q of each group, in group order
+            const float* kb = ksbuf + abuf * kKsumFloats + q * 32 + lane;
+            const float ks = kb[0] + kb[4 * 32];
+            mbar_arrive(&ksempty[abuf]);
             ++seg;
 
             const int64_t r = i / a.R;
             const int b = (int)(r / a.G), g = (int)(r % a.G);
-            const int64_t first_owner = owner_cta(r * a.R, a.T, a.P);
-            const int nslots = (int)(owner_cta(r * a.R + a.R - 1, a.T, a.P) - first_owner + 1);
-            const int slot = (int)(c - first_owner);
+            const int slot = (int)(c - owner_cta(r * a.R, a.T, a.P));
             const int h = g * kGroupHeads + q;
             if (h < a.H) {
-                float* o = a.part + (((size_t)b * a.H + h) * a.Smax + slot) * kStateFloats + lane * kDP;
+                // lane = d; element (e, d) at e * 32 + d: one 128-byte row per store
+                float* o = a.part + (((size_t)b * a.H + h) * a.Smax + slot) * kStateFloats + lane;
 #pragma unroll
-                for (int e = 0; e < kD; ++e) o[e] = v[e];
-                o[kD] = ks;
+                for (int e = 0; e < kD; ++e) o[e * kD] = v[e];
+                o[kD * kD] = ks;
             }
-            __threadfence();
-            named_barrier_sync(1, 32 * kEpilogueWarps);
-            if (et == 0) *last_flag = (atomicAdd(&a.counters[r], 1) == nslots - 1);
-            named_barrier_sync(1, 32 * kEpilogueWarps);
-            if (*last_flag) {
-                __threadfence();
-                // sum the row's partial slots in slot order; float4 lanes, all loads of
-                // a slot issued before any add so they overlap
-                constexpr int kVec = kStateFloats / 4;                    // 264 float4 per head
-                for (int base = et; base < kGroupHeads * kVec; base += 3 * 32 * kEpilogueWarps) {
-                    float4 acc[3];
-                    int hh[3], e4[3];
-#pragma unroll
-                    for (int u = 0; u < 3; ++u) {
-                        const int idx = base + u * 32 * kEpilogueWarps;
-                        hh[u] = g * kGroupHeads + idx / kVec;
-                        e4[u] = idx % kVec;
-                        if (idx >= kGroupHeads * kVec) hh[u] = a.H;       // past the group
-                        acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-                    for (int s = 0; s < nslots; s += 2) {      // two slots in flight
-                        float4 x[2][3];
-#pragma unroll
-                        for (int w2 = 0; w2 < 2; ++w2)
-#pragma unroll
-                            for (int u = 0; u < 3; ++u)
-                                if (hh[u] < a.H && s + w2 < nslots)
-                                    x[w2][u] = __ldcg(reinterpret_cast<const float4*>(
-                                                   a.part + (((size_t)b * a.H + hh[u]) * a.Smax +
-                                                             s + w2) * kStateFloats) + e4[u]);
-#pragma unroll
-                        for (int w2 = 0; w2 < 2; ++w2)
-#pragma unroll
-                            for (int u = 0; u < 3; ++u)
-                                if (hh[u] < a.H && s + w2 < nslots) {
-                                    acc[u].x += x[w2][u].x; acc[u].y += x[w2][u].y;
-                                    acc[u].z += x[w2][u].z; acc[u].w += x[w2][u].w;
-                                }
-                    }
-#pragma unroll
-                    for (int u = 0; u < 3; ++u)
-                        if (hh[u] < a.H)
-                            reinterpret_cast<float4*>(a.kv + ((size_t)b * a.H + hh[u]) * kStateFloats)
-                                [e4[u]] = acc[u];
-                }
-            }
-            named_barrier_sync(1, 32 * kEpilogueWarps);
         }
     }
     tc_fence_before_sync();
@@ -391,33 +393,64 @@ kv_reduce_persistent(const __grid_constant__ CUtensorMap tmap_k,
     }
 }
 
+// The number of partial slots of pass-1 row r (CTAs whose ranges meet it).
+__host__ __device__ __forceinline__ int p1_row_slots(int64_t r, int64_t R, int64_t T, int64_t P) {
+    return (int)(owner_cta(r * R + R - 1, T, P) - owner_cta(r * R, T, P) + 1);
+}
+
+// State of each (b, h) from pass-1 partials, summed in slot order: grid B * H,
+// kv[d][e] = sum_s part[s][e][d].  Launched right behind pass 1.
+__global__ void __launch_bounds__(256)
+kv_combine_partials(const float* __restrict__ part, float* __restrict__ kv, int H, int G,
+                    int64_t R, int64_t T, int64_t P, int Smax)
+{
+    pdl_wait_primary();
+    const int64_t bh = blockIdx.x;
+    const int64_t b = bh / H, h = bh % H;
+    const int ns = p1_row_slots(b * G + h / p1::kGroupHeads, R, T, P);
+    const float* src = part + bh * Smax * (int64_t)kStateFloats;
+    for (int idx = threadIdx.x; idx < kStateFloats; idx += blockDim.x) {
+        float acc = 0.f;
+        for (int s = 0; s < ns; ++s) acc += src[(int64_t)s * kStateFloats + idx];
+        const int e = idx / kD, d = idx % kD;
+        kv[bh * kStateFloats + d * kDP + e] = acc;
+    }
+}
+
 // ============================================================================ pass 2
 namespace p2 {
 constexpr int kTileTok = 128;                      // UMMA M
 constexpr int kPairHeads = 2;                      // 64 channels = one swizzled row
 constexpr int kTileBytes = kTileTok * 128;         // 16 KB
 constexpr int kStages = 10;
-constexpr int kN = 48;                             // 32 value columns, normaliser, padding
-constexpr int kBopBytes = kN * 128;                // per head: rows n, [hi d0..31 | lo d0..31]
-constexpr int kBopSetBytes = kPairHeads * kBopBytes;
+constexpr int kN = 80;                             // B rows per head (see the file comment)
+constexpr int kLoRow = 48;                         // first row of the value columns' lo parts
+constexpr int kDenHi = 32, kDenLo = 33;            // rows of the normaliser's hi / lo parts
+constexpr int kBopBytes = kN * 128;                // both heads side by side in each row
 constexpr int kBopRing = 2;
-constexpr int kBufCols = kPairHeads * kN;          // 96 TMEM columns per tile
-constexpr int kTmemBufs = 4;
+constexpr int kBufCols = kPairHeads * kN;          // 160 TMEM columns per tile
+constexpr int kTmemBufs = 3;
 constexpr int kTmemCols = 512;
+constexpr int kSlotsPerRound = 3;                  // partial slots staged per bulk copy round
+constexpr int kStagingBytes = kPairHeads * kSlotsPerRound * kStateFloats * 4;
 constexpr int kWorkerWarps = 8;                    // two groups of 4, alternating tiles
-static_assert(kStages % 2 == 0, "each ring slot must belong to one worker group");
-constexpr int kThreads = 32 * (3 + kWorkerWarps);
+constexpr int kThreads = 32 * (4 + kWorkerWarps);  // TMA, UMMA, builder, store, workers
 constexpr int kGainCache = 4096;
-constexpr int kStateStageBytes = kPairHeads * kStateFloats * 4;   // fp32 states of a pair
-constexpr int kSmemBytes = 1024 + kStages * kTileBytes + kBopRing * kBopSetBytes +
-                           kStateStageBytes + kGainCache * 4 + 1024;
+constexpr int kSmemBytes = 1024 + kStages * kTileBytes + kBopRing * kBopBytes + kStagingBytes +
+                           kGainCache * 4 + 512;
+static_assert(kStages % 2 == 0, "each ring slot must belong to one worker group");
+static_assert(kTmemBufs * kBufCols <= kTmemCols, "TMEM buffers");
+static_assert(kSmemBytes <= 232448, "shared memory");
 }  // namespace p2
 
 struct P2Args {
-    const float* kv;     // states [B][H][D][D+1] (written by pass 1 when chained)
+    const float* kv;     // states [B][H][D][D+1]; nullptr: sum pass-1 partials instead
+    const float* part;   // pass-1 partials [B][H][Smax1][D+1][D] (when kv is nullptr)
     const float* gq;     // gains [C] or nullptr
     int64_t T;           // work items: B * Pp rows x R tiles
     int N, H, Pp, R, P;
+    int64_t T1, P1;      // pass-1 plan: items, CTAs, stages per row, groups, slots per row
+    int R1, G1, Smax1;
     float eps;
     int norm;
 };
@@ -431,12 +464,13 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
     uint8_t* smem = align_1024(smem_raw);
     uint8_t* stages = smem;
     uint8_t* bop = stages + kStages * kTileBytes;
-    float* sstate = (float*)(bop + kBopRing * kBopSetBytes);
-    float* sgain = sstate + kPairHeads * kStateFloats;
+    float* staging = (float*)(bop + kBopRing * kBopBytes);
+    float* sgain = staging + kStagingBytes / 4;
     uint64_t* full = (uint64_t*)(sgain + kGainCache);
     uint64_t* aready = full + kStages;
     uint64_t* mmadone = aready + kStages;
-    uint64_t* empty = mmadone + kStages;
+    uint64_t* tready = mmadone + kStages;
+    uint64_t* empty = tready + kStages;
     uint64_t* tfree = empty + kStages;
     uint64_t* bfull = tfree + kTmemBufs;
     uint64_t* bempty = bfull + kBopRing;
@@ -444,6 +478,8 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
     uint64_t* sready = drain + 1;
     uint32_t* tmem_slot = (uint32_t*)(sready + 1);
 
+    // The next grid may launch now; it waits for this one before touching memory.
+    pdl_launch_dependents();
     const int64_t c = blockIdx.x;
     const int64_t i0 = range_begin(c, a.T, a.P), i1 = range_begin(c + 1, a.T, a.P);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -455,6 +491,7 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(&full[i], 1);
             mbar_init(&aready[i], 128);
             mbar_init(&mmadone[i], 1);
+            mbar_init(&tready[i], 128);
             mbar_init(&empty[i], 1);
         }
         for (int i = 0; i < kTmemBufs; ++i) mbar_init(&tfree[i], 128);
@@ -469,12 +506,19 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
         prefetch_tmap(&tmap_q);
         prefetch_tmap(&tmap_o);
     }
+    // B operand rows that never carry data stay zero
+    for (int i = threadIdx.x; i < kBopRing * (kLoRow - kDenLo - 1) * 8; i += blockDim.x) {
+        const int rb = i / ((kLoRow - kDenLo - 1) * 8), rem = i % ((kLoRow - kDenLo - 1) * 8);
+        *reinterpret_cast<uint4*>(bop + rb * kBopBytes + (kDenLo + 1 + rem / 8) * 128 +
+                                  (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
+    }
     if (a.norm)
         for (int i = threadIdx.x; i < C; i += blockDim.x) sgain[i] = a.gq[i];
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
+    fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -504,8 +548,9 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ UMMA issuer
-        if (lane == 0 && ok) {
+        // ------------------------------------------------ UMMA issuer (whole warp,
+        // one elected lane issues)
+        if (ok) {
             const uint32_t idesc = make_idesc_bf16(128, kN, false, false);
             int seg = 0;
             for (int64_t li = 0; i0 + li < i1 && ok; ++li) {
@@ -514,41 +559,46 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
                 const bool first = (li == 0) || (t == 0);
                 const bool lastt = (i + 1 == i1) || (t == a.R - 1);
                 const int rb = seg & 1, tb = (int)(li % kTmemBufs);
-                if (first) ok = mbar_wait(&bfull[rb], (uint32_t)(seg >> 1) & 1, 403);
-                if (ok) ok = mbar_wait(&aready[st], (uint32_t)(li / kStages) & 1, 404);
-                if (ok && li >= kTmemBufs)
-                    ok = mbar_wait(&tfree[tb], (uint32_t)((li / kTmemBufs) - 1) & 1, 405);
+                if (lane == 0) {
+                    if (first) ok = mbar_wait(&bfull[rb], (uint32_t)(seg >> 1) & 1, 403);
+                    if (ok) ok = mbar_wait(&aready[st], (uint32_t)(li / kStages) & 1, 404);
+                    if (ok && li >= kTmemBufs)
+                        ok = mbar_wait(&tfree[tb], (uint32_t)((li / kTmemBufs) - 1) & 1, 405);
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 tc_fence_after_sync();
                 const uint32_t ab = smem_u32(stages + st * kTileBytes);
-                const uint32_t bb0 = smem_u32(bop + rb * kBopSetBytes);
+                const uint32_t bb = smem_u32(bop + rb * kBopBytes);
 #pragma unroll
                 for (int j = 0; j < kPairHeads; ++j) {
                     const uint32_t d = tmem + tb * kBufCols + j * kN;
-                    const uint32_t bb = bb0 + j * kBopBytes;
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk) {
                         const uint64_t ad = make_smem_desc(ab + j * 64 + kk * 32, 16, 1024, kSwizzle128B);
-                        const uint64_t hi = make_smem_desc(bb + kk * 32, 16, 1024, kSwizzle128B);
-                        const uint64_t lo = make_smem_desc(bb + 64 + kk * 32, 16, 1024, kSwizzle128B);
-                        umma_bf16(d, ad, hi, idesc, kk > 0);
-                        umma_bf16(d, ad, lo, idesc, true);
+                        const uint64_t bd = make_smem_desc(bb + j * 64 + kk * 32, 16, 1024, kSwizzle128B);
+                        umma_bf16_elect(d, ad, bd, idesc, kk > 0);
                     }
                 }
-                umma_commit(&mmadone[st]);
+                umma_commit_elect(&mmadone[st]);
                 if (lastt) {
-                    umma_commit(&bempty[rb]);
+                    umma_commit_elect(&bempty[rb]);
                     ++seg;
                 }
             }
-            umma_commit(drain);
-            mbar_wait(drain, 0, 406);
+            umma_commit_elect(drain);
+            if (lane == 0) mbar_wait(drain, 0, 406);
+            __syncwarp();
         }
     } else if (warp == 2) {
         // ------------------------------------------------ B operand builder
-        // Per row segment: one bulk copy brings the pair's fp32 states into smem,
-        // then the 32 lanes write the swizzled bf16 hi/lo operand from there.
+        // Per row segment: the pair's state S_j[d][e] (j = head of the pair) lands in
+        // registers, lane = d: either the sum of the pass-1 partials of the row, slot
+        // by slot in slot order (bulk copies of up to kSlotsPerRound slots at a time),
+        // or the given state.  Lane pairs (d, d + 1) then write one bf16x2 each: even
+        // lanes the hi parts, odd lanes the lo parts.
         int seg = 0;
+        uint32_t sphase = 0;
         for (int64_t li = 0; i0 + li < i1 && ok; ++li) {
             const int64_t i = i0 + li;
             if (!(li == 0 || i % a.R == 0)) continue;              // not a segment start
@@ -558,44 +608,105 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
             if (seg == 0) pdl_wait_primary();                     // the states come from pass 1
             const int64_t r = i / a.R;
             const int b = (int)(r / a.Pp), p = (int)(r % a.Pp);
-            const int nh = min(kPairHeads, a.H - p * kPairHeads);
-            if (lane == 0) {
-                const uint32_t bytes = (uint32_t)(nh * kStateFloats * 4);
-                mbar_arrive_expect_tx(sready, bytes);
-                bulk_load(sstate, a.kv + ((size_t)b * a.H + p * kPairHeads) * kStateFloats, bytes,
-                          sready);
-            }
-            ok = mbar_wait(sready, (uint32_t)seg & 1, 410);
-            if (!ok) break;
-            uint8_t* dst = bop + rb * kBopSetBytes;
-            for (int idx = lane; idx < kPairHeads * kN * 8; idx += 32) {
-                const int j = idx / (kN * 8), rem = idx % (kN * 8), n = rem >> 3, ch = rem & 7;
-                const float* src = sstate + j * kStateFloats;
-                float vals[8];
+            const int h0 = p * kPairHeads;
+            const int nh = min(kPairHeads, a.H - h0);
+            float acc[kPairHeads][kDP];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int dd = (ch & 3) * 8 + u;
-                    const float x = (j < nh && n <= kD) ? src[dd * kDP + n] : 0.f;
-                    const float hi = __bfloat162float(__float2bfloat16_rn(x));
-                    vals[u] = (ch < 4) ? hi : (x - hi);
+            for (int j = 0; j < kPairHeads; ++j)
+#pragma unroll
+                for (int e = 0; e < kDP; ++e) acc[j][e] = 0.f;
+            if (a.kv == nullptr) {
+                const int64_t r1 = (int64_t)b * a.G1 + h0 / p1::kGroupHeads;
+                const int ns = p1_row_slots(r1, a.R1, a.T1, a.P1);
+                for (int s0 = 0; s0 < ns && ok; s0 += kSlotsPerRound) {
+                    const int n = min(kSlotsPerRound, ns - s0);
+                    __syncwarp();                                 // staging is free again
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(sready, (uint32_t)(nh * n * kStateFloats * 4));
+                        for (int j = 0; j < nh; ++j)
+                            bulk_load(staging + j * kSlotsPerRound * kStateFloats,
+                                      a.part + (((size_t)b * a.H + h0 + j) * a.Smax1 + s0) *
+                                                   kStateFloats,
+                                      (uint32_t)(n * kStateFloats * 4), sready);
+                    }
+                    ok = mbar_wait(sready, sphase, 410);
+                    sphase ^= 1;
+                    if (!ok) break;
+                    for (int s = 0; s < n; ++s)
+#pragma unroll
+                        for (int j = 0; j < kPairHeads; ++j)
+#pragma unroll
+                            for (int e = 0; e < kDP; ++e)
+                                acc[j][e] += staging[(j * kSlotsPerRound + s) * kStateFloats +
+                                                     e * kD + lane];
                 }
-                uint4 w;
-                w.x = pack_bf16x2(vals[0], vals[1]);
-                w.y = pack_bf16x2(vals[2], vals[3]);
-                w.z = pack_bf16x2(vals[4], vals[5]);
-                w.w = pack_bf16x2(vals[6], vals[7]);
-                *reinterpret_cast<uint4*>(dst + j * kBopBytes + sw128_offset(n, ch)) = w;
+            } else {
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(sready, (uint32_t)(nh * kStateFloats * 4));
+                    bulk_load(staging, a.kv + ((size_t)b * a.H + h0) * kStateFloats,
+                              (uint32_t)(nh * kStateFloats * 4), sready);
+                }
+                ok = mbar_wait(sready, sphase, 411);
+                sphase ^= 1;
+                if (ok) {
+#pragma unroll
+                    for (int j = 0; j < kPairHeads; ++j)
+#pragma unroll
+                        for (int e = 0; e < kDP; ++e)
+                            acc[j][e] = staging[j * kStateFloats + lane * kDP + e];
+                }
+            }
+            if (!ok) break;
+#pragma unroll
+            for (int j = 0; j < kPairHeads; ++j)
+                if (j >= nh)
+#pragma unroll
+                    for (int e = 0; e < kDP; ++e) acc[j][e] = 0.f;
+            uint8_t* dst = bop + rb * kBopBytes;
+            const int d0 = lane & ~1;                              // even d of the lane pair
+#pragma unroll
+            for (int j = 0; j < kPairHeads; ++j) {
+                const int chunk = j * 4 + d0 / 8, off = (d0 % 8) * 2;
+#pragma unroll
+                for (int e = 0; e < kDP; ++e) {
+                    const float x = acc[j][e];
+                    const float xp = __shfl_xor_sync(0xffffffffu, x, 1);
+                    const float xe = (lane & 1) ? xp : x, xo = (lane & 1) ? x : xp;
+                    const float he = __bfloat162float(__float2bfloat16_rn(xe));
+                    const float ho = __bfloat162float(__float2bfloat16_rn(xo));
+                    const int row = (lane & 1) ? (e < kD ? kLoRow + e : kDenLo) : e;
+                    const uint32_t w = (lane & 1) ? pack_bf16x2(xe - he, xo - ho) : pack_bf16x2(he, ho);
+                    *reinterpret_cast<uint32_t*>(dst + sw128_offset(row, chunk) + off) = w;
+                }
             }
             fence_proxy_async_smem();
-            __syncwarp();                                         // sstate is reused next segment
+            __syncwarp();
             mbar_arrive(&bfull[rb]);
             ++seg;
         }
+    } else if (warp == 3) {
+        // ------------------------------------------------ output stores
+        // Tiles go out in order; a slot returns to the producer as soon as its
+        // store has read it.
+        if (lane == 0 && ok) {
+            for (int64_t li = 0; i0 + li < i1 && ok; ++li) {
+                const int st = (int)(li % kStages);
+                ok = mbar_wait(&tready[st], (uint32_t)(li / kStages) & 1, 412);
+                if (!ok) break;
+                const int64_t i = i0 + li, r = i / a.R;
+                const int t = (int)(i % a.R), b = (int)(r / a.Pp), p = (int)(r % a.Pp);
+                tma_store_3d(&tmap_o, stages + st * kTileBytes, p * 64, t * kTileTok, b);
+                bulk_commit_group();
+                bulk_wait_group_read<0>();
+                mbar_arrive(&empty[st]);
+            }
+            bulk_wait_group<0>();
+        }
     } else {
-        // ------------------------------------------------ phi(Q), epilogue, TMA store
-        const int wi = warp - 3;                          // 0..7
+        // ------------------------------------------------ phi(Q), epilogue
+        const int wi = warp - 4;                          // 0..7
         const int grp = wi >> 2;                          // tiles with li % 2 == grp
-        const int gt = (wi & 3) * 32 + lane;              // 0..127 within the group
         const int q = warp & 3;                           // TMEM lane quadrant
         const int row = 32 * q + lane;                    // token row of the tile
 
@@ -625,40 +736,37 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
             if (!mbar_wait(&mmadone[st], (uint32_t)(li / kStages) & 1, 409)) return false;
             tc_fence_after_sync();
             const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * kBufCols;
-            float v[kPairHeads][kD + 1];
-#pragma unroll
-            for (int j = 0; j < kPairHeads; ++j) {
-                tmem_ld16(ta + j * kN, v[j]);
-                tmem_ld16(ta + j * kN + 16, v[j] + 16);
-                tmem_ld1(ta + j * kN + kD, v[j] + kD);
-            }
-            tmem_wait_ld();
-            tc_fence_before_sync();
-            mbar_arrive(&tfree[tb]);
             uint8_t* tile = stages + st * kTileBytes;
 #pragma unroll
-            for (int j = 0; j < kPairHeads; ++j) {
-                const float scale = rq[j] * __frcp_rn(fmaf(rq[j], v[j][kD], a.eps));
+            for (int j = 0; j < kPairHeads; ++j) {       // one head at a time (registers)
+                float hi[kD + 2], lo[kD];
+                tmem_ld16(ta + j * kN, hi);
+                tmem_ld16(ta + j * kN + 16, hi + 16);
+                tmem_ld2(ta + j * kN + kDenHi, hi + kD);
+                tmem_ld16(ta + j * kN + kLoRow, lo);
+                tmem_ld16(ta + j * kN + kLoRow + 16, lo + 16);
+                tmem_wait_ld();
+                if (j == kPairHeads - 1) {
+                    tc_fence_before_sync();
+                    mbar_arrive(&tfree[tb]);
+                }
+                const float den = hi[kD] + hi[kD + 1];
+                const float scale = rq[j] * __frcp_rn(fmaf(rq[j], den, a.eps));
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
+                    float o[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) o[u] = (hi[8 * cc + u] + lo[8 * cc + u]) * scale;
                     uint4 w;
-                    w.x = pack_bf16x2(v[j][8 * cc + 0] * scale, v[j][8 * cc + 1] * scale);
-                    w.y = pack_bf16x2(v[j][8 * cc + 2] * scale, v[j][8 * cc + 3] * scale);
-                    w.z = pack_bf16x2(v[j][8 * cc + 4] * scale, v[j][8 * cc + 5] * scale);
-                    w.w = pack_bf16x2(v[j][8 * cc + 6] * scale, v[j][8 * cc + 7] * scale);
+                    w.x = pack_bf16x2(o[0], o[1]);
+                    w.y = pack_bf16x2(o[2], o[3]);
+                    w.z = pack_bf16x2(o[4], o[5]);
+                    w.w = pack_bf16x2(o[6], o[7]);
                     *reinterpret_cast<uint4*>(tile + sw128_offset(row, j * 4 + cc)) = w;
                 }
             }
             fence_proxy_async_smem();
-            named_barrier_sync(1 + grp, 128);
-            if (gt == 0) {
-                const int64_t i = i0 + li, r = i / a.R;
-                const int t = (int)(i % a.R), b = (int)(r / a.Pp), p = (int)(r % a.Pp);
-                tma_store_3d(&tmap_o, tile, p * 64, t * kTileTok, b);
-                bulk_commit_group();
-                bulk_wait_group_read<1>();                // this group's previous store has read smem
-                if (li >= 2) mbar_arrive(&empty[(li - 2) % kStages]);
-            }
+            mbar_arrive(&tready[st]);
             return true;
         };
 
@@ -672,7 +780,6 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
             for (int j = 0; j < kPairHeads; ++j) r_prev[j] = r_cur[j];
         }
         if (ok && prev >= 0) ok = epilogue(prev, r_prev);
-        if (gt == 0) bulk_wait_group<0>();
     }
     tc_fence_before_sync();
     __syncthreads();
