@@ -387,7 +387,7 @@ def run_ours(args, rank, world, local):
                           "pass1_ms": a, "pass2_ms": b,
                           "hbm_frac_of_measured": 2 * by / ((a + b) * 1e-3) / 1e9 / hbm_gbs})
         # roofline of the dominant pass, on the largest launch shape of the sweep
-        dom_name, dom_kernel = ("pass 1 (state)", "kv_reduce_persistent") if p1_ms >= p2_ms else \
+        dom_name, dom_kernel = ("pass 1 (state)", "kv_partials_persistent") if p1_ms >= p2_ms else \
             ("pass 2 (apply)", "apply_persistent")
         big = max(range(len(sets)), key=lambda i: sets[i][0].tokens * 1e9 + sets[i][0].N)
         wb = sets[big][0]
@@ -412,8 +412,9 @@ def run_ours(args, rank, world, local):
                                   / hbm_gbs},
                      "parts": parts,
                      "gpu_launches": args.steps * len(sets) * 2,
-                     "per_pass_timing": "a second K-step loop of kv_state + apply with CUDA "
-                                        "events between the passes",
+                     "per_pass_timing": "a second K-step loop of kv_state (pass 1 + the small "
+                                        "partial-sum kernel) and apply (pass 2 from a given "
+                                        "state), CUDA events between the passes",
                      "clocks": clk.summary()})
 
         # e2e: the public call with host buffers, copies inside the timed region

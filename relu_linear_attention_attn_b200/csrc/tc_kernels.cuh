@@ -115,6 +115,75 @@ __device__ __forceinline__ float phi_inplace_sw128(uint8_t* tile, int row, int c
     return kScaleByRms ? 1.f : r;
 }
 
+// Two items of phi_inplace_sw128 at once: both items' loads are issued before
+// either item's stores, so their latencies overlap (the compiler cannot reorder
+// shared-memory stores and loads that may alias).
+template <bool kScaleByRms>
+__device__ __forceinline__ void phi2_inplace_sw128(uint8_t* const tile[2], const int row[2],
+                                                   const int chunk0[2], const float* const g[2],
+                                                   float eps, bool norm, const bool zero[2],
+                                                   float r_out[2], float* sum) {
+    uint4 u[2][4];
+#pragma unroll
+    for (int it = 0; it < 2; ++it)
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            u[it][c] = *reinterpret_cast<const uint4*>(tile[it] + sw128_offset(row[it], chunk0[it] + c));
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+        float x[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            x[8 * c + 0] = bf16lo(u[it][c].x); x[8 * c + 1] = bf16hi(u[it][c].x);
+            x[8 * c + 2] = bf16lo(u[it][c].y); x[8 * c + 3] = bf16hi(u[it][c].y);
+            x[8 * c + 4] = bf16lo(u[it][c].z); x[8 * c + 5] = bf16hi(u[it][c].z);
+            x[8 * c + 6] = bf16lo(u[it][c].w); x[8 * c + 7] = bf16hi(u[it][c].w);
+        }
+        float r = 1.f;
+        if (norm && !zero[it]) {
+            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                s0 = fmaf(x[i], x[i], s0);
+                s1 = fmaf(x[i + 1], x[i + 1], s1);
+                s2 = fmaf(x[i + 2], x[i + 2], s2);
+                s3 = fmaf(x[i + 3], x[i + 3], s3);
+            }
+            r = rsqrtf(((s0 + s1) + (s2 + s3)) * (1.f / kD) + eps);
+            const float* gi = g[it];
+            if (kScaleByRms) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[i] = fmaxf(gi[i] * (x[i] * r), 0.f);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[i] = fmaxf(gi[i] * x[i], 0.f);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = zero[it] ? 0.f : fmaxf(x[i], 0.f);
+        }
+        r_out[it] = kScaleByRms ? 1.f : r;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            u[it][c].x = pack_bf16x2(x[8 * c + 0], x[8 * c + 1]);
+            u[it][c].y = pack_bf16x2(x[8 * c + 2], x[8 * c + 3]);
+            u[it][c].z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
+            u[it][c].w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
+            if (sum) {
+                sum[8 * c + 0] += bf16lo(u[it][c].x); sum[8 * c + 1] += bf16hi(u[it][c].x);
+                sum[8 * c + 2] += bf16lo(u[it][c].y); sum[8 * c + 3] += bf16hi(u[it][c].y);
+                sum[8 * c + 4] += bf16lo(u[it][c].z); sum[8 * c + 5] += bf16hi(u[it][c].z);
+                sum[8 * c + 6] += bf16lo(u[it][c].w); sum[8 * c + 7] += bf16hi(u[it][c].w);
+            }
+        }
+    }
+#pragma unroll
+    for (int it = 0; it < 2; ++it)
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(tile[it] + sw128_offset(row[it], chunk0[it] + c)) = u[it][c];
+}
+
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
     return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
 }
@@ -324,14 +393,14 @@ kv_partials_persistent(const __grid_constant__ CUtensorMap tmap_k,
                 ok = mbar_wait(&full[st], (uint32_t)(li / kStages) & 1, 306);
                 if (!ok) break;
                 const int t = (int)((i0 + li) % a.R);
-#pragma unroll
-                for (int it = 0; it < 2; ++it) {
-                    const int row = lane + 32 * it;
-                    const bool live = (t * kStageTok + row < a.N) && (h < a.H);
-                    phi_inplace_sw128<true>(stages + st * kStageBytes + (hl >> 1) * kBoxBytes, row,
-                                            (hl & 1) * 4, sgain + (live ? h : 0) * kD, a.eps,
-                                            a.norm != 0, !live, ks);
-                }
+                uint8_t* const tl[2] = {stages + st * kStageBytes + (hl >> 1) * kBoxBytes,
+                                        stages + st * kStageBytes + (hl >> 1) * kBoxBytes};
+                const int rows[2] = {lane, lane + 32}, ch[2] = {(hl & 1) * 4, (hl & 1) * 4};
+                const bool dead[2] = {!((t * kStageTok + lane < a.N) && (h < a.H)),
+                                      !((t * kStageTok + lane + 32 < a.N) && (h < a.H))};
+                const float* gg[2] = {sgain + (h < a.H ? h : 0) * kD, sgain + (h < a.H ? h : 0) * kD};
+                float rr[2];
+                phi2_inplace_sw128<true>(tl, rows, ch, gg, a.eps, a.norm != 0, dead, rr, ks);
                 fence_proxy_async_smem();
                 mbar_arrive(&aready[st]);
             }
@@ -423,6 +492,7 @@ constexpr int kTileTok = 128;                      // UMMA M
 constexpr int kPairHeads = 2;                      // 64 channels = one swizzled row
 constexpr int kTileBytes = kTileTok * 128;         // 16 KB
 constexpr int kStages = 10;
+constexpr int kStoresInFlight = 2;                 // TMA stores the store warp keeps open
 constexpr int kN = 80;                             // B rows per head (see the file comment)
 constexpr int kLoRow = 48;                         // first row of the value columns' lo parts
 constexpr int kDenHi = 32, kDenLo = 33;            // rows of the normaliser's hi / lo parts
@@ -433,7 +503,8 @@ constexpr int kTmemBufs = 3;
 constexpr int kTmemCols = 512;
 constexpr int kSlotsPerRound = 3;                  // partial slots staged per bulk copy round
 constexpr int kStagingBytes = kPairHeads * kSlotsPerRound * kStateFloats * 4;
-constexpr int kWorkerWarps = 8;                    // two groups of 4, alternating tiles
+constexpr int kWorkerWarps = 16;                   // two tile groups of 8, alternating tiles
+constexpr int kGroupThreads = 32 * kWorkerWarps / 2;   // a tile group: 4 quadrants x 2 heads
 constexpr int kThreads = 32 * (4 + kWorkerWarps);  // TMA, UMMA, builder, store, workers
 constexpr int kGainCache = 4096;
 constexpr int kSmemBytes = 1024 + kStages * kTileBytes + kBopRing * kBopBytes + kStagingBytes +
@@ -455,7 +526,7 @@ struct P2Args {
     int norm;
 };
 
-__global__ void __launch_bounds__(p2::kThreads, 1)
+__global__ void __launch_bounds__(p2::kThreads, 1)   // 640 threads: at most 96 registers
 apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
                  const __grid_constant__ CUtensorMap tmap_o, const P2Args a)
 {
@@ -489,12 +560,12 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
         mbar_init(sready, 1);
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&aready[i], 128);
+            mbar_init(&aready[i], kGroupThreads);
             mbar_init(&mmadone[i], 1);
-            mbar_init(&tready[i], 128);
+            mbar_init(&tready[i], kGroupThreads);
             mbar_init(&empty[i], 1);
         }
-        for (int i = 0; i < kTmemBufs; ++i) mbar_init(&tfree[i], 128);
+        for (int i = 0; i < kTmemBufs; ++i) mbar_init(&tfree[i], kGroupThreads);
         for (int i = 0; i < kBopRing; ++i) {
             mbar_init(&bfull[i], 32);
             mbar_init(&bempty[i], 1);
@@ -610,67 +681,54 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
             const int b = (int)(r / a.Pp), p = (int)(r % a.Pp);
             const int h0 = p * kPairHeads;
             const int nh = min(kPairHeads, a.H - h0);
-            float acc[kPairHeads][kDP];
-#pragma unroll
-            for (int j = 0; j < kPairHeads; ++j)
-#pragma unroll
-                for (int e = 0; e < kDP; ++e) acc[j][e] = 0.f;
-            if (a.kv == nullptr) {
-                const int64_t r1 = (int64_t)b * a.G1 + h0 / p1::kGroupHeads;
-                const int ns = p1_row_slots(r1, a.R1, a.T1, a.P1);
-                for (int s0 = 0; s0 < ns && ok; s0 += kSlotsPerRound) {
-                    const int n = min(kSlotsPerRound, ns - s0);
-                    __syncwarp();                                 // staging is free again
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(sready, (uint32_t)(nh * n * kStateFloats * 4));
-                        for (int j = 0; j < nh; ++j)
-                            bulk_load(staging + j * kSlotsPerRound * kStateFloats,
-                                      a.part + (((size_t)b * a.H + h0 + j) * a.Smax1 + s0) *
-                                                   kStateFloats,
-                                      (uint32_t)(n * kStateFloats * 4), sready);
-                    }
-                    ok = mbar_wait(sready, sphase, 410);
-                    sphase ^= 1;
-                    if (!ok) break;
-                    for (int s = 0; s < n; ++s)
-#pragma unroll
-                        for (int j = 0; j < kPairHeads; ++j)
-#pragma unroll
-                            for (int e = 0; e < kDP; ++e)
-                                acc[j][e] += staging[(j * kSlotsPerRound + s) * kStateFloats +
-                                                     e * kD + lane];
-                }
-            } else {
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(sready, (uint32_t)(nh * kStateFloats * 4));
-                    bulk_load(staging, a.kv + ((size_t)b * a.H + h0) * kStateFloats,
-                              (uint32_t)(nh * kStateFloats * 4), sready);
-                }
-                ok = mbar_wait(sready, sphase, 411);
-                sphase ^= 1;
-                if (ok) {
-#pragma unroll
-                    for (int j = 0; j < kPairHeads; ++j)
-#pragma unroll
-                        for (int e = 0; e < kDP; ++e)
-                            acc[j][e] = staging[j * kStateFloats + lane * kDP + e];
-                }
-            }
-            if (!ok) break;
-#pragma unroll
-            for (int j = 0; j < kPairHeads; ++j)
-                if (j >= nh)
-#pragma unroll
-                    for (int e = 0; e < kDP; ++e) acc[j][e] = 0.f;
             uint8_t* dst = bop + rb * kBopBytes;
             const int d0 = lane & ~1;                              // even d of the lane pair
+            int ns = 1;
+            if (a.kv == nullptr)
+                ns = p1_row_slots((int64_t)b * a.G1 + h0 / p1::kGroupHeads, a.R1, a.T1, a.P1);
+            // heads one at a time (registers); the bulk copies of a round bring both
+            for (int j = 0; j < kPairHeads && ok; ++j) {
+                float acc[kDP];
 #pragma unroll
-            for (int j = 0; j < kPairHeads; ++j) {
+                for (int e = 0; e < kDP; ++e) acc[e] = 0.f;
+                for (int s0 = 0; s0 < ns && ok; s0 += kSlotsPerRound) {
+                    const int n = min(kSlotsPerRound, ns - s0);
+                    if (j == 0 || ns > kSlotsPerRound) {          // (re)fill the staging area
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (a.kv == nullptr) {
+                                mbar_arrive_expect_tx(sready, (uint32_t)(nh * n * kStateFloats * 4));
+                                for (int jj = 0; jj < nh; ++jj)
+                                    bulk_load(staging + jj * kSlotsPerRound * kStateFloats,
+                                              a.part + (((size_t)b * a.H + h0 + jj) * a.Smax1 + s0) *
+                                                           kStateFloats,
+                                              (uint32_t)(n * kStateFloats * 4), sready);
+                            } else {
+                                mbar_arrive_expect_tx(sready, (uint32_t)(nh * kStateFloats * 4));
+                                bulk_load(staging, a.kv + ((size_t)b * a.H + h0) * kStateFloats,
+                                          (uint32_t)(nh * kStateFloats * 4), sready);
+                            }
+                        }
+                        ok = mbar_wait(sready, sphase, 410);
+                        sphase ^= 1;
+                        if (!ok) break;
+                    }
+                    if (j >= nh) continue;                        // missing head: zeros
+                    if (a.kv == nullptr) {
+                        for (int s = 0; s < n; ++s)
+#pragma unroll
+                            for (int e = 0; e < kDP; ++e)
+                                acc[e] += staging[(j * kSlotsPerRound + s) * kStateFloats + e * kD + lane];
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < kDP; ++e) acc[e] = staging[j * kStateFloats + lane * kDP + e];
+                    }
+                }
+                if (!ok) break;
                 const int chunk = j * 4 + d0 / 8, off = (d0 % 8) * 2;
 #pragma unroll
                 for (int e = 0; e < kDP; ++e) {
-                    const float x = acc[j][e];
+                    const float x = acc[e];
                     const float xp = __shfl_xor_sync(0xffffffffu, x, 1);
                     const float xe = (lane & 1) ? xp : x, xo = (lane & 1) ? x : xp;
                     const float he = __bfloat162float(__float2bfloat16_rn(xe));
@@ -680,6 +738,7 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
                     *reinterpret_cast<uint32_t*>(dst + sw128_offset(row, chunk) + off) = w;
                 }
             }
+            if (!ok) break;
             fence_proxy_async_smem();
             __syncwarp();
             mbar_arrive(&bfull[rb]);
@@ -690,7 +749,8 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
         // Tiles go out in order; a slot returns to the producer as soon as its
         // store has read it.
         if (lane == 0 && ok) {
-            for (int64_t li = 0; i0 + li < i1 && ok; ++li) {
+            int64_t li = 0;
+            for (; i0 + li < i1 && ok; ++li) {
                 const int st = (int)(li % kStages);
                 ok = mbar_wait(&tready[st], (uint32_t)(li / kStages) & 1, 412);
                 if (!ok) break;
@@ -698,72 +758,70 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
                 const int t = (int)(i % a.R), b = (int)(r / a.Pp), p = (int)(r % a.Pp);
                 tma_store_3d(&tmap_o, stages + st * kTileBytes, p * 64, t * kTileTok, b);
                 bulk_commit_group();
-                bulk_wait_group_read<0>();
-                mbar_arrive(&empty[st]);
+                if (li >= kStoresInFlight - 1) {       // the oldest store in flight has read its tile
+                    bulk_wait_group_read<kStoresInFlight - 1>();
+                    mbar_arrive(&empty[(li - (kStoresInFlight - 1)) % kStages]);
+                }
             }
+            bulk_wait_group_read<0>();
+            for (int64_t lj = li - (kStoresInFlight - 1) > 0 ? li - (kStoresInFlight - 1) : 0; lj < li; ++lj)
+                mbar_arrive(&empty[lj % kStages]);
             bulk_wait_group<0>();
         }
     } else {
         // ------------------------------------------------ phi(Q), epilogue
-        const int wi = warp - 4;                          // 0..7
-        const int grp = wi >> 2;                          // tiles with li % 2 == grp
+        // Two tile groups of 8 warps take alternate tiles; in a group, warp w takes
+        // TMEM quadrant w % 4 (token rows 32 (w % 4) ..) and head (w / 4) % 2 of the pair.
+        const int wi = warp - 4;                          // 0..15
+        const int grp = wi >> 3;                          // tiles with li % 2 == grp
+        const int j = (wi >> 2) & 1;                      // head of the pair
         const int q = warp & 3;                           // TMEM lane quadrant
         const int row = 32 * q + lane;                    // token row of the tile
 
         // The per-token factor r = rsqrt(mean(q^2) + eps) of phi(Q) is positive, so it
         // is left out of the A operand and applied in the epilogue:
         //   O = (r num') / (r den' + eps),  num', den' computed with ReLU(g * q).
-        auto transform = [&](int64_t li, float* rq) -> bool {
+        auto transform = [&](int64_t li, float& rq) -> bool {
             const int st = (int)(li % kStages);
             if (!mbar_wait(&full[st], (uint32_t)(li / kStages) & 1, 408)) return false;
             const int64_t i = i0 + li, r = i / a.R;
             const int t = (int)(i % a.R), p = (int)(r % a.Pp);
-            uint8_t* tile = stages + st * kTileBytes;
-            const bool row_live = t * kTileTok + row < a.N;
-#pragma unroll
-            for (int j = 0; j < kPairHeads; ++j) {
-                const int h = p * kPairHeads + j;
-                const bool live = row_live && h < a.H;
-                rq[j] = phi_inplace_sw128<false>(tile, row, j * 4, sgain + (live ? h : 0) * kD,
-                                                 a.eps, a.norm != 0, !live);
-            }
+            const int h = p * kPairHeads + j;
+            const bool live = (t * kTileTok + row < a.N) && h < a.H;
+            rq = phi_inplace_sw128<false>(stages + st * kTileBytes, row, j * 4,
+                                          sgain + (live ? h : 0) * kD, a.eps, a.norm != 0, !live);
             fence_proxy_async_smem();
             mbar_arrive(&aready[st]);
             return true;
         };
-        auto epilogue = [&](int64_t li, const float* rq) -> bool {
+        auto epilogue = [&](int64_t li, float rq) -> bool {
             const int st = (int)(li % kStages), tb = (int)(li % kTmemBufs);
             if (!mbar_wait(&mmadone[st], (uint32_t)(li / kStages) & 1, 409)) return false;
             tc_fence_after_sync();
-            const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * kBufCols;
+            const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * kBufCols + j * kN;
+            float hi[kD + 2], lo[kD];
+            tmem_ld16(ta, hi);
+            tmem_ld16(ta + 16, hi + 16);
+            tmem_ld2(ta + kDenHi, hi + kD);
+            tmem_ld16(ta + kLoRow, lo);
+            tmem_ld16(ta + kLoRow + 16, lo + 16);
+            tmem_wait_ld();
+            tc_fence_before_sync();
+            mbar_arrive(&tfree[tb]);
+            const float den = hi[kD] + hi[kD + 1];
+            const float scale = rq * __frcp_rn(fmaf(rq, den, a.eps));
             uint8_t* tile = stages + st * kTileBytes;
 #pragma unroll
-            for (int j = 0; j < kPairHeads; ++j) {       // one head at a time (registers)
-                float hi[kD + 2], lo[kD];
-                tmem_ld16(ta + j * kN, hi);
-                tmem_ld16(ta + j * kN + 16, hi + 16);
-                tmem_ld2(ta + j * kN + kDenHi, hi + kD);
-                tmem_ld16(ta + j * kN + kLoRow, lo);
-                tmem_ld16(ta + j * kN + kLoRow + 16, lo + 16);
-                tmem_wait_ld();
-                if (j == kPairHeads - 1) {
-                    tc_fence_before_sync();
-                    mbar_arrive(&tfree[tb]);
-                }
-                const float den = hi[kD] + hi[kD + 1];
-                const float scale = rq[j] * __frcp_rn(fmaf(rq[j], den, a.eps));
+            for (int cc = 0; cc < 4; ++cc) {
+                float o[8];
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    float o[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) o[u] = (hi[8 * cc + u] + lo[8 * cc + u]) * scale;
-                    uint4 w;
-                    w.x = pack_bf16x2(o[0], o[1]);
-                    w.y = pack_bf16x2(o[2], o[3]);
-                    w.z = pack_bf16x2(o[4], o[5]);
-                    w.w = pack_bf16x2(o[6], o[7]);
-                    *reinterpret_cast<uint4*>(tile + sw128_offset(row, j * 4 + cc)) = w;
-                }
+                for (int u = 0; u < 8; ++u) o[u] = (hi[8 * cc + u] + lo[8 * cc + u]) * scale;
+                uint4 w;
+                w.x = pack_bf16x2(o[0], o[1]);
+                w.y = pack_bf16x2(o[2], o[3]);
+                w.z = pack_bf16x2(o[4], o[5]);
+                w.w = pack_bf16x2(o[6], o[7]);
+                *reinterpret_cast<uint4*>(tile + sw128_offset(row, j * 4 + cc)) = w;
             }
             fence_proxy_async_smem();
             mbar_arrive(&tready[st]);
@@ -771,13 +829,12 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
         };
 
         int64_t prev = -1;
-        float r_prev[kPairHeads] = {1.f, 1.f}, r_cur[kPairHeads];
+        float r_prev = 1.f, r_cur = 1.f;
         for (int64_t li = grp; i0 + li < i1 && ok; li += 2) {
             ok = transform(li, r_cur);
             if (ok && prev >= 0) ok = epilogue(prev, r_prev);
             prev = li;
-#pragma unroll
-            for (int j = 0; j < kPairHeads; ++j) r_prev[j] = r_cur[j];
+            r_prev = r_cur;
         }
         if (ok && prev >= 0) ok = epilogue(prev, r_prev);
     }
