@@ -56,6 +56,19 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 
 // One bounded try: the thread may be suspended (not spinning) until the phase
 // completes or about `suspend_ns` pass; returns whether the phase completed.
+// Non-blocking test: has the phase with this parity completed?
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity,
                                               uint32_t suspend_ns) {
     uint32_t done;
@@ -76,6 +89,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity,
 // records kErrWaitTimeout with `site`, and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site,
                                           uint64_t limit_ns = 2000000000ull) {
+    if (mbar_test(bar, parity)) return true;                 // already complete: no suspend
     const uint32_t hint = limit_ns < 1000000ull ? (uint32_t)limit_ns : 1000000u;
     if (mbar_try_wait(bar, parity, hint)) return true;
     const uint64_t t0 = global_timer_ns();

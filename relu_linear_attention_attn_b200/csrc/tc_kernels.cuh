@@ -327,37 +327,41 @@ kv_partials_persistent(const __grid_constant__ CUtensorMap tmap_k,
     } else if (warp == 1) {
         // ------------------------------------------------ UMMA issuer (whole warp,
         // one elected lane issues)
+        // Ring position, phase bit and descriptors advance as counters (no divisions or
+        // descriptor packing per stage).
         if (ok) {
             const uint32_t idesc = make_idesc_bf16(128, 128, true, true);
-            int seg = 0;
-            for (int64_t li = 0; i0 + li < i1 && ok; ++li) {
-                const int64_t i = i0 + li;
-                const int t = (int)(i % a.R), st = (int)(li % kStages);
+            const uint64_t k0 = make_smem_desc(smem_u32(stages), kBoxBytes, 1024, kSwizzle128B);
+            const uint64_t v0 = k0 + (uint64_t)((2 * kBoxBytes) >> 4);
+            const int64_t n = i1 - i0;
+            int st = 0, seg = 0;
+            uint32_t fpar = 0;
+            int64_t t = i0 % a.R;
+            for (int64_t li = 0; li < n; ++li) {
                 const bool first = (li == 0) || (t == 0);
-                const bool lastst = (i + 1 == i1) || (t == a.R - 1);
+                const bool lastst = (li + 1 == n) || (t == a.R - 1);
                 const int abuf = seg & 1;
                 if (lane == 0) {
                     if (first && seg >= 2)
                         ok = mbar_wait(&accempty[abuf], (uint32_t)((seg >> 1) - 1) & 1, 303);
-                    if (ok) ok = mbar_wait(&aready[st], (uint32_t)(li / kStages) & 1, 304);
+                    if (ok) ok = mbar_wait(&aready[st], fpar, 304);
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 tc_fence_after_sync();
                 const uint32_t d = tmem + abuf * kAccCols;
-                const uint32_t kb = smem_u32(stages + st * kStageBytes);
-                const uint32_t vb = kb + 2 * kBoxBytes;
+                const uint64_t so = (uint64_t)((st * kStageBytes) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kStageTok / 16; ++kk) {
-                    const uint64_t ad = make_smem_desc(kb + kk * 2048, kBoxBytes, 1024, kSwizzle128B);
-                    const uint64_t bd = make_smem_desc(vb + kk * 2048, kBoxBytes, 1024, kSwizzle128B);
-                    umma_bf16_elect(d, ad, bd, idesc, !(first && kk == 0));
-                }
+                for (int kk = 0; kk < kStageTok / 16; ++kk)   // 16 token rows = 2048 bytes a step
+                    umma_bf16_elect(d, k0 + so + kk * 128, v0 + so + kk * 128, idesc,
+                                    !(first && kk == 0));
                 umma_commit_elect(&empty[st]);
                 if (lastst) {
                     umma_commit_elect(&accfull[abuf]);
                     ++seg;
                 }
+                if (++st == kStages) { st = 0; fpar ^= 1; }
+                if (++t == a.R) t = 0;
             }
             umma_commit_elect(drain);
             if (lane == 0) mbar_wait(drain, 0, 305);
@@ -621,41 +625,43 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
     } else if (warp == 1) {
         // ------------------------------------------------ UMMA issuer (whole warp,
         // one elected lane issues)
+        // Ring / TMEM positions and phase bits advance as counters, and descriptors are
+        // stepped from precomputed ones (their start address is in 16-byte units).
         if (ok) {
             const uint32_t idesc = make_idesc_bf16(128, kN, false, false);
-            int seg = 0;
-            for (int64_t li = 0; i0 + li < i1 && ok; ++li) {
-                const int64_t i = i0 + li;
-                const int t = (int)(i % a.R), st = (int)(li % kStages);
+            const uint64_t a0 = make_smem_desc(smem_u32(stages), 16, 1024, kSwizzle128B);
+            const uint64_t b0 = make_smem_desc(smem_u32(bop), 16, 1024, kSwizzle128B);
+            const int64_t n = i1 - i0;
+            int st = 0, tb = 0, seg = 0;
+            uint32_t fpar = 0, tpar = 0;
+            int64_t t = i0 % a.R;
+            for (int64_t li = 0; li < n; ++li) {
                 const bool first = (li == 0) || (t == 0);
-                const bool lastt = (i + 1 == i1) || (t == a.R - 1);
-                const int rb = seg & 1, tb = (int)(li % kTmemBufs);
+                const bool lastt = (li + 1 == n) || (t == a.R - 1);
+                const int rb = seg & 1;
                 if (lane == 0) {
                     if (first) ok = mbar_wait(&bfull[rb], (uint32_t)(seg >> 1) & 1, 403);
-                    if (ok) ok = mbar_wait(&aready[st], (uint32_t)(li / kStages) & 1, 404);
-                    if (ok && li >= kTmemBufs)
-                        ok = mbar_wait(&tfree[tb], (uint32_t)((li / kTmemBufs) - 1) & 1, 405);
+                    if (ok) ok = mbar_wait(&aready[st], fpar, 404);
+                    if (ok && li >= kTmemBufs) ok = mbar_wait(&tfree[tb], tpar ^ 1, 405);
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 tc_fence_after_sync();
-                const uint32_t ab = smem_u32(stages + st * kTileBytes);
-                const uint32_t bb = smem_u32(bop + rb * kBopBytes);
-#pragma unroll
-                for (int j = 0; j < kPairHeads; ++j) {
-                    const uint32_t d = tmem + tb * kBufCols + j * kN;
-#pragma unroll
-                    for (int kk = 0; kk < 2; ++kk) {
-                        const uint64_t ad = make_smem_desc(ab + j * 64 + kk * 32, 16, 1024, kSwizzle128B);
-                        const uint64_t bd = make_smem_desc(bb + j * 64 + kk * 32, 16, 1024, kSwizzle128B);
-                        umma_bf16_elect(d, ad, bd, idesc, kk > 0);
-                    }
-                }
+                const uint64_t ad = a0 + (uint64_t)((st * kTileBytes) >> 4);
+                const uint64_t bd = b0 + (uint64_t)((rb * kBopBytes) >> 4);
+                const uint32_t d = tmem + tb * kBufCols;
+                umma_bf16_elect(d, ad, bd, idesc, false);
+                umma_bf16_elect(d, ad + 2, bd + 2, idesc, true);
+                umma_bf16_elect(d + kN, ad + 4, bd + 4, idesc, false);
+                umma_bf16_elect(d + kN, ad + 6, bd + 6, idesc, true);
                 umma_commit_elect(&mmadone[st]);
                 if (lastt) {
                     umma_commit_elect(&bempty[rb]);
                     ++seg;
                 }
+                if (++st == kStages) { st = 0; fpar ^= 1; }
+                if (++tb == kTmemBufs) { tb = 0; tpar ^= 1; }
+                if (++t == a.R) t = 0;
             }
             umma_commit_elect(drain);
             if (lane == 0) mbar_wait(drain, 0, 406);
