@@ -557,6 +557,30 @@ def fused_measure(args, sla, w, rank, dev, stream, world, bf16_tf, peak_kind):
             "gpu_launches": steps * 2, "clocks": clk.summary()}
 
 
+def profile_case(args):
+    """--warmup calls of sana_linattn_forward (two kernel launches each) on one
+    workload, optionally with another batch size; prints a checksum."""
+    import torch
+
+    import relu_linear_attention_attn_b200 as sla
+    from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
+
+    w = CONFIGS[4] if args.workload == "fused" else select(args.workload)[-1]
+    if args.batch:
+        w = w.scaled(B=args.batch)
+    x = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in make_inputs(w).items()}
+    ws = torch.empty(sla.workspace_bytes(w.B, w.N, w.C, w.H, fused=args.workload == "fused"),
+                     dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        if args.workload == "fused":
+            out = sla.qkv_fused(x["x"], x["W"], x["gq"], x["gk"], w.H, w.eps, workspace=ws)
+        else:
+            out = sla.forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps, workspace=ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": w.name, "B": w.B, "N": w.N, "calls": args.warmup,
+                      "checksum": float(out.float().abs().mean())}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -569,7 +593,15 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches, no CUDA graph")
+    ap.add_argument("--profile-case", action="store_true",
+                    help="no timing: run --warmup forward calls of --workload and exit (a small, "
+                         "fixed launch sequence for ncu captures)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="with --profile-case: batch size override for the workload")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
