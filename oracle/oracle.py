@@ -20,6 +20,12 @@ brute-forced on tiny inputs, hand-derived worked examples in
 ``tests/golden/``, closed forms (N = 1, one-hot keys, constant values),
 invariants (linearity in V, token permutation, scale invariance), and
 torch's own ``rms_norm`` for the feature map.
+
+The W8A8 prologue (``quantize_i8``, ``w8a8_project``, ``w8a8_fused_forward``)
+is pinned by ``tests/test_oracle_w8a8.py``: hand-derived codes and a
+hand-derived projection (``tests/golden/w8a8_quantize.json``), a pure-Python
+integer brute force, the half-step rounding bound, and equality with the fused
+forward on the dequantised tensors.
 """
 from __future__ import annotations
 
@@ -225,6 +231,66 @@ def fused_forward(x, W, gq, gk, H: int, eps: float, tokens=None, nthreads: int =
     q = qkv_project(xs, W, rows=(0, C))
     # apply() indexes q by flat token; give it a (B, N, C) view with only the
     # sampled rows filled, which it never reads past.
+    qfull = np.zeros((B * N, C), dtype=np.float64)
+    qfull[tok] = q
+    return apply(qfull.reshape(B, N, C), gq, S, H, eps, tokens=tok, nthreads=nthreads)
+
+
+# ----------------------------------------------------------------------------- W8A8
+# The W8A8 prologue of the fused variant ("Sana: Efficient High-Resolution Image
+# Synthesis with Linear Diffusion Transformers", section 7, on-device deployment:
+# linear layers in 8-bit weights and activations, attention kept in full
+# precision).  The pages do not state the scale granularity; the reading here is
+# symmetric int8 with one scale per token of x and one per output channel of Wqkv.
+# Codes are integers decided by floating point, so they are formed in fp32 exactly
+# as stated below (IEEE division, round half to even), the precision the kernels
+# use, and compared bit for bit.
+
+def quantize_i8(x, axis: int = -1):
+    """Symmetric int8 codes along `axis`: scale = max|x| / 127 (fp32), code =
+    round_half_even(x / scale) in fp32, clipped to [-127, 127].  A slice that is
+    all zero gets scale 0 and zero codes.  Returns (codes int8, scales fp32 with
+    `axis` removed)."""
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.max(np.abs(x32), axis=axis, keepdims=True)
+    s = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    q = np.rint((x32 / safe).astype(np.float32))
+    q = np.where(s > 0, q, np.float32(0.0))
+    q = np.clip(q, -127, 127).astype(np.int8)
+    return q, np.squeeze(s, axis=axis)
+
+
+def w8a8_project(xq, sx, Wq, sw, rows=None) -> np.ndarray:
+    """Dequantised projection of int8 codes: (xq @ Wq)[n, c] * sx[n] * sw[c].
+    xq: (..., C) int8, sx: (...) scales; Wq: (C, 3C) int8, sw: (3C,) scales.
+    The integer products sum exactly in fp64 (|sum| <= 127^2 * C < 2^53)."""
+    xq = np.asarray(xq).astype(np.float64)
+    Wq = np.asarray(Wq).astype(np.float64)
+    sw = np.asarray(sw, dtype=np.float64)
+    if rows is not None:
+        Wq = Wq[:, rows[0]:rows[1]]
+        sw = sw[rows[0]:rows[1]]
+    acc = np.matmul(xq, Wq)
+    return acc * np.asarray(sx, dtype=np.float64)[..., None] * sw
+
+
+def w8a8_fused_forward(xq, sx, Wq, sw, gq, gk, H: int, eps: float, tokens=None,
+                       nthreads: int = 0):
+    """The fused variant on int8 codes: dequantised projection, then Eq. (1) with
+    QK-RMSNorm in fp64.  tokens: optional flat token indices of O to form."""
+    xq = np.asarray(xq)
+    B, N, C = xq.shape
+    kvp = w8a8_project(xq, sx, Wq, sw, rows=(C, 3 * C))
+    k, v = kvp[..., :C], kvp[..., C:]
+    S = kv_state(np.ascontiguousarray(k), np.ascontiguousarray(v), gk, H, eps,
+                 nthreads=nthreads, norm=gk is not None)
+    if tokens is None:
+        q = w8a8_project(xq, sx, Wq, sw, rows=(0, C))
+        return apply(q, gq, S, H, eps, nthreads=nthreads)
+    tok = np.asarray(tokens, dtype=np.int64)
+    q = w8a8_project(xq.reshape(B * N, C)[tok], np.asarray(sx).reshape(B * N)[tok], Wq, sw,
+                     rows=(0, C))
     qfull = np.zeros((B * N, C), dtype=np.float64)
     qfull[tok] = q
     return apply(qfull.reshape(B, N, C), gq, S, H, eps, tokens=tok, nthreads=nthreads)
