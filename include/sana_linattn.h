@@ -115,6 +115,43 @@ SANA_API int sana_linattn_qkv_fused(const void* x, const void* Wqkv,
                            int64_t B, int64_t N, int C, int H, float eps,
                            void* workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* The fused variant with a W8A8 prologue (section 7 of the Sana notes, on-device
+ * deployment: linear layers in 8-bit weights and activations, attention in full
+ * precision).  The pages leave the scale granularity open; this library uses
+ * symmetric int8 with one scale per token of x and one per output channel of
+ * Wqkv, as produced by sana_quantize_rows_i8 / sana_quantize_cols_i8:
+ *     [Q | K | V][n, c] = (sum_k xq[n, k] Wq[k, c]) * sx[n] * sw[c]
+ * with the integer sum exact (int32) and the scaling in fp32; the norm, feature
+ * map and Eq. (1) then run exactly as in sana_linattn_qkv_fused.
+ * xq: (B, N, C) int8, 16-byte aligned; sx: fp32 [B * N]; Wq: (C, 3C) int8
+ * row-major, columns [Q | K | V], 16-byte aligned; sw: fp32 [3C]; gq, gk: fp32
+ * [C] or both NULL; out: (B, N, C) bf16.  workspace: at least
+ * sana_linattn_workspace_bytes(B, N, C, H, 1) bytes.  Errors as for
+ * sana_linattn_qkv_fused; out must not overlap any input. */
+SANA_API int sana_linattn_qkv_fused_w8a8(const int8_t* xq, const float* sx,
+                                         const int8_t* Wq, const float* sw,
+                                         const float* gq, const float* gk, void* out,
+                                         int64_t B, int64_t N, int C, int H, float eps,
+                                         void* workspace, size_t ws_bytes,
+                                         cudaStream_t stream);
+
+/* Symmetric int8 quantisation of each row of x (rows, cols) in `dtype`
+ * (row-major, cols % 8 == 0, x 16-byte aligned for bf16 / 32 for fp32, xq
+ * 8-byte aligned): scales[r] = max_c |x[r, c]| / 127 (fp32, IEEE division) and
+ * xq[r, c] = round_half_even(x[r, c] / scales[r]) in fp32, clamped to
+ * [-127, 127]; an all-zero row gets scale 0 and zero codes.  xq and scales are
+ * caller-owned device memory and must not overlap x or each other. */
+SANA_API int sana_quantize_rows_i8(const void* x, sana_dtype dtype, int8_t* xq,
+                                   float* scales, int64_t rows, int cols,
+                                   cudaStream_t stream);
+
+/* The same per column of a (K, cols) row-major matrix (e.g. Wqkv with
+ * cols = 3C): scales[c] = max_k |w[k, c]| / 127, wq[k, c] = round_half_even(
+ * w[k, c] / scales[c]) clamped to [-127, 127]. */
+SANA_API int sana_quantize_cols_i8(const void* w, sana_dtype dtype, int8_t* wq,
+                                   float* scales, int64_t K, int cols,
+                                   cudaStream_t stream);
+
 /* sana_linattn_forward without a caller-provided workspace, for callers that
  * cannot allocate device memory: code running inside a CUDA-graph capture or a
  * framework hook where cudaMalloc is forbidden, allocators that must not be

@@ -16,6 +16,7 @@ import os
 import threading
 
 __all__ = ["load", "lib_path", "workspace_bytes", "forward", "forward_noalloc", "kv_state", "apply", "qkv_fused",
+           "qkv_fused_w8a8", "quantize_rows_i8", "quantize_cols_i8",
            "device_error", "selftest_wait_timeout", "SanaError", "STATUS", "BF16", "F32"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -52,6 +53,13 @@ def _declare(lib):
     for f in (lib.sana_linattn_forward, lib.sana_linattn_kv_state, lib.sana_linattn_apply,
               lib.sana_linattn_qkv_fused):
         f.restype = ctypes.c_int
+    lib.sana_linattn_qkv_fused_w8a8.argtypes = [vp, fp, vp, fp, fp, fp, vp, i64, i64, ci, ci, cf,
+                                                vp, sz, vp]
+    lib.sana_linattn_qkv_fused_w8a8.restype = ctypes.c_int
+    lib.sana_quantize_rows_i8.argtypes = [vp, ci, vp, fp, i64, ci, vp]
+    lib.sana_quantize_rows_i8.restype = ctypes.c_int
+    lib.sana_quantize_cols_i8.argtypes = [vp, ci, vp, fp, i64, ci, vp]
+    lib.sana_quantize_cols_i8.restype = ctypes.c_int
     lib.sana_linattn_forward_noalloc.argtypes = [vp, vp, vp, fp, fp, vp, i64, i64, ci, ci, cf, ci,
                                                  vp]
     lib.sana_linattn_forward_noalloc.restype = ctypes.c_int
@@ -215,6 +223,61 @@ def selftest_wait_timeout(limit_us: int = 20000, stream=None):
     """Enqueue the bounded-wait self-test (see include/sana_linattn.h)."""
     _check("sana_linattn_selftest_wait_timeout",
            load().sana_linattn_selftest_wait_timeout(int(limit_us), _stream(stream)))
+
+
+def quantize_rows_i8(x, out=None, scales=None, stream=None):
+    """Symmetric int8 codes of each row of x (..., cols) (bf16 or fp32): returns
+    (codes int8 of x's shape, scales fp32 of x.shape[:-1]); scale = max|row| / 127,
+    code = round_half_even(x / scale) clamped to [-127, 127]."""
+    torch = _torch()
+    cols = x.shape[-1]
+    rows = x.numel() // cols if cols else 0
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    rc = load().sana_quantize_rows_i8(_dev(x, "x"), _dtype_code(x), _dev(out, "codes"),
+                                      _dev(scales, "scales"), rows, cols, _stream(stream))
+    _check("sana_quantize_rows_i8", rc)
+    return out, scales
+
+
+def quantize_cols_i8(w, out=None, scales=None, stream=None):
+    """Symmetric int8 codes of each column of w (K, cols) (bf16 or fp32): returns
+    (codes int8 (K, cols), scales fp32 (cols,))."""
+    torch = _torch()
+    K, cols = w.shape
+    if out is None:
+        out = torch.empty(w.shape, dtype=torch.int8, device=w.device)
+    if scales is None:
+        scales = torch.empty((cols,), dtype=torch.float32, device=w.device)
+    rc = load().sana_quantize_cols_i8(_dev(w, "w"), _dtype_code(w), _dev(out, "codes"),
+                                      _dev(scales, "scales"), K, cols, _stream(stream))
+    _check("sana_quantize_cols_i8", rc)
+    return out, scales
+
+
+def qkv_fused_w8a8(xq, sx, Wq, sw, gq, gk, H: int, eps: float, out=None, workspace=None,
+                   stream=None):
+    """The fused variant with a W8A8 prologue: int8 codes xq (B, N, C) with
+    per-token scales sx (B, N), int8 Wq (C, 3C) with per-channel scales sw (3C,);
+    returns O (B, N, C) bf16."""
+    torch = _torch()
+    B, N, C = xq.shape
+    if xq.dtype != torch.int8 or Wq.dtype != torch.int8:
+        raise TypeError("the W8A8 path takes int8 xq and Wq")
+    if tuple(Wq.shape) != (C, 3 * C) or tuple(sx.shape) != (B, N) or tuple(sw.shape) != (3 * C,):
+        raise ValueError("shapes: xq (B, N, C), sx (B, N), Wq (C, 3C), sw (3C,)")
+    if out is None:
+        out = torch.empty((B, N, C), dtype=torch.bfloat16, device=xq.device)
+    ws, wsb = _workspace(workspace_bytes(B, N, C, H, fused=True), xq.device, workspace)
+    rc = load().sana_linattn_qkv_fused_w8a8(_dev(xq, "xq"), _dev(sx, "sx"), _dev(Wq, "Wq"),
+                                            _dev(sw, "sw"), _gain(gq, "gq"), _gain(gk, "gk"),
+                                            _dev(out, "out"), B, N, C, H, float(eps),
+                                            None if ws is None else ws.data_ptr(), wsb,
+                                            _stream(stream))
+    _check("sana_linattn_qkv_fused_w8a8", rc)
+    return out
 
 
 def qkv_fused(x, W, gq, gk, H: int, eps: float, out=None, workspace=None, stream=None):

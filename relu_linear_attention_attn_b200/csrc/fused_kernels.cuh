@@ -20,6 +20,14 @@
 //                  Only the B-operand build reads the states F1 wrote, so under
 //                  programmatic dependent launch the Q projection overlaps F1's tail.
 //
+// W8A8 (template kI8): x and Wqkv arrive as int8 codes with one fp32 scale per
+// token of x and per output channel of Wqkv.  The projection runs as a kind::i8
+// UMMA (int32 accumulator in TMEM, exact), the epilogue dequantises
+// q = acc * sx[token] * sw[channel] in fp32, and everything after that (feature
+// map, state, apply: bf16 operands, fp32 accumulation) is the same as for bf16.
+// A stage then covers 128 k (128 bytes of an x row, as for bf16's 64 k), a UMMA
+// K = 32, and a W box is 128 k x 128 n.
+//
 // Operand layouts (all 128-byte swizzle, 1024-byte aligned):
 //   x tile        K-major: [128 tokens][64 k] per stage (TMA 3-D map over (C, N, B))
 //   W blocks      MN-major: [64 k][64 n] boxes (TMA 3-D map over (n, section, k)),
@@ -37,15 +45,25 @@ namespace sana {
 namespace fz {
 constexpr int kTileTok = 128;                      // UMMA M
 constexpr int kGroupHeads = 4;                     // heads per CTA
-constexpr int kKStep = 64;                         // k elements per pipeline stage
-constexpr int kXBytes = kTileTok * 128;            // x box: 128 tokens x 64 k = 16 KB
-constexpr int kWBox = kKStep * 128;                // W box: 64 k x 64 n = 8 KB
+constexpr int kXBytes = kTileTok * 128;            // x box: 128 tokens x 128 bytes of k = 16 KB
+constexpr int kSectionBytes = 16 * 1024;           // W rows of one stage for a group's 128 n
 constexpr int kBlock = kTileTok * 128;             // 128 tokens x 64 channels = 16 KB
+
+// Element-type dependent geometry (bf16 or int8 x and Wqkv).
+template <bool kI8>
+struct Geom {
+    static constexpr int kKStep = kI8 ? 128 : 64;      // k per stage: 128 bytes of an x row
+    static constexpr int kKSlice = kI8 ? 32 : 16;      // k per UMMA (32 bytes of a K-major row)
+    static constexpr int kWAtomN = kI8 ? 128 : 64;     // n in one 128-byte W row (MN-major atom)
+    static constexpr int kWBox = kKStep * 128;         // W box: kKStep k rows x 128 bytes
+    static constexpr int kWBoxes = 128 / kWAtomN;      // boxes per section of a group
+    static_assert(kWBoxes * kWBox == kSectionBytes, "section size");
+};
 }  // namespace fz
 
 // ============================================================================ F1
 namespace f1 {
-constexpr int kStageBytes = fz::kXBytes + 4 * fz::kWBox;   // x + K (2 boxes) + V (2 boxes)
+constexpr int kStageBytes = fz::kXBytes + 2 * fz::kSectionBytes;   // x + K section + V section
 constexpr int kStages = 3;
 constexpr int kOpBytes = 2 * fz::kBlock;                   // phi(K) or V: 128 tokens x 128 ch
 constexpr int kOnesBytes = 16 * 128;
@@ -54,10 +72,12 @@ constexpr int kKvCol = 256;                                // state accumulator 
 constexpr int kTmemCols = 512;
 constexpr int kEpiWarps = 8;                               // two per TMEM lane quadrant
 constexpr int kThreads = 32 * (2 + kEpiWarps);             // TMA, UMMA, epilogue
-constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 2 * kOpBytes + kOnesBytes + 2048;
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 2 * kOpBytes + kOnesBytes + 1024 + 2048;
 }  // namespace f1
 
 struct F1Args {
+    const float* sx;     // W8A8: per-token scales of x [B * N]
+    const float* sw;     // W8A8: per-channel scales of Wqkv [3C]
     const float* gk;     // [C] or nullptr (norm off)
     float* part;         // [B][H][S][D][D+1]
     float* kv;           // [B][H][D][D+1]
@@ -67,11 +87,13 @@ struct F1Args {
     int norm;
 };
 
+template <bool kI8>
 __global__ void __launch_bounds__(f1::kThreads, 1)
 fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
          const F1Args a)
 {
     using namespace f1;
+    using G = fz::Geom<kI8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_1024(smem_raw);
     uint8_t* stages = smem;
@@ -79,7 +101,8 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
     uint8_t* opv = opk + kOpBytes;                          // V: B operand
     uint8_t* ones = opv + kOpBytes;
     float* sg = (float*)(ones + kOnesBytes);                // 128 gains of the group
-    uint64_t* full = (uint64_t*)(sg + 128);
+    float* ssw = sg + 128;                                  // W8A8: 256 K, V channel scales
+    uint64_t* full = (uint64_t*)(ssw + 256);
     uint64_t* empty = full + kStages;
     uint64_t* accfull = empty + kStages;
     uint64_t* accempty = accfull + 1;
@@ -96,7 +119,7 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
     const int tiles = (a.N + fz::kTileTok - 1) / fz::kTileTok;
     const int t0 = s * a.tps;
     const int nt = min(a.tps, tiles - t0);
-    const int ksteps = (a.C + fz::kKStep - 1) / fz::kKStep;
+    const int ksteps = (a.C + G::kKStep - 1) / G::kKStep;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -119,6 +142,11 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
     for (int i = threadIdx.x; i < 128; i += blockDim.x) {
         const int h = g * fz::kGroupHeads + i / kD;
         sg[i] = (a.norm && h < a.H) ? a.gk[(size_t)h * kD + (i % kD)] : 1.f;
+        if (kI8) {
+            const bool live = h < a.H;
+            ssw[i] = live ? a.sw[a.C + g * 128 + i] : 0.f;             // K section
+            ssw[128 + i] = live ? a.sw[2 * a.C + g * 128 + i] : 0.f;   // V section
+        }
     }
     __syncthreads();
     if (threadIdx.x < 16)
@@ -147,15 +175,15 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
                     if (!ok) break;
                     uint8_t* sb = stages + st * kStageBytes;
                     mbar_arrive_expect_tx(&full[st], kStageBytes);
-                    tma_load_3d(sb, &tmap_x, &full[st], kk * fz::kKStep, y, b);
+                    tma_load_3d(sb, &tmap_x, &full[st], kk * G::kKStep, y, b);
                     const int n0 = g * 128;
-                    tma_load_3d(sb + fz::kXBytes, &tmap_w, &full[st], n0, 1, kk * fz::kKStep);
-                    tma_load_3d(sb + fz::kXBytes + fz::kWBox, &tmap_w, &full[st], n0 + 64, 1,
-                                kk * fz::kKStep);
-                    tma_load_3d(sb + fz::kXBytes + 2 * fz::kWBox, &tmap_w, &full[st], n0, 2,
-                                kk * fz::kKStep);
-                    tma_load_3d(sb + fz::kXBytes + 3 * fz::kWBox, &tmap_w, &full[st], n0 + 64, 2,
-                                kk * fz::kKStep);
+#pragma unroll
+                    for (int sec = 1; sec <= 2; ++sec)          // K, then V columns of the group
+#pragma unroll
+                        for (int j = 0; j < G::kWBoxes; ++j)
+                            tma_load_3d(sb + fz::kXBytes + (sec - 1) * fz::kSectionBytes + j * G::kWBox,
+                                        &tmap_w, &full[st], n0 + j * G::kWAtomN, sec,
+                                        kk * G::kKStep);
                     last = step;
                 }
             }
@@ -170,7 +198,8 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
     } else if (warp == 1) {
         // ------------------------------------------------ UMMA issuer
         if (lane == 0 && ok) {
-            const uint32_t idesc_g = make_idesc_bf16(128, 256, false, true);   // x K-major, W MN-major
+            const uint32_t idesc_g = kI8 ? make_idesc_s8(128, 256, false, true)       // x K-major,
+                                         : make_idesc_bf16(128, 256, false, true);  // W MN-major
             const uint32_t idesc_v = make_idesc_bf16(128, 128, true, true);    // phi(K), V MN-major
             const uint32_t idesc_1 = make_idesc_bf16(128, 64, true, true);
             const uint64_t ones_desc = make_smem_desc(smem_u32(ones), fz::kBlock, 1024, kSwizzle128B);
@@ -187,10 +216,12 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
                     const uint32_t xb = smem_u32(stages + st * kStageBytes);
                     const uint32_t wb = xb + fz::kXBytes;
 #pragma unroll
-                    for (int k4 = 0; k4 < fz::kKStep / 16; ++k4) {
+                    for (int k4 = 0; k4 < G::kKStep / G::kKSlice; ++k4) {
                         const uint64_t ad = make_smem_desc(xb + k4 * 32, 16, 1024, kSwizzle128B);
-                        const uint64_t bd = make_smem_desc(wb + k4 * 2048, fz::kWBox, 1024, kSwizzle128B);
-                        umma_bf16(tmem, ad, bd, idesc_g, kk > 0 || k4 > 0);
+                        const uint64_t bd = make_smem_desc(wb + k4 * G::kKSlice * 128, G::kWBox, 1024,
+                                                           kSwizzle128B);
+                        if (kI8) umma_s8(tmem, ad, bd, idesc_g, kk > 0 || k4 > 0);
+                        else umma_bf16(tmem, ad, bd, idesc_g, kk > 0 || k4 > 0);
                     }
                     umma_commit(&empty[st]);
                 }
@@ -229,6 +260,8 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             if (!ok) break;
             tc_fence_after_sync();
             const bool row_live = (t0 + ti) * fz::kTileTok + row < a.N;
+            const float sxr = (kI8 && row_live)
+                ? a.sx[(int64_t)b * a.N + (t0 + ti) * fz::kTileTok + row] : 0.f;
 #pragma unroll 1
             for (int j = 2 * half; j < 2 * half + 2; ++j) {
                 float kx[32], vx[32];
@@ -237,6 +270,13 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
                 tmem_ld16(lane_base + 128 + 32 * j, vx);
                 tmem_ld16(lane_base + 128 + 32 * j + 16, vx + 16);
                 tmem_wait_ld();
+                if (kI8) {                    // int32 accumulators -> dequantised fp32
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        kx[i] = __int2float_rn(__float_as_int(kx[i])) * sxr * ssw[j * kD + i];
+                        vx[i] = __int2float_rn(__float_as_int(vx[i])) * sxr * ssw[128 + j * kD + i];
+                    }
+                }
                 const bool live = row_live && (g * fz::kGroupHeads + j < a.H);
                 if (a.norm) {
                     float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
@@ -332,7 +372,7 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
 
 // ============================================================================ F2
 namespace f2 {
-constexpr int kStageBytes = fz::kXBytes + 2 * fz::kWBox;   // x + Q (2 boxes)
+constexpr int kStageBytes = fz::kXBytes + fz::kSectionBytes;   // x + Q section
 constexpr int kStages = 5;
 constexpr int kN = 48;                                     // 32 value columns, normaliser, padding
 constexpr int kBopBytes = kN * 128;                        // per head
@@ -344,11 +384,13 @@ constexpr int kTmemCols = 512;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kSmemBytes = 1024 + kStages * kStageBytes + fz::kGroupHeads * kBopBytes +
-                           kQoBytes + 2048;
+                           kQoBytes + 512 + 2048;
 static_assert(kStateBytes <= kQoBytes, "states must fit the staging buffer");
 }  // namespace f2
 
 struct F2Args {
+    const float* sx;     // W8A8: per-token scales of x [B * N]
+    const float* sw;     // W8A8: per-channel scales of Wqkv [3C]
     const float* kv;     // states [B][H][D][D+1] (F1's output)
     const float* gq;     // [C] or nullptr
     int N, H, C, tps;
@@ -356,11 +398,13 @@ struct F2Args {
     int norm;
 };
 
+template <bool kI8>
 __global__ void __launch_bounds__(f2::kThreads, 1)
 fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
          const __grid_constant__ CUtensorMap tmap_o, const F2Args a)
 {
     using namespace f2;
+    using G = fz::Geom<kI8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_1024(smem_raw);
     uint8_t* stages = smem;
@@ -368,7 +412,8 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
     uint8_t* qo = bop + fz::kGroupHeads * kBopBytes;
     float* sstate = (float*)qo;                             // states before the first tile
     float* sg = (float*)(qo + kQoBytes);                    // 128 gains
-    uint64_t* full = (uint64_t*)(sg + 128);
+    float* ssw = sg + 128;                                  // W8A8: 128 Q channel scales
+    uint64_t* full = (uint64_t*)(ssw + 128);
     uint64_t* empty = full + kStages;
     uint64_t* accfull = empty + kStages;                    // [2]
     uint64_t* accempty = accfull + 2;                       // [2]
@@ -384,7 +429,7 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
     const int tiles = (a.N + fz::kTileTok - 1) / fz::kTileTok;
     const int t0 = s * a.tps;
     const int nt = min(a.tps, tiles - t0);
-    const int ksteps = (a.C + fz::kKStep - 1) / fz::kKStep;
+    const int ksteps = (a.C + G::kKStep - 1) / G::kKStep;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -410,6 +455,7 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
     for (int i = threadIdx.x; i < 128; i += blockDim.x) {
         const int h = g * fz::kGroupHeads + i / kD;
         sg[i] = (a.norm && h < a.H) ? a.gq[(size_t)h * kD + (i % kD)] : 1.f;
+        if (kI8) ssw[i] = h < a.H ? a.sw[g * 128 + i] : 0.f;       // Q section
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -434,10 +480,11 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
                     if (!ok) break;
                     uint8_t* sb = stages + st * kStageBytes;
                     mbar_arrive_expect_tx(&full[st], kStageBytes);
-                    tma_load_3d(sb, &tmap_x, &full[st], kk * fz::kKStep, y, b);
-                    tma_load_3d(sb + fz::kXBytes, &tmap_w, &full[st], g * 128, 0, kk * fz::kKStep);
-                    tma_load_3d(sb + fz::kXBytes + fz::kWBox, &tmap_w, &full[st], g * 128 + 64, 0,
-                                kk * fz::kKStep);
+                    tma_load_3d(sb, &tmap_x, &full[st], kk * G::kKStep, y, b);
+#pragma unroll
+                    for (int j = 0; j < G::kWBoxes; ++j)        // Q columns of the group
+                        tma_load_3d(sb + fz::kXBytes + j * G::kWBox, &tmap_w, &full[st],
+                                    g * 128 + j * G::kWAtomN, 0, kk * G::kKStep);
                     last = step;
                 }
             }
@@ -455,7 +502,8 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
         // tile is issued after the next tile's projection, so the tensor pipe keeps
         // busy while the epilogue turns the tile's Q into the A' operand.
         if (lane == 0 && ok) {
-            const uint32_t idesc_g = make_idesc_bf16(128, 128, false, true);
+            const uint32_t idesc_g = kI8 ? make_idesc_s8(128, 128, false, true)
+                                         : make_idesc_bf16(128, 128, false, true);
             const uint32_t idesc_a = make_idesc_bf16(128, kN, false, false);
             int64_t step = 0;
             auto gemm = [&](int ti) -> bool {
@@ -470,10 +518,12 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
                     const uint32_t xb = smem_u32(stages + st * kStageBytes);
                     const uint32_t wb = xb + fz::kXBytes;
 #pragma unroll
-                    for (int k4 = 0; k4 < fz::kKStep / 16; ++k4) {
+                    for (int k4 = 0; k4 < G::kKStep / G::kKSlice; ++k4) {
                         const uint64_t ad = make_smem_desc(xb + k4 * 32, 16, 1024, kSwizzle128B);
-                        const uint64_t bd = make_smem_desc(wb + k4 * 2048, fz::kWBox, 1024, kSwizzle128B);
-                        umma_bf16(tmem + ab * kAccCols, ad, bd, idesc_g, kk > 0 || k4 > 0);
+                        const uint64_t bd = make_smem_desc(wb + k4 * G::kKSlice * 128, G::kWBox, 1024,
+                                                           kSwizzle128B);
+                        if (kI8) umma_s8(tmem + ab * kAccCols, ad, bd, idesc_g, kk > 0 || k4 > 0);
+                        else umma_bf16(tmem + ab * kAccCols, ad, bd, idesc_g, kk > 0 || k4 > 0);
                     }
                     umma_commit(&empty[st]);
                 }
@@ -558,6 +608,8 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             if (et == 0) bulk_wait_group_read<0>();
             named_barrier_sync(1, 32 * kEpiWarps);
             const bool row_live = (t0 + ti) * fz::kTileTok + row < a.N;
+            const float sxr = (kI8 && row_live)
+                ? a.sx[(int64_t)b * a.N + (t0 + ti) * fz::kTileTok + row] : 0.f;
             float rq[2];
 #pragma unroll 1
             for (int j = 2 * half; j < 2 * half + 2; ++j) {
@@ -565,6 +617,11 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
                 tmem_ld16(lane_base + ab * kAccCols + 32 * j, x);
                 tmem_ld16(lane_base + ab * kAccCols + 32 * j + 16, x + 16);
                 tmem_wait_ld();
+                if (kI8) {                    // int32 accumulators -> dequantised fp32
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        x[i] = __int2float_rn(__float_as_int(x[i])) * sxr * ssw[j * kD + i];
+                }
                 const bool live = row_live && (g * fz::kGroupHeads + j < a.H);
                 float r = 1.f;
                 if (a.norm) {

@@ -23,6 +23,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&p);
 }
 
+__device__ __forceinline__ float to_float(bf16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float to_float(float v) { return v; }
+
 // Load / store 8 consecutive elements (16-byte aligned for bf16, 32 for fp32).
 __device__ __forceinline__ void load8(const bf16* p, float* x) {
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));

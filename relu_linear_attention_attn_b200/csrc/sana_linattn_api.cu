@@ -12,6 +12,7 @@
 #include "sm100_primitives.cuh"
 #include "tc_kernels.cuh"
 #include "fused_kernels.cuh"
+#include "quant_kernels.cuh"
 
 namespace sana {
 namespace {
@@ -204,36 +205,42 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// A (B, N, C) bf16 tensor seen by TMA as 3-D (C, N, B), boxes of 64 channels x
-// `rows` tokens x 1 batch, 128-byte swizzle.  Rows past N read as zeros and are
-// not written by stores, so a tile never crosses into the next batch item.
-bool make_tmap_bnc(CUtensorMap* m, const void* base, int64_t B, int64_t N, int C, int rows) {
+// A (B, N, C) bf16 (or int8) tensor seen by TMA as 3-D (C, N, B), boxes of 128
+// bytes of channels (64 bf16 or 128 int8) x `rows` tokens x 1 batch, 128-byte
+// swizzle.  Rows past N read as zeros and are not written by stores, so a tile
+// never crosses into the next batch item.
+bool make_tmap_bnc(CUtensorMap* m, const void* base, int64_t B, int64_t N, int C, int rows,
+                   bool i8 = false) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
+    const cuuint64_t es = i8 ? 1 : 2;
     const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)N, (cuuint64_t)B};
-    const cuuint64_t strides[2] = {(cuuint64_t)C * 2, (cuuint64_t)N * C * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)N * C * es};
+    const cuuint32_t box[3] = {i8 ? 128u : 64u, (cuuint32_t)rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-           CUDA_SUCCESS;
+    return fn(m, i8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Wqkv (C, 3C) row-major seen by TMA as 3-D (n within a section, section, k) =
-// (C, 3, C): boxes of 64 n x 1 section x 64 k, 128-byte swizzle.  Columns past a
-// section's C read as zeros, so head groups past H never pick up the next section.
-bool make_tmap_w(CUtensorMap* m, const void* W, int C) {
+// (C, 3, C): boxes of 128 bytes of n (64 bf16 or 128 int8) x 1 section x as many
+// k, 128-byte swizzle.  Columns past a section's C read as zeros, so head groups
+// past H never pick up the next section.  (Bytes are moved as unsigned 8-bit; the
+// UMMA reads them as signed int8.)
+bool make_tmap_w(CUtensorMap* m, const void* W, int C, bool i8 = false) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
+    const cuuint64_t es = i8 ? 1 : 2;
     const cuuint64_t dims[3] = {(cuuint64_t)C, 3, (cuuint64_t)C};
-    const cuuint64_t strides[2] = {(cuuint64_t)C * 2, (cuuint64_t)C * 3 * 2};
-    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)C * 3 * es};
+    const cuuint32_t box[3] = {i8 ? 128u : 64u, 1, i8 ? 128u : 64u};
     const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(W), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-           CUDA_SUCCESS;
+    return fn(m, i8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+              const_cast<void*>(W), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // The tensor-core kernels keep the gains of every channel in shared memory, so they
@@ -255,9 +262,13 @@ int persistent_ctas() {
                              p1::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(apply_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              p2::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(fused_kv, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(fused_kv<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              f1::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(fused_qo, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(fused_qo<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             f2::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(fused_kv<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             f1::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(fused_qo<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              f2::kSmemBytes) != cudaSuccess)
         return 0;
     // each persistent kernel must fit one CTA on an SM (registers, threads, smem)
@@ -266,11 +277,17 @@ int persistent_ctas() {
                                                       p1::kSmemBytes) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n2, apply_persistent, p2::kThreads,
                                                       p2::kSmemBytes) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n3, fused_kv, f1::kThreads,
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n3, fused_kv<false>, f1::kThreads,
                                                       f1::kSmemBytes) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n4, fused_qo, f2::kThreads,
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n4, fused_qo<false>, f2::kThreads,
                                                       f2::kSmemBytes) != cudaSuccess ||
         n1 < 1 || n2 < 1 || n3 < 1 || n4 < 1)
+        return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n3, fused_kv<true>, f1::kThreads,
+                                                      f1::kSmemBytes) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n4, fused_qo<true>, f2::kThreads,
+                                                      f2::kSmemBytes) != cudaSuccess ||
+        n3 < 1 || n4 < 1)
         return 0;
     ctas[dev] = sms < kMaxPersistentCtas ? sms : kMaxPersistentCtas;
     return ctas[dev];
@@ -350,25 +367,28 @@ int launch_apply_tc(const void* q, const float* gq, const float* kv, const float
 
 // The fused variant: F1 (K, V projection + state), then F2 (Q projection + apply)
 // as a programmatic dependent launch.
-int launch_fused(const void* x, const void* W, const float* gq, const float* gk, void* out,
-                 int* counters, float* part, float* kv, int64_t B, int64_t N, int C, int H,
-                 float eps, cudaStream_t st) {
+template <bool kI8>
+int launch_fused(const void* x, const void* W, const float* sx, const float* sw, const float* gq,
+                 const float* gk, void* out, int* counters, float* part, float* kv, int64_t B,
+                 int64_t N, int C, int H, float eps, cudaStream_t st) {
     const int P = persistent_ctas();
     if (P == 0) return SANA_ECUDA;
     CUtensorMap tx, tw, to;
-    if (!make_tmap_bnc(&tx, x, B, N, C, fz::kTileTok) || !make_tmap_w(&tw, W, C) ||
+    if (!make_tmap_bnc(&tx, x, B, N, C, fz::kTileTok, kI8) || !make_tmap_w(&tw, W, C, kI8) ||
         !make_tmap_bnc(&to, out, B, N, C, fz::kTileTok))
         return SANA_ECUDA;
     const FusedPlan pl = make_plan_fused(B, N, H, P);
     if (cudaMemsetAsync(counters, 0, (size_t)B * pl.G * sizeof(int), st) != cudaSuccess)
         return SANA_ECUDA;
     F1Args a1{};
+    a1.sx = sx; a1.sw = sw;
     a1.gk = gk; a1.part = part; a1.kv = kv; a1.counters = counters;
     a1.N = (int)N; a1.H = H; a1.C = C; a1.S = pl.S; a1.tps = pl.tps; a1.eps = eps;
     a1.norm = gk != nullptr;
     const dim3 grid(pl.S, pl.G, (unsigned)B);
-    fused_kv<<<grid, f1::kThreads, f1::kSmemBytes, st>>>(tx, tw, a1);
+    fused_kv<kI8><<<grid, f1::kThreads, f1::kSmemBytes, st>>>(tx, tw, a1);
     F2Args a2{};
+    a2.sx = sx; a2.sw = sw;
     a2.kv = kv; a2.gq = gq; a2.N = (int)N; a2.H = H; a2.C = C; a2.tps = pl.tps; a2.eps = eps;
     a2.norm = gq != nullptr;
     cudaLaunchConfig_t cfg = {};
@@ -381,7 +401,7 @@ int launch_fused(const void* x, const void* W, const float* gq, const float* gk,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, fused_qo, tx, tw, to, a2) != cudaSuccess) return SANA_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, fused_qo<kI8>, tx, tw, to, a2) != cudaSuccess) return SANA_ECUDA;
     return SANA_OK;
 }
 
@@ -589,9 +609,81 @@ int sana_linattn_qkv_fused(const void* x, const void* Wqkv, const float* gq, con
     float* part = (float*)((char*)workspace + L.part_off);
     float* kv = (float*)((char*)workspace + L.kv_off);
     int* counters = (int*)((char*)workspace + L.counters_off);
-    if ((rc = launch_fused(x, Wqkv, gq, gk, out, counters, part, kv, B, N, C, H, eps, stream)) !=
-        SANA_OK)
+    if ((rc = launch_fused<false>(x, Wqkv, nullptr, nullptr, gq, gk, out, counters, part, kv, B, N,
+                                  C, H, eps, stream)) != SANA_OK)
         return rc;
+    return launch_status();
+}
+
+int sana_linattn_qkv_fused_w8a8(const int8_t* xq, const float* sx, const int8_t* Wq,
+                                const float* sw, const float* gq, const float* gk, void* out,
+                                int64_t B, int64_t N, int C, int H, float eps, void* workspace,
+                                size_t ws_bytes, cudaStream_t stream) {
+    int rc;
+    if ((rc = check_dims(B, N, C, H)) != SANA_OK) return rc;
+    if ((rc = check_eps(eps)) != SANA_OK) return rc;
+    if ((rc = check_gains(gq, gk)) != SANA_OK) return rc;
+    if (B == 0 || N == 0) return SANA_OK;
+    if (!xq || !sx || !Wq || !sw || !out) return SANA_EINVAL;
+    if (!aligned(xq, 16) || !aligned(Wq, 16) || !aligned(out, 16) || !aligned(sx, 4) ||
+        !aligned(sw, 4))
+        return SANA_EALIGN;
+    const size_t xb = (size_t)B * N * C, wb = (size_t)C * 3 * C, ob = (size_t)B * N * C * 2;
+    if (overlaps(out, ob, xq, xb) || overlaps(out, ob, Wq, wb) ||
+        overlaps(out, ob, sx, (size_t)B * N * 4) || overlaps(out, ob, sw, (size_t)3 * C * 4))
+        return SANA_EINVAL;
+    const WsLayout L = ws_layout(B, N, C, H, true);
+    if ((rc = validate_ws(workspace, ws_bytes, L.total)) != SANA_OK) return rc;
+    if (overlaps(workspace, L.total, out, ob) || overlaps(workspace, L.total, xq, xb) ||
+        overlaps(workspace, L.total, Wq, wb))
+        return SANA_EINVAL;
+    if (B * (int64_t)((H + 3) / 4) > 65535 * 65535LL) return SANA_EUNSUPPORTED;
+    float* part = (float*)((char*)workspace + L.part_off);
+    float* kv = (float*)((char*)workspace + L.kv_off);
+    int* counters = (int*)((char*)workspace + L.counters_off);
+    if ((rc = launch_fused<true>(xq, Wq, sx, sw, gq, gk, out, counters, part, kv, B, N, C, H, eps,
+                                 stream)) != SANA_OK)
+        return rc;
+    return launch_status();
+}
+
+int sana_quantize_rows_i8(const void* x, sana_dtype dtype, int8_t* xq, float* scales,
+                          int64_t rows, int cols, cudaStream_t stream) {
+    if (rows < 0 || cols <= 0 || cols % 8 != 0) return SANA_EINVAL;
+    if (dtype != SANA_BF16 && dtype != SANA_F32) return SANA_EINVAL;
+    if (rows == 0) return SANA_OK;
+    if (!x || !xq || !scales) return SANA_EINVAL;
+    if (!aligned(x, dtype == SANA_BF16 ? 16 : 32) || !aligned(xq, 8) || !aligned(scales, 4))
+        return SANA_EALIGN;
+    const size_t in = (size_t)rows * cols * elem_size(dtype), qb = (size_t)rows * cols;
+    if (overlaps(xq, qb, x, in) || overlaps(scales, (size_t)rows * 4, x, in) ||
+        overlaps(scales, (size_t)rows * 4, xq, qb))
+        return SANA_EINVAL;
+    if ((rows + 7) / 8 > 0x7fffffffLL) return SANA_EUNSUPPORTED;
+    const dim3 grid((unsigned)((rows + 7) / 8));
+    if (dtype == SANA_BF16)
+        quantize_rows_i8<bf16><<<grid, 256, 0, stream>>>((const bf16*)x, xq, scales, rows, cols);
+    else
+        quantize_rows_i8<float><<<grid, 256, 0, stream>>>((const float*)x, xq, scales, rows, cols);
+    return launch_status();
+}
+
+int sana_quantize_cols_i8(const void* w, sana_dtype dtype, int8_t* wq, float* scales, int64_t K,
+                          int cols, cudaStream_t stream) {
+    if (K < 0 || cols <= 0) return SANA_EINVAL;
+    if (dtype != SANA_BF16 && dtype != SANA_F32) return SANA_EINVAL;
+    if (K == 0) return SANA_OK;
+    if (!w || !wq || !scales) return SANA_EINVAL;
+    if (!aligned(w, elem_size(dtype)) || !aligned(scales, 4)) return SANA_EALIGN;
+    const size_t in = (size_t)K * cols * elem_size(dtype), qb = (size_t)K * cols;
+    if (overlaps(wq, qb, w, in) || overlaps(scales, (size_t)cols * 4, w, in) ||
+        overlaps(scales, (size_t)cols * 4, wq, qb))
+        return SANA_EINVAL;
+    const dim3 grid((unsigned)((cols + 31) / 32)), block(32, 8);
+    if (dtype == SANA_BF16)
+        quantize_cols_i8<bf16><<<grid, block, 0, stream>>>((const bf16*)w, wq, scales, K, cols);
+    else
+        quantize_cols_i8<float><<<grid, block, 0, stream>>>((const float*)w, wq, scales, K, cols);
     return launch_status();
 }
 

@@ -60,8 +60,9 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The five workloads: a tiny Eq. (1) check, then SANA latents at 1024px, a
-# 2048px batch, a 4K overflow stress with the norm off, and the fused path.
+# The workloads: a tiny Eq. (1) check, then SANA latents at 1024px, a 2048px
+# batch, a 4K overflow stress with the norm off, the fused path, and the fused
+# path with a W8A8 prologue (same recipe; x and Wqkv are quantised by the op).
 CONFIGS = (
     Workload("tiny-512px-f32", B=1, N=256, C=64, H=2, dtype="f32", recipe="gaussian",
              gains="ones", eps=1e-6, seed=0),
@@ -73,6 +74,8 @@ CONFIGS = (
              recipe="overflow", gains="off", eps=1e-6, seed=3),
     Workload("fused-2048px-b4", B=4, N=4096, C=2240, H=70, dtype="bf16", recipe="fused",
              gains="random", eps=1e-6, seed=4),
+    Workload("w8a8-2048px-b4", B=4, N=4096, C=2240, H=70, dtype="bf16", recipe="fused",
+             gains="random", eps=1e-6, seed=5),
 )
 
 

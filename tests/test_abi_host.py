@@ -140,3 +140,38 @@ def test_other_entry_points_reject_bad_arguments(lib):
     a = list(args)
     a[2] = FAKE + (3 << 30)
     assert lib.sana_linattn_qkv_fused(*a) == EINVAL
+
+
+def test_w8a8_and_quantize_entry_points_reject_bad_arguments(lib):
+    # W8A8 fused: misaligned xq, one gain, too-small workspace, overlap of out and xq
+    args = [FAKE, FAKE + (1 << 30), FAKE + (2 << 30), FAKE + (3 << 30), None, None,
+            FAKE + (4 << 30), 4, 4096, 2240, 70, 1e-6, FAKE + (5 << 30), 1 << 34, None]
+    a = list(args)
+    a[0] += 8
+    assert lib.sana_linattn_qkv_fused_w8a8(*a) == EALIGN
+    a = list(args)
+    a[4] = FAKE + (6 << 30)
+    assert lib.sana_linattn_qkv_fused_w8a8(*a) == EINVAL
+    a = list(args)
+    a[13] = 4096
+    assert lib.sana_linattn_qkv_fused_w8a8(*a) == EWS
+    a = list(args)
+    a[6] = FAKE + 64
+    assert lib.sana_linattn_qkv_fused_w8a8(*a) == EINVAL
+    a = list(args)
+    a[10] = 35                                   # D = 64
+    assert lib.sana_linattn_qkv_fused_w8a8(*a) == EUNSUP
+    # quantisation: cols not a multiple of 8, bad dtype, misaligned, overlapping
+    assert lib.sana_quantize_rows_i8(FAKE, 0, FAKE + (1 << 30), FAKE + (2 << 30), 16, 12,
+                                     None) == EINVAL
+    assert lib.sana_quantize_rows_i8(FAKE, 5, FAKE + (1 << 30), FAKE + (2 << 30), 16, 16,
+                                     None) == EINVAL
+    assert lib.sana_quantize_rows_i8(FAKE + 2, 0, FAKE + (1 << 30), FAKE + (2 << 30), 16, 16,
+                                     None) == EALIGN
+    assert lib.sana_quantize_rows_i8(FAKE, 0, FAKE + 8, FAKE + (2 << 30), 16, 16, None) == EINVAL
+    assert lib.sana_quantize_rows_i8(FAKE, 0, FAKE + (1 << 30), FAKE + (2 << 30), 0, 16,
+                                     None) == OK
+    assert lib.sana_quantize_cols_i8(FAKE, 0, FAKE + 4, FAKE + (2 << 30), 64, 64, None) == EINVAL
+    assert lib.sana_quantize_cols_i8(FAKE, 0, FAKE + (1 << 30), FAKE + (2 << 30) + 2, 64, 64,
+                                     None) == EALIGN
+
