@@ -212,19 +212,36 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     from oracle import oracle as O
-    from relu_linear_attention_attn_b200.synthetic import make_inputs
-    wl = select(args.workload)
+    from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
+    fused = args.workload in ("fused", "w8a8")
+    wl = [CONFIGS[4] if args.workload == "fused" else CONFIGS[5]] if fused else \
+        select(args.workload)
     # each step: one whole batch item of every workload in the sweep, bounded so
     # the --steps/--warmup run stays within a few minutes
     data = []
     for w in wl:
         x = make_inputs(w)
-        data.append((w, x["q"][:1], x["k"][:1], x["v"][:1], x["gq"], x["gk"]))
-    per_step_tokens = sum(w.N for w, *_ in data)
+        if args.workload == "fused":
+            data.append((w, x["x"][:1], x["W"], x["gq"], x["gk"]))
+        elif args.workload == "w8a8":
+            Wq, sw = O.quantize_i8(x["W"].float().numpy(), axis=0)
+            data.append((w, x["x"][:1], (Wq, sw), x["gq"], x["gk"]))
+        else:
+            data.append((w, x["q"][:1], x["k"][:1], x["v"][:1], x["gq"], x["gk"]))
+    per_step_tokens = sum(d[0].N for d in data)
 
     def step():
-        for w, q, k, v, gq, gk in data:
-            O.forward(q, k, v, gq, gk, w.H, w.eps)
+        for d in data:
+            if args.workload == "fused":
+                w, xx, W, gq, gk = d
+                O.fused_forward(xx, W, gq, gk, w.H, w.eps)
+            elif args.workload == "w8a8":
+                w, xx, (Wq, sw), gq, gk = d
+                xq, sx = O.quantize_i8(xx.float().numpy())
+                O.w8a8_fused_forward(xq, sx, Wq, sw, gq, gk, w.H, w.eps)
+            else:
+                w, q, k, v, gq, gk = d
+                O.forward(q, k, v, gq, gk, w.H, w.eps)
     for _ in range(args.warmup):
         step()
     t0 = time.perf_counter()
@@ -233,7 +250,7 @@ def run_reference(args, rank, world):
     dt = time.perf_counter() - t0
     value = per_step_tokens * args.steps / dt / 1e6
     sample = (f"one batch item of each workload per step ({per_step_tokens} tokens): "
-              + ", ".join(f"{w.name} N={w.N}" for w, *_ in data))
+              + ", ".join(f"{d[0].name} N={d[0].N}" for d in data))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "Mtokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -269,7 +286,7 @@ def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = measured_peaks()
-    wl = select(args.workload) if args.workload != "fused" else []
+    wl = select(args.workload) if args.workload not in ("fused", "w8a8") else []
 
     # inputs resident in HBM; each rank works on its own batch (weak scaling)
     sets = []
@@ -421,6 +438,16 @@ def run_ours(args, rank, world, local):
         if not args.no_e2e:
             line["e2e"] = e2e_measure(args, sla, sets, stream, world)
 
+    if args.workload == "w8a8" or (args.workload == "sweep" and not args.no_fused):
+        line["w8a8"] = w8a8_measure(args, sla, CONFIGS[5], rank, dev, stream, world, bf16_tf,
+                                    peak_kind)
+        if args.workload == "w8a8":
+            f = line["w8a8"]
+            line.update({"value": f["value"], "ms_per_step": f["ms_per_step"],
+                         "roofline": f["roofline"], "gpu_launches": f["gpu_launches"],
+                         "clocks": f.get("clocks")})
+            line["config"] = {"workload": CONFIGS[5].name, "B": 4, "N": 4096, "C": 2240,
+                              "H": 70, "parallelism": f"dp{args.gpus}"}
     if args.workload == "fused" or (args.workload == "sweep" and not args.no_fused):
         line["fused"] = fused_measure(args, sla, CONFIGS[4], rank, dev, stream, world, bf16_tf,
                                       peak_kind)
@@ -557,6 +584,64 @@ def fused_measure(args, sla, w, rank, dev, stream, world, bf16_tf, peak_kind):
             "gpu_launches": steps * 2, "clocks": clk.summary()}
 
 
+def w8a8_measure(args, sla, w, rank, dev, stream, world, bf16_tf, peak_kind):
+    """The fused op with the W8A8 prologue: Wqkv is quantised once (untimed, as a
+    deployment would store it); each step quantises x per token and runs the W8A8
+    fused kernels.  The projection's roofline is the int8 tensor peak, taken as
+    the measured bf16 burst x 2 (the nominal dense int8 : bf16 ratio, 4.5 : 2.25
+    PFLOP/s)."""
+    import torch
+    from relu_linear_attention_attn_b200.synthetic import make_inputs
+    x = make_inputs(w.scaled(seed=w.seed + 1000 * rank) if rank else w)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    Wq, sw = sla.quantize_cols_i8(d["W"])
+    xq = torch.empty(d["x"].shape, dtype=torch.int8, device=dev)
+    sx = torch.empty(d["x"].shape[:-1], dtype=torch.float32, device=dev)
+    out = torch.empty_like(d["x"])
+    ws = torch.empty(sla.workspace_bytes(w.B, w.N, w.C, w.H, fused=True), dtype=torch.uint8,
+                     device=dev)
+    steps = max(3, min(args.steps, 20))
+
+    def fused():
+        sla.qkv_fused_w8a8(xq, sx, Wq, sw, d["gq"], d["gk"], w.H, w.eps, out=out, workspace=ws)
+
+    def step():
+        sla.quantize_rows_i8(d["x"], out=xq, scales=sx)
+        fused()
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    with ClockSampler(dev.index) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        for e in ev:
+            e[0].record(stream)
+            sla.quantize_rows_i8(d["x"], out=xq, scales=sx)
+            e[1].record(stream)
+            fused()
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    q_ms = max_over_ranks(statistics.fmean(e[0].elapsed_time(e[1]) for e in ev), world)
+    f_ms = max_over_ranks(statistics.fmean(e[1].elapsed_time(e[2]) for e in ev), world)
+    ops = 2.0 * w.tokens * w.C * 3 * w.C
+    i8_peak = 2.0 * bf16_tf
+    tops = ops / (f_ms * 1e-3) / 1e12
+    return {"workload": w.name, "value": w.tokens * world / ((q_ms + f_ms) * 1e-3) / 1e6,
+            "unit": "Mtokens/s", "ms_per_step": q_ms + f_ms, "quantize_x_ms": q_ms,
+            "fused_ms": f_ms, "steps": steps,
+            "granularity": "int8 symmetric, one scale per token of x and per output channel "
+                           "of Wqkv (Wqkv quantised once, untimed)",
+            "roofline": {"bound": "tensor", "achieved": tops, "peak": i8_peak, "unit": "TOPS",
+                         "frac": tops / i8_peak, "traffic": None,
+                         "kernel": "fused_kv<int8> + fused_qo<int8> (the projection is kind::i8)",
+                         "op_per_launch": ops,
+                         "peak_kind": f"int8 = 2 x {peak_kind} bf16 burst (bf16_tflops), the "
+                                      "nominal dense int8:bf16 ratio"},
+            "gpu_launches": steps * 3, "clocks": clk.summary()}
+
+
 def profile_case(args):
     """--warmup calls of sana_linattn_forward (two kernel launches each) on one
     workload, optionally with another batch size; prints a checksum."""
@@ -565,15 +650,21 @@ def profile_case(args):
     import relu_linear_attention_attn_b200 as sla
     from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
 
-    w = CONFIGS[4] if args.workload == "fused" else select(args.workload)[-1]
+    fused = args.workload in ("fused", "w8a8")
+    w = {"fused": CONFIGS[4], "w8a8": CONFIGS[5]}.get(args.workload) or select(args.workload)[-1]
     if args.batch:
         w = w.scaled(B=args.batch)
     x = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in make_inputs(w).items()}
-    ws = torch.empty(sla.workspace_bytes(w.B, w.N, w.C, w.H, fused=args.workload == "fused"),
+    ws = torch.empty(sla.workspace_bytes(w.B, w.N, w.C, w.H, fused=fused),
                      dtype=torch.uint8, device="cuda")
+    if args.workload == "w8a8":
+        Wq, sw = sla.quantize_cols_i8(x["W"])
     for _ in range(args.warmup):
         if args.workload == "fused":
             out = sla.qkv_fused(x["x"], x["W"], x["gq"], x["gk"], w.H, w.eps, workspace=ws)
+        elif args.workload == "w8a8":
+            xq, sx = sla.quantize_rows_i8(x["x"])
+            out = sla.qkv_fused_w8a8(xq, sx, Wq, sw, x["gq"], x["gk"], w.H, w.eps, workspace=ws)
         else:
             out = sla.forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps, workspace=ws)
     torch.cuda.synchronize()
@@ -588,7 +679,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="sweep",
-                    choices=["sweep", "fused", "1024px", "2048px", "4096px"])
+                    choices=["sweep", "fused", "w8a8", "1024px", "2048px", "4096px"])
     ap.add_argument("--no-fused", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
