@@ -26,6 +26,11 @@ is pinned by ``tests/test_oracle_w8a8.py``: hand-derived codes and a
 hand-derived projection (``tests/golden/w8a8_quantize.json``), a pure-Python
 integer brute force, the half-step rounding bound, and equality with the fused
 forward on the dequantised tensors.
+
+The prefix (causal) form ``causal_forward`` (C: ``oracle_causal_forward_f64``,
+the running state over tokens) is pinned by ``tests/test_oracle_causal.py``:
+hand-derived examples, a masked quadratic form with a textbook RMSNorm, the last
+token against the non-causal forward, the first token's closed form, causality.
 """
 from __future__ import annotations
 
@@ -71,8 +76,10 @@ def _bind(lib):
     lib.oracle_kv_state_f64.argtypes = [dp, dp, dp, dp, i64, i64, ci, ci, cd, ci, ci]
     lib.oracle_apply_f64.argtypes = [dp, dp, dp, dp, i64p, i64, i64, i64, ci, ci, cd, ci, ci]
     lib.oracle_forward_f64.argtypes = [dp, dp, dp, dp, dp, dp, i64, i64, ci, ci, cd, ci, ci]
+    lib.oracle_causal_forward_f64.argtypes = [dp, dp, dp, dp, dp, dp, i64, i64, ci, ci, cd, ci,
+                                              ci]
     for f in (lib.oracle_phi_f64, lib.oracle_kv_state_f64, lib.oracle_apply_f64,
-              lib.oracle_forward_f64):
+              lib.oracle_forward_f64, lib.oracle_causal_forward_f64):
         f.restype = ctypes.c_int
     return lib
 
@@ -198,6 +205,23 @@ def forward(q, k, v, gq, gk, H: int, eps: float, scope: str = "head",
                                     B, N, C, H, float(eps), mode, nthreads or host_threads())
     if rc != 0:
         raise ValueError("oracle_forward_f64 rejected its arguments")
+    return out
+
+
+def causal_forward(q, k, v, gq, gk, H: int, eps: float, nthreads: int = 0) -> np.ndarray:
+    """The prefix form: token n attends to keys j <= n only (the running sums
+    of the state), per-head QK-RMSNorm as in forward().  (B, N, C) fp64."""
+    mode = _norm_mode(gq, gk, "head")
+    q, k, v, gq, gk = (_f64(a) for a in (q, k, v, gq, gk))
+    B, N, C = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same (B, N, C) shape")
+    out = np.empty((B, N, C), dtype=np.float64)
+    rc = _load().oracle_causal_forward_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(gq), _ptr(gk),
+                                           _ptr(out), B, N, C, H, float(eps), mode,
+                                           nthreads or host_threads())
+    if rc != 0:
+        raise ValueError("oracle_causal_forward_f64 rejected its arguments")
     return out
 
 

@@ -272,3 +272,59 @@ int oracle_forward_f64(const double* q, const double* k, const double* v,
     free(S);
     return rc;
 }
+
+/* The prefix (causal) form: "Sana ..." notes describe linear attention as a
+ * cumulative prefix sum (the explainer page's O(N) prefix form).  Token n only
+ * sees keys j <= n:
+ *   S_n[d][e] = sum_{j <= n} phi(K_j)[d] V_j[e],  S_n[d][D] = sum_{j <= n} phi(K_j)[d],
+ *   O_n[e]    = (sum_d phi(Q_n)[d] S_n[d][e]) / (sum_d phi(Q_n)[d] S_n[d][D] + eps).
+ * Written as the running sum over tokens, one (b, h) at a time.  out: (B, N, C). */
+typedef struct {
+    const double* q; const double* k; const double* v;
+    const double* gq; const double* gk; double* out;
+    int64_t N; int C, H; double eps; int norm;
+} causal_ctx;
+
+static void causal_one(int64_t bh, void* vctx)
+{
+    causal_ctx* c = (causal_ctx*)vctx;
+    const int D = c->C / c->H;
+    const int64_t b = bh / c->H;
+    const int h = (int)(bh % c->H);
+    double* S = (double*)calloc((size_t)D * (D + 1), sizeof(double));
+    double* kk = (double*)malloc(sizeof(double) * (size_t)D);
+    double* qq = (double*)malloc(sizeof(double) * (size_t)D);
+    for (int64_t n = 0; n < c->N; ++n) {
+        const size_t row = ((size_t)b * c->N + n) * c->C;
+        phi_head(c->k + row, c->gk, kk, c->C, c->H, h, c->eps, c->norm);
+        const double* vv = c->v + row + (size_t)h * D;
+        for (int d = 0; d < D; ++d) {
+            for (int e = 0; e < D; ++e) S[d * (D + 1) + e] += kk[d] * vv[e];
+            S[d * (D + 1) + D] += kk[d];
+        }
+        phi_head(c->q + row, c->gq, qq, c->C, c->H, h, c->eps, c->norm);
+        double den = 0.0;
+        for (int d = 0; d < D; ++d) den += qq[d] * S[d * (D + 1) + D];
+        double* o = c->out + row + (size_t)h * D;
+        for (int e = 0; e < D; ++e) {
+            double num = 0.0;
+            for (int d = 0; d < D; ++d) num += qq[d] * S[d * (D + 1) + e];
+            o[e] = num / (den + c->eps);
+        }
+    }
+    free(S);
+    free(kk);
+    free(qq);
+}
+
+int oracle_causal_forward_f64(const double* q, const double* k, const double* v,
+                              const double* gq, const double* gk, double* out,
+                              int64_t B, int64_t N, int C, int H, double eps,
+                              int norm, int nthreads)
+{
+    if (B < 0 || N < 0 || C <= 0 || H <= 0 || C % H != 0) return -1;
+    if (norm != ORACLE_NORM_OFF && (gq == NULL || gk == NULL)) return -1;
+    causal_ctx c = { q, k, v, gq, gk, out, N, C, H, eps, norm };
+    parallel_for(B * H, nthreads, causal_one, &c);
+    return 0;
+}
