@@ -291,30 +291,32 @@ static void causal_one(int64_t bh, void* vctx)
     const int D = c->C / c->H;
     const int64_t b = bh / c->H;
     const int h = (int)(bh % c->H);
-    double* S = (double*)calloc((size_t)D * (D + 1), sizeof(double));
-    double* kk = (double*)malloc(sizeof(double) * (size_t)D);
-    double* qq = (double*)malloc(sizeof(double) * (size_t)D);
-    for (int64_t n = 0; n < c->N; ++n) {
-        const size_t row = ((size_t)b * c->N + n) * c->C;
-        phi_head(c->k + row, c->gk, kk, c->C, c->H, h, c->eps, c->norm);
-        const double* vv = c->v + row + (size_t)h * D;
-        for (int d = 0; d < D; ++d) {
-            for (int e = 0; e < D; ++e) S[d * (D + 1) + e] += kk[d] * vv[e];
-            S[d * (D + 1) + D] += kk[d];
+    double* run = (double*)calloc((size_t)D * (D + 1), sizeof(double));   /* S_n */
+    double* fk = (double*)malloc(sizeof(double) * (size_t)D);
+    double* fq = (double*)malloc(sizeof(double) * (size_t)D);
+    for (int64_t t = 0; t < c->N; ++t) {              /* tokens in order */
+        const size_t at = ((size_t)b * c->N + t) * c->C;
+        /* S_n = S_{n-1} + phi(K_n)^T [V_n | 1] */
+        phi_head(c->k + at, c->gk, fk, c->C, c->H, h, c->eps, c->norm);
+        const double* vn = c->v + at + (size_t)h * D;
+        for (int i = 0; i < D; ++i) {
+            for (int j = 0; j < D; ++j) run[i * (D + 1) + j] += fk[i] * vn[j];
+            run[i * (D + 1) + D] += fk[i];
         }
-        phi_head(c->q + row, c->gq, qq, c->C, c->H, h, c->eps, c->norm);
-        double den = 0.0;
-        for (int d = 0; d < D; ++d) den += qq[d] * S[d * (D + 1) + D];
-        double* o = c->out + row + (size_t)h * D;
-        for (int e = 0; e < D; ++e) {
-            double num = 0.0;
-            for (int d = 0; d < D; ++d) num += qq[d] * S[d * (D + 1) + e];
-            o[e] = num / (den + c->eps);
+        /* O_n = phi(Q_n) S_n[:, :D] / (phi(Q_n) S_n[:, D] + eps) */
+        phi_head(c->q + at, c->gq, fq, c->C, c->H, h, c->eps, c->norm);
+        double dn = 0.0;
+        for (int i = 0; i < D; ++i) dn += fq[i] * run[i * (D + 1) + D];
+        double* on = c->out + at + (size_t)h * D;
+        for (int j = 0; j < D; ++j) {
+            double nm = 0.0;
+            for (int i = 0; i < D; ++i) nm += fq[i] * run[i * (D + 1) + j];
+            on[j] = nm / (dn + c->eps);
         }
     }
-    free(S);
-    free(kk);
-    free(qq);
+    free(run);
+    free(fk);
+    free(fq);
 }
 
 int oracle_causal_forward_f64(const double* q, const double* k, const double* v,

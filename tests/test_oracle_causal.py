@@ -86,17 +86,17 @@ def test_causal_pins_hold():
 
 SRC = os.path.join(os.path.dirname(O.__file__), "sana_oracle.c")
 MUTATIONS = {
-    "apply_before_accumulating": (
-        "        phi_head(c->q + row, c->gq, qq, c->C, c->H, h, c->eps, c->norm);\n        double den = 0.0;",
-        "        phi_head(c->q + row, c->gq, qq, c->C, c->H, h, c->eps, c->norm);\n"
-        "        for (int d = 0; d < D; ++d) { for (int e = 0; e < D; ++e) S[d * (D + 1) + e] -= kk[d] * vv[e];"
-        " S[d * (D + 1) + D] -= kk[d]; }\n        double den = 0.0;"),
-    "causal_normaliser_counts_tokens": ("            S[d * (D + 1) + D] += kk[d];\n        }\n        phi_head(c->q",
-                                        "            S[d * (D + 1) + D] += 1.0;\n        }\n        phi_head(c->q"),
-    "causal_eps_dropped": ("            o[e] = num / (den + c->eps);\n        }\n    }\n    free(S);",
-                           "            o[e] = num / den;\n        }\n    }\n    free(S);"),
-    "causal_value_head_offset_lost": ("        const double* vv = c->v + row + (size_t)h * D;\n        for (int d = 0; d < D; ++d) {\n            for (int e = 0; e < D; ++e) S[d * (D + 1) + e] += kk[d] * vv[e];\n            S[d * (D + 1) + D] += kk[d];\n        }\n        phi_head(c->q",
-                                      "        const double* vv = c->v + row;\n        for (int d = 0; d < D; ++d) {\n            for (int e = 0; e < D; ++e) S[d * (D + 1) + e] += kk[d] * vv[e];\n            S[d * (D + 1) + D] += kk[d];\n        }\n        phi_head(c->q"),
+    "state_updated_after_apply": (
+        "        /* O_n = phi(Q_n) S_n[:, :D] / (phi(Q_n) S_n[:, D] + eps) */",
+        "        for (int i = 0; i < D; ++i) { for (int j = 0; j < D; ++j) run[i * (D + 1) + j] -= fk[i] * vn[j];"
+        " run[i * (D + 1) + D] -= fk[i]; }"),
+    "causal_normaliser_counts_tokens": ("            run[i * (D + 1) + D] += fk[i];",
+                                        "            run[i * (D + 1) + D] += 1.0;"),
+    "causal_eps_dropped": ("            on[j] = nm / (dn + c->eps);", "            on[j] = nm / dn;"),
+    "causal_value_head_offset_lost": ("        const double* vn = c->v + at + (size_t)h * D;",
+                                      "        const double* vn = c->v + at;"),
+    "causal_state_transposed": ("            for (int j = 0; j < D; ++j) run[i * (D + 1) + j] += fk[i] * vn[j];",
+                                "            for (int j = 0; j < D; ++j) run[i * (D + 1) + j] += fk[j] * vn[i];"),
 }
 
 
