@@ -70,8 +70,9 @@ typedef enum {
 } sana_dtype;
 
 /* Bytes of device workspace that sana_linattn_forward (fused == 0),
- * sana_linattn_kv_state (fused == 0) or sana_linattn_qkv_fused (fused != 0)
- * needs for this shape.  Returns 0 for an invalid or empty shape. */
+ * sana_linattn_kv_state (fused == 0), sana_linattn_qkv_fused and
+ * sana_linattn_qkv_fused_w8a8 (fused == 1) or sana_linattn_forward_causal
+ * (fused == 2) needs for this shape.  Returns 0 for an invalid or empty shape. */
 SANA_API size_t sana_linattn_workspace_bytes(int64_t B, int64_t N, int C, int H, int fused);
 
 /* Eq. (1) end to end on projected q, k, v.
@@ -83,6 +84,21 @@ SANA_API int sana_linattn_forward(const void* q, const void* k, const void* v,
                          int64_t B, int64_t N, int C, int H, float eps,
                          sana_dtype dtype, void* workspace, size_t ws_bytes,
                          cudaStream_t stream);
+
+/* The prefix (causal) form of Eq. (1): the explainer page of the Sana notes
+ * describes linear attention as a cumulative prefix sum; here token n sees keys
+ * j <= n only:
+ *   O_n = phi(Q_n) S_n[:, :D] / (phi(Q_n) S_n[:, D] + eps),
+ *   S_n = sum_{j <= n} phi(K_j)^T [V_j | 1].
+ * Arguments, dtypes, layouts and errors as for sana_linattn_forward; workspace:
+ * at least sana_linattn_workspace_bytes(B, N, C, H, 2) bytes (one fp32 state per
+ * 128-token chunk of every (b, h)).  Chunk states are combined in chunk order, so
+ * results are reproducible. */
+SANA_API int sana_linattn_forward_causal(const void* q, const void* k, const void* v,
+                                         const float* gq, const float* gk, void* out,
+                                         int64_t B, int64_t N, int C, int H, float eps,
+                                         sana_dtype dtype, void* workspace, size_t ws_bytes,
+                                         cudaStream_t stream);
 
 /* The state half of Eq. (1) (the sums formed once and reused by every query,
  * section 2.1 of the Sana notes): kv (B, H, D, D+1) fp32 receives

@@ -16,7 +16,7 @@ import os
 import threading
 
 __all__ = ["load", "lib_path", "workspace_bytes", "forward", "forward_noalloc", "kv_state", "apply", "qkv_fused",
-           "qkv_fused_w8a8", "quantize_rows_i8", "quantize_cols_i8",
+           "qkv_fused_w8a8", "quantize_rows_i8", "quantize_cols_i8", "forward_causal",
            "device_error", "selftest_wait_timeout", "SanaError", "STATUS", "BF16", "F32"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -53,6 +53,9 @@ def _declare(lib):
     for f in (lib.sana_linattn_forward, lib.sana_linattn_kv_state, lib.sana_linattn_apply,
               lib.sana_linattn_qkv_fused):
         f.restype = ctypes.c_int
+    lib.sana_linattn_forward_causal.argtypes = [vp, vp, vp, fp, fp, vp, i64, i64, ci, ci, cf, ci,
+                                                vp, sz, vp]
+    lib.sana_linattn_forward_causal.restype = ctypes.c_int
     lib.sana_linattn_qkv_fused_w8a8.argtypes = [vp, fp, vp, fp, fp, fp, vp, i64, i64, ci, ci, cf,
                                                 vp, sz, vp]
     lib.sana_linattn_qkv_fused_w8a8.restype = ctypes.c_int
@@ -160,6 +163,26 @@ def forward(q, k, v, gq, gk, H: int, eps: float, out=None, workspace=None, strea
                                      _gain(gk, "gk"), _dev(out, "out"), B, N, C, H, float(eps), dt,
                                      None if ws is None else ws.data_ptr(), wsb, _stream(stream))
     _check("sana_linattn_forward", rc)
+    return out
+
+
+def forward_causal(q, k, v, gq, gk, H: int, eps: float, out=None, workspace=None, stream=None):
+    """The prefix (causal) form: token n attends to keys j <= n.  Same arguments as
+    forward()."""
+    B, N, C = q.shape
+    if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share shape and dtype")
+    dt = _dtype_code(q)
+    if out is None:
+        out = _torch().empty_like(q)
+    ws, wsb = _workspace(int(load().sana_linattn_workspace_bytes(B, N, C, H, 2)), q.device,
+                         workspace)
+    rc = load().sana_linattn_forward_causal(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
+                                            _gain(gq, "gq"), _gain(gk, "gk"), _dev(out, "out"),
+                                            B, N, C, H, float(eps), dt,
+                                            None if ws is None else ws.data_ptr(), wsb,
+                                            _stream(stream))
+    _check("sana_linattn_forward_causal", rc)
     return out
 
 

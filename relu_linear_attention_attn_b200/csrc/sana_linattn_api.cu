@@ -13,6 +13,7 @@
 #include "tc_kernels.cuh"
 #include "fused_kernels.cuh"
 #include "quant_kernels.cuh"
+#include "causal_kernels.cuh"
 
 namespace sana {
 namespace {
@@ -464,7 +465,52 @@ extern "C" {
 
 size_t sana_linattn_workspace_bytes(int64_t B, int64_t N, int C, int H, int fused) {
     if (check_dims(B, N, C, H) != SANA_OK || B == 0 || N == 0) return 0;
+    if (fused == 2) {        // the prefix form: one state per chunk of every (b, h)
+        const int64_t S = (N + kCausalChunk - 1) / kCausalChunk;
+        return align_up((size_t)B * H * S * kStateFloats * sizeof(float), 256);
+    }
     return ws_layout(B, N, C, H, fused != 0).total;
+}
+
+int sana_linattn_forward_causal(const void* q, const void* k, const void* v, const float* gq,
+                                const float* gk, void* out, int64_t B, int64_t N, int C, int H,
+                                float eps, sana_dtype dtype, void* workspace, size_t ws_bytes,
+                                cudaStream_t stream) {
+    int rc;
+    if ((rc = check_dims(B, N, C, H)) != SANA_OK) return rc;
+    if ((rc = check_eps(eps)) != SANA_OK) return rc;
+    if ((rc = check_gains(gq, gk)) != SANA_OK) return rc;
+    if (dtype != SANA_BF16 && dtype != SANA_F32) return SANA_EINVAL;
+    if (B == 0 || N == 0) return SANA_OK;
+    if ((rc = validate_qkv(q, k, v, out, B, N, C, dtype)) != SANA_OK) return rc;
+    const int64_t S = (N + kCausalChunk - 1) / kCausalChunk;
+    const size_t need = sana_linattn_workspace_bytes(B, N, C, H, 2);
+    if ((rc = validate_ws(workspace, ws_bytes, need)) != SANA_OK) return rc;
+    const size_t bytes = (size_t)B * N * C * elem_size(dtype);
+    if (overlaps(workspace, need, out, bytes) || overlaps(workspace, need, q, bytes) ||
+        overlaps(workspace, need, k, bytes) || overlaps(workspace, need, v, bytes))
+        return SANA_EINVAL;
+    if (S > 0x7fffffffLL) return SANA_EUNSUPPORTED;
+    float* part = (float*)workspace;
+    const dim3 g1((unsigned)S, H, (unsigned)B);
+    const int norm = gk != nullptr;
+    if (dtype == SANA_BF16) {
+        kv_partial_simt<bf16><<<g1, 128, 0, stream>>>((const bf16*)k, (const bf16*)v, gk, part, N,
+                                                      H, C, C, (int)S, kCausalChunk, eps, norm);
+        causal_scan<<<(unsigned)(B * H), 256, 0, stream>>>(part, (int)S);
+        causal_apply_simt<bf16><<<g1, kCausalChunk, 0, stream>>>(
+            (const bf16*)q, (const bf16*)k, (const bf16*)v, gq, gk, part, (bf16*)out, N, H,
+            (int)S, eps, norm);
+    } else {
+        kv_partial_simt<float><<<g1, 128, 0, stream>>>((const float*)k, (const float*)v, gk, part,
+                                                       N, H, C, C, (int)S, kCausalChunk, eps,
+                                                       norm);
+        causal_scan<<<(unsigned)(B * H), 256, 0, stream>>>(part, (int)S);
+        causal_apply_simt<float><<<g1, kCausalChunk, 0, stream>>>(
+            (const float*)q, (const float*)k, (const float*)v, gq, gk, part, (float*)out, N, H,
+            (int)S, eps, norm);
+    }
+    return launch_status();
 }
 
 const char* sana_linattn_strerror(int status) {

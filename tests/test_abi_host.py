@@ -175,3 +175,25 @@ def test_w8a8_and_quantize_entry_points_reject_bad_arguments(lib):
     assert lib.sana_quantize_cols_i8(FAKE, 0, FAKE + (1 << 30), FAKE + (2 << 30) + 2, 64, 64,
                                      None) == EALIGN
 
+
+def test_causal_entry_point_rejects_bad_arguments(lib):
+    ws_need = lib.sana_linattn_workspace_bytes(2, 1000, 2240, 70, 2)
+    assert ws_need == 2 * 70 * 8 * 1056 * 4                 # one state per 128-token chunk
+    args = [FAKE, FAKE + (1 << 30), FAKE + (2 << 30), None, None, FAKE + (4 << 30), 2, 1000,
+            2240, 70, 1e-6, 0, FAKE + (6 << 30), ws_need, None]
+    a = list(args)
+    a[0] += 2
+    assert lib.sana_linattn_forward_causal(*a) == EALIGN
+    a = list(args)
+    a[13] = ws_need - 4
+    assert lib.sana_linattn_forward_causal(*a) == EWS
+    a = list(args)
+    a[3] = FAKE + (3 << 30)
+    assert lib.sana_linattn_forward_causal(*a) == EINVAL
+    a = list(args)
+    a[9] = 35
+    assert lib.sana_linattn_forward_causal(*a) == EUNSUP
+    a = list(args)
+    a[5] = FAKE + 64
+    assert lib.sana_linattn_forward_causal(*a) == EINVAL
+
