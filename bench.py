@@ -434,6 +434,9 @@ def run_ours(args, rank, world, local):
                                         "state), CUDA events between the passes",
                      "clocks": clk.summary()})
 
+        if not args.no_fused:
+            line["causal"] = causal_measure(args, sla, sets, stream, world, hbm_gbs)
+
         # e2e: the public call with host buffers, copies inside the timed region
         if not args.no_e2e:
             line["e2e"] = e2e_measure(args, sla, sets, stream, world)
@@ -582,6 +585,51 @@ def fused_measure(args, sla, w, rank, dev, stream, world, bf16_tf, peak_kind):
                          "flop_per_launch": flops,
                          "peak_kind": f"{peak_kind} bf16 burst (bf16_tflops)"},
             "gpu_launches": steps * 2, "clocks": clk.summary()}
+
+
+def causal_measure(args, sla, sets, stream, world, hbm_gbs):
+    """The prefix (causal) form over the sweep's workloads (inputs resident, K steps
+    of sana_linattn_forward_causal per workload, CUDA events per call)."""
+    import torch
+    steps = max(3, min(args.steps, 10))
+    parts, tot_tok, tot_ms = [], 0, 0.0
+    for w, d, _ in sets:
+        ws = torch.empty(int(sla.load().sana_linattn_workspace_bytes(w.B, w.N, w.C, w.H, 2)),
+                         dtype=torch.uint8, device=d["q"].device)
+
+        def call():
+            sla.forward_causal(d["q"], d["k"], d["v"], d["gq"], d["gk"], w.H, w.eps,
+                               out=d["out"], workspace=ws)
+        for _ in range(max(args.warmup, 3)):
+            call()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for a, b in evs:
+            a.record(stream)
+            call()
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(statistics.fmean(a.elapsed_time(b) for a, b in evs), world)
+        by = w.tokens * 2 * PASS_BYTES_PER_TOKEN
+        parts.append({"workload": w.name, "ms": ms, "Mtokens_per_s": w.tokens / (ms * 1e-3) / 1e6,
+                      "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / hbm_gbs})
+        tot_tok += w.tokens
+        tot_ms += ms
+    big = max(range(len(sets)), key=lambda i: sets[i][0].tokens * 1e9 + sets[i][0].N)
+    wb = sets[big][0]
+    achieved = wb.tokens * 2 * PASS_BYTES_PER_TOKEN / (parts[big]["ms"] * 1e-3) / 1e9
+    return {"value": tot_tok * world / (tot_ms * 1e-3) / 1e6, "unit": "Mtokens/s",
+            "ms_per_step": tot_ms, "steps": steps, "parts": parts,
+            "chunk_tokens": 128,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": achieved / hbm_gbs, "traffic": None,
+                         "kernel": "kv_partial_simt + causal_scan + causal_apply_simt (CUDA cores)",
+                         "workload": wb.name,
+                         "algorithmic_bytes_per_launch": wb.tokens * 2 * PASS_BYTES_PER_TOKEN},
+            "gpu_launches": steps * len(sets) * 3}
 
 
 def w8a8_measure(args, sla, w, rank, dev, stream, world, bf16_tf, peak_kind):

@@ -17,6 +17,7 @@
 namespace sana {
 
 constexpr int kCausalChunk = 128;
+constexpr int kRowPad = 36;
 
 // Exclusive prefix over chunks: grid B * H, 256 threads; part[bh][c] becomes
 // sum_{c' < c} part[bh][c'] (the first chunk's becomes zero).
@@ -57,8 +58,9 @@ causal_apply_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __r
                   const float* __restrict__ pre, T* __restrict__ out, int64_t N, int H, int S,
                   float eps, int norm)
 {
-    __shared__ float sK[kCausalChunk][kDP];     // phi(K) of the chunk (padded rows)
-    __shared__ float sV[kCausalChunk][kDP];     // V of the chunk
+    // phi(K) and V of the chunk; rows padded to 36 floats so they read as float4
+    __shared__ __align__(16) float sK[kCausalChunk][kRowPad];
+    __shared__ __align__(16) float sV[kCausalChunk][kRowPad];
     __shared__ float sP[kStateFloats];          // prefix state of the chunk
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, t = threadIdx.x;
     const int64_t n = (int64_t)c * kCausalChunk + t;
@@ -102,15 +104,26 @@ causal_apply_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         for (int e = 0; e < kDP; ++e) num[e] = fmaf(a, sP[d * kDP + e], num[e]);
     }
     for (int j = 0; j <= t; ++j) {               // keys of this chunk up to the query
+        const float4* kr = reinterpret_cast<const float4*>(sK[j]);
+        const float4* vr = reinterpret_cast<const float4*>(sV[j]);
         float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-        for (int d = 0; d < kD; d += 2) {
-            a0 = fmaf(fq[d], sK[j][d], a0);
-            a1 = fmaf(fq[d + 1], sK[j][d + 1], a1);
+        for (int d4 = 0; d4 < kD / 4; ++d4) {
+            const float4 kk = kr[d4];
+            a0 = fmaf(fq[4 * d4 + 0], kk.x, a0);
+            a1 = fmaf(fq[4 * d4 + 1], kk.y, a1);
+            a0 = fmaf(fq[4 * d4 + 2], kk.z, a0);
+            a1 = fmaf(fq[4 * d4 + 3], kk.w, a1);
         }
         const float a = a0 + a1;
 #pragma unroll
-        for (int e = 0; e < kD; ++e) num[e] = fmaf(a, sV[j][e], num[e]);
+        for (int e4 = 0; e4 < kD / 4; ++e4) {
+            const float4 vv = vr[e4];
+            num[4 * e4 + 0] = fmaf(a, vv.x, num[4 * e4 + 0]);
+            num[4 * e4 + 1] = fmaf(a, vv.y, num[4 * e4 + 1]);
+            num[4 * e4 + 2] = fmaf(a, vv.z, num[4 * e4 + 2]);
+            num[4 * e4 + 3] = fmaf(a, vv.w, num[4 * e4 + 3]);
+        }
         num[kD] += a;
     }
     if (!live) return;
