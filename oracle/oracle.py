@@ -31,6 +31,11 @@ The prefix (causal) form ``causal_forward`` (C: ``oracle_causal_forward_f64``,
 the running state over tokens) is pinned by ``tests/test_oracle_causal.py``:
 hand-derived examples, a masked quadratic form with a textbook RMSNorm, the last
 token against the non-causal forward, the first token's closed form, causality.
+
+The backward (``backward``: hand-derived gradients of the forward with respect to
+q, k, v and the gains) is pinned by ``tests/test_oracle_backward.py``: automatic
+differentiation of an independently written fp64 torch forward, central
+finite differences of ``forward``, and the closed form of dV.
 """
 from __future__ import annotations
 
@@ -318,3 +323,72 @@ def w8a8_fused_forward(xq, sx, Wq, sw, gq, gk, H: int, eps: float, tokens=None,
     qfull = np.zeros((B * N, C), dtype=np.float64)
     qfull[tok] = q
     return apply(qfull.reshape(B, N, C), gq, S, H, eps, tokens=tok, nthreads=nthreads)
+
+
+# ----------------------------------------------------------------------------- backward
+# Gradients of Eq. (1) with the per-head QK-RMSNorm feature map, for training with
+# the op ("Sana ..." section 2.1 defines only the forward; the gradients below are
+# derived from it).  Per (b, h), with u = g * x * r, r = (mean_d x^2 + eps)^(-1/2),
+# phi = ReLU(u), S = sum_j phi(K_j)^T V_j, z = sum_j phi(K_j):
+#   num_i = phi(Q_i) S,  den_i = phi(Q_i) . z + eps,  O_i = num_i / den_i
+#   dnum_i = dO_i / den_i,               dden_i = -(dO_i . O_i) / den_i
+#   dphi(Q_i) = dnum_i S^T + dden_i z
+#   dS = sum_i phi(Q_i)^T dnum_i,        dz = sum_i phi(Q_i) dden_i
+#   dphi(K_j) = dS V_j + dz,             dV_j = phi(K_j) dS
+# and through the feature map (du = dphi where u > 0, else 0):
+#   dg[d] += du[d] x[d] r,   dx[c] = g[c] r du[c] - (r^3 x[c] / D) sum_d du[d] g[d] x[d]
+# (norm off: dx = dphi where x > 0).
+
+def _phi_fwd(x, g, H: int, eps: float):
+    """(phi, u, r) of x (B, N, C) per head; r has shape (B, N, H, 1)."""
+    B, N, C = x.shape
+    D = C // H
+    xh = x.reshape(B, N, H, D)
+    if g is None:
+        return np.maximum(xh, 0.0), xh, None
+    r = 1.0 / np.sqrt((xh * xh).mean(-1, keepdims=True) + eps)
+    u = g.reshape(1, 1, H, D) * xh * r
+    return np.maximum(u, 0.0), u, r
+
+
+def _phi_bwd(dphi, x, g, u, r, H: int):
+    """(dx (B, N, C), dg (C,) or None) through the feature map."""
+    B, N, C = x.shape
+    D = C // H
+    xh = x.reshape(B, N, H, D)
+    du = np.where(u > 0.0, dphi, 0.0)
+    if g is None:
+        return du.reshape(B, N, C), None
+    gh = g.reshape(1, 1, H, D)
+    dg = (du * xh * r).sum(axis=(0, 1)).reshape(C)
+    t = (du * gh * xh).sum(-1, keepdims=True)
+    dx = gh * r * du - (r ** 3) * xh * t / D
+    return dx.reshape(B, N, C), dg
+
+
+def backward(q, k, v, gq, gk, dout, H: int, eps: float):
+    """Gradients of the forward() output with respect to q, k, v and the gains:
+    returns (dq, dk, dv, dgq, dgk), fp64; dgq, dgk are None with the norm off."""
+    q, k, v, dout = (_f64(a) for a in (q, k, v, dout))
+    gq, gk = _f64(gq), _f64(gk)
+    B, N, C = q.shape
+    D = C // H
+    pq, uq, rq = _phi_fwd(q, gq, H, eps)
+    pk, uk, rk = _phi_fwd(k, gk, H, eps)
+    vh = v.reshape(B, N, H, D)
+    do = dout.reshape(B, N, H, D)
+    S = np.einsum("bnhd,bnhe->bhde", pk, vh)
+    z = pk.sum(axis=1)                                        # (B, H, D)
+    num = np.einsum("bnhd,bhde->bnhe", pq, S)
+    den = np.einsum("bnhd,bhd->bnh", pq, z)[..., None] + eps
+    o = num / den
+    dnum = do / den
+    dden = -(do * o).sum(-1, keepdims=True) / den
+    dpq = np.einsum("bnhe,bhde->bnhd", dnum, S) + dden * z[:, None]
+    dS = np.einsum("bnhd,bnhe->bhde", pq, dnum)
+    dz = np.einsum("bnhd,bnh->bhd", pq, dden[..., 0])
+    dpk = np.einsum("bhde,bnhe->bnhd", dS, vh) + dz[:, None]
+    dv = np.einsum("bnhd,bhde->bnhe", pk, dS)
+    dq, dgq = _phi_bwd(dpq, q, gq, uq, rq, H)
+    dk, dgk = _phi_bwd(dpk, k, gk, uk, rk, H)
+    return dq, dk, dv.reshape(B, N, C), dgq, dgk
