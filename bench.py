@@ -156,8 +156,10 @@ def max_over_ranks(x: float, world: int) -> float:
     return x if world == 1 else mor(x, device="cuda")
 
 
+# the sources the two pass kernels compile from: a recorded ncu traffic figure is
+# reported only while these hash to the value stored beside it
 KERNEL_SOURCES = ("relu_linear_attention_attn_b200/csrc/tc_kernels.cuh",
-                  "relu_linear_attention_attn_b200/csrc/fused_kernels.cuh",
+                  "relu_linear_attention_attn_b200/csrc/sana_common.cuh",
                   "relu_linear_attention_attn_b200/csrc/sm100_primitives.cuh")
 
 
@@ -436,6 +438,7 @@ def run_ours(args, rank, world, local):
 
         if not args.no_fused:
             line["causal"] = causal_measure(args, sla, sets, stream, world, hbm_gbs)
+            line["backward"] = backward_measure(args, sla, sets, stream, world, hbm_gbs)
 
         # e2e: the public call with host buffers, copies inside the timed region
         if not args.no_e2e:
@@ -630,6 +633,62 @@ def causal_measure(args, sla, sets, stream, world, hbm_gbs):
                          "workload": wb.name,
                          "algorithmic_bytes_per_launch": wb.tokens * 2 * PASS_BYTES_PER_TOKEN},
             "gpu_launches": steps * len(sets) * 3}
+
+
+def backward_measure(args, sla, sets, stream, world, hbm_gbs):
+    """The backward of the op (dq, dk, dv and the gain gradients from dO) over the
+    sweep's workloads: inputs and dO resident, K steps of sana_linattn_backward per
+    workload, CUDA events per call.  Algorithmic bytes: read q, k, v, dO and write
+    dq, dk, dv once each (7 x C x 2 B per token in bf16)."""
+    import torch
+    from relu_linear_attention_attn_b200.synthetic import make_output_grad
+    steps = max(3, min(args.steps, 10))
+    parts, tot_tok, tot_ms = [], 0, 0.0
+    launches = 0
+    for w, d, _ in sets:
+        dev = d["q"].device
+        do = make_output_grad(w).to(dev)
+        grads = (torch.empty_like(d["q"]), torch.empty_like(d["q"]), torch.empty_like(d["q"]),
+                 None if d["gq"] is None else torch.empty(w.C, dtype=torch.float32, device=dev),
+                 None if d["gk"] is None else torch.empty(w.C, dtype=torch.float32, device=dev))
+        ws = torch.empty(int(sla.load().sana_linattn_backward_workspace_bytes(w.B, w.N, w.C, w.H)),
+                         dtype=torch.uint8, device=dev)
+
+        def call():
+            sla.backward(d["q"], d["k"], d["v"], d["gq"], d["gk"], do, w.H, w.eps, grads=grads,
+                         workspace=ws)
+        for _ in range(max(args.warmup, 3)):
+            call()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for a, b in evs:
+            a.record(stream)
+            call()
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(statistics.fmean(a.elapsed_time(b) for a, b in evs), world)
+        by = w.tokens * 7 * PASS_BYTES_PER_TOKEN // 2
+        parts.append({"workload": w.name, "ms": ms, "Mtokens_per_s": w.tokens / (ms * 1e-3) / 1e6,
+                      "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / hbm_gbs})
+        tot_tok += w.tokens
+        tot_ms += ms
+        launches += steps * (8 if d["gq"] is not None else 6)
+        del do, grads, ws
+    big = max(range(len(sets)), key=lambda i: sets[i][0].tokens * 1e9 + sets[i][0].N)
+    wb = sets[big][0]
+    by_big = wb.tokens * 7 * PASS_BYTES_PER_TOKEN // 2
+    achieved = by_big / (parts[big]["ms"] * 1e-3) / 1e9
+    return {"value": tot_tok * world / (tot_ms * 1e-3) / 1e6, "unit": "Mtokens/s",
+            "ms_per_step": tot_ms, "steps": steps, "parts": parts,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": achieved / hbm_gbs, "traffic": None,
+                         "kernel": "kv state + bwd_query_simt + outer_partial_simt + "
+                                   "bwd_key_simt + gain_combine (CUDA cores)",
+                         "workload": wb.name, "algorithmic_bytes_per_launch": by_big},
+            "gpu_launches": launches}
 
 
 def w8a8_measure(args, sla, w, rank, dev, stream, world, bf16_tf, peak_kind):

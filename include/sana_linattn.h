@@ -100,6 +100,24 @@ SANA_API int sana_linattn_forward_causal(const void* q, const void* k, const voi
                                          sana_dtype dtype, void* workspace, size_t ws_bytes,
                                          cudaStream_t stream);
 
+/* Gradients of sana_linattn_forward's output for training (the pages define
+ * only the forward; the gradients follow from Eq. (1) and the feature map):
+ * given dout = dL/dO (B, N, C), writes dq, dk, dv (B, N, C) in `dtype` and, with
+ * the norm on, dgq, dgk = dL/dgq, dL/dgk (fp32 [C]; both NULL with the norm off,
+ * when gq = gk = NULL).  Recomputes the forward state itself.  All tensors
+ * 16-byte aligned (gains and their gradients 4-byte); outputs must not overlap
+ * inputs or each other.  workspace: at least
+ * sana_linattn_backward_workspace_bytes(B, N, C, H) bytes.  Sums are formed in a
+ * fixed order, so results are reproducible.  B == 0 or N == 0 zero-fills
+ * dgq, dgk. */
+SANA_API size_t sana_linattn_backward_workspace_bytes(int64_t B, int64_t N, int C, int H);
+SANA_API int sana_linattn_backward(const void* q, const void* k, const void* v,
+                                   const float* gq, const float* gk, const void* dout,
+                                   void* dq, void* dk, void* dv, float* dgq, float* dgk,
+                                   int64_t B, int64_t N, int C, int H, float eps,
+                                   sana_dtype dtype, void* workspace, size_t ws_bytes,
+                                   cudaStream_t stream);
+
 /* The state half of Eq. (1) (the sums formed once and reused by every query,
  * section 2.1 of the Sana notes): kv (B, H, D, D+1) fp32 receives
  * S_{b,h}[d][e] = sum_n phi(K)[d] V[e] for e < D and S_{b,h}[d][D] =

@@ -17,6 +17,7 @@ import threading
 
 __all__ = ["load", "lib_path", "workspace_bytes", "forward", "forward_noalloc", "kv_state", "apply", "qkv_fused",
            "qkv_fused_w8a8", "quantize_rows_i8", "quantize_cols_i8", "forward_causal",
+           "backward",
            "device_error", "selftest_wait_timeout", "SanaError", "STATUS", "BF16", "F32"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -53,6 +54,11 @@ def _declare(lib):
     for f in (lib.sana_linattn_forward, lib.sana_linattn_kv_state, lib.sana_linattn_apply,
               lib.sana_linattn_qkv_fused):
         f.restype = ctypes.c_int
+    lib.sana_linattn_backward_workspace_bytes.argtypes = [i64, i64, ci, ci]
+    lib.sana_linattn_backward_workspace_bytes.restype = sz
+    lib.sana_linattn_backward.argtypes = [vp, vp, vp, fp, fp, vp, vp, vp, vp, fp, fp, i64, i64,
+                                          ci, ci, cf, ci, vp, sz, vp]
+    lib.sana_linattn_backward.restype = ctypes.c_int
     lib.sana_linattn_forward_causal.argtypes = [vp, vp, vp, fp, fp, vp, i64, i64, ci, ci, cf, ci,
                                                 vp, sz, vp]
     lib.sana_linattn_forward_causal.restype = ctypes.c_int
@@ -164,6 +170,43 @@ def forward(q, k, v, gq, gk, H: int, eps: float, out=None, workspace=None, strea
                                      None if ws is None else ws.data_ptr(), wsb, _stream(stream))
     _check("sana_linattn_forward", rc)
     return out
+
+
+def backward(q, k, v, gq, gk, dout, H: int, eps: float, grads=None, workspace=None,
+             stream=None):
+    """Gradients of forward()'s output: returns (dq, dk, dv, dgq, dgk); dgq, dgk
+    (float32 [C]) are None with the norm off.  `grads`, when given, is that tuple
+    preallocated (the results are written into it)."""
+    torch = _torch()
+    B, N, C = q.shape
+    for t, n in ((k, "k"), (v, "v"), (dout, "dout")):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError(f"{n} must match q in shape and dtype")
+    dt = _dtype_code(q)
+    if grads is not None:
+        dq, dk, dv, dgq, dgk = grads
+        for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+            if t.shape != q.shape or t.dtype != q.dtype:
+                raise ValueError(f"{n} must match q in shape and dtype")
+        for t, n in ((dgq, "dgq"), (dgk, "dgk")):
+            if (t is None) != (gq is None) or (t is not None and (t.shape != (C,) or
+                                                                   t.dtype != torch.float32)):
+                raise ValueError(f"{n} must be float32 [C] exactly when the gains are given")
+    else:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        dgq = dgk = None
+        if gq is not None:
+            dgq = torch.empty(C, dtype=torch.float32, device=q.device)
+            dgk = torch.empty(C, dtype=torch.float32, device=q.device)
+    ws, wsb = _workspace(int(load().sana_linattn_backward_workspace_bytes(B, N, C, H)), q.device,
+                         workspace)
+    rc = load().sana_linattn_backward(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _gain(gq, "gq"),
+                                      _gain(gk, "gk"), _dev(dout, "dout"), _dev(dq, "dq"),
+                                      _dev(dk, "dk"), _dev(dv, "dv"), _dev(dgq, "dgq"),
+                                      _dev(dgk, "dgk"), B, N, C, H, float(eps), dt,
+                                      None if ws is None else ws.data_ptr(), wsb, _stream(stream))
+    _check("sana_linattn_backward", rc)
+    return dq, dk, dv, dgq, dgk
 
 
 def forward_causal(q, k, v, gq, gk, H: int, eps: float, out=None, workspace=None, stream=None):

@@ -14,6 +14,7 @@
 #include "fused_kernels.cuh"
 #include "quant_kernels.cuh"
 #include "causal_kernels.cuh"
+#include "backward_kernels.cuh"
 
 namespace sana {
 namespace {
@@ -470,6 +471,97 @@ size_t sana_linattn_workspace_bytes(int64_t B, int64_t N, int C, int H, int fuse
         return align_up((size_t)B * H * S * kStateFloats * sizeof(float), 256);
     }
     return ws_layout(B, N, C, H, fused != 0).total;
+}
+
+size_t sana_linattn_backward_workspace_bytes(int64_t B, int64_t N, int C, int H) {
+    if (check_dims(B, N, C, H) != SANA_OK || B == 0 || N == 0) return 0;
+    const Plan p = make_plan(B, N, H);
+    const int64_t tiles = (N + kBwdTile - 1) / kBwdTile;
+    size_t off = 0;
+    off = align_up(off + (size_t)B * H * p.S * kStateFloats * 4, 256);   // split partials
+    off = align_up(off + (size_t)B * H * kStateFloats * 4, 256);         // forward states
+    off = align_up(off + (size_t)B * H * kStateFloats * 4, 256);         // [dS | dz]
+    off = align_up(off + (size_t)B * N * H * kGrow * 4, 256);            // [dnum | dden] rows
+    off = align_up(off + (size_t)2 * B * tiles * C * 4, 256);            // gain partials
+    return off;
+}
+
+int sana_linattn_backward(const void* q, const void* k, const void* v, const float* gq,
+                          const float* gk, const void* dout, void* dq, void* dk, void* dv,
+                          float* dgq, float* dgk, int64_t B, int64_t N, int C, int H, float eps,
+                          sana_dtype dtype, void* workspace, size_t ws_bytes,
+                          cudaStream_t stream) {
+    int rc;
+    if ((rc = check_dims(B, N, C, H)) != SANA_OK) return rc;
+    if ((rc = check_eps(eps)) != SANA_OK) return rc;
+    if ((rc = check_gains(gq, gk)) != SANA_OK) return rc;
+    if (dtype != SANA_BF16 && dtype != SANA_F32) return SANA_EINVAL;
+    const bool norm = gq != nullptr;
+    if (norm != (dgq != nullptr) || norm != (dgk != nullptr)) return SANA_EINVAL;
+    if (norm && (!aligned(dgq, 4) || !aligned(dgk, 4))) return SANA_EALIGN;
+    if (B == 0 || N == 0) {
+        if (norm && (cudaMemsetAsync(dgq, 0, (size_t)C * 4, stream) != cudaSuccess ||
+                     cudaMemsetAsync(dgk, 0, (size_t)C * 4, stream) != cudaSuccess))
+            return SANA_ECUDA;
+        return SANA_OK;
+    }
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return SANA_EINVAL;
+    const void* ins[4] = {q, k, v, dout};
+    void* outs[3] = {dq, dk, dv};
+    for (const void* p : ins) if (!aligned(p, 16)) return SANA_EALIGN;
+    for (void* p : outs) if (!aligned(p, 16)) return SANA_EALIGN;
+    const size_t bytes = (size_t)B * N * C * elem_size(dtype);
+    for (void* o : outs) {
+        for (const void* i : ins) if (overlaps(o, bytes, i, bytes)) return SANA_EINVAL;
+        for (void* o2 : outs) if (o2 != o && overlaps(o, bytes, o2, bytes)) return SANA_EINVAL;
+    }
+    const size_t need = sana_linattn_backward_workspace_bytes(B, N, C, H);
+    if ((rc = validate_ws(workspace, ws_bytes, need)) != SANA_OK) return rc;
+    for (const void* i : ins) if (overlaps(workspace, need, i, bytes)) return SANA_EINVAL;
+    for (void* o : outs) if (overlaps(workspace, need, o, bytes)) return SANA_EINVAL;
+    const Plan p = make_plan(B, N, H);
+    const int64_t tiles = (N + kBwdTile - 1) / kBwdTile;
+    char* w = (char*)workspace;
+    size_t off = 0;
+    float* part = (float*)(w + off);
+    off = align_up(off + (size_t)B * H * p.S * kStateFloats * 4, 256);
+    float* Sz = (float*)(w + off);
+    off = align_up(off + (size_t)B * H * kStateFloats * 4, 256);
+    float* dSz = (float*)(w + off);
+    off = align_up(off + (size_t)B * H * kStateFloats * 4, 256);
+    float* G = (float*)(w + off);
+    off = align_up(off + (size_t)B * N * H * kGrow * 4, 256);
+    float* gpq = (float*)(w + off);
+    float* gpk = gpq + (size_t)B * tiles * C;
+    const dim3 gs(p.S, H, (unsigned)B), gt((unsigned)tiles, H, (unsigned)B);
+    const int nrm = norm ? 1 : 0;
+    if (dtype == SANA_BF16) {
+        launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, Sz, B, N, H, C, C, eps, p,
+                           stream);
+        bwd_query_simt<bf16><<<gt, kBwdTile, 0, stream>>>((const bf16*)q, (const bf16*)dout, gq, Sz,
+                                                          (bf16*)dq, G, gpq, N, H, eps, nrm);
+        outer_partial_simt<bf16><<<gs, 128, 0, stream>>>((const bf16*)q, gq, G, part, N, H, p.S,
+                                                         p.tps, eps, nrm);
+        kv_combine<<<(unsigned)(B * H), 256, 0, stream>>>(part, dSz, p.S);
+        bwd_key_simt<bf16><<<gt, kBwdTile, 0, stream>>>((const bf16*)k, (const bf16*)v, gk, dSz,
+                                                        (bf16*)dk, (bf16*)dv, gpk, N, H, eps, nrm);
+    } else {
+        launch_state<float>((const float*)k, (const float*)v, gk, part, Sz, B, N, H, C, C, eps, p,
+                            stream);
+        bwd_query_simt<float><<<gt, kBwdTile, 0, stream>>>((const float*)q, (const float*)dout, gq,
+                                                           Sz, (float*)dq, G, gpq, N, H, eps, nrm);
+        outer_partial_simt<float><<<gs, 128, 0, stream>>>((const float*)q, gq, G, part, N, H, p.S,
+                                                          p.tps, eps, nrm);
+        kv_combine<<<(unsigned)(B * H), 256, 0, stream>>>(part, dSz, p.S);
+        bwd_key_simt<float><<<gt, kBwdTile, 0, stream>>>((const float*)k, (const float*)v, gk, dSz,
+                                                         (float*)dk, (float*)dv, gpk, N, H, eps,
+                                                         nrm);
+    }
+    if (norm) {
+        gain_combine<<<(C + 255) / 256, 256, 0, stream>>>(gpq, dgq, B * tiles, C);
+        gain_combine<<<(C + 255) / 256, 256, 0, stream>>>(gpk, dgk, B * tiles, C);
+    }
+    return launch_status();
 }
 
 int sana_linattn_forward_causal(const void* q, const void* k, const void* v, const float* gq,

@@ -134,3 +134,11 @@ def make_inputs(w: Workload) -> dict:
     gq, gk = _gains(rng, w.C, w.gains)
     return dict(q=_store(q, w.dtype), k=_store(k, w.dtype), v=_store(v, w.dtype),
                 gq=gq, gk=gk, eps=w.eps)
+
+
+def make_output_grad(w: Workload, seed_offset: int = 100) -> torch.Tensor:
+    """dL/dO for backward tests and timing: N(0, 1) of shape (B, N, C) in the
+    workload's storage dtype, from default_rng(w.seed + seed_offset)."""
+    rng = np.random.default_rng(w.seed + seed_offset)
+    return _store(rng.standard_normal((w.B, w.N, w.C), dtype=np.float32), w.dtype)
+

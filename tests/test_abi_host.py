@@ -197,3 +197,27 @@ def test_causal_entry_point_rejects_bad_arguments(lib):
     a[5] = FAKE + 64
     assert lib.sana_linattn_forward_causal(*a) == EINVAL
 
+
+def test_backward_entry_point_rejects_bad_arguments(lib):
+    need = lib.sana_linattn_backward_workspace_bytes(1, 256, 2240, 70)
+    assert need > 1 * 256 * 70 * 33 * 4
+    base = [FAKE, FAKE + (1 << 30), FAKE + (2 << 30), FAKE + (3 << 30), FAKE + (3 << 30) + 65536,
+            FAKE + (4 << 30), FAKE + (5 << 30), FAKE + (6 << 30), FAKE + (7 << 30),
+            FAKE + (8 << 30), FAKE + (8 << 30) + 65536, 1, 256, 2240, 70, 1e-6, 0,
+            FAKE + (9 << 30), need, None]
+    a = list(base)
+    a[9] = None                                  # gains given, one gain gradient missing
+    assert lib.sana_linattn_backward(*a) == EINVAL
+    a = list(base)
+    a[6] += 2                                    # misaligned dq
+    assert lib.sana_linattn_backward(*a) == EALIGN
+    a = list(base)
+    a[7] = FAKE + 64                             # dk overlaps q
+    assert lib.sana_linattn_backward(*a) == EINVAL
+    a = list(base)
+    a[18] = need - 256
+    assert lib.sana_linattn_backward(*a) == EWS
+    a = list(base)
+    a[14] = 35
+    assert lib.sana_linattn_backward(*a) == EUNSUP
+

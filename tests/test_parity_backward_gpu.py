@@ -1,0 +1,74 @@
+"""Parity of the backward (through the C ABI) with the fp64 oracle's hand-derived
+gradients (themselves pinned against autograd and finite differences).
+
+Tolerances (gradients have no fixed scale, so they are normwise against a scale
+s = max(max|g_ref|, max|dV_ref|)): bf16 outputs max|g - g_ref| <= 2e-2 * s and
+||g - g_ref||_2 <= 2e-2 * max(||g_ref||_2, s * sqrt(size) * 1e-2); fp32 outputs
+max|g - g_ref| <= 1e-4 * s (the backward chains more roundings than the forward:
+the RMS term of the feature-map gradient cancels).  dV sets the floor of the
+scale because dQ, dK and the gain gradients vanish where the output barely
+depends on them (N = 1: O = V den / (den + eps)), and their relative error is then
+ill-posed; with the normalised features of unit RMS, one token's share of a gain
+gradient is of the order of its dQ, so the same floor serves the gains."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from parity import to_dev, to_np
+from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs, make_output_grad
+
+pytestmark = pytest.mark.gpu
+
+
+def _close(got, ref, dtype, what, scale):
+    g, r = to_np(got), to_np(ref)
+    assert np.isfinite(g).all(), f"{what}: non-finite"
+    s = max(float(np.abs(r).max()), scale)
+    err = float(np.abs(g - r).max())
+    if dtype == "f32":
+        assert err <= 1e-4 * s, f"{what}: max err {err:.3e}, scale {s:.3e}"
+    else:
+        l2 = float(np.linalg.norm(g - r))
+        ref_l2 = max(float(np.linalg.norm(r)), s * np.sqrt(r.size) * 1e-2)
+        assert err <= 2e-2 * s and l2 <= 2e-2 * ref_l2, \
+            f"{what}: max err {err:.3e} (scale {s:.3e}), l2 {l2:.3e} vs {ref_l2:.3e}"
+
+
+def _check(cuda_lib, w):
+    x = make_inputs(w)
+    do = make_output_grad(w)
+    d = to_dev(x)
+    got = cuda_lib.backward(d["q"], d["k"], d["v"], d["gq"], d["gk"], do.cuda(), w.H, w.eps)
+    torch.cuda.synchronize()
+    ref = O.backward(x["q"], x["k"], x["v"], x["gq"], x["gk"], do, w.H, w.eps)
+    dv_scale = float(np.abs(ref[2]).max())
+    for name, g, r in zip(("dq", "dk", "dv", "dgq", "dgk"), got, ref):
+        if r is None:
+            assert g is None
+            continue
+        # gain gradients are fp32 outputs whatever the dtype
+        _close(g, r, "f32" if name.startswith("dg") and w.dtype == "f32" else w.dtype,
+               f"{w.name} {name}", dv_scale)
+
+
+@pytest.mark.parametrize("w", [CONFIGS[0], CONFIGS[0].scaled(N=300, gains="random", seed=80),
+                               CONFIGS[1].scaled(N=1, seed=81),
+                               CONFIGS[1].scaled(N=333, seed=82),
+                               CONFIGS[1].scaled(B=2, N=129, gains="off", seed=83),
+                               CONFIGS[1],
+                               CONFIGS[2].scaled(B=2, seed=84)],
+                         ids=lambda w: f"{w.dtype}-B{w.B}-N{w.N}-{w.gains}")
+def test_backward_parity(cuda_lib, w):
+    _check(cuda_lib, w)
+
+
+def test_backward_is_deterministic(cuda_lib):
+    w = CONFIGS[1].scaled(B=2, N=1000, seed=85)
+    d = to_dev(make_inputs(w))
+    do = make_output_grad(w).cuda()
+    a = cuda_lib.backward(d["q"], d["k"], d["v"], d["gq"], d["gk"], do, w.H, w.eps)
+    b = cuda_lib.backward(d["q"], d["k"], d["v"], d["gq"], d["gk"], do, w.H, w.eps)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
