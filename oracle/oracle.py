@@ -32,6 +32,12 @@ the running state over tokens) is pinned by ``tests/test_oracle_causal.py``:
 hand-derived examples, a masked quadratic form with a textbook RMSNorm, the last
 token against the non-causal forward, the first token's closed form, causality.
 
+The Mix-FFN (``linear``, ``depthwise_conv3x3``, ``glu``, ``dwconv_glu``,
+``mixffn_forward``) is pinned by ``tests/test_oracle_mixffn.py``: a hand-derived
+3x3 worked example (cross-correlation orientation, zero padding, exact gate
+values), a pure-Python brute force, torch's grouped ``conv2d``, ``glu`` and
+``silu``, and closed forms of a constant input and of a centre-only kernel.
+
 The backward (``backward``: hand-derived gradients of the forward with respect to
 q, k, v and the gains) is pinned by ``tests/test_oracle_backward.py``: automatic
 differentiation of an independently written fp64 torch forward, central
@@ -392,3 +398,98 @@ def backward(q, k, v, gq, gk, dout, H: int, eps: float):
     dq, dgq = _phi_bwd(dpq, q, gq, uq, rq, H)
     dk, dgk = _phi_bwd(dpk, k, gk, uk, rk, H)
     return dq, dk, dv.reshape(B, N, C), dgq, dgk
+
+
+# ----------------------------------------------------------------------------- Mix-FFN
+# The Mix-FFN of the Linear DiT block ("Sana: Efficient High-Resolution Image
+# Synthesis with Linear Diffusion Transformers", section 2.2: an inverted residual
+# block, a 3x3 depthwise convolution and a GLU take the place of the MLP FFN;
+# section 2.3: the convolution's zero padding is what carries position; "SANA 1.5",
+# section "Model architecture": C = 2240, FFN width 5600).  The pages leave the
+# rest open; the reading here, with tokens n = y * Ws + x on an (Hs, Ws) grid:
+#   U  = X W1 + b1                                  1x1 expand, C -> 2F
+#   Cv[y, x, c] = bdw[c] + sum_{i, j in 0..2} wdw[c, i, j] U[y + i - 1, x + j - 1, c]
+#                                                   depthwise 3x3 cross-correlation,
+#                                                   zero outside the grid
+#   Hg = Cv[..., :F] * gate(Cv[..., F:])            GLU: the first half gated by the
+#                                                   second; gate = sigmoid (the GLU's
+#                                                   definition) or SiLU
+#   Y  = Hg W2 + b2                                 1x1 project, F -> C
+# Biases are optional (None: no bias).
+
+def linear(x, W, b=None) -> np.ndarray:
+    """x @ W (+ b) in fp64: x (..., K), W (K, Nc) row-major, b (Nc,) or None."""
+    y = np.matmul(_f64(x), _f64(W))
+    if b is not None:
+        y = y + _f64(b)
+    return y
+
+
+def depthwise_conv3x3(u, wdw, bdw, Hs: int, Ws: int) -> np.ndarray:
+    """Depthwise 3x3 cross-correlation with zero padding of u (B, Hs*Ws, Cc) on the
+    row-major (Hs, Ws) token grid; wdw (Cc, 3, 3), tap (i, j) reads the token at
+    (y + i - 1, x + j - 1); bdw (Cc,) or None."""
+    u = _f64(u)
+    B, N, Cc = u.shape
+    if N != Hs * Ws:
+        raise ValueError("N must equal Hs * Ws")
+    w = _f64(wdw).reshape(Cc, 3, 3)
+    padded = np.zeros((B, Hs + 2, Ws + 2, Cc))
+    padded[:, 1:Hs + 1, 1:Ws + 1, :] = u.reshape(B, Hs, Ws, Cc)
+    out = np.zeros((B, Hs, Ws, Cc))
+    for i in range(3):
+        for j in range(3):
+            out += w[:, i, j] * padded[:, i:i + Hs, j:j + Ws, :]
+    if bdw is not None:
+        out += _f64(bdw)
+    return out.reshape(B, N, Cc)
+
+
+def glu(c, gate: str = "sigmoid") -> np.ndarray:
+    """GLU over the last axis (2F -> F): value c[..., :F] times gate(c[..., F:]),
+    gate = sigmoid(z) = 1 / (1 + exp(-z)) or silu(z) = z * sigmoid(z)."""
+    c = _f64(c)
+    F = c.shape[-1] // 2
+    a, z = c[..., :F], c[..., F:]
+    with np.errstate(over="ignore"):
+        sig = 1.0 / (1.0 + np.exp(-z))
+    if gate == "sigmoid":
+        return a * sig
+    if gate == "silu":
+        return a * (z * sig)
+    raise ValueError(f"unknown gate {gate!r}")
+
+
+def dwconv_glu(u, wdw, bdw, Hs: int, Ws: int, gate: str = "sigmoid") -> np.ndarray:
+    """The Mix-FFN middle: GLU of the depthwise 3x3 convolution of u (B, N, 2F)."""
+    return glu(depthwise_conv3x3(u, wdw, bdw, Hs, Ws), gate)
+
+
+def mixffn_forward(x, W1, b1, wdw, bdw, W2, b2, Hs: int, Ws: int, gate: str = "sigmoid",
+                   tokens=None) -> np.ndarray:
+    """The whole Mix-FFN: x (B, N, C) -> (B, N, C).  tokens: optional flat token
+    indices (b * N + n) of Y to form; only the expand of their 3x3 neighbourhoods is
+    computed, and the result has shape (len(tokens), C)."""
+    x = _f64(x)
+    B, N, C = x.shape
+    if tokens is None:
+        return linear(dwconv_glu(linear(x, W1, b1), wdw, bdw, Hs, Ws, gate), W2, b2)
+    tok = np.asarray(tokens, dtype=np.int64)
+    rows = []
+    for t in tok:
+        b, n = divmod(int(t), N)
+        y0, x0 = divmod(n, Ws)
+        # the 3x3 neighbourhood as its own 3x3 grid, zero where it leaves the grid
+        xs = np.zeros((1, 9, C))
+        for i in range(3):
+            for j in range(3):
+                yy, xx = y0 + i - 1, x0 + j - 1
+                if 0 <= yy < Hs and 0 <= xx < Ws:
+                    xs[0, 3 * i + j] = x[b, yy * Ws + xx]
+        u = linear(xs, W1, b1)
+        inside = np.array([[0 <= y0 + i - 1 < Hs and 0 <= x0 + j - 1 < Ws for j in range(3)]
+                           for i in range(3)], dtype=np.float64).reshape(1, 9, 1)
+        u = u * inside                      # outside the grid U is zero, bias included
+        c = depthwise_conv3x3(u, wdw, bdw, 3, 3)[:, 4]
+        rows.append(linear(glu(c, gate), W2, b2)[0])
+    return np.stack(rows) if rows else np.zeros((0, _f64(W2).shape[-1]))
