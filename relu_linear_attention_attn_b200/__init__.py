@@ -17,13 +17,15 @@ import threading
 
 __all__ = ["load", "lib_path", "workspace_bytes", "forward", "forward_noalloc", "kv_state", "apply", "qkv_fused",
            "qkv_fused_w8a8", "quantize_rows_i8", "quantize_cols_i8", "forward_causal",
-           "backward",
+           "backward", "gemm_bias", "mixffn_dwconv_glu", "mixffn_workspace_bytes",
+           "mixffn_forward", "GATES",
            "device_error", "selftest_wait_timeout", "SanaError", "STATUS", "BF16", "F32"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libsana_linattn.so"
 
 BF16, F32 = 0, 1
+GATES = {"sigmoid": 0, "silu": 1}
 STATUS = {0: "SANA_OK", -1: "SANA_EINVAL", -2: "SANA_EALIGN", -3: "SANA_EUNSUPPORTED",
           -4: "SANA_EWORKSPACE", -5: "SANA_ECUDA", -6: "SANA_ESCRATCH"}
 
@@ -76,6 +78,15 @@ def _declare(lib):
     lib.sana_linattn_device_error.restype = ctypes.c_int
     lib.sana_linattn_selftest_wait_timeout.argtypes = [i64, vp]
     lib.sana_linattn_selftest_wait_timeout.restype = ctypes.c_int
+    lib.sana_gemm_bias_bf16.argtypes = [vp, vp, fp, vp, i64, ci, ci, vp]
+    lib.sana_gemm_bias_bf16.restype = ctypes.c_int
+    lib.sana_mixffn_dwconv_glu.argtypes = [vp, fp, fp, vp, i64, ci, ci, ci, ci, vp]
+    lib.sana_mixffn_dwconv_glu.restype = ctypes.c_int
+    lib.sana_mixffn_workspace_bytes.argtypes = [i64, ci, ci, ci, ci]
+    lib.sana_mixffn_workspace_bytes.restype = sz
+    lib.sana_mixffn_forward.argtypes = [vp, vp, fp, fp, fp, vp, fp, vp, i64, ci, ci, ci, ci, ci,
+                                        vp, sz, vp]
+    lib.sana_mixffn_forward.restype = ctypes.c_int
     lib.sana_linattn_strerror.argtypes = [ci]
     lib.sana_linattn_strerror.restype = ctypes.c_char_p
     return lib
@@ -362,4 +373,80 @@ def qkv_fused(x, W, gq, gk, H: int, eps: float, out=None, workspace=None, stream
                                        None if ws is None else ws.data_ptr(), wsb,
                                        _stream(stream))
     _check("sana_linattn_qkv_fused", rc)
+    return out
+
+
+# --------------------------------------------------------------------------- Mix-FFN
+# (declared in include/sana_mixffn.h)
+def _bf16(t, name: str):
+    if t.dtype != _torch().bfloat16:
+        raise TypeError(f"{name} must be bfloat16")
+    return _dev(t, name)
+
+
+def _gate(gate: str) -> int:
+    if gate not in GATES:
+        raise ValueError(f"gate must be one of {sorted(GATES)}")
+    return GATES[gate]
+
+
+def gemm_bias(A, W, bias=None, out=None, stream=None):
+    """out[M, Nc] = A[M, K] @ W[K, Nc] (+ bias) in bf16 with fp32 accumulation.
+    A may have leading batch dimensions (flattened into M)."""
+    K, Nc = W.shape
+    if A.shape[-1] != K:
+        raise ValueError("A's last dimension must equal W's first")
+    M = A.numel() // K
+    if out is None:
+        out = _torch().empty(*A.shape[:-1], Nc, dtype=A.dtype, device=A.device)
+    if out.numel() != M * Nc:
+        raise ValueError("out must hold M x Nc elements")
+    rc = load().sana_gemm_bias_bf16(_bf16(A, "A"), _bf16(W, "W"), _gain(bias, "bias"),
+                                    _bf16(out, "out"), M, K, Nc, _stream(stream))
+    _check("sana_gemm_bias_bf16", rc)
+    return out
+
+
+def mixffn_dwconv_glu(u, wdw, bdw, Hs: int, Ws: int, gate: str = "sigmoid", out=None,
+                      stream=None):
+    """GLU of the depthwise 3x3 convolution of u (B, Hs*Ws, 2F) bf16 on the row-major
+    (Hs, Ws) grid; wdw float32 (2F, 3, 3), bdw float32 [2F] or None -> (B, N, F)."""
+    B, N, C2 = u.shape
+    if N != Hs * Ws or C2 % 2:
+        raise ValueError("u must be (B, Hs*Ws, 2F)")
+    F = C2 // 2
+    if tuple(wdw.shape) != (C2, 3, 3):
+        raise ValueError("wdw must be (2F, 3, 3)")
+    if out is None:
+        out = _torch().empty(B, N, F, dtype=u.dtype, device=u.device)
+    rc = load().sana_mixffn_dwconv_glu(_bf16(u, "u"), _gain(wdw, "wdw"), _gain(bdw, "bdw"),
+                                       _bf16(out, "out"), B, Hs, Ws, F, _gate(gate),
+                                       _stream(stream))
+    _check("sana_mixffn_dwconv_glu", rc)
+    return out
+
+
+def mixffn_workspace_bytes(B: int, Hs: int, Ws: int, C: int, F: int) -> int:
+    return int(load().sana_mixffn_workspace_bytes(B, Hs, Ws, C, F))
+
+
+def mixffn_forward(x, W1, b1, wdw, bdw, W2, b2, Hs: int, Ws: int, gate: str = "sigmoid",
+                   out=None, workspace=None, stream=None):
+    """The Mix-FFN of x (B, Hs*Ws, C) bf16: 1x1 expand (W1: (C, 2F)), depthwise 3x3 +
+    GLU, 1x1 project (W2: (F, C)); biases float32 or None."""
+    B, N, C = x.shape
+    F = W2.shape[0]
+    if N != Hs * Ws or tuple(W1.shape) != (C, 2 * F) or tuple(W2.shape) != (F, C):
+        raise ValueError("shapes must be x (B, Hs*Ws, C), W1 (C, 2F), W2 (F, C)")
+    if tuple(wdw.shape) != (2 * F, 3, 3):
+        raise ValueError("wdw must be (2F, 3, 3)")
+    if out is None:
+        out = _torch().empty_like(x)
+    ws, wsb = _workspace(mixffn_workspace_bytes(B, Hs, Ws, C, F), x.device, workspace)
+    rc = load().sana_mixffn_forward(_bf16(x, "x"), _bf16(W1, "W1"), _gain(b1, "b1"),
+                                    _gain(wdw, "wdw"), _gain(bdw, "bdw"), _bf16(W2, "W2"),
+                                    _gain(b2, "b2"), _bf16(out, "out"), B, Hs, Ws, C, F,
+                                    _gate(gate), None if ws is None else ws.data_ptr(), wsb,
+                                    _stream(stream))
+    _check("sana_mixffn_forward", rc)
     return out

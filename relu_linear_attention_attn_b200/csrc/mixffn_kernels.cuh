@@ -1,0 +1,349 @@
+// The Mix-FFN of the Linear DiT block ("Sana: Efficient High-Resolution Image
+// Synthesis with Linear Diffusion Transformers", section 2.2: an inverted residual
+// block, a 3x3 depthwise convolution and a GLU in place of the MLP FFN; section
+// 2.3: the convolution's zero padding carries position; "SANA 1.5", section
+// "Model architecture": C = 2240, FFN width F = 5600).  Tokens n = y * Ws + x of a
+// row-major (Hs, Ws) grid:
+//   U  = X W1 + b1                    gemm_bias_bf16     (1x1 expand, C -> 2F)
+//   Hg = Cv[:, :F] * gate(Cv[:, F:]), dwconv3x3_glu      (depthwise 3x3 with zero
+//        Cv = dwconv3x3(U) + bdw                          padding, then the GLU)
+//   Y  = Hg W2 + b2                   gemm_bias_bf16     (1x1 project, F -> C)
+// U and Hg are stored in bf16; every sum accumulates in fp32.
+//
+// gemm_bias_bf16: D[M][Nc] = A[M][K] W[K][Nc] (+ bias) on the sm_100a tensor cores.
+//   Persistent: CTA c takes tiles c, c + grid, ... of 128 rows x 256 columns, the
+//   column tile fastest, so concurrent CTAs share A rows through L2.  Warp 0 is
+//   the TMA producer (4-stage ring of A 128 x 64 k, K-major, and W 64 k x 256 n,
+//   MN-major, both 128-byte swizzled), warp 1 issues 128x256x16 UMMAs into one
+//   of two TMEM accumulators, warps 2-9 drain the other (bias, bf16, stores), so
+//   a tile's epilogue overlaps the next tile's main loop.
+// dwconv3x3_glu: CTA (channel chunk, column strip, batch) marches down the grid
+//   rows of a 32-token strip for 32 value channels and the 32 matching gate
+//   channels.  An 8-row TMA ring brings in each input row once, with one halo
+//   token on each side (coordinates outside the grid read as zeros: the padding);
+//   each thread keeps three rolling output rows in registers, so input row r is
+//   added to outputs r + 1, r and r - 1 with kernel rows 0, 1 and 2, and output
+//   r - 1 is complete after input r.
+#pragma once
+
+#include "sana_common.cuh"
+#include "sm100_primitives.cuh"
+#include "tc_kernels.cuh"
+
+namespace sana {
+
+enum GateKind : int { kGateSigmoid = 0, kGateSilu = 1 };
+
+__device__ __forceinline__ void tma_load_4d_u(void* dst, const CUtensorMap* m, uint64_t* bar,
+                                              int x, int y, int z, int w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(m), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
+}
+
+// ============================================================================ GEMM
+namespace gm {
+constexpr int kBM = 128;                        // UMMA M: rows per tile
+constexpr int kBN = 256;                        // UMMA N: columns per tile
+constexpr int kBK = 64;                         // k per stage: 128 bytes of an A row
+constexpr int kABytes = kBM * 128;              // 16 KB
+constexpr int kWBox = kBK * 128;                // 8 KB: 64 k rows x 64 n
+constexpr int kWBoxes = kBN / 64;
+constexpr int kStageBytes = kABytes + kWBoxes * kWBox;   // 48 KB
+constexpr int kStages = 4;
+constexpr int kTmemCols = 2 * kBN;              // two accumulators
+constexpr int kEpiWarps = 8;                    // two per TMEM lane quadrant
+constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+}  // namespace gm
+
+struct GemmArgs {
+    const float* bias;   // [Nc] or nullptr
+    bf16* d;             // [M][Nc] row-major
+    int64_t M;
+    int Nc, K;
+    int mb, nb;          // tiles along M and along Nc
+};
+
+__global__ void __launch_bounds__(gm::kThreads, 1)
+gemm_bias_bf16(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
+               const GemmArgs a)
+{
+    using namespace gm;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align_1024(smem_raw);
+    uint8_t* stages = smem;
+    uint64_t* full = (uint64_t*)(stages + kStages * kStageBytes);
+    uint64_t* empty = full + kStages;
+    uint64_t* accfull = empty + kStages;         // [2]
+    uint64_t* accempty = accfull + 2;            // [2]
+    uint64_t* drained = accempty + 2;
+    uint32_t* tmem_slot = (uint32_t*)(drained + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t tiles = (int64_t)a.mb * a.nb;
+    const int ksteps = (a.K + kBK - 1) / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&accfull[i], 1);
+            mbar_init(&accempty[i], 32 * kEpiWarps);
+        }
+        mbar_init(drained, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmap_a);
+        prefetch_tmap(&tmap_w);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int64_t step = 0, last = -1;
+            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int m0 = (int)(t / a.nb) * kBM;
+                const int n0 = (int)(t % a.nb) * kBN;
+                for (int kk = 0; kk < ksteps; ++kk, ++step) {
+                    const int st = (int)(step % kStages);
+                    if (step >= kStages)
+                        ok = mbar_wait(&empty[st], (uint32_t)((step / kStages) - 1) & 1, 601);
+                    if (!ok) break;
+                    uint8_t* sb = stages + st * kStageBytes;
+                    mbar_arrive_expect_tx(&full[st], kStageBytes);
+                    tma_load_2d(sb, &tmap_a, &full[st], kk * kBK, m0);
+#pragma unroll
+                    for (int j = 0; j < kWBoxes; ++j)
+                        tma_load_2d(sb + kABytes + j * kWBox, &tmap_w, &full[st], n0 + 64 * j,
+                                    kk * kBK);
+                    last = step;
+                }
+            }
+            if (!ok) {        // let every copy already issued land before the CTA exits
+                for (int st = 0; st < kStages; ++st) {
+                    const int64_t li = last - ((last - st) % kStages + kStages) % kStages;
+                    if (last >= 0 && li >= 0)
+                        mbar_wait(&full[st], (uint32_t)(li / kStages) & 1, 602);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ UMMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = make_idesc_bf16(kBM, kBN, false, true);   // A K-, W MN-major
+            int64_t step = 0;
+            int lt = 0;
+            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++lt) {
+                const int buf = lt & 1;
+                if (lt >= 2) ok = mbar_wait(&accempty[buf], (uint32_t)((lt >> 1) - 1) & 1, 603);
+                if (!ok) break;
+                tc_fence_after_sync();
+                const uint32_t acc = tmem + buf * kBN;
+                for (int kk = 0; kk < ksteps; ++kk, ++step) {
+                    const int st = (int)(step % kStages);
+                    ok = mbar_wait(&full[st], (uint32_t)(step / kStages) & 1, 604);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    const uint32_t ab = smem_u32(stages + st * kStageBytes);
+                    const uint32_t wb = ab + kABytes;
+#pragma unroll
+                    for (int k4 = 0; k4 < kBK / 16; ++k4) {
+                        const uint64_t ad = make_smem_desc(ab + k4 * 32, 16, 1024, kSwizzle128B);
+                        const uint64_t bd = make_smem_desc(wb + k4 * 16 * 128, kWBox, 1024,
+                                                           kSwizzle128B);
+                        umma_bf16(acc, ad, bd, idesc, kk > 0 || k4 > 0);
+                    }
+                    umma_commit(&empty[st]);
+                }
+                if (!ok) break;
+                umma_commit(&accfull[buf]);
+            }
+            // every UMMA issued has completed before the TMEM is released
+            umma_commit(drained);
+            mbar_wait(drained, 0, 605);
+        }
+    } else {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;                        // TMEM lane quadrant
+        const int half = (warp - 2) >> 2;              // columns [128 half, 128 half + 128)
+        int lt = 0;
+        for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++lt) {
+            const int buf = lt & 1;
+            ok = mbar_wait(&accfull[buf], (uint32_t)(lt >> 1) & 1, 606);
+            if (!ok) break;
+            tc_fence_after_sync();
+            const int64_t row = (t / a.nb) * kBM + 32 * q + lane;
+            const int n0 = (int)(t % a.nb) * kBN;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                const int col = half * 128 + c * 32;
+                float v[32];
+                const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + buf * kBN + col;
+                tmem_ld16(ta, v);
+                tmem_ld16(ta + 16, v + 16);
+                tmem_wait_ld();
+                const int n = n0 + col;
+                if (n >= a.Nc) break;
+                if (a.bias) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (n + i < a.Nc) v[i] += __ldg(a.bias + n + i);
+                }
+                if (row < a.M) {
+                    bf16* dst = a.d + row * a.Nc + n;
+#pragma unroll
+                    for (int g8 = 0; g8 < 4; ++g8)
+                        if (n + 8 * g8 < a.Nc) store8(dst + 8 * g8, v + 8 * g8);
+                }
+            }
+            tc_fence_before_sync();
+            mbar_arrive(&accempty[buf]);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ============================================================================ dwconv + GLU
+namespace dw {
+constexpr int kTX = 32;                         // output tokens per CTA along a grid row
+constexpr int kCh = 32;                         // value channels per CTA (+ 32 gate channels)
+constexpr int kBoxTok = kTX + 2;                // one halo token on each side
+constexpr int kTokBytes = kCh * 2;              // 64 B of one token in a ring row
+constexpr int kRowBytes = kBoxTok * kTokBytes;  // 2176 B
+constexpr int kSlotBytes = 2 * kRowBytes;       // value row + gate row
+constexpr int kSlots = 8;                       // input rows in flight
+constexpr int kThreads = 256;                   // (token x: 32) x (4-channel group: 8)
+}  // namespace dw
+
+template <int kGate>
+__device__ __forceinline__ void glu_store4(bf16* p, const float* av, const float* ag) {
+    float o[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const float z = ag[c];
+        const float sg = 1.f / (1.f + expf(-z));
+        o[c] = av[c] * (kGate == kGateSigmoid ? sg : z * sg);
+    }
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+}
+
+// u: (B, Hs, Ws, 2F) bf16 seen by TMA as 4-D (2F, Ws, Hs, B), boxes of 32 channels
+// x 34 tokens x 1 row x 1 batch.  wdw [2F][3][3] fp32, bdw [2F] fp32 or nullptr,
+// h (B, Hs*Ws, F) bf16.  grid (ceil(F / 32), ceil(Ws / 32), B).  F % 8 == 0.
+template <int kGate>
+__global__ void __launch_bounds__(dw::kThreads, 2)
+dwconv3x3_glu(const __grid_constant__ CUtensorMap tmap_u, const float* __restrict__ wdw,
+              const float* __restrict__ bdw, bf16* __restrict__ h, int Hs, int Ws, int F)
+{
+    using namespace dw;
+    __shared__ __align__(128) uint8_t ring[kSlots][kSlotBytes];
+    __shared__ __align__(8) uint64_t full[kSlots];
+    const int c0 = blockIdx.x * kCh, x0 = blockIdx.y * kTX, b = blockIdx.z;
+    const int t = threadIdx.x, cg = t & 7, x = t >> 3;
+    const int j0 = c0 + 4 * cg;                        // first value channel of the thread
+    const bool chan_live = j0 < F;                     // F % 4 == 0: all 4 or none
+    const bool live = chan_live && x0 + x < Ws;
+
+    if (t == 0) {
+        for (int s = 0; s < kSlots; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+        prefetch_tmap(&tmap_u);
+    }
+    __syncthreads();
+    int issued = 0;                                    // rows issued (thread 0)
+    if (t == 0) {
+        for (; issued < kSlots && issued < Hs; ++issued) {
+            const int s = issued % kSlots;
+            mbar_arrive_expect_tx(&full[s], kSlotBytes);
+            tma_load_4d_u(ring[s], &tmap_u, &full[s], c0, x0 - 1, issued, b);
+            tma_load_4d_u(ring[s] + kRowBytes, &tmap_u, &full[s], F + c0, x0 - 1, issued, b);
+        }
+    }
+
+    float wv[4][9], wg[4][9], bv[4], bg[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int jv = chan_live ? j0 + c : 0, jg = chan_live ? F + j0 + c : 0;
+#pragma unroll
+        for (int k = 0; k < 9; ++k) {
+            wv[c][k] = __ldg(wdw + (int64_t)jv * 9 + k);
+            wg[c][k] = __ldg(wdw + (int64_t)jg * 9 + k);
+        }
+        bv[c] = bdw ? __ldg(bdw + jv) : 0.f;
+        bg[c] = bdw ? __ldg(bdw + jg) : 0.f;
+    }
+    // a0: output row r - 1, a1: row r, a2: row r + 1 while input row r is added
+    float a0v[4], a0g[4], a1v[4], a1g[4], a2v[4], a2g[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        a0v[c] = a1v[c] = a2v[c] = bv[c];
+        a0g[c] = a1g[c] = a2g[c] = bg[c];
+    }
+    bool ok = true;
+    int waited = 0;                                    // rows this thread has waited for
+    const int64_t out_row0 = ((int64_t)b * Hs) * Ws + x0 + x;
+    for (int r = 0; r < Hs; ++r) {
+        const int s = r % kSlots;
+        if (ok) ok = mbar_wait(&full[s], (uint32_t)(r / kSlots) & 1, 701);
+        if (ok) waited = r + 1;
+        const uint8_t* rv = ring[s] + x * kTokBytes + cg * 8;
+#pragma unroll
+        for (int dx = 0; dx < 3; ++dx) {
+            const uint2 pv = *reinterpret_cast<const uint2*>(rv + dx * kTokBytes);
+            const uint2 pg = *reinterpret_cast<const uint2*>(rv + kRowBytes + dx * kTokBytes);
+            const float v[4] = {bf16lo(pv.x), bf16hi(pv.x), bf16lo(pv.y), bf16hi(pv.y)};
+            const float g[4] = {bf16lo(pg.x), bf16hi(pg.x), bf16lo(pg.y), bf16hi(pg.y)};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                a2v[c] = fmaf(wv[c][dx], v[c], a2v[c]);          // kernel row 0 -> output r + 1
+                a1v[c] = fmaf(wv[c][3 + dx], v[c], a1v[c]);      // kernel row 1 -> output r
+                a0v[c] = fmaf(wv[c][6 + dx], v[c], a0v[c]);      // kernel row 2 -> output r - 1
+                a2g[c] = fmaf(wg[c][dx], g[c], a2g[c]);
+                a1g[c] = fmaf(wg[c][3 + dx], g[c], a1g[c]);
+                a0g[c] = fmaf(wg[c][6 + dx], g[c], a0g[c]);
+            }
+        }
+        __syncthreads();                               // slot s is free
+        if (t == 0 && ok && issued < Hs) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(&full[s], kSlotBytes);
+            tma_load_4d_u(ring[s], &tmap_u, &full[s], c0, x0 - 1, issued, b);
+            tma_load_4d_u(ring[s] + kRowBytes, &tmap_u, &full[s], F + c0, x0 - 1, issued, b);
+            ++issued;
+        }
+        if (r >= 1 && live) glu_store4<kGate>(h + (out_row0 + (int64_t)(r - 1) * Ws) * F + j0, a0v, a0g);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            a0v[c] = a1v[c]; a0g[c] = a1g[c];
+            a1v[c] = a2v[c]; a1g[c] = a2g[c];
+            a2v[c] = bv[c];  a2g[c] = bg[c];
+        }
+    }
+    if (Hs >= 1 && live) glu_store4<kGate>(h + (out_row0 + (int64_t)(Hs - 1) * Ws) * F + j0, a0v, a0g);
+    // after a timeout, let the copies already issued land before the CTA exits
+    if (t == 0 && !ok)
+        for (int r = waited; r < issued; ++r)
+            mbar_wait(&full[r % kSlots], (uint32_t)(r / kSlots) & 1, 702);
+}
+
+}  // namespace sana

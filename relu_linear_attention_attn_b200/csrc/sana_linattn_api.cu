@@ -1,6 +1,7 @@
 // C ABI of the SANA linear-attention library: argument validation, workspace
 // planning and kernel launches.  No allocation, no host synchronisation.
 #include "../../include/sana_linattn.h"
+#include "../../include/sana_mixffn.h"
 
 #include <math.h>
 #include <stdint.h>
@@ -15,6 +16,7 @@
 #include "quant_kernels.cuh"
 #include "causal_kernels.cuh"
 #include "backward_kernels.cuh"
+#include "mixffn_kernels.cuh"
 
 namespace sana {
 namespace {
@@ -861,6 +863,214 @@ int sana_linattn_device_error(int* code, int* site, int clear) {
             return SANA_ECUDA;
     }
     return SANA_OK;
+}
+
+}  // extern "C"
+
+// ============================================================================ Mix-FFN
+namespace sana {
+namespace {
+
+// A row-major (rows, cols) bf16 matrix seen by TMA as 2-D (cols, rows), boxes of
+// 64 columns (128 bytes) x box_rows rows, 128-byte swizzle; out-of-range reads
+// are zeros (ragged M, N and K tails).
+bool make_tmap_rowmajor(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
+                        uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64u, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// u (B, Hs, Ws, 2F) bf16 as 4-D (2F, Ws, Hs, B), boxes of 32 channels x 34 tokens x
+// 1 row x 1 batch, no swizzle; coordinates outside the grid read as zeros.
+bool make_tmap_grid(CUtensorMap* m, const void* u, int64_t B, int Hs, int Ws, int F) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t ch = 2 * (cuuint64_t)F;
+    const cuuint64_t dims[4] = {ch, (cuuint64_t)Ws, (cuuint64_t)Hs, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {ch * 2, ch * 2 * Ws, ch * 2 * Ws * Hs};
+    const cuuint32_t box[4] = {(cuuint32_t)dw::kCh, (cuuint32_t)dw::kBoxTok, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(u), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// CTAs of the persistent GEMM: one per SM (its shared memory and 512 TMEM columns
+// allow no second).  0 on failure.
+int gemm_ctas() {
+    static int ctas[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (ctas[dev]) return ctas[dev];
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms <= 0)
+        return 0;
+    if (cudaFuncSetAttribute(gemm_bias_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gm::kSmemBytes) != cudaSuccess)
+        return 0;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemm_bias_bf16, gm::kThreads,
+                                                      gm::kSmemBytes) != cudaSuccess ||
+        per_sm < 1)
+        return 0;
+    ctas[dev] = sms;
+    return sms;
+}
+
+int check_gemm(const void* A, const void* W, const float* bias, const void* D, int64_t M, int K,
+               int Nc) {
+    if (M < 0 || K <= 0 || Nc <= 0 || K % 8 != 0 || Nc % 8 != 0) return SANA_EINVAL;
+    if (M >= ((int64_t)1 << 31)) return SANA_EUNSUPPORTED;
+    if (M == 0) return SANA_OK;
+    if (!A || !W || !D) return SANA_EINVAL;
+    if (!aligned(A, 16) || !aligned(W, 16) || !aligned(D, 16)) return SANA_EALIGN;
+    if (bias && !aligned(bias, 4)) return SANA_EALIGN;
+    const size_t nd = (size_t)M * Nc * 2;
+    if (overlaps(D, nd, A, (size_t)M * K * 2) || overlaps(D, nd, W, (size_t)K * Nc * 2) ||
+        overlaps(D, nd, bias, (size_t)Nc * 4))
+        return SANA_EINVAL;
+    return SANA_OK;
+}
+
+int launch_gemm(const void* A, const void* W, const float* bias, void* D, int64_t M, int K, int Nc,
+                cudaStream_t st) {
+    if (M == 0) return SANA_OK;
+    const int P = gemm_ctas();
+    if (!P) return SANA_EUNSUPPORTED;
+    CUtensorMap ta, tw;
+    if (!make_tmap_rowmajor(&ta, A, M, K, gm::kBM) || !make_tmap_rowmajor(&tw, W, K, Nc, gm::kBK))
+        return SANA_ECUDA;
+    GemmArgs a{};
+    a.bias = bias;
+    a.d = (bf16*)D;
+    a.M = M;
+    a.Nc = Nc;
+    a.K = K;
+    a.mb = (int)((M + gm::kBM - 1) / gm::kBM);
+    a.nb = (Nc + gm::kBN - 1) / gm::kBN;
+    const int64_t tiles = (int64_t)a.mb * a.nb;
+    const unsigned grid = (unsigned)(tiles < P ? tiles : P);
+    gemm_bias_bf16<<<grid, gm::kThreads, gm::kSmemBytes, st>>>(ta, tw, a);
+    return launch_status();
+}
+
+int check_grid(int64_t B, int Hs, int Ws, int F) {
+    if (B < 0 || Hs < 0 || Ws < 0 || F <= 0 || F % 8 != 0) return SANA_EINVAL;
+    if (B > 65535 || Hs >= (1 << 24) || Ws >= (1 << 24)) return SANA_EUNSUPPORTED;
+    if ((F + dw::kCh - 1) / dw::kCh > (1 << 30)) return SANA_EUNSUPPORTED;
+    return SANA_OK;
+}
+
+int launch_dwconv(const void* u, const float* wdw, const float* bdw, void* h, int64_t B, int Hs,
+                  int Ws, int F, int gate, cudaStream_t st) {
+    if (B == 0 || Hs == 0 || Ws == 0) return SANA_OK;
+    CUtensorMap tu;
+    if (!make_tmap_grid(&tu, u, B, Hs, Ws, F)) return SANA_ECUDA;
+    const dim3 grid((unsigned)((F + dw::kCh - 1) / dw::kCh), (unsigned)((Ws + dw::kTX - 1) / dw::kTX),
+                    (unsigned)B);
+    if (gate == SANA_GATE_SIGMOID)
+        dwconv3x3_glu<kGateSigmoid><<<grid, dw::kThreads, 0, st>>>(tu, wdw, bdw, (bf16*)h, Hs, Ws, F);
+    else
+        dwconv3x3_glu<kGateSilu><<<grid, dw::kThreads, 0, st>>>(tu, wdw, bdw, (bf16*)h, Hs, Ws, F);
+    return launch_status();
+}
+
+int check_dwconv(const void* u, const float* wdw, const float* bdw, const void* h, int64_t B,
+                 int Hs, int Ws, int F, int gate) {
+    int rc;
+    if ((rc = check_grid(B, Hs, Ws, F)) != SANA_OK) return rc;
+    if (gate != SANA_GATE_SIGMOID && gate != SANA_GATE_SILU) return SANA_EINVAL;
+    if (B == 0 || Hs == 0 || Ws == 0) return SANA_OK;
+    if (!u || !wdw || !h) return SANA_EINVAL;
+    if (!aligned(u, 16) || !aligned(h, 16)) return SANA_EALIGN;
+    if (!aligned(wdw, 4) || (bdw && !aligned(bdw, 4))) return SANA_EALIGN;
+    const size_t tok = (size_t)B * Hs * Ws;
+    if (overlaps(h, tok * F * 2, u, tok * 2 * F * 2) ||
+        overlaps(h, tok * F * 2, wdw, (size_t)2 * F * 9 * 4) ||
+        overlaps(h, tok * F * 2, bdw, (size_t)2 * F * 4))
+        return SANA_EINVAL;
+    return SANA_OK;
+}
+
+struct MixLayout {
+    size_t u_off, h_off, total;
+};
+
+MixLayout mix_layout(int64_t B, int Hs, int Ws, int F) {
+    const size_t tok = (size_t)B * Hs * Ws;
+    MixLayout l{};
+    l.u_off = 0;
+    l.h_off = align_up(tok * 2 * F * 2, 256);
+    l.total = align_up(l.h_off + tok * F * 2, 256);
+    return l;
+}
+
+}  // namespace
+}  // namespace sana
+
+extern "C" {
+
+int sana_gemm_bias_bf16(const void* A, const void* W, const float* bias, void* D, int64_t M, int K,
+                        int Nc, cudaStream_t stream) {
+    int rc;
+    if ((rc = check_gemm(A, W, bias, D, M, K, Nc)) != SANA_OK) return rc;
+    return launch_gemm(A, W, bias, D, M, K, Nc, stream);
+}
+
+int sana_mixffn_dwconv_glu(const void* u, const float* wdw, const float* bdw, void* h, int64_t B,
+                           int Hs, int Ws, int F, int gate, cudaStream_t stream) {
+    int rc;
+    if ((rc = check_dwconv(u, wdw, bdw, h, B, Hs, Ws, F, gate)) != SANA_OK) return rc;
+    return launch_dwconv(u, wdw, bdw, h, B, Hs, Ws, F, gate, stream);
+}
+
+size_t sana_mixffn_workspace_bytes(int64_t B, int Hs, int Ws, int C, int F) {
+    if (check_grid(B, Hs, Ws, F) != SANA_OK || C <= 0 || C % 8 != 0) return 0;
+    if (B == 0 || Hs == 0 || Ws == 0) return 0;
+    return mix_layout(B, Hs, Ws, F).total;
+}
+
+int sana_mixffn_forward(const void* x, const void* W1, const float* b1, const float* wdw,
+                        const float* bdw, const void* W2, const float* b2, void* y, int64_t B,
+                        int Hs, int Ws, int C, int F, int gate, void* workspace, size_t ws_bytes,
+                        cudaStream_t stream) {
+    int rc;
+    if ((rc = check_grid(B, Hs, Ws, F)) != SANA_OK) return rc;
+    if (C <= 0 || C % 8 != 0) return SANA_EINVAL;
+    if (gate != SANA_GATE_SIGMOID && gate != SANA_GATE_SILU) return SANA_EINVAL;
+    if (B == 0 || Hs == 0 || Ws == 0) return SANA_OK;
+    const int64_t M = B * (int64_t)Hs * Ws;
+    if (M >= ((int64_t)1 << 31)) return SANA_EUNSUPPORTED;
+    if (!x || !W1 || !wdw || !W2 || !y) return SANA_EINVAL;
+    const MixLayout l = mix_layout(B, Hs, Ws, F);
+    if ((rc = validate_ws(workspace, ws_bytes, l.total)) != SANA_OK) return rc;
+    uint8_t* ws = (uint8_t*)workspace;
+    void* U = ws + l.u_off;
+    void* Hg = ws + l.h_off;
+    const void* args[] = {x, W1, b1, wdw, bdw, W2, b2, y};
+    const size_t sizes[] = {(size_t)M * C * 2, (size_t)C * 2 * F * 2, (size_t)2 * F * 4,
+                            (size_t)2 * F * 9 * 4, (size_t)2 * F * 4, (size_t)F * C * 2,
+                            (size_t)C * 4, (size_t)M * C * 2};
+    for (int i = 0; i < 8; ++i)
+        if (overlaps(workspace, l.total, args[i], sizes[i])) return SANA_EINVAL;
+    if ((rc = check_gemm(x, W1, b1, U, M, C, 2 * F)) != SANA_OK) return rc;
+    if ((rc = check_dwconv(U, wdw, bdw, Hg, B, Hs, Ws, F, gate)) != SANA_OK) return rc;
+    if ((rc = check_gemm(Hg, W2, b2, y, M, F, C)) != SANA_OK) return rc;
+    for (int i = 0; i < 6; ++i)
+        if (overlaps(y, sizes[7], args[i], sizes[i])) return SANA_EINVAL;
+    if ((rc = launch_gemm(x, W1, b1, U, M, C, 2 * F, stream)) != SANA_OK) return rc;
+    if ((rc = launch_dwconv(U, wdw, bdw, Hg, B, Hs, Ws, F, gate, stream)) != SANA_OK) return rc;
+    return launch_gemm(Hg, W2, b2, y, M, F, C, stream);
 }
 
 }  // extern "C"

@@ -142,3 +142,83 @@ def make_output_grad(w: Workload, seed_offset: int = 100) -> torch.Tensor:
     rng = np.random.default_rng(w.seed + seed_offset)
     return _store(rng.standard_normal((w.B, w.N, w.C), dtype=np.float32), w.dtype)
 
+
+
+# ----------------------------------------------------------------------------- Mix-FFN
+@dataclasses.dataclass(frozen=True)
+class MixFFNWorkload:
+    """One Mix-FFN input configuration: tokens on a row-major (Hs, Ws) latent grid.
+
+    Recipe (numpy ``default_rng(seed)``, float32 draws in this order, then the
+    storage rounding): x ~ N(0, 1) (B, Hs*Ws, C) bf16; W1 ~ N(0, 1/C) (C, 2F) bf16;
+    b1 ~ 0.1 N(0, 1) [2F]; wdw ~ N(0, 1/9) (2F, 3, 3); bdw ~ 0.1 N(0, 1) [2F];
+    W2 ~ N(0, 1/F) (F, C) bf16; b2 ~ 0.1 N(0, 1) [C] (fp32 biases and depthwise
+    weights; the biases are None when ``bias`` is False, after being drawn)."""
+    name: str
+    B: int
+    Hs: int
+    Ws: int
+    C: int
+    F: int
+    gate: str           # sigmoid | silu
+    bias: bool
+    seed: int
+
+    @property
+    def N(self) -> int:
+        return self.Hs * self.Ws
+
+    @property
+    def tokens(self) -> int:
+        return self.B * self.N
+
+    def scaled(self, **kw) -> "MixFFNWorkload":
+        return dataclasses.replace(self, **kw)
+
+
+# A tiny grid, SANA-1.6B's widths (C = 2240, F = 5600) on the 1024px latent grid
+# (32 x 32 tokens), and a 2048px batch of 4 (64 x 64 tokens).
+MIXFFN_CONFIGS = (
+    MixFFNWorkload("mixffn-tiny", B=1, Hs=8, Ws=8, C=64, F=96, gate="sigmoid", bias=True,
+                   seed=31),
+    MixFFNWorkload("mixffn-1024px-b1", B=1, Hs=32, Ws=32, C=2240, F=5600, gate="sigmoid",
+                   bias=True, seed=32),
+    MixFFNWorkload("mixffn-2048px-b4", B=4, Hs=64, Ws=64, C=2240, F=5600, gate="sigmoid",
+                   bias=True, seed=33),
+)
+
+
+def make_mixffn_inputs(w: MixFFNWorkload) -> dict:
+    """CPU tensors x, W1, b1, wdw, bdw, W2, b2 of one Mix-FFN workload."""
+    rng = np.random.default_rng(w.seed)
+    x = rng.standard_normal((w.B, w.N, w.C), dtype=np.float32)
+    W1 = rng.standard_normal((w.C, 2 * w.F), dtype=np.float32) / np.float32(np.sqrt(w.C))
+    b1 = 0.1 * rng.standard_normal(2 * w.F, dtype=np.float32)
+    wdw = rng.standard_normal((2 * w.F, 3, 3), dtype=np.float32) / np.float32(3.0)
+    bdw = 0.1 * rng.standard_normal(2 * w.F, dtype=np.float32)
+    W2 = rng.standard_normal((w.F, w.C), dtype=np.float32) / np.float32(np.sqrt(w.F))
+    b2 = 0.1 * rng.standard_normal(w.C, dtype=np.float32)
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return dict(x=_store(x, "bf16"), W1=_store(W1, "bf16"), W2=_store(W2, "bf16"),
+                wdw=f32(wdw), b1=f32(b1) if w.bias else None, bdw=f32(bdw) if w.bias else None,
+                b2=f32(b2) if w.bias else None)
+
+
+def make_gemm_inputs(M: int, K: int, Nc: int, seed: int, bias: bool = True) -> dict:
+    """A ~ N(0, 1) (M, K) bf16, W ~ N(0, 1/K) (K, Nc) bf16, bias ~ 0.1 N(0, 1) fp32."""
+    rng = np.random.default_rng(seed)
+    A = rng.standard_normal((M, K), dtype=np.float32)
+    W = rng.standard_normal((K, Nc), dtype=np.float32) / np.float32(np.sqrt(K))
+    b = 0.1 * rng.standard_normal(Nc, dtype=np.float32)
+    return dict(A=_store(A, "bf16"), W=_store(W, "bf16"),
+                bias=torch.from_numpy(b) if bias else None)
+
+
+def make_dwconv_inputs(B: int, Hs: int, Ws: int, F: int, seed: int, bias: bool = True) -> dict:
+    """u ~ N(0, 1) (B, Hs*Ws, 2F) bf16, wdw ~ N(0, 1/9) (2F, 3, 3), bdw ~ 0.1 N(0, 1)."""
+    rng = np.random.default_rng(seed)
+    u = rng.standard_normal((B, Hs * Ws, 2 * F), dtype=np.float32)
+    wdw = rng.standard_normal((2 * F, 3, 3), dtype=np.float32) / np.float32(3.0)
+    bdw = 0.1 * rng.standard_normal(2 * F, dtype=np.float32)
+    return dict(u=_store(u, "bf16"), wdw=torch.from_numpy(wdw),
+                bdw=torch.from_numpy(bdw) if bias else None)

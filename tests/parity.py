@@ -4,7 +4,8 @@ Tolerances (applied to the library's output against the fp64 oracle on the
 same dtype-rounded inputs):
   bf16 output : max|O - O_ref| <= 2e-2 and mean|O - O_ref| <= 2e-3, and, as a
                 stricter guard derived from the arithmetic (bf16 operands carry
-                a relative rounding of 2^-9 ~ 2e-3 and the output one more), the
+                a relative rounding of up to 2^-8 ~ 3.9e-3, the unit roundoff of
+                bf16's 8 significant bits, and the output one more), the
                 normwise relative error ||O - O_ref||_2 / ||O_ref||_2 <= 2e-2.
   fp32 output : max|O - O_ref| <= 5e-5 * max|O_ref| (normwise relative).
 """

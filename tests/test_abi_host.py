@@ -221,3 +221,75 @@ def test_backward_entry_point_rejects_bad_arguments(lib):
     a[14] = 35
     assert lib.sana_linattn_backward(*a) == EUNSUP
 
+
+
+def test_mixffn_entry_points_reject_bad_arguments(lib):
+    G = 1 << 30
+    # GEMM: K and Nc multiples of 8, aligned pointers, D apart from the operands
+    base = [FAKE, FAKE + G, FAKE + 2 * G, FAKE + 3 * G, 1000, 2240, 11200, None]
+    a = list(base)
+    a[5] = 2244
+    assert lib.sana_gemm_bias_bf16(*a) == EINVAL
+    a = list(base)
+    a[6] = 0
+    assert lib.sana_gemm_bias_bf16(*a) == EINVAL
+    a = list(base)
+    a[0] += 8
+    assert lib.sana_gemm_bias_bf16(*a) == EALIGN
+    a = list(base)
+    a[2] += 2
+    assert lib.sana_gemm_bias_bf16(*a) == EALIGN
+    a = list(base)
+    a[3] = FAKE + 64                              # D overlaps A
+    assert lib.sana_gemm_bias_bf16(*a) == EINVAL
+    a = list(base)
+    a[4] = 1 << 31
+    assert lib.sana_gemm_bias_bf16(*a) == EUNSUP
+    a = list(base)
+    a[4] = 0                                      # empty: nothing to do
+    assert lib.sana_gemm_bias_bf16(*a) == OK
+    # depthwise conv + GLU
+    base = [FAKE, FAKE + G, FAKE + 2 * G, FAKE + 3 * G, 2, 64, 64, 5600, 0, None]
+    a = list(base)
+    a[7] = 5604
+    assert lib.sana_mixffn_dwconv_glu(*a) == EINVAL
+    a = list(base)
+    a[8] = 2
+    assert lib.sana_mixffn_dwconv_glu(*a) == EINVAL
+    a = list(base)
+    a[3] += 4
+    assert lib.sana_mixffn_dwconv_glu(*a) == EALIGN
+    a = list(base)
+    a[3] = FAKE + 128                             # h overlaps u
+    assert lib.sana_mixffn_dwconv_glu(*a) == EINVAL
+    a = list(base)
+    a[4] = 70000
+    assert lib.sana_mixffn_dwconv_glu(*a) == EUNSUP
+    # the whole Mix-FFN
+    need = lib.sana_mixffn_workspace_bytes(2, 64, 64, 2240, 5600)
+    tok = 2 * 64 * 64
+    assert need == tok * 2 * 5600 * 2 + tok * 5600 * 2
+    assert lib.sana_mixffn_workspace_bytes(2, 64, 64, 2240, 5601) == 0
+    base = [FAKE, FAKE + G, None, FAKE + 2 * G, None, FAKE + 3 * G, None, FAKE + 4 * G, 2, 64, 64,
+            2240, 5600, 0, FAKE + 5 * G, need, None]
+    a = list(base)
+    a[15] = need - 256
+    assert lib.sana_mixffn_forward(*a) == EWS
+    a = list(base)
+    a[14] = FAKE + 5 * G + 16
+    assert lib.sana_mixffn_forward(*a) == EALIGN
+    a = list(base)
+    a[14] = FAKE + 4 * G                          # workspace overlaps y
+    assert lib.sana_mixffn_forward(*a) == EINVAL
+    a = list(base)
+    a[7] = FAKE + 64                              # y overlaps x
+    assert lib.sana_mixffn_forward(*a) == EINVAL
+    a = list(base)
+    a[11] = 2242
+    assert lib.sana_mixffn_forward(*a) == EINVAL
+    a = list(base)
+    a[13] = 5
+    assert lib.sana_mixffn_forward(*a) == EINVAL
+    a = list(base)
+    a[0] += 2
+    assert lib.sana_mixffn_forward(*a) == EALIGN
