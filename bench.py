@@ -215,6 +215,8 @@ def run_reference(args, rank, world):
         return
     from oracle import oracle as O
     from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
+    if args.workload == "mixffn":
+        return run_reference_mixffn(args, O)
     fused = args.workload in ("fused", "w8a8")
     wl = [CONFIGS[4] if args.workload == "fused" else CONFIGS[5]] if fused else \
         select(args.workload)
@@ -266,6 +268,58 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def mixffn_cpu_sample():
+    """The oracle's Mix-FFN as it stands on a bounded sample (128 tokens of the
+    2048px batch of 4, about 10 s of host work)."""
+    from oracle import oracle as O
+    from relu_linear_attention_attn_b200.synthetic import MIXFFN_CONFIGS, make_mixffn_inputs
+    w = MIXFFN_CONFIGS[2]
+    x = make_mixffn_inputs(w)
+    f = lambda t: None if t is None else t.float().numpy()
+    tok = [(i * 1031) % w.tokens for i in range(128)]
+    t0 = time.perf_counter()
+    O.mixffn_forward(f(x["x"]), f(x["W1"]), f(x["b1"]), f(x["wdw"]), f(x["bdw"]), f(x["W2"]),
+                     f(x["b2"]), w.Hs, w.Ws, w.gate, tokens=tok)
+    dt = time.perf_counter() - t0
+    return {"value": len(tok) / dt / 1e6, "unit": "Mtokens/s", "cores": O.host_threads(),
+            "kind": "oracle", "sample": f"{len(tok)} tokens of {w.name} (3x3 neighbourhoods), "
+                                        f"fp64 numpy oracle, {dt:.1f} s"}
+
+
+def run_reference_mixffn(args, O):
+    """The oracle's Mix-FFN on a bounded sample of the 2048px batch of 4: each step
+    forms Y for 64 tokens spread over the grids (their 3x3 neighbourhoods' expand,
+    the depthwise conv + GLU, the project), in fp64 on the host cores."""
+    from relu_linear_attention_attn_b200.synthetic import MIXFFN_CONFIGS, make_mixffn_inputs
+    w = MIXFFN_CONFIGS[2]
+    x = make_mixffn_inputs(w)
+    f = lambda t: None if t is None else t.float().numpy()
+    args_np = (f(x["x"]), f(x["W1"]), f(x["b1"]), f(x["wdw"]), f(x["bdw"]), f(x["W2"]), f(x["b2"]))
+    tok = [(i * 1031) % w.tokens for i in range(64)]
+
+    def step():
+        O.mixffn_forward(*args_np, w.Hs, w.Ws, w.gate, tokens=tok)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = len(tok) * args.steps / dt / 1e6
+    sample = f"64 tokens of {w.name} per step (3x3 neighbourhoods, fp64 oracle)"
+    line = {"impl": "reference", "metric": "Mix-FFN tokens per second", "value": value,
+            "unit": "Mtokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hs": w.Hs, "Ws": w.Ws, "C": w.C, "F": w.F},
+            "cpu_baseline": {"value": value, "unit": "Mtokens/s", "cores": O.host_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "Mtokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
 def config_block(args, wl):
     return {"workload": "sana-latent-sweep-N1K-16K" if args.workload == "sweep" else
             args.workload,
@@ -288,7 +342,7 @@ def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = measured_peaks()
-    wl = select(args.workload) if args.workload not in ("fused", "w8a8") else []
+    wl = select(args.workload) if args.workload not in ("fused", "w8a8", "mixffn") else []
 
     # inputs resident in HBM; each rank works on its own batch (weak scaling)
     sets = []
@@ -454,6 +508,17 @@ def run_ours(args, rank, world, local):
                          "clocks": f.get("clocks")})
             line["config"] = {"workload": CONFIGS[5].name, "B": 4, "N": 4096, "C": 2240,
                               "H": 70, "parallelism": f"dp{args.gpus}"}
+    if args.workload == "mixffn" or (args.workload == "sweep" and not args.no_fused):
+        line["mixffn"] = mixffn_measure(args, sla, rank, dev, stream, world, bf16_tf, hbm_gbs,
+                                        peak_kind)
+        if args.workload == "mixffn":
+            f = line["mixffn"]
+            line.update({"metric": "Mix-FFN tokens per second", "value": f["value"],
+                         "ms_per_step": f["ms_per_step"], "roofline": f["roofline"],
+                         "gpu_launches": f["gpu_launches"], "clocks": f.get("clocks"),
+                         "e2e": f["e2e"]})
+            line["config"] = {"workload": f["workload"], "B": 4, "Hs": 64, "Ws": 64, "C": 2240,
+                              "F": 5600, "parallelism": f"dp{args.gpus}"}
     if args.workload == "fused" or (args.workload == "sweep" and not args.no_fused):
         line["fused"] = fused_measure(args, sla, CONFIGS[4], rank, dev, stream, world, bf16_tf,
                                       peak_kind)
@@ -465,7 +530,9 @@ def run_ours(args, rank, world, local):
             line["config"] = {"workload": CONFIGS[4].name, "B": 4, "N": 4096, "C": 2240, "H": 70,
                               "parallelism": f"dp{args.gpus}"}
 
-    if rank == 0 and world == 1 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu and args.workload == "mixffn":
+        line["cpu_baseline"] = mixffn_cpu_sample()
+    elif rank == 0 and world == 1 and not args.no_cpu:
         pairs = [(w, x) for w, _, x in sets]
         if not pairs:
             w = CONFIGS[1]
@@ -749,6 +816,87 @@ def w8a8_measure(args, sla, w, rank, dev, stream, world, bf16_tf, peak_kind):
             "gpu_launches": steps * 3, "clocks": clk.summary()}
 
 
+def mixffn_measure(args, sla, rank, dev, stream, world, bf16_tf, hbm_gbs, peak_kind):
+    """The Mix-FFN tail of the block on the 2048px batch of 4 (64 x 64 latent grid,
+    C = 2240, F = 5600): one step = expand GEMM -> depthwise 3x3 + GLU -> project
+    GEMM (sana_mixffn_forward's three kernels, inputs resident), CUDA events between
+    the launches.  The dominant kernel is the expand GEMM, bound by the tensor peak;
+    the depthwise conv + GLU is HBM-bound (reads U, writes Hg: 3F x 2 B per token)."""
+    import torch
+    from relu_linear_attention_attn_b200.synthetic import MIXFFN_CONFIGS, make_mixffn_inputs
+    w = MIXFFN_CONFIGS[2]
+    x = make_mixffn_inputs(w.scaled(seed=w.seed + 1000 * rank) if rank else w)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    M = w.tokens
+    u = torch.empty(M, 2 * w.F, dtype=torch.bfloat16, device=dev)
+    h = torch.empty(M, w.F, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(M, w.C, dtype=torch.bfloat16, device=dev)
+    xf = d["x"].reshape(M, w.C)
+    steps = max(3, min(args.steps, 20))
+    stages = (lambda: sla.gemm_bias(xf, d["W1"], d["b1"], out=u),
+              lambda: sla.mixffn_dwconv_glu(u.view(w.B, w.N, 2 * w.F), d["wdw"], d["bdw"], w.Hs,
+                                            w.Ws, w.gate, out=h.view(w.B, w.N, w.F)),
+              lambda: sla.gemm_bias(h, d["W2"], d["b2"], out=y))
+    for _ in range(max(args.warmup, 3)):
+        for f in stages:
+            f()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    with ClockSampler(dev.index) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        for e in ev:
+            e[0].record(stream)
+            for i, f in enumerate(stages):
+                f()
+                e[i + 1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = [max_over_ranks(statistics.fmean(e[i].elapsed_time(e[i + 1]) for e in ev), world)
+          for i in range(3)]
+    # e2e: the public call with host buffers (pinned x uploaded, y downloaded each step)
+    hx = x["x"].pin_memory()
+    hy = torch.empty_like(hx).pin_memory()
+    ws = torch.empty(sla.mixffn_workspace_bytes(w.B, w.Hs, w.Ws, w.C, w.F), dtype=torch.uint8,
+                     device=dev)
+    dx, dy = torch.empty_like(d["x"]), torch.empty_like(d["x"])
+
+    def e2e_step():
+        dx.copy_(hx, non_blocking=True)
+        sla.mixffn_forward(dx, d["W1"], d["b1"], d["wdw"], d["bdw"], d["W2"], d["b2"], w.Hs, w.Ws,
+                           w.gate, out=dy, workspace=ws)
+        hy.copy_(dy, non_blocking=True)
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / steps, world)
+    fl_expand = 2.0 * M * w.C * 2 * w.F
+    fl_project = 2.0 * M * w.F * w.C
+    dw_bytes = M * 3 * w.F * 2
+    tf = fl_expand / (ms[0] * 1e-3) / 1e12
+    return {"workload": w.name, "value": M * world / (sum(ms) * 1e-3) / 1e6,
+            "unit": "Mtokens/s", "ms_per_step": sum(ms), "steps": steps,
+            "expand_ms": ms[0], "dwconv_glu_ms": ms[1], "project_ms": ms[2],
+            "expand_tflops": tf, "project_tflops": fl_project / (ms[2] * 1e-3) / 1e12,
+            "dwconv_glu_hbm_frac": dw_bytes / (ms[1] * 1e-3) / 1e9 / hbm_gbs,
+            "step_tflops": (fl_expand + fl_project) / (sum(ms) * 1e-3) / 1e12,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16_tf, "unit": "TFLOP/s",
+                         "frac": tf / bf16_tf, "traffic": None,
+                         "kernel": "gemm_bias_bf16 (expand, 16384 x 2240 x 11200)",
+                         "flop_per_launch": fl_expand,
+                         "peak_kind": f"{peak_kind} bf16 burst (bf16_tflops)"},
+            "e2e": {"value": M * world / (e2e_ms * 1e-3) / 1e6, "unit": "Mtokens/s",
+                    "h2d_bytes_per_step": hx.numel() * 2, "d2h_bytes_per_step": hy.numel() * 2},
+            "gpu_launches": steps * 3, "clocks": clk.summary()}
+
+
 def profile_case(args):
     """--warmup calls of sana_linattn_forward (two kernel launches each) on one
     workload, optionally with another batch size; prints a checksum."""
@@ -786,7 +934,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="sweep",
-                    choices=["sweep", "fused", "w8a8", "1024px", "2048px", "4096px"])
+                    choices=["sweep", "fused", "w8a8", "mixffn", "1024px", "2048px", "4096px"])
     ap.add_argument("--no-fused", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

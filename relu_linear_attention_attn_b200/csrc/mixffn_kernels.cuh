@@ -235,14 +235,41 @@ constexpr int kSlots = 8;                       // input rows in flight
 constexpr int kThreads = 256;                   // (token x: 32) x (4-channel group: 8)
 }  // namespace dw
 
+// Two fp32 lanes in one 64-bit register, for the packed fma.rn.f32x2 of sm_100a
+// (each lane an IEEE fma with round-to-nearest, as fmaf).
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t p, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+// bf16 pair (lo in the low half-word) -> two fp32 lanes; exact.
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t u) {
+    return pack2(bf16lo(u), bf16hi(u));
+}
+
+// Output row of 4 value + 4 gate channels: pairs 0, 1 value, 2, 3 gate.
+// GLU with the gate sigmoid(z) = 1 / (1 + e^-z) from __expf and __fdividef (a
+// few fp32 ulps; e^-z = inf gives 0), then bf16 rounding and one 8-byte store.
 template <int kGate>
-__device__ __forceinline__ void glu_store4(bf16* p, const float* av, const float* ag) {
+__device__ __forceinline__ void glu_store4(bf16* p, const uint64_t* acc) {
+    float a[4], z[4];
+    unpack2(acc[0], a[0], a[1]);
+    unpack2(acc[1], a[2], a[3]);
+    unpack2(acc[2], z[0], z[1]);
+    unpack2(acc[3], z[2], z[3]);
     float o[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        const float z = ag[c];
-        const float sg = 1.f / (1.f + expf(-z));
-        o[c] = av[c] * (kGate == kGateSigmoid ? sg : z * sg);
+        const float sg = __fdividef(1.f, 1.f + __expf(-z[c]));
+        o[c] = a[c] * (kGate == kGateSigmoid ? sg : z[c] * sg);
     }
     *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
 }
@@ -250,6 +277,9 @@ __device__ __forceinline__ void glu_store4(bf16* p, const float* av, const float
 // u: (B, Hs, Ws, 2F) bf16 seen by TMA as 4-D (2F, Ws, Hs, B), boxes of 32 channels
 // x 34 tokens x 1 row x 1 batch.  wdw [2F][3][3] fp32, bdw [2F] fp32 or nullptr,
 // h (B, Hs*Ws, F) bf16.  grid (ceil(F / 32), ceil(Ws / 32), B).  F % 8 == 0.
+// Thread (x, cg) owns value channels j0..j0+3 (j0 = c0 + 4 cg) and the matching gate
+// channels of grid column x0 + x; output row y lives in the accumulator set
+// acc[y % 3] (4 packed pairs), so the march needs no register moves.
 template <int kGate>
 __global__ void __launch_bounds__(dw::kThreads, 2)
 dwconv3x3_glu(const __grid_constant__ CUtensorMap tmap_u, const float* __restrict__ wdw,
@@ -271,75 +301,85 @@ dwconv3x3_glu(const __grid_constant__ CUtensorMap tmap_u, const float* __restric
     }
     __syncthreads();
     int issued = 0;                                    // rows issued (thread 0)
-    if (t == 0) {
-        for (; issued < kSlots && issued < Hs; ++issued) {
-            const int s = issued % kSlots;
-            mbar_arrive_expect_tx(&full[s], kSlotBytes);
-            tma_load_4d_u(ring[s], &tmap_u, &full[s], c0, x0 - 1, issued, b);
-            tma_load_4d_u(ring[s] + kRowBytes, &tmap_u, &full[s], F + c0, x0 - 1, issued, b);
-        }
-    }
+    auto issue = [&]() {
+        const int s = issued % kSlots;
+        mbar_arrive_expect_tx(&full[s], kSlotBytes);
+        tma_load_4d_u(ring[s], &tmap_u, &full[s], c0, x0 - 1, issued, b);
+        tma_load_4d_u(ring[s] + kRowBytes, &tmap_u, &full[s], F + c0, x0 - 1, issued, b);
+        ++issued;
+    };
+    if (t == 0)
+        while (issued < kSlots && issued < Hs) issue();
 
-    float wv[4][9], wg[4][9], bv[4], bg[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const int jv = chan_live ? j0 + c : 0, jg = chan_live ? F + j0 + c : 0;
+    // w2[k][p]: tap k (= 3 i + j) of channel pair p (0, 1 value; 2, 3 gate)
+    uint64_t w2[9][4], bias2[4];
+    {
+        const int jv = chan_live ? j0 : 0, jg = chan_live ? F + j0 : 0;
+        const float* wv = wdw + (int64_t)jv * 9;
+        const float* wg = wdw + (int64_t)jg * 9;
 #pragma unroll
         for (int k = 0; k < 9; ++k) {
-            wv[c][k] = __ldg(wdw + (int64_t)jv * 9 + k);
-            wg[c][k] = __ldg(wdw + (int64_t)jg * 9 + k);
+            w2[k][0] = pack2(__ldg(wv + k), __ldg(wv + 9 + k));
+            w2[k][1] = pack2(__ldg(wv + 18 + k), __ldg(wv + 27 + k));
+            w2[k][2] = pack2(__ldg(wg + k), __ldg(wg + 9 + k));
+            w2[k][3] = pack2(__ldg(wg + 18 + k), __ldg(wg + 27 + k));
         }
-        bv[c] = bdw ? __ldg(bdw + jv) : 0.f;
-        bg[c] = bdw ? __ldg(bdw + jg) : 0.f;
+        bias2[0] = bdw ? pack2(__ldg(bdw + jv), __ldg(bdw + jv + 1)) : 0ull;
+        bias2[1] = bdw ? pack2(__ldg(bdw + jv + 2), __ldg(bdw + jv + 3)) : 0ull;
+        bias2[2] = bdw ? pack2(__ldg(bdw + jg), __ldg(bdw + jg + 1)) : 0ull;
+        bias2[3] = bdw ? pack2(__ldg(bdw + jg + 2), __ldg(bdw + jg + 3)) : 0ull;
     }
-    // a0: output row r - 1, a1: row r, a2: row r + 1 while input row r is added
-    float a0v[4], a0g[4], a1v[4], a1g[4], a2v[4], a2g[4];
+    // Output row y accumulates in A[y % 3].  Its first term (kernel row 0, input
+    // row y - 1) starts from the bias; output 0 has no such term and starts there.
+    uint64_t A0[4], A1[4], A2[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        a0v[c] = a1v[c] = a2v[c] = bv[c];
-        a0g[c] = a1g[c] = a2g[c] = bg[c];
-    }
+    for (int p = 0; p < 4; ++p) A0[p] = A1[p] = A2[p] = bias2[p];
+
     bool ok = true;
     int waited = 0;                                    // rows this thread has waited for
-    const int64_t out_row0 = ((int64_t)b * Hs) * Ws + x0 + x;
-    for (int r = 0; r < Hs; ++r) {
+    const int roff = x * kTokBytes + cg * 8;
+    const int64_t row_pitch = (int64_t)Ws * F;                 // elements between grid rows
+    bf16* out = h + (((int64_t)b * Hs) * Ws + x0 + x) * F + j0;   // output row 0
+
+    // input row r: up = output r + 1 (kernel row 0), mid = output r (row 1),
+    // dn = output r - 1 (row 2), complete after this row
+    auto row = [&](int r, uint64_t (&up)[4], uint64_t (&mid)[4], uint64_t (&dn)[4]) {
         const int s = r % kSlots;
         if (ok) ok = mbar_wait(&full[s], (uint32_t)(r / kSlots) & 1, 701);
         if (ok) waited = r + 1;
-        const uint8_t* rv = ring[s] + x * kTokBytes + cg * 8;
+        const uint8_t* rv = ring[s] + roff;
 #pragma unroll
         for (int dx = 0; dx < 3; ++dx) {
             const uint2 pv = *reinterpret_cast<const uint2*>(rv + dx * kTokBytes);
             const uint2 pg = *reinterpret_cast<const uint2*>(rv + kRowBytes + dx * kTokBytes);
-            const float v[4] = {bf16lo(pv.x), bf16hi(pv.x), bf16lo(pv.y), bf16hi(pv.y)};
-            const float g[4] = {bf16lo(pg.x), bf16hi(pg.x), bf16lo(pg.y), bf16hi(pg.y)};
+            const uint64_t in[4] = {bf16x2_to_f32x2(pv.x), bf16x2_to_f32x2(pv.y),
+                                    bf16x2_to_f32x2(pg.x), bf16x2_to_f32x2(pg.y)};
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                a2v[c] = fmaf(wv[c][dx], v[c], a2v[c]);          // kernel row 0 -> output r + 1
-                a1v[c] = fmaf(wv[c][3 + dx], v[c], a1v[c]);      // kernel row 1 -> output r
-                a0v[c] = fmaf(wv[c][6 + dx], v[c], a0v[c]);      // kernel row 2 -> output r - 1
-                a2g[c] = fmaf(wg[c][dx], g[c], a2g[c]);
-                a1g[c] = fmaf(wg[c][3 + dx], g[c], a1g[c]);
-                a0g[c] = fmaf(wg[c][6 + dx], g[c], a0g[c]);
+            for (int p = 0; p < 4; ++p) {
+                up[p] = fma2(w2[dx][p], in[p], dx == 0 ? bias2[p] : up[p]);   // a new row
+                mid[p] = fma2(w2[3 + dx][p], in[p], mid[p]);
+                dn[p] = fma2(w2[6 + dx][p], in[p], dn[p]);
             }
         }
         __syncthreads();                               // slot s is free
         if (t == 0 && ok && issued < Hs) {
             fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&full[s], kSlotBytes);
-            tma_load_4d_u(ring[s], &tmap_u, &full[s], c0, x0 - 1, issued, b);
-            tma_load_4d_u(ring[s] + kRowBytes, &tmap_u, &full[s], F + c0, x0 - 1, issued, b);
-            ++issued;
+            issue();
         }
-        if (r >= 1 && live) glu_store4<kGate>(h + (out_row0 + (int64_t)(r - 1) * Ws) * F + j0, a0v, a0g);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            a0v[c] = a1v[c]; a0g[c] = a1g[c];
-            a1v[c] = a2v[c]; a1g[c] = a2g[c];
-            a2v[c] = bv[c];  a2g[c] = bg[c];
+        if (r >= 1) {
+            if (live) glu_store4<kGate>(out, dn);
+            out += row_pitch;
         }
+    };
+    for (int r = 0; r < Hs; r += 3) {
+        row(r, A1, A0, A2);
+        if (r + 1 < Hs) row(r + 1, A2, A1, A0);
+        if (r + 2 < Hs) row(r + 2, A0, A2, A1);
     }
-    if (Hs >= 1 && live) glu_store4<kGate>(h + (out_row0 + (int64_t)(Hs - 1) * Ws) * F + j0, a0v, a0g);
+    if (Hs >= 1 && live) {               // out now points at output row Hs - 1
+        const uint64_t* last = (Hs - 1) % 3 == 0 ? A0 : ((Hs - 1) % 3 == 1 ? A1 : A2);
+        glu_store4<kGate>(out, last);
+    }
     // after a timeout, let the copies already issued land before the CTA exits
     if (t == 0 && !ok)
         for (int r = waited; r < issued; ++r)
