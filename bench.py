@@ -693,7 +693,7 @@ def causal_measure(args, sla, sets, stream, world, hbm_gbs):
     achieved = wb.tokens * 2 * PASS_BYTES_PER_TOKEN / (parts[big]["ms"] * 1e-3) / 1e9
     return {"value": tot_tok * world / (tot_ms * 1e-3) / 1e6, "unit": "Mtokens/s",
             "ms_per_step": tot_ms, "steps": steps, "parts": parts,
-            "chunk_tokens": 128,
+            "chunk_tokens": 64,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
                          "frac": achieved / hbm_gbs, "traffic": None,
                          "kernel": "kv_partial_simt + causal_scan + causal_apply_simt (CUDA cores)",

@@ -92,7 +92,7 @@ SANA_API int sana_linattn_forward(const void* q, const void* k, const void* v,
  *   S_n = sum_{j <= n} phi(K_j)^T [V_j | 1].
  * Arguments, dtypes, layouts and errors as for sana_linattn_forward; workspace:
  * at least sana_linattn_workspace_bytes(B, N, C, H, 2) bytes (one fp32 state per
- * 128-token chunk of every (b, h)).  Chunk states are combined in chunk order, so
+ * 64-token chunk of every (b, h)).  Chunk states are combined in chunk order, so
  * results are reproducible. */
 SANA_API int sana_linattn_forward_causal(const void* q, const void* k, const void* v,
                                          const float* gq, const float* gk, void* out,

@@ -18,14 +18,68 @@
 //                    combined by kv_combine
 //   bwd_key_simt     one thread per (key token, head): dK, dV, gain partial
 //   gain_combine     gain partials summed over CTAs in order
+// The 32 x 33 products run as packed fp32 pairs (fma.rn.f32x2) on state rows
+// staged in shared memory with an even pitch.
 #pragma once
 
+#include "f32x2.cuh"
 #include "sana_common.cuh"
 
 namespace sana {
 
 constexpr int kBwdTile = 128;      // tokens per CTA of the per-token kernels
 constexpr int kGrow = kDP;         // [dnum | dden] floats per token-head
+constexpr int kSPitch = kDP + 1;   // shared-memory pitch of a state row (even)
+
+// A (D, D+1) state into shared memory rows of pitch kSPitch.
+__device__ __forceinline__ void stage_state(const float* st, float (*sS)[kSPitch], int t,
+                                            int nthreads) {
+    for (int i = t; i < kStateFloats; i += nthreads) sS[i / kDP][i % kDP] = st[i];
+}
+
+// y[e] = sum_d a[d] S[d][e] for e < D (packed pairs), and the normaliser column
+// sum_d a[d] S[d][D] (scalar), on a staged state.
+__device__ __forceinline__ void vec_state(const float* a, const float (*sS)[kSPitch], float* y,
+                                          float& yz) {
+    uint64_t y2[kD / 2];
+#pragma unroll
+    for (int i = 0; i < kD / 2; ++i) y2[i] = 0ull;
+    float z = 0.f;
+#pragma unroll 4
+    for (int d = 0; d < kD; ++d) {
+        const uint64_t a2 = pack2(a[d], a[d]);
+        const float2* row = reinterpret_cast<const float2*>(sS[d]);
+#pragma unroll
+        for (int i = 0; i < kD / 2; ++i) {
+            const float2 sv = row[i];
+            y2[i] = fma2(a2, pack2(sv.x, sv.y), y2[i]);
+        }
+        z = fmaf(a[d], sS[d][kD], z);
+    }
+#pragma unroll
+    for (int i = 0; i < kD / 2; ++i) unpack2(y2[i], y[2 * i], y[2 * i + 1]);
+    yz = z;
+}
+
+// y[d] = sum_{e < D} S[d][e] b[e] (packed pairs over e, lanes added at the end).
+__device__ __forceinline__ void state_vec(const float (*sS)[kSPitch], const float* b, float* y) {
+    uint64_t b2[kD / 2];
+#pragma unroll
+    for (int i = 0; i < kD / 2; ++i) b2[i] = pack2(b[2 * i], b[2 * i + 1]);
+#pragma unroll
+    for (int d = 0; d < kD; ++d) {
+        const float2* row = reinterpret_cast<const float2*>(sS[d]);
+        uint64_t acc = 0ull;
+#pragma unroll
+        for (int i = 0; i < kD / 2; ++i) {
+            const float2 sv = row[i];
+            acc = fma2(b2[i], pack2(sv.x, sv.y), acc);
+        }
+        float lo, hi;
+        unpack2(acc, lo, hi);
+        y[d] = lo + hi;
+    }
+}
 
 // u, r and phi of one head's 32 values; returns r (1 with the norm off).
 __device__ __forceinline__ float phi_fwd32(const float* x, const float* g, float eps, bool norm,
@@ -104,11 +158,10 @@ bwd_query_simt(const T* __restrict__ q, const T* __restrict__ dout,
                T* __restrict__ dq, float* __restrict__ G, float* __restrict__ gpart,
                int64_t N, int H, float eps, int norm)
 {
-    __shared__ float sS[kStateFloats];
+    __shared__ __align__(16) float sS[kD][kSPitch];
     __shared__ float red[kBwdTile];
     const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z, t = threadIdx.x;
-    const float* st = Sz + ((int64_t)b * H + h) * kStateFloats;
-    for (int i = t; i < kStateFloats; i += kBwdTile) sS[i] = st[i];
+    stage_state(Sz + ((int64_t)b * H + h) * kStateFloats, sS, t, kBwdTile);
     __syncthreads();
     const int64_t n = (int64_t)tile * kBwdTile + t;
     const bool live = n < N;
@@ -120,14 +173,9 @@ bwd_query_simt(const T* __restrict__ q, const T* __restrict__ dout,
 #pragma unroll
         for (int i = 0; i < kD; i += 8) load8(q + row + i, x + i);
         r = phi_fwd32(x, gq + h * kD, eps, norm != 0, u, p);
-        float num[kDP];
-#pragma unroll
-        for (int e = 0; e < kDP; ++e) num[e] = 0.f;
-#pragma unroll 4
-        for (int d = 0; d < kD; ++d)
-#pragma unroll
-            for (int e = 0; e < kDP; ++e) num[e] = fmaf(p[d], sS[d * kDP + e], num[e]);
-        const float den = num[kD] + eps;
+        float num[kD], numz;
+        vec_state(p, sS, num, numz);
+        const float den = numz + eps;
         float go[kD];
 #pragma unroll
         for (int i = 0; i < kD; i += 8) load8(dout + row + i, go + i);
@@ -143,13 +191,9 @@ bwd_query_simt(const T* __restrict__ q, const T* __restrict__ dout,
         }
         gr[kD] = dden;
         float dp[kD];
+        state_vec(sS, go, dp);                    // dnum S^T
 #pragma unroll
-        for (int d = 0; d < kD; ++d) {
-            float a = dden * sS[d * kDP + kD];
-#pragma unroll
-            for (int e = 0; e < kD; ++e) a = fmaf(go[e], sS[d * kDP + e], a);
-            dp[d] = a;
-        }
+        for (int d = 0; d < kD; ++d) dp[d] = fmaf(dden, sS[d][kD], dp[d]);   // + dden z
         phi_bwd32(dp, x, u, gq + h * kD, r, norm != 0, dg);
 #pragma unroll
         for (int i = 0; i < kD; i += 8) store8(dq + row + i, dp + i);
@@ -171,14 +215,15 @@ outer_partial_simt(const T* __restrict__ x, const float* __restrict__ gx,
                    int S, int64_t tps, float eps, int norm)
 {
     __shared__ float sA[64][kDP];
-    __shared__ float sB[64][kDP + 1];
+    __shared__ __align__(16) float sB[64][kSPitch];
     const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
     const int64_t n0 = (int64_t)s * tps, n1 = min(N, n0 + tps);
     const int64_t C = (int64_t)H * kD;
     const int d = tid >> 2, e0 = (tid & 3) * 8;
-    float acc[8], acc_last = 0.f;
+    uint64_t acc2[4];                 // columns e0 .. e0 + 7 in pairs
+    float acc_last = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 4; ++i) acc2[i] = 0ull;
     for (int64_t c0 = n0; c0 < n1; c0 += 64) {
         // load role: thread t < 64 forms phi of token c0 + t, threads 64..127 copy its G row
         const int lt = tid & 63;
@@ -209,12 +254,20 @@ outer_partial_simt(const T* __restrict__ x, const float* __restrict__ gx,
         const int cnt = (int)min((int64_t)64, n1 - c0);
         for (int tt = 0; tt < cnt; ++tt) {
             const float a = sA[tt][d];
+            const uint64_t a2 = pack2(a, a);
+            const float2* br = reinterpret_cast<const float2*>(&sB[tt][e0]);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = fmaf(a, sB[tt][e0 + i], acc[i]);
+            for (int i = 0; i < 4; ++i) {
+                const float2 bv = br[i];
+                acc2[i] = fma2(a2, pack2(bv.x, bv.y), acc2[i]);
+            }
             acc_last = fmaf(a, sB[tt][kD], acc_last);
         }
         __syncthreads();
     }
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) unpack2(acc2[i], acc[2 * i], acc[2 * i + 1]);
     float* out = part + (((int64_t)b * H + h) * S + s) * kStateFloats;
 #pragma unroll
     for (int i = 0; i < 8; ++i) out[d * kDP + e0 + i] = acc[i];
@@ -228,11 +281,10 @@ bwd_key_simt(const T* __restrict__ k, const T* __restrict__ v, const float* __re
              const float* __restrict__ dSz, T* __restrict__ dk, T* __restrict__ dv,
              float* __restrict__ gpart, int64_t N, int H, float eps, int norm)
 {
-    __shared__ float sS[kStateFloats];
+    __shared__ __align__(16) float sS[kD][kSPitch];
     __shared__ float red[kBwdTile];
     const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z, t = threadIdx.x;
-    const float* st = dSz + ((int64_t)b * H + h) * kStateFloats;
-    for (int i = t; i < kStateFloats; i += kBwdTile) sS[i] = st[i];
+    stage_state(dSz + ((int64_t)b * H + h) * kStateFloats, sS, t, kBwdTile);
     __syncthreads();
     const int64_t n = (int64_t)tile * kBwdTile + t;
     const bool live = n < N;
@@ -246,23 +298,14 @@ bwd_key_simt(const T* __restrict__ k, const T* __restrict__ v, const float* __re
         const float r = phi_fwd32(x, gk + h * kD, eps, norm != 0, u, p);
 #pragma unroll
         for (int i = 0; i < kD; i += 8) load8(v + row + i, vv + i);
-        float dvv[kD];
-#pragma unroll
-        for (int e = 0; e < kD; ++e) dvv[e] = 0.f;
-#pragma unroll 4
-        for (int d = 0; d < kD; ++d)
-#pragma unroll
-            for (int e = 0; e < kD; ++e) dvv[e] = fmaf(p[d], sS[d * kDP + e], dvv[e]);
+        float dvv[kD], unused;
+        vec_state(p, sS, dvv, unused);            // phi(K) dS
 #pragma unroll
         for (int i = 0; i < kD; i += 8) store8(dv + row + i, dvv + i);
         float dp[kD];
+        state_vec(sS, vv, dp);                    // dS V
 #pragma unroll
-        for (int d = 0; d < kD; ++d) {
-            float a = sS[d * kDP + kD];
-#pragma unroll
-            for (int e = 0; e < kD; ++e) a = fmaf(sS[d * kDP + e], vv[e], a);
-            dp[d] = a;
-        }
+        for (int d = 0; d < kD; ++d) dp[d] += sS[d][kD];                      // + dz
         phi_bwd32(dp, x, u, gk + h * kD, r, norm != 0, dg);
 #pragma unroll
         for (int i = 0; i < kD; i += 8) store8(dk + row + i, dp + i);

@@ -10,14 +10,20 @@
 //   3. causal_apply_simt: per chunk, the prefix state applied to every query plus
 //      the masked quadratic form inside the chunk:
 //        num_n = phi(Q_n) P_c + sum_{j in chunk, j <= n} (phi(Q_n).phi(K_j)) [V_j | 1].
+// Per query and head the chunk costs about 1,056 FMA for the prefix state and
+// 65 (L + 1) / 2 on average for the quadratic form, so L = 64 balances the two
+// against the chunk states' traffic (one 4,224-byte state per chunk and head).
+// The inner products run as packed fp32 pairs (fma.rn.f32x2).
 #pragma once
 
+#include "f32x2.cuh"
 #include "sana_common.cuh"
 
 namespace sana {
 
-constexpr int kCausalChunk = 128;
+constexpr int kCausalChunk = 64;
 constexpr int kRowPad = 36;
+constexpr int kStateRowPad = 34;     // prefix-state rows padded to an even length
 
 // Exclusive prefix over chunks: grid B * H, 256 threads; part[bh][c] becomes
 // sum_{c' < c} part[bh][c'] (the first chunk's becomes zero).
@@ -61,13 +67,13 @@ causal_apply_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     // phi(K) and V of the chunk; rows padded to 36 floats so they read as float4
     __shared__ __align__(16) float sK[kCausalChunk][kRowPad];
     __shared__ __align__(16) float sV[kCausalChunk][kRowPad];
-    __shared__ float sP[kStateFloats];          // prefix state of the chunk
+    __shared__ __align__(16) float sP[kD][kStateRowPad];   // prefix state of the chunk
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, t = threadIdx.x;
     const int64_t n = (int64_t)c * kCausalChunk + t;
     const bool live = n < N;
     const int64_t C = (int64_t)H * kD;
     const float* ps = pre + (((int64_t)b * H + h) * S + c) * kStateFloats;
-    for (int i = t; i < kStateFloats; i += kCausalChunk) sP[i] = ps[i];
+    for (int i = t; i < kStateFloats; i += kCausalChunk) sP[i / kDP][i % kDP] = ps[i];
     float x[kD];
     const int64_t row = ((int64_t)b * N + n) * C + (int64_t)h * kD;
     if (live) {
@@ -94,43 +100,57 @@ causal_apply_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         for (int i = 0; i < kD; ++i) fq[i] = 0.f;
     }
     __syncthreads();
-    float num[kDP];
+    // num2[i]: value columns 2i, 2i + 1; numz: the normaliser column
+    uint64_t num2[kD / 2], fq2[kD / 2];
 #pragma unroll
-    for (int e = 0; e < kDP; ++e) num[e] = 0.f;
+    for (int i = 0; i < kD / 2; ++i) {
+        num2[i] = 0ull;
+        fq2[i] = pack2(fq[2 * i], fq[2 * i + 1]);
+    }
+    float numz = 0.f;
 #pragma unroll 4
     for (int d = 0; d < kD; ++d) {
-        const float a = fq[d];
+        const uint64_t a2 = pack2(fq[d], fq[d]);
+        const float2* pr = reinterpret_cast<const float2*>(sP[d]);
 #pragma unroll
-        for (int e = 0; e < kDP; ++e) num[e] = fmaf(a, sP[d * kDP + e], num[e]);
+        for (int i = 0; i < kD / 2; ++i) {
+            const float2 pp = pr[i];
+            num2[i] = fma2(a2, pack2(pp.x, pp.y), num2[i]);
+        }
+        numz = fmaf(fq[d], sP[d][kD], numz);
     }
     for (int j = 0; j <= t; ++j) {               // keys of this chunk up to the query
         const float4* kr = reinterpret_cast<const float4*>(sK[j]);
         const float4* vr = reinterpret_cast<const float4*>(sV[j]);
-        float a0 = 0.f, a1 = 0.f;
+        uint64_t acc = 0ull;                     // even and odd channels of the dot product
 #pragma unroll
         for (int d4 = 0; d4 < kD / 4; ++d4) {
             const float4 kk = kr[d4];
-            a0 = fmaf(fq[4 * d4 + 0], kk.x, a0);
-            a1 = fmaf(fq[4 * d4 + 1], kk.y, a1);
-            a0 = fmaf(fq[4 * d4 + 2], kk.z, a0);
-            a1 = fmaf(fq[4 * d4 + 3], kk.w, a1);
+            acc = fma2(fq2[2 * d4], pack2(kk.x, kk.y), acc);
+            acc = fma2(fq2[2 * d4 + 1], pack2(kk.z, kk.w), acc);
         }
+        float a0, a1;
+        unpack2(acc, a0, a1);
         const float a = a0 + a1;
+        const uint64_t aa = pack2(a, a);
 #pragma unroll
         for (int e4 = 0; e4 < kD / 4; ++e4) {
             const float4 vv = vr[e4];
-            num[4 * e4 + 0] = fmaf(a, vv.x, num[4 * e4 + 0]);
-            num[4 * e4 + 1] = fmaf(a, vv.y, num[4 * e4 + 1]);
-            num[4 * e4 + 2] = fmaf(a, vv.z, num[4 * e4 + 2]);
-            num[4 * e4 + 3] = fmaf(a, vv.w, num[4 * e4 + 3]);
+            num2[2 * e4] = fma2(aa, pack2(vv.x, vv.y), num2[2 * e4]);
+            num2[2 * e4 + 1] = fma2(aa, pack2(vv.z, vv.w), num2[2 * e4 + 1]);
         }
-        num[kD] += a;
+        numz += a;
     }
     if (!live) return;
-    const float inv = 1.f / (num[kD] + eps);
+    const float inv = 1.f / (numz + eps);
     float o[kD];
 #pragma unroll
-    for (int e = 0; e < kD; ++e) o[e] = num[e] * inv;
+    for (int i = 0; i < kD / 2; ++i) {
+        float lo, hi;
+        unpack2(num2[i], lo, hi);
+        o[2 * i] = lo * inv;
+        o[2 * i + 1] = hi * inv;
+    }
 #pragma unroll
     for (int i = 0; i < kD; i += 8) store8(out + row + i, o + i);
 }

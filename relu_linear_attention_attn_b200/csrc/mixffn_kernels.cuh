@@ -26,6 +26,7 @@
 //   r - 1 is complete after input r.
 #pragma once
 
+#include "f32x2.cuh"
 #include "sana_common.cuh"
 #include "sm100_primitives.cuh"
 #include "tc_kernels.cuh"
@@ -234,26 +235,6 @@ constexpr int kSlotBytes = 2 * kRowBytes;       // value row + gate row
 constexpr int kSlots = 8;                       // input rows in flight
 constexpr int kThreads = 256;                   // (token x: 32) x (4-channel group: 8)
 }  // namespace dw
-
-// Two fp32 lanes in one 64-bit register, for the packed fma.rn.f32x2 of sm_100a
-// (each lane an IEEE fma with round-to-nearest, as fmaf).
-__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void unpack2(uint64_t p, float& lo, float& hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-// bf16 pair (lo in the low half-word) -> two fp32 lanes; exact.
-__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t u) {
-    return pack2(bf16lo(u), bf16hi(u));
-}
 
 // Output row of 4 value + 4 gate channels: pairs 0, 1 value, 2, 3 gate.
 // GLU with the gate sigmoid(z) = 1 / (1 + e^-z) from __expf and __fdividef (a
