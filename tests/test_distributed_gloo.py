@@ -91,3 +91,89 @@ def test_even_split_edges():
     assert [even_split(10, r, 3) for r in range(3)] == [(0, 3), (3, 3), (6, 4)]
     with pytest.raises(ValueError):
         even_split(3, 4, 4)
+
+
+# ----------------------------------------------------------------------------- Mix-FFN rows
+MIX_WORLD = 3          # a middle rank exchanges with both neighbours
+
+
+def _mix_case():
+    from relu_linear_attention_attn_b200.synthetic import MIXFFN_CONFIGS
+    return MIXFFN_CONFIGS[0].scaled(B=2, Hs=8, Ws=5, C=16, F=8, gate="silu", seed=92)
+
+
+def _mix_worker(rank, world, port, outdir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import sys
+        root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+        sys.path.insert(0, root)
+        from oracle import oracle as O
+        from relu_linear_attention_attn_b200 import sharding
+        from relu_linear_attention_attn_b200.synthetic import make_mixffn_inputs
+
+        w = _mix_case()
+        x = make_mixffn_inputs(w)
+        f = lambda t: None if t is None else t.double().numpy()
+        y0, cnt = sharding.row_shard(w.Hs, rank, world)
+        x_r = f(x["x"])[:, y0 * w.Ws:(y0 + cnt) * w.Ws]
+        # the expand of this rank's rows, with the fp64 oracle standing in for the GPU
+        U = torch.from_numpy(O.linear(x_r, f(x["W1"]), f(x["b1"]))).reshape(w.B, cnt, w.Ws,
+                                                                         2 * w.F)
+        top, bottom = sharding.exchange_halo_rows(U[:, 0].contiguous(), U[:, -1].contiguous(),
+                                                  rank, world)
+        U_ext = torch.cat([top[:, None], U, bottom[:, None]], dim=1).numpy()
+        Hg = O.dwconv_glu(U_ext.reshape(w.B, (cnt + 2) * w.Ws, 2 * w.F), f(x["wdw"]), f(x["bdw"]),
+                          cnt + 2, w.Ws, w.gate).reshape(w.B, cnt + 2, w.Ws, w.F)[:, 1:cnt + 1]
+        y = O.linear(Hg.reshape(w.B, cnt * w.Ws, w.F), f(x["W2"]), f(x["b2"]))
+        np.savez(os.path.join(outdir, f"mix{rank}.npz"), y=y, y0=y0, cnt=cnt,
+                 top=top.numpy(), bottom=bottom.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.fixture(scope="module")
+def mix_results(tmp_path_factory):
+    outdir = str(tmp_path_factory.mktemp("gloo_mix"))
+    mp.start_processes(_mix_worker, args=(MIX_WORLD, _free_port(), outdir), nprocs=MIX_WORLD,
+                       join=True, start_method="spawn")
+    return [dict(np.load(os.path.join(outdir, f"mix{r}.npz"))) for r in range(MIX_WORLD)]
+
+
+def test_row_sharded_mixffn_matches_single_process(mix_results):
+    from oracle import oracle as O
+    from relu_linear_attention_attn_b200.synthetic import make_mixffn_inputs
+    w = _mix_case()
+    x = make_mixffn_inputs(w)
+    f = lambda t: None if t is None else t.double().numpy()
+    ref = O.mixffn_forward(f(x["x"]), f(x["W1"]), f(x["b1"]), f(x["wdw"]), f(x["bdw"]), f(x["W2"]),
+                           f(x["b2"]), w.Hs, w.Ws, w.gate)
+    got = np.concatenate([r["y"] for r in mix_results], axis=1)
+    assert [int(r["cnt"]) for r in mix_results] == [2, 3, 3]
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_halo_rows_are_the_neighbours_rows_and_zero_at_the_edges(mix_results):
+    from oracle import oracle as O
+    from relu_linear_attention_attn_b200.synthetic import make_mixffn_inputs
+    w = _mix_case()
+    x = make_mixffn_inputs(w)
+    U = O.linear(x["x"].double().numpy(), x["W1"].double().numpy(),
+                 x["b1"].double().numpy()).reshape(w.B, w.Hs, w.Ws, 2 * w.F)
+    for r in mix_results:
+        y0, cnt = int(r["y0"]), int(r["cnt"])
+        exp_top = U[:, y0 - 1] if y0 > 0 else np.zeros_like(U[:, 0])
+        exp_bot = U[:, y0 + cnt] if y0 + cnt < w.Hs else np.zeros_like(U[:, 0])
+        np.testing.assert_array_equal(r["top"], exp_top)
+        np.testing.assert_array_equal(r["bottom"], exp_bot)
+
+
+def test_row_shard_needs_a_row_per_rank():
+    from relu_linear_attention_attn_b200.sharding import row_shard
+    assert [row_shard(8, r, 3) for r in range(3)] == [(0, 2), (2, 3), (5, 3)]
+    with pytest.raises(ValueError):
+        row_shard(2, 0, 3)

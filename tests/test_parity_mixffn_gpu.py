@@ -128,3 +128,26 @@ def test_mixffn_is_deterministic(cuda_lib):
                                 w.Hs, w.Ws, w.gate)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def test_row_shards_reassemble_the_unsharded_forward(cuda_lib):
+    """Three row shards of the 1024px grid (the halo rows copied between them as the
+    ranks' exchange would) give the one-call forward bit for bit."""
+    from relu_linear_attention_attn_b200 import sharding
+    w = MIXFFN_CONFIGS[1].scaled(Hs=17, seed=41)            # ragged: 5, 6, 6 rows
+    d = _dev(make_mixffn_inputs(w))
+    ref = cuda_lib.mixffn_forward(d["x"], d["W1"], d["b1"], d["wdw"], d["bdw"], d["W2"], d["b2"],
+                                  w.Hs, w.Ws, w.gate)
+    world = 3
+    shards = [sharding.row_shard(w.Hs, r, world) for r in range(world)]
+    Us = [sharding.mixffn_shard_expand(d["x"][:, y0 * w.Ws:(y0 + c) * w.Ws].contiguous(), d["W1"],
+                                       d["b1"], w.Ws) for y0, c in shards]
+    parts = []
+    for r, (y0, c) in enumerate(shards):
+        zero = torch.zeros_like(Us[r][:, 0])
+        top = Us[r - 1][:, -2] if r > 0 else zero              # the neighbour's last own row
+        bottom = Us[r + 1][:, 1] if r < world - 1 else zero    # and its first
+        parts.append(sharding.mixffn_shard_finish(Us[r], top, bottom, d["wdw"], d["bdw"], d["W2"],
+                                                  d["b2"], w.Ws, w.gate))
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(parts, dim=1), ref)
