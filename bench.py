@@ -163,16 +163,24 @@ KERNEL_SOURCES = ("relu_linear_attention_attn_b200/csrc/tc_kernels.cuh",
                   "relu_linear_attention_attn_b200/csrc/sm100_primitives.cuh")
 
 
-def kernel_source_hash() -> str:
+# the sources the Mix-FFN kernels compile from
+MIXFFN_SOURCES = ("relu_linear_attention_attn_b200/csrc/mixffn_kernels.cuh",
+                  "relu_linear_attention_attn_b200/csrc/f32x2.cuh",
+                  "relu_linear_attention_attn_b200/csrc/tc_kernels.cuh",
+                  "relu_linear_attention_attn_b200/csrc/sana_common.cuh",
+                  "relu_linear_attention_attn_b200/csrc/sm100_primitives.cuh")
+
+
+def kernel_source_hash(sources=KERNEL_SOURCES) -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in sources:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str, workload: str):
+def ncu_traffic(kernel: str, workload: str, sources=KERNEL_SOURCES):
     """DRAM bytes per launch of `kernel` on `workload` from the committed ncu record,
     or None when there is none or the kernel sources changed since it was taken."""
     try:
@@ -180,7 +188,7 @@ def ncu_traffic(kernel: str, workload: str):
             rec = json.load(f).get(f"{kernel}@{workload}")
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or rec.get("source_hash") != kernel_source_hash(sources):
         return None
     return rec["dram_read_bytes"] + rec["dram_write_bytes"]
 
@@ -888,7 +896,8 @@ def mixffn_measure(args, sla, rank, dev, stream, world, bf16_tf, hbm_gbs, peak_k
             "dwconv_glu_hbm_frac": dw_bytes / (ms[1] * 1e-3) / 1e9 / hbm_gbs,
             "step_tflops": (fl_expand + fl_project) / (sum(ms) * 1e-3) / 1e12,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16_tf, "unit": "TFLOP/s",
-                         "frac": tf / bf16_tf, "traffic": None,
+                         "frac": tf / bf16_tf,
+                         "traffic": ncu_traffic("gemm_bias_bf16", w.name, MIXFFN_SOURCES),
                          "kernel": "gemm_bias_bf16 (expand, 16384 x 2240 x 11200)",
                          "flop_per_launch": fl_expand,
                          "peak_kind": f"{peak_kind} bf16 burst (bf16_tflops)"},
