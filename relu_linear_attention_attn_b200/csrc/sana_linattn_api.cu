@@ -477,10 +477,10 @@ size_t sana_linattn_workspace_bytes(int64_t B, int64_t N, int C, int H, int fuse
 
 size_t sana_linattn_backward_workspace_bytes(int64_t B, int64_t N, int C, int H) {
     if (check_dims(B, N, C, H) != SANA_OK || B == 0 || N == 0) return 0;
-    const Plan p = make_plan(B, N, H);
     const int64_t tiles = (N + kBwdTile - 1) / kBwdTile;
     size_t off = 0;
-    off = align_up(off + (size_t)B * H * p.S * kStateFloats * 4, 256);   // split partials
+    // split partials: the forward state's (either plan), then dS, dz's
+    off = align_up(off + (size_t)B * H * max_splits(B, N, H) * kStateFloats * 4, 256);
     off = align_up(off + (size_t)B * H * kStateFloats * 4, 256);         // forward states
     off = align_up(off + (size_t)B * H * kStateFloats * 4, 256);         // [dS | dz]
     off = align_up(off + (size_t)B * N * H * kGrow * 4, 256);            // [dnum | dden] rows
@@ -526,7 +526,7 @@ int sana_linattn_backward(const void* q, const void* k, const void* v, const flo
     char* w = (char*)workspace;
     size_t off = 0;
     float* part = (float*)(w + off);
-    off = align_up(off + (size_t)B * H * p.S * kStateFloats * 4, 256);
+    off = align_up(off + (size_t)B * H * max_splits(B, N, H) * kStateFloats * 4, 256);
     float* Sz = (float*)(w + off);
     off = align_up(off + (size_t)B * H * kStateFloats * 4, 256);
     float* dSz = (float*)(w + off);
@@ -538,8 +538,16 @@ int sana_linattn_backward(const void* q, const void* k, const void* v, const flo
     const dim3 gs(p.S, H, (unsigned)B), gt((unsigned)tiles, H, (unsigned)B);
     const int nrm = norm ? 1 : 0;
     if (dtype == SANA_BF16) {
-        launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, Sz, B, N, H, C, C, eps, p,
-                           stream);
+        // the forward state as the bf16 forward forms it (tensor-core pass 1 + combine)
+        if (tc_path(dtype, C)) {
+            PersistPlan1 pl{};
+            if ((rc = launch_partials_tc(k, v, gk, part, B, N, C, H, eps, stream, &pl)) != SANA_OK ||
+                (rc = launch_combine_tc(part, Sz, B, H, pl, stream)) != SANA_OK)
+                return rc;
+        } else {
+            launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, Sz, B, N, H, C, C, eps, p,
+                               stream);
+        }
         bwd_query_simt<bf16><<<gt, kBwdTile, 0, stream>>>((const bf16*)q, (const bf16*)dout, gq, Sz,
                                                           (bf16*)dq, G, gpq, N, H, eps, nrm);
         outer_partial_simt<bf16><<<gs, 128, 0, stream>>>((const bf16*)q, gq, G, part, N, H, p.S,
