@@ -53,8 +53,8 @@ def measured_peaks():
 
 # ----------------------------------------------------------------------------- workloads
 def sweep_workloads():
-    from relu_linear_attention_attn_b200.synthetic import CONFIGS
-    return {"1024px": CONFIGS[1], "2048px": CONFIGS[2], "4096px": CONFIGS[3]}
+    from relu_linear_attention_attn_b200.synthetic import WORKLOADS
+    return {"1024px": WORKLOADS["1024px-b1"], "2048px": WORKLOADS["2048px-b8-lognormal"], "4096px": WORKLOADS["4096px-b2-overflow"]}
 
 
 def select(workload: str):
@@ -222,11 +222,11 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     from oracle import oracle as O
-    from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
+    from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs
     if args.workload == "mixffn":
         return run_reference_mixffn(args, O)
     fused = args.workload in ("fused", "w8a8")
-    wl = [CONFIGS[4] if args.workload == "fused" else CONFIGS[5]] if fused else \
+    wl = [WORKLOADS["fused-2048px-b4"] if args.workload == "fused" else WORKLOADS["w8a8-2048px-b4"]] if fused else \
         select(args.workload)
     # each step: one whole batch item of every workload in the sweep, bounded so
     # the --steps/--warmup run stays within a few minutes
@@ -280,8 +280,8 @@ def mixffn_cpu_sample():
     """The oracle's Mix-FFN as it stands on a bounded sample (128 tokens of the
     2048px batch of 4, about 10 s of host work)."""
     from oracle import oracle as O
-    from relu_linear_attention_attn_b200.synthetic import MIXFFN_CONFIGS, make_mixffn_inputs
-    w = MIXFFN_CONFIGS[2]
+    from relu_linear_attention_attn_b200.synthetic import MIXFFN_WORKLOADS, make_mixffn_inputs
+    w = MIXFFN_WORKLOADS["mixffn-2048px-b4"]
     x = make_mixffn_inputs(w)
     f = lambda t: None if t is None else t.float().numpy()
     tok = [(i * 1031) % w.tokens for i in range(128)]
@@ -298,8 +298,8 @@ def run_reference_mixffn(args, O):
     """The oracle's Mix-FFN on a bounded sample of the 2048px batch of 4: each step
     forms Y for 64 tokens spread over the grids (their 3x3 neighbourhoods' expand,
     the depthwise conv + GLU, the project), in fp64 on the host cores."""
-    from relu_linear_attention_attn_b200.synthetic import MIXFFN_CONFIGS, make_mixffn_inputs
-    w = MIXFFN_CONFIGS[2]
+    from relu_linear_attention_attn_b200.synthetic import MIXFFN_WORKLOADS, make_mixffn_inputs
+    w = MIXFFN_WORKLOADS["mixffn-2048px-b4"]
     x = make_mixffn_inputs(w)
     f = lambda t: None if t is None else t.float().numpy()
     args_np = (f(x["x"]), f(x["W1"]), f(x["b1"]), f(x["wdw"]), f(x["bdw"]), f(x["W2"]), f(x["b2"]))
@@ -344,7 +344,7 @@ def run_ours(args, rank, world, local):
     import torch
 
     import relu_linear_attention_attn_b200 as sla
-    from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
+    from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs
 
     sla.load()
     dev = torch.device("cuda", local)
@@ -507,14 +507,14 @@ def run_ours(args, rank, world, local):
             line["e2e"] = e2e_measure(args, sla, sets, stream, world)
 
     if args.workload == "w8a8" or (args.workload == "sweep" and not args.no_fused):
-        line["w8a8"] = w8a8_measure(args, sla, CONFIGS[5], rank, dev, stream, world, bf16_tf,
+        line["w8a8"] = w8a8_measure(args, sla, WORKLOADS["w8a8-2048px-b4"], rank, dev, stream, world, bf16_tf,
                                     peak_kind)
         if args.workload == "w8a8":
             f = line["w8a8"]
             line.update({"value": f["value"], "ms_per_step": f["ms_per_step"],
                          "roofline": f["roofline"], "gpu_launches": f["gpu_launches"],
                          "clocks": f.get("clocks")})
-            line["config"] = {"workload": CONFIGS[5].name, "B": 4, "N": 4096, "C": 2240,
+            line["config"] = {"workload": WORKLOADS["w8a8-2048px-b4"].name, "B": 4, "N": 4096, "C": 2240,
                               "H": 70, "parallelism": f"dp{args.gpus}"}
     if args.workload == "mixffn" or (args.workload == "sweep" and not args.no_fused):
         line["mixffn"] = mixffn_measure(args, sla, rank, dev, stream, world, bf16_tf, hbm_gbs,
@@ -528,14 +528,14 @@ def run_ours(args, rank, world, local):
             line["config"] = {"workload": f["workload"], "B": 4, "Hs": 64, "Ws": 64, "C": 2240,
                               "F": 5600, "parallelism": f"dp{args.gpus}"}
     if args.workload == "fused" or (args.workload == "sweep" and not args.no_fused):
-        line["fused"] = fused_measure(args, sla, CONFIGS[4], rank, dev, stream, world, bf16_tf,
+        line["fused"] = fused_measure(args, sla, WORKLOADS["fused-2048px-b4"], rank, dev, stream, world, bf16_tf,
                                       peak_kind)
         if not sets:
             f = line["fused"]
             line.update({"value": f["value"], "ms_per_step": f["ms_per_step"],
                          "roofline": f["roofline"], "gpu_launches": f["gpu_launches"],
                          "clocks": f.get("clocks"), "e2e": f.get("e2e")})
-            line["config"] = {"workload": CONFIGS[4].name, "B": 4, "N": 4096, "C": 2240, "H": 70,
+            line["config"] = {"workload": WORKLOADS["fused-2048px-b4"].name, "B": 4, "N": 4096, "C": 2240, "H": 70,
                               "parallelism": f"dp{args.gpus}"}
 
     if rank == 0 and world == 1 and not args.no_cpu and args.workload == "mixffn":
@@ -543,7 +543,7 @@ def run_ours(args, rank, world, local):
     elif rank == 0 and world == 1 and not args.no_cpu:
         pairs = [(w, x) for w, _, x in sets]
         if not pairs:
-            w = CONFIGS[1]
+            w = WORKLOADS["1024px-b1"]
             pairs = [(w, make_inputs(w))]
         line["cpu_baseline"] = cpu_oracle_sample(pairs)
     if rank == 0:
@@ -831,8 +831,8 @@ def mixffn_measure(args, sla, rank, dev, stream, world, bf16_tf, hbm_gbs, peak_k
     the launches.  The dominant kernel is the expand GEMM, bound by the tensor peak;
     the depthwise conv + GLU is HBM-bound (reads U, writes Hg: 3F x 2 B per token)."""
     import torch
-    from relu_linear_attention_attn_b200.synthetic import MIXFFN_CONFIGS, make_mixffn_inputs
-    w = MIXFFN_CONFIGS[2]
+    from relu_linear_attention_attn_b200.synthetic import MIXFFN_WORKLOADS, make_mixffn_inputs
+    w = MIXFFN_WORKLOADS["mixffn-2048px-b4"]
     x = make_mixffn_inputs(w.scaled(seed=w.seed + 1000 * rank) if rank else w)
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     M = w.tokens
@@ -912,10 +912,10 @@ def profile_case(args):
     import torch
 
     import relu_linear_attention_attn_b200 as sla
-    from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
+    from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs
 
     fused = args.workload in ("fused", "w8a8")
-    w = {"fused": CONFIGS[4], "w8a8": CONFIGS[5]}.get(args.workload) or select(args.workload)[-1]
+    w = {"fused": WORKLOADS["fused-2048px-b4"], "w8a8": WORKLOADS["w8a8-2048px-b4"]}.get(args.workload) or select(args.workload)[-1]
     if args.batch:
         w = w.scaled(B=args.batch)
     x = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in make_inputs(w).items()}

@@ -63,7 +63,7 @@ class Workload:
 # The workloads: a tiny Eq. (1) check, then SANA latents at 1024px, a 2048px
 # batch, a 4K overflow stress with the norm off, the fused path, and the fused
 # path with a W8A8 prologue (same recipe; x and Wqkv are quantised by the op).
-CONFIGS = (
+WORKLOAD_LIST = (
     Workload("tiny-512px-f32", B=1, N=256, C=64, H=2, dtype="f32", recipe="gaussian",
              gains="ones", eps=1e-6, seed=0),
     Workload("1024px-b1", B=1, N=1024, C=2240, H=70, dtype="bf16", recipe="gaussian",
@@ -77,6 +77,7 @@ CONFIGS = (
     Workload("w8a8-2048px-b4", B=4, N=4096, C=2240, H=70, dtype="bf16", recipe="fused",
              gains="random", eps=1e-6, seed=5),
 )
+WORKLOADS = {w.name: w for w in WORKLOAD_LIST}
 
 
 def _store(a: np.ndarray, dtype: str) -> torch.Tensor:
@@ -178,7 +179,7 @@ class MixFFNWorkload:
 
 # A tiny grid, SANA-1.6B's widths (C = 2240, F = 5600) on the 1024px latent grid
 # (32 x 32 tokens), and a 2048px batch of 4 (64 x 64 tokens).
-MIXFFN_CONFIGS = (
+MIXFFN_WORKLOAD_LIST = (
     MixFFNWorkload("mixffn-tiny", B=1, Hs=8, Ws=8, C=64, F=96, gate="sigmoid", bias=True,
                    seed=31),
     MixFFNWorkload("mixffn-1024px-b1", B=1, Hs=32, Ws=32, C=2240, F=5600, gate="sigmoid",
@@ -186,6 +187,7 @@ MIXFFN_CONFIGS = (
     MixFFNWorkload("mixffn-2048px-b4", B=4, Hs=64, Ws=64, C=2240, F=5600, gate="sigmoid",
                    bias=True, seed=33),
 )
+MIXFFN_WORKLOADS = {w.name: w for w in MIXFFN_WORKLOAD_LIST}
 
 
 def make_mixffn_inputs(w: MixFFNWorkload) -> dict:

@@ -35,9 +35,9 @@ def _worker(rank, world, port, outdir):
         sys.path.insert(0, root)
         from oracle import oracle as O
         from relu_linear_attention_attn_b200 import sharding
-        from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
+        from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs
 
-        w = CONFIGS[2].scaled(B=2, N=301, C=128, H=4, seed=91)      # ragged split
+        w = WORKLOADS["2048px-b8-lognormal"].scaled(B=2, N=301, C=128, H=4, seed=91)      # ragged split
         x = make_inputs(w)
         n0, cnt = sharding.token_shard(w.N, rank, world)
         sl = slice(n0, n0 + cnt)
@@ -62,8 +62,8 @@ def results(tmp_path_factory):
 
 def test_sequence_sharded_state_and_output_match_single_process(results):
     from oracle import oracle as O
-    from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
-    w = CONFIGS[2].scaled(B=2, N=301, C=128, H=4, seed=91)
+    from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs
+    w = WORKLOADS["2048px-b8-lognormal"].scaled(B=2, N=301, C=128, H=4, seed=91)
     x = make_inputs(w)
     S_full = O.kv_state(x["k"], x["v"], x["gk"], w.H, w.eps)
     ref = O.forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps)
@@ -98,8 +98,8 @@ MIX_WORLD = 3          # a middle rank exchanges with both neighbours
 
 
 def _mix_case():
-    from relu_linear_attention_attn_b200.synthetic import MIXFFN_CONFIGS
-    return MIXFFN_CONFIGS[0].scaled(B=2, Hs=8, Ws=5, C=16, F=8, gate="silu", seed=92)
+    from relu_linear_attention_attn_b200.synthetic import MIXFFN_WORKLOADS
+    return MIXFFN_WORKLOADS["mixffn-tiny"].scaled(B=2, Hs=8, Ws=5, C=16, F=8, gate="silu", seed=92)
 
 
 def _mix_worker(rank, world, port, outdir):

@@ -49,8 +49,8 @@ def test_quadratic_form(B, N, H, D, norm):
 
 def test_tiny_config_matches_quadratic_form():
     """The whole tiny configuration (B=1, H=2, D=32, N=256, fp32 inputs, g=1)."""
-    from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
-    w = CONFIGS[0]
+    from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs
+    w = WORKLOADS["tiny-512px-f32"]
     x = make_inputs(w)
     got = O.forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps)
     ref = quadratic_form(x["q"].double().numpy(), x["k"].double().numpy(),

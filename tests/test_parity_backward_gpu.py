@@ -16,7 +16,7 @@ import torch
 
 from oracle import oracle as O
 from parity import to_dev, to_np
-from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs, make_output_grad
+from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs, make_output_grad
 
 pytestmark = pytest.mark.gpu
 
@@ -52,19 +52,19 @@ def _check(cuda_lib, w):
                f"{w.name} {name}", dv_scale)
 
 
-@pytest.mark.parametrize("w", [CONFIGS[0], CONFIGS[0].scaled(N=300, gains="random", seed=80),
-                               CONFIGS[1].scaled(N=1, seed=81),
-                               CONFIGS[1].scaled(N=333, seed=82),
-                               CONFIGS[1].scaled(B=2, N=129, gains="off", seed=83),
-                               CONFIGS[1],
-                               CONFIGS[2].scaled(B=2, seed=84)],
+@pytest.mark.parametrize("w", [WORKLOADS["tiny-512px-f32"], WORKLOADS["tiny-512px-f32"].scaled(N=300, gains="random", seed=80),
+                               WORKLOADS["1024px-b1"].scaled(N=1, seed=81),
+                               WORKLOADS["1024px-b1"].scaled(N=333, seed=82),
+                               WORKLOADS["1024px-b1"].scaled(B=2, N=129, gains="off", seed=83),
+                               WORKLOADS["1024px-b1"],
+                               WORKLOADS["2048px-b8-lognormal"].scaled(B=2, seed=84)],
                          ids=lambda w: f"{w.dtype}-B{w.B}-N{w.N}-{w.gains}")
 def test_backward_parity(cuda_lib, w):
     _check(cuda_lib, w)
 
 
 def test_backward_is_deterministic(cuda_lib):
-    w = CONFIGS[1].scaled(B=2, N=1000, seed=85)
+    w = WORKLOADS["1024px-b1"].scaled(B=2, N=1000, seed=85)
     d = to_dev(make_inputs(w))
     do = make_output_grad(w).cuda()
     a = cuda_lib.backward(d["q"], d["k"], d["v"], d["gq"], d["gk"], do, w.H, w.eps)

@@ -9,7 +9,7 @@ import torch
 
 from oracle import oracle as O
 from parity import assert_close, to_dev
-from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
+from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -20,11 +20,11 @@ def run(lib, d, w):
     return out
 
 
-@pytest.mark.parametrize("w", [CONFIGS[0], CONFIGS[0].scaled(N=300, seed=90),
-                               CONFIGS[1].scaled(N=1, seed=91),
-                               CONFIGS[1].scaled(N=333, seed=92),
-                               CONFIGS[1].scaled(B=2, N=129, gains="off", seed=93),
-                               CONFIGS[2].scaled(B=1, N=1000, seed=94)],
+@pytest.mark.parametrize("w", [WORKLOADS["tiny-512px-f32"], WORKLOADS["tiny-512px-f32"].scaled(N=300, seed=90),
+                               WORKLOADS["1024px-b1"].scaled(N=1, seed=91),
+                               WORKLOADS["1024px-b1"].scaled(N=333, seed=92),
+                               WORKLOADS["1024px-b1"].scaled(B=2, N=129, gains="off", seed=93),
+                               WORKLOADS["2048px-b8-lognormal"].scaled(B=1, N=1000, seed=94)],
                          ids=lambda w: f"{w.dtype}-B{w.B}-N{w.N}-{w.gains}")
 def test_causal_small_full_parity(cuda_lib, w):
     x = make_inputs(w)
@@ -33,9 +33,9 @@ def test_causal_small_full_parity(cuda_lib, w):
     assert_close(out, ref, w.dtype, w.name)
 
 
-@pytest.mark.parametrize("idx", [2, 3])
-def test_causal_full_size_parity(cuda_lib, idx):
-    w = CONFIGS[idx]
+@pytest.mark.parametrize("name", ["2048px-b8-lognormal", "4096px-b2-overflow"])
+def test_causal_full_size_parity(cuda_lib, name):
+    w = WORKLOADS[name]
     x = make_inputs(w)
     out = run(cuda_lib, to_dev(x), w)
     ref = O.causal_forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps)
@@ -43,7 +43,7 @@ def test_causal_full_size_parity(cuda_lib, idx):
 
 
 def test_causal_last_token_matches_noncausal_and_is_deterministic(cuda_lib):
-    w = CONFIGS[1].scaled(B=2, N=777, seed=95)
+    w = WORKLOADS["1024px-b1"].scaled(B=2, N=777, seed=95)
     d = to_dev(make_inputs(w))
     a = run(cuda_lib, d, w)
     b = run(cuda_lib, d, w)

@@ -11,7 +11,7 @@ import torch
 import relu_linear_attention_attn_b200 as sla
 from oracle import oracle as O
 from parity import assert_close, errors, sample_tokens, to_dev, to_np
-from relu_linear_attention_attn_b200.synthetic import CONFIGS, Workload, make_inputs
+from relu_linear_attention_attn_b200.synthetic import WORKLOADS, Workload, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -20,9 +20,9 @@ def run_forward(lib, d, w):
     return lib.forward(d["q"], d["k"], d["v"], d["gq"], d["gk"], w.H, w.eps)
 
 
-@pytest.mark.parametrize("idx", [0, 1])
-def test_config_full_parity(cuda_lib, idx):
-    w = CONFIGS[idx]
+@pytest.mark.parametrize("name", ["tiny-512px-f32", "1024px-b1"])
+def test_workload_full_parity(cuda_lib, name):
+    w = WORKLOADS[name]
     x = make_inputs(w)
     out = run_forward(cuda_lib, to_dev(x), w)
     torch.cuda.synchronize()
@@ -30,9 +30,9 @@ def test_config_full_parity(cuda_lib, idx):
     assert_close(out, ref, w.dtype, w.name)
 
 
-@pytest.mark.parametrize("idx", [2, 3])
-def test_config_full_size_sampled_parity(cuda_lib, idx):
-    w = CONFIGS[idx]
+@pytest.mark.parametrize("name", ["2048px-b8-lognormal", "4096px-b2-overflow"])
+def test_workload_full_size_sampled_parity(cuda_lib, name):
+    w = WORKLOADS[name]
     x = make_inputs(w)
     d = to_dev(x)
     out = run_forward(cuda_lib, d, w)
@@ -50,7 +50,7 @@ def test_config_full_size_sampled_parity(cuda_lib, idx):
 
 def test_gains_reading_random_on_lognormal_recipe(cuda_lib):
     """The 2048px recipe under the other reading of its gains (1 + 0.1 N(0,1))."""
-    w = CONFIGS[2].scaled(B=2, N=1500, gains="random", seed=12)
+    w = WORKLOADS["2048px-b8-lognormal"].scaled(B=2, N=1500, gains="random", seed=12)
     x = make_inputs(w)
     out = run_forward(cuda_lib, to_dev(x), w)
     torch.cuda.synchronize()
@@ -84,7 +84,7 @@ def test_fp32_path(cuda_lib, B, N, H):
 
 
 def test_fused_full_size_sampled_parity(cuda_lib):
-    w = CONFIGS[4]
+    w = WORKLOADS["fused-2048px-b4"]
     x = make_inputs(w)
     d = to_dev(x)
     out = cuda_lib.qkv_fused(d["x"], d["W"], d["gq"], d["gk"], w.H, w.eps)
@@ -98,7 +98,7 @@ def test_fused_full_size_sampled_parity(cuda_lib):
 @pytest.mark.parametrize("B,N,gains", [(1, 1, "random"), (1, 300, "random"), (2, 129, "off"),
                                        (1, 1000, "ones")])
 def test_fused_small_full_parity(cuda_lib, B, N, gains):
-    w = CONFIGS[4].scaled(B=B, N=N, gains=gains, seed=40 + N)
+    w = WORKLOADS["fused-2048px-b4"].scaled(B=B, N=N, gains=gains, seed=40 + N)
     x = make_inputs(w)
     d = to_dev(x)
     out = cuda_lib.qkv_fused(d["x"], d["W"], d["gq"], d["gk"], w.H, w.eps)
@@ -108,7 +108,7 @@ def test_fused_small_full_parity(cuda_lib, B, N, gains):
 
 
 def test_apply_with_oracle_state(cuda_lib):
-    w = CONFIGS[1]
+    w = WORKLOADS["1024px-b1"]
     x = make_inputs(w)
     S = O.kv_state(x["k"], x["v"], x["gk"], w.H, w.eps)
     kv = torch.from_numpy(S).float().cuda()
@@ -120,7 +120,7 @@ def test_apply_with_oracle_state(cuda_lib):
 def test_sequence_shards_sum_to_the_whole_state(cuda_lib):
     """States of disjoint token ranges add up to the state of the whole sequence,
     so a sequence-sharded run needs one sum all-reduce of the state."""
-    w = CONFIGS[2].scaled(B=2, N=2000, seed=21)
+    w = WORKLOADS["2048px-b8-lognormal"].scaled(B=2, N=2000, seed=21)
     x = to_dev(make_inputs(w))
     full = cuda_lib.kv_state(x["k"], x["v"], x["gk"], w.H, w.eps)
     a = cuda_lib.kv_state(x["k"][:, :700].contiguous(), x["v"][:, :700].contiguous(), x["gk"],
@@ -133,7 +133,7 @@ def test_sequence_shards_sum_to_the_whole_state(cuda_lib):
 
 
 def test_bitwise_determinism(cuda_lib):
-    w = CONFIGS[2].scaled(B=2, N=3000, seed=22)
+    w = WORKLOADS["2048px-b8-lognormal"].scaled(B=2, N=3000, seed=22)
     d = to_dev(make_inputs(w))
     o1 = run_forward(cuda_lib, d, w)
     o2 = run_forward(cuda_lib, d, w)
@@ -142,7 +142,7 @@ def test_bitwise_determinism(cuda_lib):
 
 
 def test_zero_denominator_row_gives_zero(cuda_lib):
-    w = CONFIGS[1].scaled(N=300, seed=23)
+    w = WORKLOADS["1024px-b1"].scaled(N=300, seed=23)
     x = make_inputs(w)
     x["q"][0, 17] = -x["q"][0, 17].abs() - 0.25     # every head of token 17 is negative
     out = run_forward(cuda_lib, to_dev(x), w)
@@ -152,7 +152,7 @@ def test_zero_denominator_row_gives_zero(cuda_lib):
 
 
 def test_overflow_stress_is_finite_and_exceeds_fp16(cuda_lib):
-    w = CONFIGS[3].scaled(B=1, N=16384, seed=24)
+    w = WORKLOADS["4096px-b2-overflow"].scaled(B=1, N=16384, seed=24)
     d = to_dev(make_inputs(w))
     kv = cuda_lib.kv_state(d["k"], d["v"], None, w.H, w.eps)
     out = run_forward(cuda_lib, d, w)
@@ -164,7 +164,7 @@ def test_overflow_stress_is_finite_and_exceeds_fp16(cuda_lib):
 def test_empty_problems(cuda_lib):
     z = torch.empty((0, 5, 2240), dtype=torch.bfloat16, device="cuda")
     assert run_forward(cuda_lib, dict(q=z, k=z, v=z, gq=None, gk=None),
-                       CONFIGS[3]).numel() == 0
+                       WORKLOADS["4096px-b2-overflow"]).numel() == 0
     e = torch.empty((2, 0, 2240), dtype=torch.bfloat16, device="cuda")
     kv = torch.full((2, 70, 32, 33), 7.0, device="cuda")
     cuda_lib.kv_state(e, e, None, 70, 1e-6, kv=kv)
@@ -174,7 +174,7 @@ def test_empty_problems(cuda_lib):
 
 def test_validation_with_real_buffers(cuda_lib):
     lib = cuda_lib.load()
-    w = CONFIGS[1]
+    w = WORKLOADS["1024px-b1"]
     d = to_dev(make_inputs(w))
     q = d["q"]
     out = torch.empty_like(q)
@@ -211,7 +211,7 @@ def test_bounded_wait_gives_up_and_reports(cuda_lib):
     cuda_lib.selftest_wait_timeout(limit_us=20000)
     torch.cuda.synchronize()
     assert cuda_lib.device_error(clear=True) == (1, 999)
-    w = CONFIGS[1].scaled(N=200, seed=31)
+    w = WORKLOADS["1024px-b1"].scaled(N=200, seed=31)
     x = make_inputs(w)
     out = run_forward(cuda_lib, to_dev(x), w)
     torch.cuda.synchronize()
@@ -230,11 +230,11 @@ def test_wide_head_count_runs_the_cuda_core_path(cuda_lib):
     assert_close(out, O.forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps), "bf16")
 
 
-@pytest.mark.parametrize("idx", [2, 3])
-def test_state_reduction_is_reproducible_at_full_size(cuda_lib, idx):
+@pytest.mark.parametrize("name", ["2048px-b8-lognormal", "4096px-b2-overflow"])
+def test_state_reduction_is_reproducible_at_full_size(cuda_lib, name):
     """Pass 1 at full size, twice: the combine order is fixed, so the states are
     bitwise equal (a race in the ring or the combine would show up here)."""
-    w = CONFIGS[idx]
+    w = WORKLOADS[name]
     d = to_dev(make_inputs(w))
     a = cuda_lib.kv_state(d["k"], d["v"], d["gk"], w.H, w.eps)
     b = cuda_lib.kv_state(d["k"], d["v"], d["gk"], w.H, w.eps)

@@ -18,7 +18,7 @@ import torch
 
 from oracle import oracle as O
 from parity import to_np
-from relu_linear_attention_attn_b200.synthetic import (MIXFFN_CONFIGS, make_dwconv_inputs,
+from relu_linear_attention_attn_b200.synthetic import (MIXFFN_WORKLOADS, make_dwconv_inputs,
                                                        make_gemm_inputs, make_mixffn_inputs)
 
 pytestmark = pytest.mark.gpu
@@ -85,9 +85,9 @@ def _oracle_args(x):
     return (f(x["x"]), f(x["W1"]), f(x["b1"]), f(x["wdw"]), f(x["bdw"]), f(x["W2"]), f(x["b2"]))
 
 
-@pytest.mark.parametrize("w", [MIXFFN_CONFIGS[0], MIXFFN_CONFIGS[0].scaled(Hs=7, Ws=13, gate="silu",
+@pytest.mark.parametrize("w", [MIXFFN_WORKLOADS["mixffn-tiny"], MIXFFN_WORKLOADS["mixffn-tiny"].scaled(Hs=7, Ws=13, gate="silu",
                                                                            bias=False, seed=40),
-                               MIXFFN_CONFIGS[1]], ids=lambda w: f"{w.name}-{w.Hs}x{w.Ws}-{w.gate}")
+                               MIXFFN_WORKLOADS["mixffn-1024px-b1"]], ids=lambda w: f"{w.name}-{w.Hs}x{w.Ws}-{w.gate}")
 def test_mixffn_forward_parity(cuda_lib, w):
     x = make_mixffn_inputs(w)
     d = _dev(x)
@@ -106,7 +106,7 @@ def test_mixffn_forward_parity(cuda_lib, w):
 def test_mixffn_full_size_sampled(cuda_lib):
     """The 2048px batch of 4, in the launch configuration the benchmark times,
     on tokens at the grid's corners, edges and interior of every batch."""
-    w = MIXFFN_CONFIGS[2]
+    w = MIXFFN_WORKLOADS["mixffn-2048px-b4"]
     x = make_mixffn_inputs(w)
     d = _dev(x)
     got = cuda_lib.mixffn_forward(d["x"], d["W1"], d["b1"], d["wdw"], d["bdw"], d["W2"], d["b2"],
@@ -120,7 +120,7 @@ def test_mixffn_full_size_sampled(cuda_lib):
 
 
 def test_mixffn_is_deterministic(cuda_lib):
-    w = MIXFFN_CONFIGS[1]
+    w = MIXFFN_WORKLOADS["mixffn-1024px-b1"]
     d = _dev(make_mixffn_inputs(w))
     a = cuda_lib.mixffn_forward(d["x"], d["W1"], d["b1"], d["wdw"], d["bdw"], d["W2"], d["b2"],
                                 w.Hs, w.Ws, w.gate)
@@ -134,7 +134,7 @@ def test_row_shards_reassemble_the_unsharded_forward(cuda_lib):
     """Three row shards of the 1024px grid (the halo rows copied between them as the
     ranks' exchange would) give the one-call forward bit for bit."""
     from relu_linear_attention_attn_b200 import sharding
-    w = MIXFFN_CONFIGS[1].scaled(Hs=17, seed=41)            # ragged: 5, 6, 6 rows
+    w = MIXFFN_WORKLOADS["mixffn-1024px-b1"].scaled(Hs=17, seed=41)            # ragged: 5, 6, 6 rows
     d = _dev(make_mixffn_inputs(w))
     ref = cuda_lib.mixffn_forward(d["x"], d["W1"], d["b1"], d["wdw"], d["bdw"], d["W2"], d["b2"],
                                   w.Hs, w.Ws, w.gate)

@@ -9,7 +9,7 @@ import torch
 
 from oracle import oracle as O
 from parity import assert_close, sample_tokens
-from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
+from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -25,7 +25,7 @@ def _codes_equal(q_gpu, s_gpu, q_ref, s_ref, what):
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_quantize_rows_bit_exact(cuda_lib, dtype):
-    w = CONFIGS[5].scaled(B=2, N=300, dtype=dtype, seed=51)
+    w = WORKLOADS["w8a8-2048px-b4"].scaled(B=2, N=300, dtype=dtype, seed=51)
     x = make_inputs(w)["x"].clone()
     x[0, 7] = 0                        # an all-zero row: scale 0, codes 0
     x[1, 3] *= 1e-30 if dtype == "f32" else 1.0   # a tiny-magnitude row
@@ -37,7 +37,7 @@ def test_quantize_rows_bit_exact(cuda_lib, dtype):
 
 
 def test_quantize_cols_bit_exact_full_wqkv(cuda_lib):
-    W = make_inputs(CONFIGS[5])["W"]
+    W = make_inputs(WORKLOADS["w8a8-2048px-b4"])["W"]
     q, s = cuda_lib.quantize_cols_i8(W.cuda())
     torch.cuda.synchronize()
     q_ref, s_ref = O.quantize_i8(W.float().numpy(), axis=0)
@@ -62,7 +62,7 @@ def _run(cuda_lib, xq, sx, Wq, sw, x, w):
 @pytest.mark.parametrize("B,N,gains", [(1, 1, "random"), (1, 300, "random"), (2, 129, "off"),
                                        (1, 1000, "ones")])
 def test_w8a8_small_full_parity(cuda_lib, B, N, gains):
-    w = CONFIGS[5].scaled(B=B, N=N, gains=gains, seed=60 + N)
+    w = WORKLOADS["w8a8-2048px-b4"].scaled(B=B, N=N, gains=gains, seed=60 + N)
     x = make_inputs(w)
     xq, sx, Wq, sw = _oracle_codes(x)
     out = _run(cuda_lib, xq, sx, Wq, sw, x, w)
@@ -71,7 +71,7 @@ def test_w8a8_small_full_parity(cuda_lib, B, N, gains):
 
 
 def test_w8a8_full_size_sampled_parity(cuda_lib):
-    w = CONFIGS[5]
+    w = WORKLOADS["w8a8-2048px-b4"]
     x = make_inputs(w)
     xq, sx, Wq, sw = _oracle_codes(x)
     out = _run(cuda_lib, xq, sx, Wq, sw, x, w)
@@ -83,7 +83,7 @@ def test_w8a8_full_size_sampled_parity(cuda_lib):
 
 def test_w8a8_with_gpu_codes_is_deterministic(cuda_lib):
     """The GPU's own quantisation feeding the W8A8 op twice gives identical bits."""
-    w = CONFIGS[5].scaled(B=1, N=1024, seed=77)
+    w = WORKLOADS["w8a8-2048px-b4"].scaled(B=1, N=1024, seed=77)
     x = make_inputs(w)
     xq, sx = cuda_lib.quantize_rows_i8(x["x"].cuda())
     Wq, sw = cuda_lib.quantize_cols_i8(x["W"].cuda())

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 from parity import assert_close, to_dev
-from relu_linear_attention_attn_b200.synthetic import CONFIGS, make_inputs
+from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -30,7 +30,7 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row(cuda_lib):
     lib = cuda_lib.load()
     # two calls in a row, different shapes, so the second one meets the first
     # one's leftovers in the shared scratch
-    for w in (CONFIGS[2].scaled(B=2, N=3000, seed=61), CONFIGS[3].scaled(B=1, N=5000, seed=62)):
+    for w in (WORKLOADS["2048px-b8-lognormal"].scaled(B=2, N=3000, seed=61), WORKLOADS["4096px-b2-overflow"].scaled(B=1, N=5000, seed=62)):
         d = to_dev(make_inputs(w))
         ref = cuda_lib.forward(d["q"], d["k"], d["v"], d["gq"], d["gk"], w.H, w.eps)
         out = torch.empty_like(d["q"])
@@ -41,9 +41,9 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row(cuda_lib):
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda_lib):
     lib = cuda_lib.load()
-    w = CONFIGS[3].scaled(B=64, N=16384)            # needs far more than 16 MiB
+    w = WORKLOADS["4096px-b2-overflow"].scaled(B=64, N=16384)            # needs far more than 16 MiB
     assert cuda_lib.workspace_bytes(w.B, w.N, w.C, w.H) > (16 << 20)
-    small = CONFIGS[1].scaled(N=8)
+    small = WORKLOADS["1024px-b1"].scaled(N=8)
     d = to_dev(make_inputs(small))
     out = torch.empty_like(d["q"])
     assert _noalloc(lib, d, w, out) == ESCRATCH      # rejected before anything is launched
