@@ -104,7 +104,9 @@ SANA_API int sana_linattn_forward_causal(const void* q, const void* k, const voi
  * only the forward; the gradients follow from Eq. (1) and the feature map):
  * given dout = dL/dO (B, N, C), writes dq, dk, dv (B, N, C) in `dtype` and, with
  * the norm on, dgq, dgk = dL/dgq, dL/dgk (fp32 [C]; both NULL with the norm off,
- * when gq = gk = NULL).  Recomputes the forward state itself.  All tensors
+ * when gq = gk = NULL).  Recomputes the forward state itself, the way
+ * sana_linattn_forward forms it (for bf16 with C <= 4096 on the tensor cores,
+ * phi(K) and V as bf16 operands, fp32 sums).  All tensors
  * 16-byte aligned (gains and their gradients 4-byte); outputs must not overlap
  * inputs or each other.  workspace: at least
  * sana_linattn_backward_workspace_bytes(B, N, C, H) bytes.  Sums are formed in a
