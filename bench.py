@@ -34,6 +34,7 @@ if ROOT not in sys.path:
 
 METRIC = "linear-attn Mtokens/s at C=2240, N=1K–16K; % of B200 HBM roofline"
 HBM_FALLBACK_GBS = 6650.0
+HBM_NOMINAL_GBS = 8000.0          # B200 HBM3e nominal (DGX figure), for context
 BF16_FALLBACK_TFLOPS = 1590.0
 # algorithmic bytes per token of each pass (bf16, C = 2240): pass 1 reads k and v,
 # pass 2 reads q and writes out; 17,920 B/token for the whole op
@@ -212,9 +213,21 @@ def cpu_oracle_sample(pairs, budget_s: float = 12.0):
                 break
         if t_total >= budget_s:
             break
+    # the O(N^2) brute force of Eq. (1), on the tiny workload only
+    from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs
+    wt = WORKLOADS["tiny-512px-f32"]
+    xt = make_inputs(wt)
+    reps, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < 0.5:
+        O.quadratic_forward(xt["q"], xt["k"], xt["v"], xt["gq"], xt["gk"], wt.H, wt.eps)
+        reps += 1
+    t_brute = (time.perf_counter() - t0) / reps
     return {"value": tokens / t_total / 1e6, "unit": "Mtokens/s", "cores": O.host_threads(),
             "kind": "oracle", "sample": f"{tokens} tokens ({', '.join(parts)}), fp64 C oracle, "
-                                        f"{t_total:.1f} s"}
+                                        f"{t_total:.1f} s",
+            "brute_force_tiny": {"value": wt.tokens / t_brute / 1e6, "unit": "Mtokens/s",
+                                 "workload": wt.name, "kind": "oracle O(N^2) form",
+                                 "ms_per_call": t_brute * 1e3}}
 
 
 def run_reference(args, rank, world):
@@ -490,7 +503,19 @@ def run_ours(args, rank, world, local):
                                   "sweep_pass_frac": (p1_b if p1_ms >= p2_ms else p2_b) /
                                   ((p1_ms if p1_ms >= p2_ms else p2_ms) * 1e-3) / 1e9 / hbm_gbs,
                                   "sweep_op_frac": 2 * p1_b / ((p1_ms + p2_ms) * 1e-3) / 1e9
-                                  / hbm_gbs},
+                                  / hbm_gbs,
+                                  # the whole op's roof in tokens/s (17,920 B/token per GPU)
+                                  "op_roof_mtok_s": {
+                                      "measured": hbm_gbs * 1e9 / (2 * PASS_BYTES_PER_TOKEN) / 1e6
+                                      * world,
+                                      "nominal_8tbs": HBM_NOMINAL_GBS * 1e9
+                                      / (2 * PASS_BYTES_PER_TOKEN) / 1e6 * world},
+                                  "value_frac_of_op_roof": {
+                                      "measured": value / (hbm_gbs * 1e9 /
+                                                           (2 * PASS_BYTES_PER_TOKEN) / 1e6 * world),
+                                      "nominal_8tbs": value / (HBM_NOMINAL_GBS * 1e9 /
+                                                               (2 * PASS_BYTES_PER_TOKEN) / 1e6 *
+                                                               world)}},
                      "parts": parts,
                      "gpu_launches": args.steps * len(sets) * 2,
                      "per_pass_timing": "a second K-step loop of kv_state (pass 1 + the small "

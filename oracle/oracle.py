@@ -15,6 +15,10 @@ the fused variant (section 7, on-device deployment, of the Sana notes: the
 ReLU(K)^T V reduction fused with the QKV projection), done as an fp64 numpy
 matmul.
 
+``quadratic_forward`` is Eq. (1) in its O(N^2) form, the CPU brute force the
+benchmark times on the tiny workload; it is pinned against ``forward`` and the
+tests' independent quadratic form.
+
 Pins (checked by ``tests/test_oracle_pins.py``): the quadratic form of Eq. (1)
 brute-forced on tiny inputs, hand-derived worked examples in
 ``tests/golden/``, closed forms (N = 1, one-hot keys, constant values),
@@ -216,6 +220,22 @@ def forward(q, k, v, gq, gk, H: int, eps: float, scope: str = "head",
                                     B, N, C, H, float(eps), mode, nthreads or host_threads())
     if rc != 0:
         raise ValueError("oracle_forward_f64 rejected its arguments")
+    return out
+
+
+def quadratic_forward(q, k, v, gq, gk, H: int, eps: float) -> np.ndarray:
+    """Eq. (1) as the O(N^2) sum it reorders: per (b, h), A_ij = phi(Q_i).phi(K_j),
+    O_i = sum_j A_ij V_j / (sum_j A_ij + eps).  Equal to ``forward`` up to rounding
+    (associativity); used as the brute-force CPU timing on small inputs."""
+    pq, pk, vv = phi(q, gq, H, eps), phi(k, gk, H, eps), _f64(v)
+    B, N, C = pq.shape
+    D = C // H
+    out = np.empty_like(vv)
+    for b in range(B):
+        for h in range(H):
+            cols = slice(h * D, (h + 1) * D)
+            A = np.matmul(pq[b, :, cols], pk[b, :, cols].T)
+            out[b, :, cols] = np.matmul(A, vv[b, :, cols]) / (A.sum(axis=1)[:, None] + eps)
     return out
 
 

@@ -305,3 +305,16 @@ def test_fused_projection_matches_brute_force_and_subset():
     tok = np.array([1, 8, 9, 17])
     np.testing.assert_allclose(O.fused_forward(x, W, g, g, H, 1e-6, tokens=tok),
                                got.reshape(B * N, C)[tok], rtol=1e-12)
+
+
+@pytest.mark.parametrize("gains", ["ones", "random", "off"])
+def test_oracle_quadratic_forward_is_eq1(gains):
+    """The oracle's O(N^2) form agrees with its linear form (associativity) and with
+    the tests' independent quadratic form (torch's rms_norm feature map)."""
+    from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs
+    w = WORKLOADS["tiny-512px-f32"].scaled(N=97, gains=gains, seed=44)
+    x = make_inputs(w)
+    q, k, v = (x[n].double().numpy() for n in ("q", "k", "v"))
+    got = O.quadratic_forward(q, k, v, x["gq"], x["gk"], w.H, w.eps)
+    assert rel_err(got, O.forward(q, k, v, x["gq"], x["gk"], w.H, w.eps)) < 1e-12
+    assert rel_err(got, quadratic_form(q, k, v, x["gq"], x["gk"], w.H, w.eps)) < 1e-12
