@@ -228,6 +228,13 @@ SANA_API int sana_linattn_device_error(int* code, int* site, int clear);
  * the context stays usable.  Returns SANA_EINVAL for a limit out of range. */
 SANA_API int sana_linattn_selftest_wait_timeout(int64_t limit_us, cudaStream_t stream);
 
+/* Self-test of the launch-error path: enqueues a launch that the CUDA runtime
+ * rejects before anything reaches the GPU (one block of 2048 threads, above the
+ * per-block limit) and returns the status the library reports for it, SANA_ECUDA,
+ * as every entry point does for a failed launch.  The error is not sticky: the
+ * context stays usable and later calls succeed. */
+SANA_API int sana_linattn_selftest_launch_failure(cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 SANA_API const char* sana_linattn_strerror(int status);
 

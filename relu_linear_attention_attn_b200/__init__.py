@@ -19,7 +19,7 @@ __all__ = ["load", "lib_path", "workspace_bytes", "forward", "forward_noalloc", 
            "qkv_fused_w8a8", "quantize_rows_i8", "quantize_cols_i8", "forward_causal",
            "backward", "gemm_bias", "mixffn_dwconv_glu", "mixffn_workspace_bytes",
            "mixffn_forward", "GATES",
-           "device_error", "selftest_wait_timeout", "SanaError", "STATUS", "BF16", "F32"]
+           "device_error", "selftest_wait_timeout", "selftest_launch_failure", "SanaError", "STATUS", "BF16", "F32"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libsana_linattn.so"
@@ -76,6 +76,8 @@ def _declare(lib):
     lib.sana_linattn_forward_noalloc.restype = ctypes.c_int
     lib.sana_linattn_device_error.argtypes = [ctypes.POINTER(ci), ctypes.POINTER(ci), ci]
     lib.sana_linattn_device_error.restype = ctypes.c_int
+    lib.sana_linattn_selftest_launch_failure.argtypes = [vp]
+    lib.sana_linattn_selftest_launch_failure.restype = ctypes.c_int
     lib.sana_linattn_selftest_wait_timeout.argtypes = [i64, vp]
     lib.sana_linattn_selftest_wait_timeout.restype = ctypes.c_int
     lib.sana_gemm_bias_bf16.argtypes = [vp, vp, fp, vp, i64, ci, ci, vp]
@@ -294,6 +296,12 @@ def device_error(clear: bool = True):
            load().sana_linattn_device_error(ctypes.byref(code), ctypes.byref(site),
                                             1 if clear else 0))
     return code.value, site.value
+
+
+def selftest_launch_failure(stream=None) -> int:
+    """Enqueue a launch the runtime rejects (see include/sana_linattn.h) and return
+    the library's status for it (SANA_ECUDA = -5); raises nothing."""
+    return int(load().sana_linattn_selftest_launch_failure(_stream(stream)))
 
 
 def selftest_wait_timeout(limit_us: int = 20000, stream=None):

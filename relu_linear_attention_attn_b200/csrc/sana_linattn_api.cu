@@ -459,6 +459,9 @@ int noalloc_scratch(void** out) {
     *out = g_noalloc_ptr[dev];
     return SANA_OK;
 }
+// Target of the launch-failure self-test; never runs.
+__global__ void launch_failure_selftest() {}
+
 }  // namespace
 }  // namespace sana
 
@@ -849,6 +852,14 @@ int sana_linattn_forward_noalloc(const void* q, const void* k, const void* v, co
     // has written earlier in the same call, so nothing needs clearing.
     return sana_linattn_forward(q, k, v, gq, gk, out, B, N, C, H, eps, dtype, scratch,
                                 kNoAllocScratchBytes, stream);
+}
+
+int sana_linattn_selftest_launch_failure(cudaStream_t stream) {
+    // 2048 threads in one block is above the per-block limit: the runtime rejects
+    // the launch (nothing reaches the GPU) and the error surfaces like any other
+    // launch failure of the library.
+    launch_failure_selftest<<<1, 2048, 0, stream>>>();
+    return launch_status();
 }
 
 int sana_linattn_selftest_wait_timeout(int64_t limit_us, cudaStream_t stream) {

@@ -62,3 +62,28 @@ def sample_tokens(B: int, N: int, n: int = 512, seed: int = 0) -> np.ndarray:
 
 def to_dev(inp: dict, device="cuda") -> dict:
     return {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+
+
+# ----------------------------------------------------------------------------- guard bands
+CANARY = 0x5A
+
+
+class Guarded:
+    """A buffer of `nbytes` (offset `align`-aligned) inside a larger uint8 buffer whose
+    `guard` bytes on each side hold a canary; `intact()` says whether anything wrote
+    outside the region.  `view(dtype, shape)` is the region as a typed tensor."""
+
+    def __init__(self, nbytes: int, device, guard: int = 4096, align: int = 256):
+        self.nbytes = int(nbytes)
+        self.buf = torch.full((self.nbytes + 2 * guard + align,), CANARY, dtype=torch.uint8,
+                              device=device)
+        base = self.buf.data_ptr()
+        self.off = guard + (-(base + guard)) % align
+        self.region = self.buf[self.off:self.off + self.nbytes]
+
+    def view(self, dtype, shape):
+        return self.region.view(dtype).view(shape)
+
+    def intact(self) -> bool:
+        return bool((self.buf[:self.off] == CANARY).all()) and \
+            bool((self.buf[self.off + self.nbytes:] == CANARY).all())

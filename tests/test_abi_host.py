@@ -293,3 +293,21 @@ def test_mixffn_entry_points_reject_bad_arguments(lib):
     a = list(base)
     a[0] += 2
     assert lib.sana_mixffn_forward(*a) == EALIGN
+
+
+def test_guard_band_helper_detects_writes_outside_the_region():
+    """The canary helper the GPU tests wrap outputs and workspaces in (checked here on
+    CPU tensors)."""
+    from parity import Guarded
+    g = Guarded(1000, "cpu", guard=64, align=256)
+    assert g.region.data_ptr() % 256 == 0 and g.region.numel() == 1000 and g.intact()
+    g.region.fill_(1)
+    assert g.intact()
+    x = g.view(torch.bfloat16, (10, 50))
+    x.fill_(3.0)
+    assert g.intact()
+    g.buf[g.off + 1000] = 0
+    assert not g.intact()
+    h = Guarded(64, "cpu", guard=64, align=256)
+    h.buf[h.off - 1] = 7
+    assert not h.intact()
