@@ -8,6 +8,11 @@ PyTorch fallback: if the shared library is missing, ``load()`` raises.
     import relu_linear_attention_attn_b200 as sla
     out = sla.forward(q, k, v, gq, gk, H=70, eps=1e-6)     # (B, N, C) bf16/fp32
     out = sla.qkv_fused(x, Wqkv, gq, gk, H=70, eps=1e-6)   # bf16
+    out = sla.forward_causal(q, k, v, gq, gk, H=70, eps=1e-6)
+    dq, dk, dv, dgq, dgk = sla.backward(q, k, v, gq, gk, dout, H=70, eps=1e-6)
+    y = sla.mixffn_forward(x, W1, b1, wdw, bdw, W2, b2, Hs=64, Ws=64)   # Mix-FFN tail
+
+The Mix-FFN calls are declared in ``include/sana_mixffn.h``.
 """
 from __future__ import annotations
 
