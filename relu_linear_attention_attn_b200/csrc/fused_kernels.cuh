@@ -323,6 +323,9 @@ fused_kv(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             mbar_arrive(opready);
         }
         if (ok) ok = mbar_wait(kvdone, 0, 509);
+        // Each thread decided `ok` on its own waits; the half-0 threads agree on it
+        // before the named barriers below, so none of them waits at one alone.
+        if (half == 0) ok = named_barrier_and(1, 128, ok);
         if (ok && half == 0) {
             // the CTA's partial state: diagonal blocks of the state accumulator
             tc_fence_after_sync();
@@ -596,17 +599,20 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             *reinterpret_cast<uint4*>(bop + j * kBopBytes + sw128_offset(n, ch)) = w;
         }
         fence_proxy_async_smem();
-        named_barrier_sync(1, 32 * kEpiWarps);             // the states in qo have been read
+        // The states in qo have been read.  Every epilogue thread reaches each named
+        // barrier from here on, and the barriers also settle `ok` (each thread's
+        // waits are bounded on their own), so the threads leave the loop together.
+        ok = named_barrier_and(1, 32 * kEpiWarps, ok);
         mbar_arrive(bready);
 
         for (int ti = 0; ti < nt && ok; ++ti) {
             const int ab = ti & 1;
-            ok = mbar_wait(&accfull[ab], (uint32_t)(ti >> 1) & 1, 609);
-            if (!ok) break;
-            tc_fence_after_sync();
+            bool wok = mbar_wait(&accfull[ab], (uint32_t)(ti >> 1) & 1, 609);
             // the previous tile's O store must have read the staging buffer
             if (et == 0) bulk_wait_group_read<0>();
-            named_barrier_sync(1, 32 * kEpiWarps);
+            ok = named_barrier_and(1, 32 * kEpiWarps, wok);
+            if (!ok) break;
+            tc_fence_after_sync();
             const bool row_live = (t0 + ti) * fz::kTileTok + row < a.N;
             const float sxr = (kI8 && row_live)
                 ? a.sx[(int64_t)b * a.N + (t0 + ti) * fz::kTileTok + row] : 0.f;
@@ -659,11 +665,10 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             fence_proxy_async_smem();
             mbar_arrive(opready);
             // O = r D[:, :32] / (r D[:, 32] + eps), written over the A' operand
-            ok = mbar_wait(ddone, (uint32_t)ti & 1, 610);
-            if (!ok) break;
+            wok = mbar_wait(ddone, (uint32_t)ti & 1, 610);
             tc_fence_after_sync();
 #pragma unroll 1
-            for (int j = 2 * half; j < 2 * half + 2; ++j) {
+            for (int j = 2 * half; j < 2 * half + 2 && wok; ++j) {
                 float v[kD + 1];
                 tmem_ld16(lane_base + kDCol + j * kN, v);
                 tmem_ld16(lane_base + kDCol + j * kN + 16, v + 16);
@@ -683,8 +688,8 @@ fused_qo(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUt
             }
             tc_fence_before_sync();
             fence_proxy_async_smem();
-            named_barrier_sync(1, 32 * kEpiWarps);
-            if (et == 0) {
+            ok = named_barrier_and(1, 32 * kEpiWarps, wok);
+            if (ok && et == 0) {
                 const int y = (t0 + ti) * fz::kTileTok;
                 tma_store_3d(&tmap_o, qo, g * 128, y, b);
                 if (g * 128 + 64 < a.C)                       // no store that starts past C

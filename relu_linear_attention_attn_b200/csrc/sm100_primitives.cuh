@@ -113,6 +113,23 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Named barrier that also returns the AND of `pred` over the participating
+// threads, so a group whose members each decided on their own (a bounded wait
+// that gave up in some threads and not in others) leaves the barrier agreeing.
+// Every participant must reach it, whatever its own pred.
+__device__ __forceinline__ bool named_barrier_and(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.b32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
 // ------------------------------------------------------------------ dependent launch
 // Programmatic dependent launch: the primary grid allows its dependent grid to be
 // scheduled; the dependent grid waits for the primary grid's completion (and the
