@@ -130,6 +130,27 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- distributed
+def spawn_ranks_if_needed(args):
+    """`--gpus N` with N > 1 runs one process per GPU.  Started without a launcher
+    (no WORLD_SIZE in the environment), the script re-executes itself under
+    torch.distributed.run with N ranks on this node; started by a launcher, the
+    launcher's world size must equal N."""
+    world = os.environ.get("WORLD_SIZE")
+    if world is None:
+        if args.gpus > 1:
+            import socket
+            with socket.socket() as s:
+                s.bind(("127.0.0.1", 0))
+                port = s.getsockname()[1]
+            cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                   f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+                   "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+            os.execv(sys.executable, cmd)
+        return
+    if int(world) != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but the launcher started {world} ranks")
+
+
 def dist_setup(args):
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -138,6 +159,9 @@ def dist_setup(args):
     if world > 1:
         import datetime
         import torch.distributed as dist
+        # NCCL reports its communicator (rank count, transport) at init
+        os.environ.setdefault("NCCL_DEBUG", "INFO")
+        os.environ.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
@@ -280,7 +304,7 @@ def run_reference(args, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_block(args, wl),
+            "config": config_block(args, wl, world),
             "cpu_baseline": {"value": value, "unit": "Mtokens/s", "cores": O.host_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "Mtokens/s", "h2d_bytes_per_step": 0,
@@ -341,7 +365,7 @@ def run_reference_mixffn(args, O):
     print(json.dumps(line), flush=True)
 
 
-def config_block(args, wl):
+def config_block(args, wl, world=1):
     return {"workload": "sana-latent-sweep-N1K-16K" if args.workload == "sweep" else
             args.workload,
             "parts": [{"name": w.name, "B": w.B, "N": w.N, "C": w.C, "H": w.H, "D": w.D,
@@ -349,7 +373,7 @@ def config_block(args, wl):
             "global_batch_tokens": sum(w.tokens for w in wl),
             "l2": "inputs larger than L2: one step streams >1.1 GB, so each workload's "
                   "inputs are evicted before they are used again",
-            "parallelism": f"dp{args.gpus} (batch-sharded, no collective)"}
+            "parallelism": f"dp{world} (batch-sharded, no collective)"}
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -394,7 +418,7 @@ def run_ours(args, rank, world, local):
     line = {"metric": METRIC, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_block(args, wl)}
+            "config": config_block(args, wl, world)}
 
     def fwd_step():
         for w, d, _ in sets:
@@ -523,6 +547,8 @@ def run_ours(args, rank, world, local):
                                         "state), CUDA events between the passes",
                      "clocks": clk.summary()})
 
+        if world == 1 and rank == 0 and not args.no_cpu and args.workload == "sweep":
+            line["configs"] = configs_measure(args, sla, sets, dev, hbm_gbs, bf16_tf, peak_kind)
         if not args.no_fused:
             line["causal"] = causal_measure(args, sla, sets, stream, world, hbm_gbs)
             line["backward"] = backward_measure(args, sla, sets, stream, world, hbm_gbs)
@@ -540,7 +566,7 @@ def run_ours(args, rank, world, local):
                          "roofline": f["roofline"], "gpu_launches": f["gpu_launches"],
                          "clocks": f.get("clocks")})
             line["config"] = {"workload": WORKLOADS["w8a8-2048px-b4"].name, "B": 4, "N": 4096, "C": 2240,
-                              "H": 70, "parallelism": f"dp{args.gpus}"}
+                              "H": 70, "parallelism": f"dp{world}"}
     if args.workload == "mixffn" or (args.workload == "sweep" and not args.no_fused):
         line["mixffn"] = mixffn_measure(args, sla, rank, dev, stream, world, bf16_tf, hbm_gbs,
                                         peak_kind)
@@ -551,7 +577,7 @@ def run_ours(args, rank, world, local):
                          "gpu_launches": f["gpu_launches"], "clocks": f.get("clocks"),
                          "e2e": f["e2e"]})
             line["config"] = {"workload": f["workload"], "B": 4, "Hs": 64, "Ws": 64, "C": 2240,
-                              "F": 5600, "parallelism": f"dp{args.gpus}"}
+                              "F": 5600, "parallelism": f"dp{world}"}
     if args.workload == "fused" or (args.workload == "sweep" and not args.no_fused):
         line["fused"] = fused_measure(args, sla, WORKLOADS["fused-2048px-b4"], rank, dev, stream, world, bf16_tf,
                                       peak_kind)
@@ -561,7 +587,7 @@ def run_ours(args, rank, world, local):
                          "roofline": f["roofline"], "gpu_launches": f["gpu_launches"],
                          "clocks": f.get("clocks"), "e2e": f.get("e2e")})
             line["config"] = {"workload": WORKLOADS["fused-2048px-b4"].name, "B": 4, "N": 4096, "C": 2240, "H": 70,
-                              "parallelism": f"dp{args.gpus}"}
+                              "parallelism": f"dp{world}"}
 
     if rank == 0 and world == 1 and not args.no_cpu and args.workload == "mixffn":
         line["cpu_baseline"] = mixffn_cpu_sample()
@@ -573,6 +599,132 @@ def run_ours(args, rank, world, local):
         line["cpu_baseline"] = cpu_oracle_sample(pairs)
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def graph_call_ms(body, steps: int) -> float:
+    """Device time per call of `body`, recorded `steps` times into one CUDA graph
+    (median of 5 replays after 2 warm-up replays)."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        body()
+        side.synchronize()
+        with torch.cuda.graph(g, stream=side):
+            for _ in range(steps):
+                body()
+    torch.cuda.synchronize()
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) / steps)
+    del g
+    return statistics.median(ts)
+
+
+def configs_measure(args, sla, sets, dev, hbm_gbs, bf16_tf, peak_kind):
+    """One record per named workload of the metric's configurations: the tiny fp32
+    check, the three SANA latent sizes and the fused-QKV 2048px batch of 4.
+
+    time: the op alone, `steps` calls in one CUDA graph, each call preceded by a
+    read of a 512 MB buffer that evicts the op's inputs from L2 (a cold L2 for every
+    call); the flush's own time, measured the same way, is subtracted.
+    cpu_baseline + parity: the fp64 oracle, as it stands, on a bounded sample of
+    the workload (batch item 0 of the attention workloads; 256 sampled tokens of
+    batch item 0 for the fused one, whose state still needs all of that item's
+    tokens), timed on the host cores; the GPU output of the same tokens is
+    compared with the oracle's (max-abs, mean-abs, normwise relative L2)."""
+    import numpy as np
+    import torch
+    from oracle import oracle as O
+    from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs
+
+    steps = max(3, min(args.steps, 20))
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    sink = torch.empty(1, dtype=torch.int64, device=dev)
+
+    def do_flush():
+        torch.sum(flush.view(torch.int64), dim=0, keepdim=True, out=sink)
+    t_flush = graph_call_ms(do_flush, steps)
+
+    def errs(got, ref):
+        g = np.asarray(got, dtype=np.float64)
+        d = np.abs(g - ref)
+        return {"max_abs": float(d.max()), "mean_abs": float(d.mean()),
+                "rel_l2": float(np.linalg.norm(g - ref) / max(np.linalg.norm(ref), 1e-300)),
+                "finite": bool(np.isfinite(g).all())}
+
+    recs = {}
+    # the tiny fp32 check and the three latent sizes
+    tiny = WORKLOADS["tiny-512px-f32"]
+    xt = make_inputs(tiny)
+    dt = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in xt.items()}
+    dt["out"] = torch.empty_like(dt["q"])
+    dt["ws"] = torch.empty(sla.workspace_bytes(tiny.B, tiny.N, tiny.C, tiny.H), dtype=torch.uint8,
+                           device=dev)
+    for w, d, x in [(tiny, dt, xt)] + [(w, d, x) for w, d, x in sets]:
+        def call(w=w, d=d):
+            sla.forward(d["q"], d["k"], d["v"], d["gq"], d["gk"], w.H, w.eps, out=d["out"],
+                        workspace=d["ws"])
+        ms = graph_call_ms(lambda: (do_flush(), call()), steps) - t_flush
+        call()
+        torch.cuda.synchronize()
+        got = d["out"][:1].float().cpu().numpy()
+        t0 = time.perf_counter()
+        ref = O.forward(x["q"][:1], x["k"][:1], x["v"][:1], x["gq"], x["gk"], w.H, w.eps)
+        t_cpu = time.perf_counter() - t0
+        by = w.tokens * (2 * w.C * (4 if w.dtype == "f32" else 2) * 2)
+        rec = {"B": w.B, "N": w.N, "C": w.C, "H": w.H, "dtype": w.dtype, "us": ms * 1e3,
+               "Mtokens_per_s": w.tokens / (ms * 1e-3) / 1e6,
+               "parity_vs_oracle": errs(got, ref) | {"sample": "batch item 0, every token"},
+               "cpu_oracle": {"Mtokens_per_s": w.N / t_cpu / 1e6, "cores": O.host_threads(),
+                              "sample": "batch item 0"}}
+        if w.dtype == "bf16":
+            rec["hbm_frac"] = {"measured": by / (ms * 1e-3) / 1e9 / hbm_gbs,
+                               "nominal_8tbs": by / (ms * 1e-3) / 1e9 / HBM_NOMINAL_GBS}
+        recs[w.name] = rec
+    del dt
+    # the fused QKV variant
+    wf = WORKLOADS["fused-2048px-b4"]
+    xf = make_inputs(wf)
+    df = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in xf.items()}
+    of = torch.empty_like(df["x"])
+    wsf = torch.empty(sla.workspace_bytes(wf.B, wf.N, wf.C, wf.H, fused=True), dtype=torch.uint8,
+                      device=dev)
+
+    def fcall():
+        sla.qkv_fused(df["x"], df["W"], df["gq"], df["gk"], wf.H, wf.eps, out=of, workspace=wsf)
+    ms = graph_call_ms(lambda: (do_flush(), fcall()), steps) - t_flush
+    fcall()
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(0)
+    tok = np.sort(rng.choice(wf.N, size=256, replace=False))
+    got = of[0].float().cpu().numpy()[tok]
+    t0 = time.perf_counter()
+    ref = O.fused_forward(xf["x"][:1], xf["W"], xf["gq"], xf["gk"], wf.H, wf.eps, tokens=tok)
+    t_cpu = time.perf_counter() - t0
+    fl = 2.0 * wf.tokens * wf.C * 3 * wf.C
+    recs[wf.name] = {"B": wf.B, "N": wf.N, "C": wf.C, "H": wf.H, "dtype": "bf16", "us": ms * 1e3,
+                     "Mtokens_per_s": wf.tokens / (ms * 1e-3) / 1e6,
+                     "tflops": fl / (ms * 1e-3) / 1e12,
+                     "tensor_frac": {"of": f"{peak_kind} bf16 burst", "value":
+                                     fl / (ms * 1e-3) / 1e12 / bf16_tf},
+                     "parity_vs_oracle": errs(got, ref.reshape(len(tok), wf.C)) |
+                     {"sample": "256 sampled tokens of batch item 0"},
+                     "cpu_oracle": {"Mtokens_per_s": len(tok) / t_cpu / 1e6,
+                                    "cores": O.host_threads(),
+                                    "sample": "256 tokens of batch item 0 (with the K, V "
+                                              "projection of all its 4096 tokens)"}}
+    return {"timing": f"{steps} calls in one CUDA graph, each after a 512 MB read that "
+                      "evicts L2; the read's own time subtracted", "workloads": recs}
 
 
 def e2e_measure(args, sla, sets, stream, world):
@@ -984,6 +1136,7 @@ def main():
         return
     if args.warmup < 3:
         args.warmup = 3
+    spawn_ranks_if_needed(args)
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -162,12 +162,16 @@ def _stream(stream) -> int:
     return s.cuda_stream
 
 
-def _workspace(nbytes: int, device, workspace):
+def _workspace(nbytes: int, device, workspace, stream=None):
     torch = _torch()
     if nbytes == 0:
         return None, 0
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        # the library runs on `stream`: keep the caching allocator from handing this
+        # block to other work on the current stream before that stream's use of it ends
+        if stream is not None and stream != torch.cuda.current_stream(device):
+            workspace.record_stream(stream)
     if workspace.numel() * workspace.element_size() < nbytes:
         raise ValueError(f"workspace needs {nbytes} bytes")
     return workspace, workspace.numel() * workspace.element_size()
@@ -182,7 +186,7 @@ def forward(q, k, v, gq, gk, H: int, eps: float, out=None, workspace=None, strea
     dt = _dtype_code(q)
     if out is None:
         out = _torch().empty_like(q)
-    ws, wsb = _workspace(workspace_bytes(B, N, C, H), q.device, workspace)
+    ws, wsb = _workspace(workspace_bytes(B, N, C, H), q.device, workspace, stream)
     rc = load().sana_linattn_forward(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _gain(gq, "gq"),
                                      _gain(gk, "gk"), _dev(out, "out"), B, N, C, H, float(eps), dt,
                                      None if ws is None else ws.data_ptr(), wsb, _stream(stream))
@@ -217,7 +221,7 @@ def backward(q, k, v, gq, gk, dout, H: int, eps: float, grads=None, workspace=No
             dgq = torch.empty(C, dtype=torch.float32, device=q.device)
             dgk = torch.empty(C, dtype=torch.float32, device=q.device)
     ws, wsb = _workspace(int(load().sana_linattn_backward_workspace_bytes(B, N, C, H)), q.device,
-                         workspace)
+                         workspace, stream)
     rc = load().sana_linattn_backward(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _gain(gq, "gq"),
                                       _gain(gk, "gk"), _dev(dout, "dout"), _dev(dq, "dq"),
                                       _dev(dk, "dk"), _dev(dv, "dv"), _dev(dgq, "dgq"),
@@ -237,7 +241,7 @@ def forward_causal(q, k, v, gq, gk, H: int, eps: float, out=None, workspace=None
     if out is None:
         out = _torch().empty_like(q)
     ws, wsb = _workspace(int(load().sana_linattn_workspace_bytes(B, N, C, H, 2)), q.device,
-                         workspace)
+                         workspace, stream)
     rc = load().sana_linattn_forward_causal(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
                                             _gain(gq, "gq"), _gain(gk, "gk"), _dev(out, "out"),
                                             B, N, C, H, float(eps), dt,
@@ -273,7 +277,7 @@ def kv_state(k, v, gk, H: int, eps: float, kv=None, workspace=None, stream=None)
     dt = _dtype_code(k)
     if kv is None:
         kv = torch.empty((B, H, D, D + 1), dtype=torch.float32, device=k.device)
-    ws, wsb = _workspace(workspace_bytes(B, N, C, H), k.device, workspace)
+    ws, wsb = _workspace(workspace_bytes(B, N, C, H), k.device, workspace, stream)
     rc = load().sana_linattn_kv_state(_dev(k, "k"), _dev(v, "v"), _gain(gk, "gk"), _dev(kv, "kv"),
                                       B, N, C, H, float(eps), dt,
                                       None if ws is None else ws.data_ptr(), wsb, _stream(stream))
@@ -360,7 +364,7 @@ def qkv_fused_w8a8(xq, sx, Wq, sw, gq, gk, H: int, eps: float, out=None, workspa
         raise ValueError("shapes: xq (B, N, C), sx (B, N), Wq (C, 3C), sw (3C,)")
     if out is None:
         out = torch.empty((B, N, C), dtype=torch.bfloat16, device=xq.device)
-    ws, wsb = _workspace(workspace_bytes(B, N, C, H, fused=True), xq.device, workspace)
+    ws, wsb = _workspace(workspace_bytes(B, N, C, H, fused=True), xq.device, workspace, stream)
     rc = load().sana_linattn_qkv_fused_w8a8(_dev(xq, "xq"), _dev(sx, "sx"), _dev(Wq, "Wq"),
                                             _dev(sw, "sw"), _gain(gq, "gq"), _gain(gk, "gk"),
                                             _dev(out, "out"), B, N, C, H, float(eps),
@@ -380,7 +384,7 @@ def qkv_fused(x, W, gq, gk, H: int, eps: float, out=None, workspace=None, stream
         raise ValueError("Wqkv must be (C, 3C)")
     if out is None:
         out = torch.empty_like(x)
-    ws, wsb = _workspace(workspace_bytes(B, N, C, H, fused=True), x.device, workspace)
+    ws, wsb = _workspace(workspace_bytes(B, N, C, H, fused=True), x.device, workspace, stream)
     rc = load().sana_linattn_qkv_fused(_dev(x, "x"), _dev(W, "Wqkv"), _gain(gq, "gq"),
                                        _gain(gk, "gk"), _dev(out, "out"), B, N, C, H, float(eps),
                                        None if ws is None else ws.data_ptr(), wsb,
@@ -455,7 +459,7 @@ def mixffn_forward(x, W1, b1, wdw, bdw, W2, b2, Hs: int, Ws: int, gate: str = "s
         raise ValueError("wdw must be (2F, 3, 3)")
     if out is None:
         out = _torch().empty_like(x)
-    ws, wsb = _workspace(mixffn_workspace_bytes(B, Hs, Ws, C, F), x.device, workspace)
+    ws, wsb = _workspace(mixffn_workspace_bytes(B, Hs, Ws, C, F), x.device, workspace, stream)
     rc = load().sana_mixffn_forward(_bf16(x, "x"), _bf16(W1, "W1"), _gain(b1, "b1"),
                                     _gain(wdw, "wdw"), _gain(bdw, "bdw"), _bf16(W2, "W2"),
                                     _gain(b2, "b2"), _bf16(out, "out"), B, Hs, Ws, C, F,

@@ -36,8 +36,12 @@ def token_shard(N: int, rank: int, world: int) -> tuple[int, int]:
 
 
 def allreduce_state(kv, group=None):
-    """Sum the ranks' partial states in place (one all-reduce of the fp32 state)."""
+    """Sum the ranks' partial states in place (one all-reduce of the fp32 state).
+    A single process (no process group, or a group of one) holds the whole state
+    already and returns it unchanged."""
     import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size(group) == 1:
+        return kv
     dist.all_reduce(kv, op=dist.ReduceOp.SUM, group=group)
     return kv
 
@@ -53,14 +57,26 @@ def max_over_ranks(x: float, device=None, group=None) -> float:
     return float(t.item())
 
 
+def _on_stream(stream):
+    """Make `stream` the current stream for the block (no-op for None), so the
+    library's launches, torch's own work and the collectives, which order
+    themselves after the current stream, all run in one order."""
+    import contextlib
+
+    import torch
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+
+
 def sequence_parallel_forward(q, k, v, gq, gk, H: int, eps: float, group=None, stream=None):
     """Eq. (1) over a sequence split across ranks.  q, k, v hold this rank's token
     range (B, N_r, C) on its GPU; returns this rank's output rows.  The state of
-    the whole sequence is the all-reduced sum of the ranks' states."""
+    the whole sequence is the all-reduced sum of the ranks' states.  Everything
+    runs on `stream` (default: the current stream), the all-reduce included."""
     import relu_linear_attention_attn_b200 as sla
-    kv = sla.kv_state(k, v, gk, H, eps, stream=stream)
-    allreduce_state(kv, group=group)
-    return sla.apply(q, gq, kv, H, eps, stream=stream)
+    with _on_stream(stream):
+        kv = sla.kv_state(k, v, gk, H, eps)
+        allreduce_state(kv, group=group)
+        return sla.apply(q, gq, kv, H, eps)
 
 
 # ----------------------------------------------------------------------------- Mix-FFN
@@ -113,9 +129,10 @@ def mixffn_shard_expand(x_r, W1, b1, Ws: int, stream=None):
     if rows * Ws != Nr:
         raise ValueError("x_r must hold whole grid rows")
     F2 = W1.shape[1]
-    U = torch.zeros(B, rows + 2, Ws, F2, dtype=x_r.dtype, device=x_r.device)
-    for b in range(B):
-        sla.gemm_bias(x_r[b], W1, b1, out=U[b, 1:rows + 1].view(rows * Ws, F2), stream=stream)
+    with _on_stream(stream):
+        U = torch.zeros(B, rows + 2, Ws, F2, dtype=x_r.dtype, device=x_r.device)
+        for b in range(B):
+            sla.gemm_bias(x_r[b], W1, b1, out=U[b, 1:rows + 1].view(rows * Ws, F2))
     return U
 
 
@@ -128,13 +145,14 @@ def mixffn_shard_finish(U, top, bottom, wdw, bdw, W2, b2, Ws: int, gate: str = "
     import relu_linear_attention_attn_b200 as sla
     B, rows2, _, F2 = U.shape
     rows, F, C = rows2 - 2, F2 // 2, W2.shape[1]
-    U[:, 0].copy_(top)
-    U[:, rows + 1].copy_(bottom)
-    Hg = sla.mixffn_dwconv_glu(U.view(B, rows2 * Ws, F2), wdw, bdw, rows2, Ws, gate,
-                               stream=stream).view(B, rows2, Ws, F)
-    y = torch.empty(B, rows * Ws, C, dtype=U.dtype, device=U.device)
-    for b in range(B):
-        sla.gemm_bias(Hg[b, 1:rows + 1].reshape(rows * Ws, F), W2, b2, out=y[b], stream=stream)
+    with _on_stream(stream):
+        U[:, 0].copy_(top)
+        U[:, rows + 1].copy_(bottom)
+        Hg = sla.mixffn_dwconv_glu(U.view(B, rows2 * Ws, F2), wdw, bdw, rows2, Ws,
+                                   gate).view(B, rows2, Ws, F)
+        y = torch.empty(B, rows * Ws, C, dtype=U.dtype, device=U.device)
+        for b in range(B):
+            sla.gemm_bias(Hg[b, 1:rows + 1].reshape(rows * Ws, F), W2, b2, out=y[b])
     return y
 
 
@@ -144,6 +162,7 @@ def sequence_parallel_mixffn(x_r, W1, b1, wdw, bdw, W2, b2, Ws: int, rank: int, 
     rows (B, rows * Ws, C) on its GPU; returns this rank's output rows."""
     U = mixffn_shard_expand(x_r, W1, b1, Ws, stream=stream)
     rows = U.shape[1] - 2
-    top, bottom = exchange_halo_rows(U[:, 1].contiguous(), U[:, rows].contiguous(), rank, world,
-                                     group=group)
+    with _on_stream(stream):
+        top, bottom = exchange_halo_rows(U[:, 1].contiguous(), U[:, rows].contiguous(), rank,
+                                         world, group=group)
     return mixffn_shard_finish(U, top, bottom, wdw, bdw, W2, b2, Ws, gate, stream=stream)
