@@ -78,7 +78,9 @@ SANA_API size_t sana_linattn_workspace_bytes(int64_t B, int64_t N, int C, int H,
 /* Eq. (1) end to end on projected q, k, v.
  * q, k, v, out: (B, N, C) in `dtype`.  gq, gk: fp32 [C] or both NULL.
  * workspace: at least sana_linattn_workspace_bytes(B, N, C, H, 0) bytes; its
- * contents on entry do not matter and are garbage on exit. */
+ * contents on entry do not matter and are garbage on exit.
+ * bf16 with C <= 4096 runs on the tensor cores as two persistent passes (the
+ * state, then its application); fp32 and wider problems run CUDA-core kernels. */
 SANA_API int sana_linattn_forward(const void* q, const void* k, const void* v,
                          const float* gq, const float* gk, void* out,
                          int64_t B, int64_t N, int C, int H, float eps,
@@ -202,8 +204,11 @@ SANA_API int sana_quantize_cols_i8(const void* w, sana_dtype dtype, int8_t* wq,
  *     exceeds 16 MiB return SANA_ESCRATCH; 2048px B=8 and 4096px B=2 at
  *     C = 2240 fit.
  *   - The first call on a device looks up the array's device address with the
- *     device current (cudaGetSymbolAddress); make that first call before any
- *     stream capture.
+ *     device current (cudaGetSymbolAddress) and keeps it for the life of the
+ *     process; make that first call before any stream capture.  The kept
+ *     address, like the library's other per-device set-up, does not survive
+ *     cudaDeviceReset or the teardown of the device's primary context: do not
+ *     call the library across one.
  *   - Every call shares the one array and leaves its contents behind; the
  *     forward path writes every scratch byte before reading it, so stale
  *     contents never matter.  Calls that overlap on the GPU (different streams,

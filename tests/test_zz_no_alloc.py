@@ -8,6 +8,7 @@ every other test; it also passes alone in a fresh process."""
 import pytest
 import torch
 
+from oracle import oracle as O
 from parity import assert_close, to_dev
 from relu_linear_attention_attn_b200.synthetic import WORKLOADS, make_inputs
 
@@ -21,22 +22,33 @@ def _noalloc(lib, d, w, out):
     s = torch.cuda.current_stream().cuda_stream
     gq = d["gq"].data_ptr() if d["gq"] is not None else None
     gk = d["gk"].data_ptr() if d["gk"] is not None else None
+    dt = 0 if w.dtype == "bf16" else 1
     return lib.sana_linattn_forward_noalloc(d["q"].data_ptr(), d["k"].data_ptr(),
                                             d["v"].data_ptr(), gq, gk, out.data_ptr(), w.B, w.N,
-                                            w.C, w.H, w.eps, 0, s)
+                                            w.C, w.H, w.eps, dt, s)
 
 
 def test_noalloc_matches_forward_on_two_calls_in_a_row(cuda_lib):
+    """Calls in a row on different shapes, so each one meets the one before's
+    leftovers in the shared scratch: the bf16 tensor-core path twice, then the
+    fp32 CUDA-core path (which also uses the scratch's state region and a
+    different split plan).  The no-allocation call runs the same kernels with the
+    same fixed plan as sana_linattn_forward, so the two agree bit for bit; each
+    is also checked against the fp64 oracle."""
     lib = cuda_lib.load()
-    # two calls in a row, different shapes, so the second one meets the first
-    # one's leftovers in the shared scratch
-    for w in (WORKLOADS["2048px-b8-lognormal"].scaled(B=2, N=3000, seed=61), WORKLOADS["4096px-b2-overflow"].scaled(B=1, N=5000, seed=62)):
-        d = to_dev(make_inputs(w))
+    cases = (WORKLOADS["2048px-b8-lognormal"].scaled(B=2, N=3000, seed=61),
+             WORKLOADS["4096px-b2-overflow"].scaled(B=1, N=5000, seed=62),
+             WORKLOADS["tiny-512px-f32"].scaled(seed=63))
+    for w in cases:
+        x = make_inputs(w)
+        d = to_dev(x)
         ref = cuda_lib.forward(d["q"], d["k"], d["v"], d["gq"], d["gk"], w.H, w.eps)
         out = torch.empty_like(d["q"])
         assert _noalloc(lib, d, w, out) == 0
         torch.cuda.synchronize()
-        assert_close(out, ref, "bf16", f"noalloc vs forward {w.name}")
+        assert torch.equal(out, ref), f"noalloc differs from forward on {w.name}"
+        assert_close(out, O.forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps),
+                     w.dtype, f"noalloc vs oracle {w.name}")
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda_lib):
