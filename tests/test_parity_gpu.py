@@ -73,6 +73,32 @@ def test_ragged_shapes_full_parity(cuda_lib, recipe, gains, B, N):
                  w.name)
 
 
+@pytest.mark.parametrize("B,N,H,recipe,gains", [
+    (1, 1, 70, "gaussian", "random"), (1, 64, 70, "lognormal", "ones"),
+    (1, 129, 70, "overflow", "off"), (1, 1000, 70, "gaussian", "random"),
+    (1, 1024, 70, "overflow", "off"), (2, 384, 6, "gaussian", "random"),
+    (1, 500, 5, "lognormal", "random"), (3, 256, 70, "gaussian", "ones")])
+def test_short_sequences_full_parity(cuda_lib, B, N, H, recipe, gains):
+    """Short sequences (N <= 1024, few work items per CTA, many partial slots per
+    row): ragged token counts and head counts that leave a head group or a head
+    pair partly or wholly empty; the one-call forward and the split kv_state +
+    apply both match the oracle, and the forward is reproducible bit for bit."""
+    w = Workload(f"short-{B}x{N}-h{H}", B=B, N=N, C=32 * H, H=H, dtype="bf16", recipe=recipe,
+                 gains=gains, eps=1e-6, seed=300 + 7 * B + N + H)
+    x = make_inputs(w)
+    d = to_dev(x)
+    out = run_forward(cuda_lib, d, w)
+    kv = cuda_lib.kv_state(d["k"], d["v"], d["gk"], w.H, w.eps)
+    two_pass = cuda_lib.apply(d["q"], d["gq"], kv, w.H, w.eps)
+    torch.cuda.synchronize()
+    ref = O.forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps)
+    assert_close(out, ref, "bf16", w.name)
+    assert_close(two_pass, ref, "bf16", w.name + " two-pass")
+    again = run_forward(cuda_lib, d, w)
+    torch.cuda.synchronize()
+    assert torch.equal(out, again), "short-sequence path is not reproducible"
+
+
 @pytest.mark.parametrize("B,N,H", [(1, 1, 2), (2, 300, 2), (1, 1000, 5), (1, 4096, 70)])
 def test_fp32_path(cuda_lib, B, N, H):
     w = Workload("f32", B=B, N=N, C=32 * H, H=H, dtype="f32", recipe="gaussian", gains="random",
