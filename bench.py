@@ -377,6 +377,64 @@ def config_block(args, wl, world=1):
 
 
 # ----------------------------------------------------------------------------- our arm
+def run_seq_shard(args, sla, rank, world, dev, stream, hbm_gbs):
+    """--shard seq: every workload's sequence split over the ranks; each step runs
+    sharding.sequence_parallel_forward (per-rank state of its token range through
+    sana_linattn_kv_state, one fp32 sum all-reduce of the state over NCCL, then
+    sana_linattn_apply on the rank's own queries).  The whole job processes each
+    workload once per step, so value = all tokens / step time (strong scaling)."""
+    import torch
+
+    from relu_linear_attention_attn_b200 import sharding
+    from relu_linear_attention_attn_b200.synthetic import make_inputs
+    wl = select(args.workload)
+    sets = []
+    for w in wl:
+        x = make_inputs(w)
+        n0, cnt = sharding.token_shard(w.N, rank, world)
+        d = {n: x[n][:, n0:n0 + cnt].contiguous().to(dev) for n in ("q", "k", "v")}
+        d["gq"] = None if x["gq"] is None else x["gq"].to(dev)
+        d["gk"] = None if x["gk"] is None else x["gk"].to(dev)
+        sets.append((w, d))
+
+    def step():
+        for w, d in sets:
+            sharding.sequence_parallel_forward(d["q"], d["k"], d["v"], d["gq"], d["gk"], w.H,
+                                               w.eps)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b), world) / args.steps
+    tokens = sum(w.tokens for w in wl)
+    value = tokens / (ms * 1e-3) / 1e6
+    state_bytes = sum(w.B * w.H * w.D * (w.D + 1) * 4 for w in wl)
+    line = {"metric": METRIC, "value": value, "unit": "Mtokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config_block(args, wl, world) |
+            {"parallelism": f"sp{world} (sequence-sharded: per-rank state, one fp32 sum "
+                            f"all-reduce of {state_bytes} B per step, per-rank apply)"},
+            "launch": "eager sequence_parallel_forward calls (NCCL all-reduce between the passes)",
+            "roofline": {"bound": "hbm", "achieved": tokens * 2 * PASS_BYTES_PER_TOKEN / world /
+                         (ms * 1e-3) / 1e9, "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": tokens * 2 * PASS_BYTES_PER_TOKEN / world / (ms * 1e-3) / 1e9 /
+                         hbm_gbs, "traffic": None,
+                         "kernel": "the whole op per rank (its token share of q, k, v, out)"},
+            "gpu_launches": args.steps * len(wl) * 3, "clocks": clk.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, rank, world, local):
     import torch
 
@@ -387,6 +445,10 @@ def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = measured_peaks()
+    if args.shard == "seq":
+        if args.workload not in ("sweep", "1024px", "2048px", "4096px"):
+            raise SystemExit("--shard seq applies to the attention workloads")
+        return run_seq_shard(args, sla, rank, world, dev, stream, hbm_gbs)
     wl = select(args.workload) if args.workload not in ("fused", "w8a8", "mixffn") else []
 
     # inputs resident in HBM; each rank works on its own batch (weak scaling)
@@ -1130,6 +1192,10 @@ def main():
                          "fixed launch sequence for ncu captures)")
     ap.add_argument("--batch", type=int, default=0,
                     help="with --profile-case: batch size override for the workload")
+    ap.add_argument("--shard", choices=["batch", "seq"], default="batch",
+                    help="batch: every rank runs its own batch (weak scaling, no collective); "
+                         "seq: the ranks split each sequence and all-reduce the state "
+                         "(sharding.sequence_parallel_forward; strong scaling)")
     args = ap.parse_args()
     if args.profile_case:
         profile_case(args)

@@ -11,8 +11,9 @@
 // U and Hg are stored in bf16; every sum accumulates in fp32.
 //
 // gemm_bias_bf16: D[M][Nc] = A[M][K] W[K][Nc] (+ bias) on the sm_100a tensor cores.
-//   Persistent: CTA c takes tiles c, c + grid, ... of 128 rows x 256 columns, the
-//   column tile fastest, so concurrent CTAs share A rows through L2.  Warp 0 is
+//   Persistent: CTA c takes tiles c, c + grid, ... of 128 rows x 256 columns, in
+//   groups of 8 row blocks with the row block fastest inside a group, so concurrent
+//   CTAs share A rows and a band of W columns through L2.  Warp 0 is
 //   the TMA producer (4-stage ring of A 128 x 64 k, K-major, and W 64 k x 256 n,
 //   MN-major, both 128-byte swizzled), warp 1 issues 128x256x16 UMMAs into one
 //   of two TMEM accumulators, warps 2-9 drain the other (bias, bf16, stores), so
@@ -68,6 +69,20 @@ struct GemmArgs {
     int mb, nb;          // tiles along M and along Nc
 };
 
+// Tile t -> (row block, column block).  Tiles go in groups of kGroupRows row blocks;
+// within a group the row block is fastest, so the CTAs running at once share a few
+// A row blocks and a band of W columns, and each W column block is used by the
+// group's row blocks back to back (it stays in L2 across the group even while the
+// output stream passes through, instead of being re-read from DRAM per row block).
+constexpr int kGroupRows = 8;
+__device__ __forceinline__ void gemm_tile(int64_t t, const GemmArgs& a, int& mblk, int& nblk) {
+    const int64_t per_group = (int64_t)kGroupRows * a.nb;
+    const int64_t grp = t / per_group, local = t % per_group;
+    const int rows = (int)min((int64_t)kGroupRows, a.mb - grp * kGroupRows);
+    nblk = (int)(local / rows);
+    mblk = (int)(grp * kGroupRows + local % rows);
+}
+
 __global__ void __launch_bounds__(gm::kThreads, 1)
 gemm_bias_bf16(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
                const GemmArgs a)
@@ -118,8 +133,10 @@ gemm_bias_bf16(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
         if (lane == 0) {
             int64_t step = 0, last = -1;
             for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-                const int m0 = (int)(t / a.nb) * kBM;
-                const int n0 = (int)(t % a.nb) * kBN;
+                int mblk, nblk;
+                gemm_tile(t, a, mblk, nblk);
+                const int m0 = mblk * kBM;
+                const int n0 = nblk * kBN;
                 for (int kk = 0; kk < ksteps; ++kk, ++step) {
                     const int st = (int)(step % kStages);
                     if (step >= kStages)
@@ -188,8 +205,10 @@ gemm_bias_bf16(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
             ok = mbar_wait(&accfull[buf], (uint32_t)(lt >> 1) & 1, 606);
             if (!ok) break;
             tc_fence_after_sync();
-            const int64_t row = (t / a.nb) * kBM + 32 * q + lane;
-            const int n0 = (int)(t % a.nb) * kBN;
+            int mblk, nblk;
+            gemm_tile(t, a, mblk, nblk);
+            const int64_t row = (int64_t)mblk * kBM + 32 * q + lane;
+            const int n0 = nblk * kBN;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 const int col = half * 128 + c * 32;

@@ -50,6 +50,23 @@
 
 namespace sana {
 
+// x[i] = ReLU(g[i] * x[i] * r) (kScaleByRms) or ReLU(g[i] * x[i]) for one head's 32
+// values, the gains read from shared memory eight at a time as 16-byte loads (g
+// must be 16-byte aligned: the gain arrays start 1024-byte aligned and a head's
+// gains are 128 bytes apart).
+template <bool kScaleByRms>
+__device__ __forceinline__ void scale_relu32(float* x, const float* g, float r) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const float4 v = reinterpret_cast<const float4*>(g)[c];
+        const float gv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            x[4 * c + u] = kScaleByRms ? fmaxf(gv[u] * (x[4 * c + u] * r), 0.f)
+                                       : fmaxf(gv[u] * x[4 * c + u], 0.f);
+    }
+}
+
 // The feature map on 32 values held as 4 swizzled 16-byte chunks of row `row`,
 // starting at chunk `chunk0`, rewritten in place as bf16.  g points at the
 // head's 32 gains in shared memory (ignored with the norm off).
@@ -86,13 +103,7 @@ __device__ __forceinline__ float phi_inplace_sw128(uint8_t* tile, int row, int c
             s3 = fmaf(x[i + 3], x[i + 3], s3);
         }
         r = rsqrtf(((s0 + s1) + (s2 + s3)) * (1.f / kD) + eps);
-        if (kScaleByRms) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] = fmaxf(g[i] * (x[i] * r), 0.f);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] = fmaxf(g[i] * x[i], 0.f);
-        }
+        scale_relu32<kScaleByRms>(x, g, r);
     } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[i] = zero ? 0.f : fmaxf(x[i], 0.f);
@@ -150,14 +161,7 @@ __device__ __forceinline__ void phi2_inplace_sw128(uint8_t* const tile[2], const
                 s3 = fmaf(x[i + 3], x[i + 3], s3);
             }
             r = rsqrtf(((s0 + s1) + (s2 + s3)) * (1.f / kD) + eps);
-            const float* gi = g[it];
-            if (kScaleByRms) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = fmaxf(gi[i] * (x[i] * r), 0.f);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = fmaxf(gi[i] * x[i], 0.f);
-            }
+            scale_relu32<kScaleByRms>(x, g[it], r);
         } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) x[i] = zero[it] ? 0.f : fmaxf(x[i], 0.f);
