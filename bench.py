@@ -508,6 +508,7 @@ def run_ours(args, rank, world, local):
         torch.cuda.synchronize()
         eager_ms = max_over_ranks(t_start.elapsed_time(t_end), world) / args.steps
         graph = None
+        graph_ms = None          # the workloads on concurrent streams
         if not args.eager:
             side = torch.cuda.Stream()
             side.wait_stream(stream)
@@ -519,6 +520,27 @@ def run_ours(args, rank, world, local):
             torch.cuda.synchronize()
             graph.replay()
             torch.cuda.synchronize()
+            if len(sets) > 1 and args.concurrency == "streams":
+                # The workloads are independent problems: each gets a stream that
+                # runs its K forward calls back to back; the graph forks from and
+                # joins to the capture stream, so the persistent kernels of one
+                # workload fill the SMs another's leave idle in its tail.
+                wstreams = [torch.cuda.Stream() for _ in sets]
+                graph_ms = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(side):
+                    with torch.cuda.graph(graph_ms, stream=side):
+                        for ws_ in wstreams:
+                            ws_.wait_stream(side)
+                        for ws_, (w, d, _) in zip(wstreams, sets):
+                            with torch.cuda.stream(ws_):
+                                for _ in range(args.steps):
+                                    sla.forward(d["q"], d["k"], d["v"], d["gq"], d["gk"], w.H,
+                                                w.eps, out=d["out"], workspace=d["ws"])
+                        for ws_ in wstreams:
+                            side.wait_stream(ws_)
+                torch.cuda.synchronize()
+                graph_ms.replay()
+                torch.cuda.synchronize()
         with ClockSampler(local) as clk:
             # keep the GPU busy for ~0.3 s inside the sampling window (untimed), so the
             # clock samples see the clocks the timed steps run at
@@ -540,6 +562,16 @@ def run_ours(args, rank, world, local):
             t_end.record(stream)
             torch.cuda.synchronize()
             barrier(world)
+            if graph_ms is not None:
+                t_s2 = torch.cuda.Event(enable_timing=True)
+                t_e2 = torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                barrier(world)
+                t_s2.record(stream)
+                graph_ms.replay()
+                t_e2.record(stream)
+                torch.cuda.synchronize()
+                barrier(world)
         # (2) per-pass durations for the roofline: the same K steps as kv_state +
         # apply (the two halves of sana_linattn_forward), events between the passes.
         barrier(world)
@@ -547,8 +579,10 @@ def run_ours(args, rank, world, local):
         for s_ in range(args.steps):
             step(ev[s_])
         torch.cuda.synchronize()
-        elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
-        ms_per_step = elapsed_ms / args.steps
+        one_stream_ms = max_over_ranks(t_start.elapsed_time(t_end), world) / args.steps
+        ms_per_step = one_stream_ms
+        if graph_ms is not None:
+            ms_per_step = max_over_ranks(t_s2.elapsed_time(t_e2), world) / args.steps
         value = tokens_per_step * world / (ms_per_step * 1e-3) / 1e6
         # per-pass durations (average per launch) and algorithmic bytes
         parts = []
@@ -576,7 +610,11 @@ def run_ours(args, rank, world, local):
         achieved = bytes_big / (ms_big * 1e-3) / 1e9
         line.update({"value": value, "ms_per_step": ms_per_step,
                      "launch": ("eager sana_linattn_forward calls" if graph is None else
-                                "one CUDA graph of the K steps of sana_linattn_forward calls"),
+                                "one CUDA graph of the K steps of sana_linattn_forward calls" +
+                                (", each workload on its own stream (independent problems "
+                                 "run concurrently; the graph forks and joins once)"
+                                 if graph_ms is not None else ", one stream")),
+                     "value_one_stream": tokens_per_step * world / (one_stream_ms * 1e-3) / 1e6,
                      "eager_value": tokens_per_step * world / (eager_ms * 1e-3) / 1e6,
                      "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs,
                                   "unit": "GB/s", "frac": achieved / hbm_gbs,
@@ -1192,6 +1230,9 @@ def main():
                          "fixed launch sequence for ncu captures)")
     ap.add_argument("--batch", type=int, default=0,
                     help="with --profile-case: batch size override for the workload")
+    ap.add_argument("--concurrency", choices=["streams", "serial"], default="streams",
+                    help="sweep: run the workloads on one stream each (independent problems "
+                         "overlapping on the SMs) or all on one stream")
     ap.add_argument("--shard", choices=["batch", "seq"], default="batch",
                     help="batch: every rank runs its own batch (weak scaling, no collective); "
                          "seq: the ranks split each sequence and all-reduce the state "

@@ -266,3 +266,30 @@ def test_state_reduction_is_reproducible_at_full_size(cuda_lib, name):
     b = cuda_lib.kv_state(d["k"], d["v"], d["gk"], w.H, w.eps)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def test_independent_problems_on_concurrent_streams(cuda_lib):
+    """Forward calls on different streams share the GPU (the persistent passes of
+    one fill SMs another leaves idle); each result equals the same call run alone,
+    bit for bit."""
+    cases = [WORKLOADS["1024px-b1"].scaled(N=700, seed=111),
+             WORKLOADS["2048px-b8-lognormal"].scaled(B=2, N=2500, seed=112),
+             WORKLOADS["4096px-b2-overflow"].scaled(B=1, N=6000, seed=113)]
+    data = [to_dev(make_inputs(w)) for w in cases]
+    alone = []
+    for w, d in zip(cases, data):
+        alone.append(run_forward(cuda_lib, d, w))
+        torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in cases]
+    outs = [torch.empty_like(d["q"]) for d in data]
+    for _ in range(3):
+        for s in streams:
+            s.wait_stream(torch.cuda.current_stream())
+        for s, w, d, o in zip(streams, cases, data, outs):
+            with torch.cuda.stream(s):
+                cuda_lib.forward(d["q"], d["k"], d["v"], d["gq"], d["gk"], w.H, w.eps, out=o)
+        for s in streams:
+            torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    for w, a, o in zip(cases, alone, outs):
+        assert torch.equal(a, o), w.name
