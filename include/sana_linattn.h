@@ -133,6 +133,25 @@ SANA_API int sana_linattn_kv_state(const void* k, const void* v, const float* gk
                           sana_dtype dtype, void* workspace, size_t ws_bytes,
                           cudaStream_t stream);
 
+/* The two passes of sana_linattn_forward as separate calls; issued one after
+ * the other on the same stream they are exactly the forward (same kernels, same
+ * plan, bit-identical output), and other work may be enqueued between them.
+ *   sana_linattn_forward_pass1: the split-N partial states of phi(K)^T [V | 1]
+ *     (one per contiguous token range of every (b, h), a fixed function of B, N, H
+ *     and the device) into `workspace`.
+ *   sana_linattn_forward_pass2: sums each (b, h)'s partials in range order and
+ *     applies the state to q, writing out.  Reads the partials pass 1 wrote into
+ *     the same workspace for the same (B, N, C, H, eps, gains) on the same device.
+ * bf16 with C <= 4096 only (the tensor-core path; SANA_EUNSUPPORTED otherwise).
+ * workspace: at least sana_linattn_workspace_bytes(B, N, C, H, 0) bytes; not
+ * touched by anything else between the two calls. */
+SANA_API int sana_linattn_forward_pass1(const void* k, const void* v, const float* gk,
+                                        int64_t B, int64_t N, int C, int H, float eps,
+                                        void* workspace, size_t ws_bytes, cudaStream_t stream);
+SANA_API int sana_linattn_forward_pass2(const void* q, const float* gq, void* out,
+                                        int64_t B, int64_t N, int C, int H, float eps,
+                                        void* workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* The query half of Eq. (1) with a given state:
  * out = phi(Q) kv[:, :D] / (phi(Q) kv[:, D] + eps).
  * q, out: (B, N, C) in `dtype`; kv: (B, H, D, D+1) fp32; gq: fp32 [C] or NULL

@@ -20,7 +20,7 @@ import ctypes
 import os
 import threading
 
-__all__ = ["load", "lib_path", "workspace_bytes", "forward", "forward_noalloc", "kv_state", "apply", "qkv_fused",
+__all__ = ["load", "lib_path", "workspace_bytes", "forward", "forward_noalloc", "forward_pass1", "forward_pass2", "kv_state", "apply", "qkv_fused",
            "qkv_fused_w8a8", "quantize_rows_i8", "quantize_cols_i8", "forward_causal",
            "backward", "gemm_bias", "mixffn_dwconv_glu", "mixffn_workspace_bytes",
            "mixffn_forward", "GATES",
@@ -57,6 +57,10 @@ def _declare(lib):
                                          vp]
     lib.sana_linattn_kv_state.argtypes = [vp, vp, fp, fp, i64, i64, ci, ci, cf, ci, vp, sz, vp]
     lib.sana_linattn_apply.argtypes = [vp, fp, fp, vp, i64, i64, ci, ci, cf, ci, vp]
+    lib.sana_linattn_forward_pass1.argtypes = [vp, vp, fp, i64, i64, ci, ci, cf, vp, sz, vp]
+    lib.sana_linattn_forward_pass2.argtypes = [vp, fp, vp, i64, i64, ci, ci, cf, vp, sz, vp]
+    lib.sana_linattn_forward_pass1.restype = ctypes.c_int
+    lib.sana_linattn_forward_pass2.restype = ctypes.c_int
     lib.sana_linattn_qkv_fused.argtypes = [vp, vp, fp, fp, vp, i64, i64, ci, ci, cf, vp, sz, vp]
     for f in (lib.sana_linattn_forward, lib.sana_linattn_kv_state, lib.sana_linattn_apply,
               lib.sana_linattn_qkv_fused):
@@ -266,6 +270,38 @@ def forward_noalloc(q, k, v, gq, gk, H: int, eps: float, out=None, stream=None):
                                              _gain(gq, "gq"), _gain(gk, "gk"), _dev(out, "out"),
                                              B, N, C, H, float(eps), dt, _stream(stream))
     _check("sana_linattn_forward_noalloc", rc)
+    return out
+
+
+def forward_pass1(k, v, gk, H: int, eps: float, workspace, stream=None):
+    """The forward's first pass alone: the split-N partial states into `workspace`
+    (uint8, at least workspace_bytes(B, N, C, H)).  bf16 only."""
+    B, N, C = k.shape
+    if v.shape != k.shape or v.dtype != k.dtype:
+        raise ValueError("k, v must share shape and dtype")
+    if _dtype_code(k) != BF16:
+        raise TypeError("the forward's passes run on bf16 inputs")
+    ws, wsb = _workspace(workspace_bytes(B, N, C, H), k.device, workspace, stream)
+    rc = load().sana_linattn_forward_pass1(_dev(k, "k"), _dev(v, "v"), _gain(gk, "gk"), B, N, C,
+                                           H, float(eps), None if ws is None else ws.data_ptr(),
+                                           wsb, _stream(stream))
+    _check("sana_linattn_forward_pass1", rc)
+    return ws
+
+
+def forward_pass2(q, gq, H: int, eps: float, workspace, out=None, stream=None):
+    """The forward's second pass alone, from the partial states forward_pass1 left
+    in `workspace` for the same shapes."""
+    B, N, C = q.shape
+    if _dtype_code(q) != BF16:
+        raise TypeError("the forward's passes run on bf16 inputs")
+    if out is None:
+        out = _torch().empty_like(q)
+    wsb = workspace.numel() * workspace.element_size()
+    rc = load().sana_linattn_forward_pass2(_dev(q, "q"), _gain(gq, "gq"), _dev(out, "out"), B, N,
+                                           C, H, float(eps), workspace.data_ptr(), wsb,
+                                           _stream(stream))
+    _check("sana_linattn_forward_pass2", rc)
     return out
 
 

@@ -17,6 +17,7 @@
 #include "causal_kernels.cuh"
 #include "backward_kernels.cuh"
 #include "mixffn_kernels.cuh"
+#include "causal_tc_kernels.cuh"
 
 namespace sana {
 namespace {
@@ -262,8 +263,10 @@ int persistent_ctas() {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         sms <= 0)
         return 0;
-    if (cudaFuncSetAttribute(kv_partials_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             p1::kSmemBytes) != cudaSuccess ||
+    if (cudaFuncSetAttribute(kv_partials_persistent<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, p1::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(kv_partials_persistent<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, p1::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(apply_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              p2::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(fused_kv<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -273,12 +276,14 @@ int persistent_ctas() {
         cudaFuncSetAttribute(fused_kv<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              f1::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(fused_qo<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             f2::kSmemBytes) != cudaSuccess)
+                             f2::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(causal_apply_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ca::kSmemBytes) != cudaSuccess)
         return 0;
     // each persistent kernel must fit one CTA on an SM (registers, threads, smem)
     int n1 = 0, n2 = 0, n3 = 0, n4 = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, kv_partials_persistent, p1::kThreads,
-                                                      p1::kSmemBytes) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, kv_partials_persistent<false>,
+                                                      p1::kThreads, p1::kSmemBytes) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n2, apply_persistent, p2::kThreads,
                                                       p2::kSmemBytes) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n3, fused_kv<false>, f1::kThreads,
@@ -329,12 +334,12 @@ int launch_partials_tc(const void* k, const void* v, const float* gk, float* par
         return SANA_ECUDA;
     const PersistPlan1 pl = make_plan_p1(B, N, H, P);
     P1Args a{};
-    a.gk = gk; a.part = part; a.T = pl.T;
+    a.gk = gk; a.part = part; a.T = pl.T; a.Cc = 1;
     a.N = (int)N; a.H = H; a.G = pl.G; a.R = pl.R; a.Smax = pl.Smax; a.P = pl.P;
     a.eps = eps; a.norm = gk != nullptr;
     if (plan_out) *plan_out = pl;
-    return launch_pdl(kv_partials_persistent, dim3(pl.P), p1::kThreads, p1::kSmemBytes, st, true,
-                      tk, tv, a);
+    return launch_pdl(kv_partials_persistent<false>, dim3(pl.P), p1::kThreads, p1::kSmemBytes, st,
+                      true, tk, tv, a);
 }
 
 // The final states kv [B][H][D][D+1] from pass-1 partials (right behind pass 1).
@@ -367,6 +372,49 @@ int launch_apply_tc(const void* q, const float* gq, const float* kv, const float
     }
     return launch_pdl(apply_persistent, dim3(pl.P), p2::kThreads, p2::kSmemBytes, st,
                       kv == nullptr, tq, to, a);
+}
+
+// The prefix (causal) form on the tensor cores (bf16): pass 1 with one row per
+// 128-token chunk (the chunks' partial states), the exclusive prefix over chunks,
+// then the chunked apply.  Workspace: [partials B*H*Cc*2 states][prefix B*H*Cc].
+int launch_causal_tc(const void* q, const void* k, const void* v, const float* gq,
+                     const float* gk, void* out, int64_t B, int64_t N, int C, int H, float eps,
+                     void* workspace, cudaStream_t st) {
+    const int P = persistent_ctas();
+    if (P == 0) return SANA_ECUDA;
+    const int64_t Cc = (N + kCausalTcChunk - 1) / kCausalTcChunk;
+    constexpr int kR = kCausalTcChunk / p1::kStageTok;      // pass-1 stages per chunk
+    const int G = (H + p1::kGroupHeads - 1) / p1::kGroupHeads;
+    const int64_t T1 = B * G * Cc * kR;
+    if (B * (int64_t)H * Cc > 0x7fffffffLL || T1 > ((int64_t)1 << 40)) return SANA_EUNSUPPORTED;
+    const int64_t cap = (T1 + kMinItemsPerCta - 1) / kMinItemsPerCta;
+    const int P1 = (int)(cap < P ? cap : P);
+    float* part = (float*)workspace;
+    float* pre = (float*)((char*)workspace +
+                          align_up((size_t)B * H * Cc * 2 * kStateFloats * sizeof(float), 256));
+    CUtensorMap tk, tv;
+    if (!make_tmap_bnc(&tk, k, B, N, C, kP1StageTok) || !make_tmap_bnc(&tv, v, B, N, C, kP1StageTok))
+        return SANA_ECUDA;
+    P1Args a1{};
+    a1.gk = gk; a1.part = part; a1.T = T1; a1.N = (int)N; a1.H = H; a1.G = G; a1.R = kR;
+    a1.Smax = 2; a1.P = P1; a1.eps = eps; a1.norm = gk != nullptr; a1.Cc = (int)Cc;
+    int rc = launch_pdl(kv_partials_persistent<true>, dim3(P1), p1::kThreads, p1::kSmemBytes, st,
+                        false, tk, tv, a1);
+    if (rc != SANA_OK) return rc;
+    PrefixArgs ap{};
+    ap.part = part; ap.pre = pre; ap.H = H; ap.G = G; ap.Cc = (int)Cc; ap.Smax = 2;
+    ap.R1 = kR; ap.T1 = T1; ap.P1 = P1;
+    causal_prefix_states<<<(unsigned)(B * H), kStateFloats / 4, 0, st>>>(ap);
+    CUtensorMap tq, tk2, tv2, to;
+    if (!make_tmap_bnc(&tq, q, B, N, C, ca::kTok) || !make_tmap_bnc(&tk2, k, B, N, C, ca::kTok) ||
+        !make_tmap_bnc(&tv2, v, B, N, C, ca::kTok) || !make_tmap_bnc(&to, out, B, N, C, ca::kTok))
+        return SANA_ECUDA;
+    CaArgs a3{};
+    a3.pre = pre; a3.gq = gq; a3.gk = gk; a3.N = (int)N; a3.H = H;
+    a3.Pp = (H + 1) / 2; a3.Cc = (int)Cc; a3.T = B * a3.Pp * Cc;
+    a3.P = (int)(a3.T < P ? a3.T : P); a3.eps = eps; a3.norm = gq != nullptr;
+    causal_apply_tc<<<a3.P, ca::kThreads, ca::kSmemBytes, st>>>(tq, tk2, tv2, to, a3);
+    return launch_status();
 }
 
 // The fused variant: F1 (K, V projection + state), then F2 (Q projection + apply)
@@ -471,9 +519,14 @@ extern "C" {
 
 size_t sana_linattn_workspace_bytes(int64_t B, int64_t N, int C, int H, int fused) {
     if (check_dims(B, N, C, H) != SANA_OK || B == 0 || N == 0) return 0;
-    if (fused == 2) {        // the prefix form: one state per chunk of every (b, h)
+    if (fused == 2) {        // the prefix form: states per chunk of every (b, h)
+        // CUDA-core path: one state per 64-token chunk; tensor-core path: up to two
+        // partial slots and the prefix per 128-token chunk
         const int64_t S = (N + kCausalChunk - 1) / kCausalChunk;
-        return align_up((size_t)B * H * S * kStateFloats * sizeof(float), 256);
+        const size_t simt = align_up((size_t)B * H * S * kStateFloats * sizeof(float), 256);
+        const int64_t Cc = (N + kCausalTcChunk - 1) / kCausalTcChunk;
+        const size_t tc = 2 * align_up((size_t)B * H * Cc * 2 * kStateFloats * sizeof(float), 256);
+        return simt > tc ? simt : tc;
     }
     return ws_layout(B, N, C, H, fused != 0).total;
 }
@@ -599,6 +652,8 @@ int sana_linattn_forward_causal(const void* q, const void* k, const void* v, con
     float* part = (float*)workspace;
     const dim3 g1((unsigned)S, H, (unsigned)B);
     const int norm = gk != nullptr;
+    if (tc_path(dtype, C) && (!norm || (aligned(gq, 16) && aligned(gk, 16))))
+        return launch_causal_tc(q, k, v, gq, gk, out, B, N, C, H, eps, workspace, stream);
     if (dtype == SANA_BF16) {
         kv_partial_simt<bf16><<<g1, 128, 0, stream>>>((const bf16*)k, (const bf16*)v, gk, part, N,
                                                       H, C, C, (int)S, kCausalChunk, eps, norm);
@@ -736,6 +791,54 @@ int sana_linattn_forward(const void* q, const void* k, const void* v, const floa
         launch_apply<float, float>((const float*)q, gq, kv, (float*)out, B, N, H, C, C, eps,
                                    stream);
     }
+    return launch_status();
+}
+
+int sana_linattn_forward_pass1(const void* k, const void* v, const float* gk, int64_t B,
+                               int64_t N, int C, int H, float eps, void* workspace,
+                               size_t ws_bytes, cudaStream_t stream) {
+    int rc;
+    if ((rc = check_dims(B, N, C, H)) != SANA_OK) return rc;
+    if ((rc = check_eps(eps)) != SANA_OK) return rc;
+    if (gk && !aligned(gk, 4)) return SANA_EALIGN;
+    if (!tc_path(SANA_BF16, C)) return SANA_EUNSUPPORTED;
+    if (B == 0 || N == 0) return SANA_OK;
+    if (!k || !v) return SANA_EINVAL;
+    if (!aligned(k, 16) || !aligned(v, 16)) return SANA_EALIGN;
+    const WsLayout L = ws_layout(B, N, C, H, false);
+    if ((rc = validate_ws(workspace, ws_bytes, L.total)) != SANA_OK) return rc;
+    const size_t bytes = (size_t)B * N * C * 2;
+    if (overlaps(workspace, L.total, k, bytes) || overlaps(workspace, L.total, v, bytes))
+        return SANA_EINVAL;
+    float* part = (float*)((char*)workspace + L.part_off);
+    if ((rc = launch_partials_tc(k, v, gk, part, B, N, C, H, eps, stream, nullptr)) != SANA_OK)
+        return rc;
+    return launch_status();
+}
+
+int sana_linattn_forward_pass2(const void* q, const float* gq, void* out, int64_t B, int64_t N,
+                               int C, int H, float eps, void* workspace, size_t ws_bytes,
+                               cudaStream_t stream) {
+    int rc;
+    if ((rc = check_dims(B, N, C, H)) != SANA_OK) return rc;
+    if ((rc = check_eps(eps)) != SANA_OK) return rc;
+    if (gq && !aligned(gq, 4)) return SANA_EALIGN;
+    if (!tc_path(SANA_BF16, C)) return SANA_EUNSUPPORTED;
+    if (B == 0 || N == 0) return SANA_OK;
+    if (!q || !out) return SANA_EINVAL;
+    if (!aligned(q, 16) || !aligned(out, 16)) return SANA_EALIGN;
+    const WsLayout L = ws_layout(B, N, C, H, false);
+    if ((rc = validate_ws(workspace, ws_bytes, L.total)) != SANA_OK) return rc;
+    const size_t bytes = (size_t)B * N * C * 2;
+    if (overlaps(out, bytes, q, bytes) || overlaps(workspace, L.total, q, bytes) ||
+        overlaps(workspace, L.total, out, bytes))
+        return SANA_EINVAL;
+    const int P = persistent_ctas();
+    if (P == 0) return SANA_ECUDA;
+    const PersistPlan1 pl = make_plan_p1(B, N, H, P);     // the plan pass 1 used
+    float* part = (float*)((char*)workspace + L.part_off);
+    if ((rc = launch_apply_tc(q, gq, nullptr, part, &pl, out, B, N, C, H, eps, stream)) != SANA_OK)
+        return rc;
     return launch_status();
 }
 

@@ -236,13 +236,19 @@ static_assert(kStages >= 2 && kStages % 2 == 0, "ring slots must be even");
 
 struct P1Args {
     const float* gk;     // gains [C], or nullptr with the norm off
-    float* part;         // partial states [B][H][Smax][D+1][D]  (column e major)
-    int64_t T;           // work items: B * G rows x R stages
+    float* part;         // partial states [B][H][Smax][D+1][D]  (column e major);
+                         // chunked: [B][H][Cc][Smax][D+1][D]
+    int64_t T;           // work items: B * G rows x R stages (chunked: B * G * Cc rows)
     int N, H, G, R, Smax, P;
     float eps;
     int norm;
+    int Cc;              // chunked: chunks of R stages each (b, g) sequence is cut into
 };
 
+// One row per (b, g) over the whole sequence (the forward's state), or, with
+// kChunked, one row per (b, g, chunk of R stages): the states of the sequence's
+// chunks, which the prefix (causal) form scans.
+template <bool kChunked>
 __global__ void __launch_bounds__(p1::kThreads, 1)
 kv_partials_persistent(const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v, const P1Args a)
@@ -310,10 +316,13 @@ kv_partials_persistent(const __grid_constant__ CUtensorMap tmap_k,
                 if (li >= kStages) ok = mbar_wait(&empty[st], (uint32_t)((li / kStages) - 1) & 1, 301);
                 if (!ok) break;
                 const int64_t i = i0 + li, r = i / a.R;
-                const int t = (int)(i % a.R), b = (int)(r / a.G), g = (int)(r % a.G);
+                const int t = (int)(i % a.R);
+                const int64_t rg = kChunked ? r / a.Cc : r;                   // (b, g)
+                const int b = (int)(rg / a.G), g = (int)(rg % a.G);
+                const int t0 = kChunked ? (int)(r % a.Cc) * a.R : 0;         // first stage
                 uint8_t* sb = stages + st * kStageBytes;
                 mbar_arrive_expect_tx(&full[st], kStageBytes);
-                const int x = g * 128, y = t * kStageTok;
+                const int x = g * 128, y = (t0 + t) * kStageTok;
                 tma_load_3d(sb, &tmap_k, &full[st], x, y, b);
                 tma_load_3d(sb + kBoxBytes, &tmap_k, &full[st], x + 64, y, b);
                 tma_load_3d(sb + 2 * kBoxBytes, &tmap_v, &full[st], x, y, b);
@@ -389,7 +398,8 @@ kv_partials_persistent(const __grid_constant__ CUtensorMap tmap_k,
             // one row segment [sb, se): this group's stages are those with li % 2 == grp
             const int64_t r = sb / a.R;
             const int64_t se = (r + 1) * a.R < i1 ? (r + 1) * a.R : i1;
-            const int g = (int)(r % a.G);
+            const int g = (int)((kChunked ? r / a.Cc : r) % a.G);
+            const int tbase = kChunked ? (int)(r % a.Cc) * a.R * kStageTok : 0;
             const int h = g * kGroupHeads + hl;
             float ks[kD];
 #pragma unroll
@@ -404,8 +414,8 @@ kv_partials_persistent(const __grid_constant__ CUtensorMap tmap_k,
                 uint8_t* const tl[2] = {stages + st * kStageBytes + (hl >> 1) * kBoxBytes,
                                         stages + st * kStageBytes + (hl >> 1) * kBoxBytes};
                 const int rows[2] = {lane, lane + 32}, ch[2] = {(hl & 1) * 4, (hl & 1) * 4};
-                const bool dead[2] = {!((t * kStageTok + lane < a.N) && (h < a.H)),
-                                      !((t * kStageTok + lane + 32 < a.N) && (h < a.H))};
+                const bool dead[2] = {!((tbase + t * kStageTok + lane < a.N) && (h < a.H)),
+                                      !((tbase + t * kStageTok + lane + 32 < a.N) && (h < a.H))};
                 const float* gg[2] = {sgain + (h < a.H ? h : 0) * kD, sgain + (h < a.H ? h : 0) * kD};
                 float rr[2];
                 phi2_inplace_sw128<true>(tl, rows, ch, gg, a.eps, a.norm != 0, dead, rr, ks);
@@ -450,12 +460,15 @@ kv_partials_persistent(const __grid_constant__ CUtensorMap tmap_k,
             ++seg;
 
             const int64_t r = i / a.R;
-            const int b = (int)(r / a.G), g = (int)(r % a.G);
+            const int64_t rg = kChunked ? r / a.Cc : r;
+            const int b = (int)(rg / a.G), g = (int)(rg % a.G);
             const int slot = (int)(c - owner_cta(r * a.R, a.T, a.P));
             const int h = g * kGroupHeads + q;
             if (h < a.H) {
                 // lane = d; element (e, d) at e * 32 + d: one 128-byte row per store
-                float* o = a.part + (((size_t)b * a.H + h) * a.Smax + slot) * kStateFloats + lane;
+                const size_t bh = (size_t)b * a.H + h;
+                const size_t row = kChunked ? bh * a.Cc + (size_t)(r % a.Cc) : bh;
+                float* o = a.part + (row * a.Smax + slot) * kStateFloats + lane;
 #pragma unroll
                 for (int e = 0; e < kD; ++e) o[e * kD] = v[e];
                 o[kD * kD] = ks;

@@ -178,7 +178,9 @@ def test_w8a8_and_quantize_entry_points_reject_bad_arguments(lib):
 
 def test_causal_entry_point_rejects_bad_arguments(lib):
     ws_need = lib.sana_linattn_workspace_bytes(2, 1000, 2240, 70, 2)
-    assert ws_need == 2 * 70 * 16 * 1056 * 4                # one state per 64-token chunk
+    simt = 2 * 70 * 16 * 1056 * 4               # one state per 64-token chunk
+    tc = 2 * (2 * 70 * 8 * 2 * 1056 * 4)        # two partial slots + the prefix per 128 tokens
+    assert ws_need == max(simt, tc)
     args = [FAKE, FAKE + (1 << 30), FAKE + (2 << 30), None, None, FAKE + (4 << 30), 2, 1000,
             2240, 70, 1e-6, 0, FAKE + (6 << 30), ws_need, None]
     a = list(args)

@@ -24,7 +24,10 @@ def run(lib, d, w):
                                WORKLOADS["1024px-b1"].scaled(N=1, seed=91),
                                WORKLOADS["1024px-b1"].scaled(N=333, seed=92),
                                WORKLOADS["1024px-b1"].scaled(B=2, N=129, gains="off", seed=93),
-                               WORKLOADS["2048px-b8-lognormal"].scaled(B=1, N=1000, seed=94)],
+                               WORKLOADS["2048px-b8-lognormal"].scaled(B=1, N=1000, seed=94),
+                               WORKLOADS["1024px-b1"].scaled(N=129, C=160, H=5, seed=96),
+                               WORKLOADS["4096px-b2-overflow"].scaled(B=3, N=640, seed=97),
+                               WORKLOADS["1024px-b1"].scaled(B=2, N=2049, seed=98)],
                          ids=lambda w: f"{w.dtype}-B{w.B}-N{w.N}-{w.gains}")
 def test_causal_small_full_parity(cuda_lib, w):
     x = make_inputs(w)
@@ -52,3 +55,20 @@ def test_causal_last_token_matches_noncausal_and_is_deterministic(cuda_lib):
     torch.cuda.synchronize()
     diff = (a[:, -1].float() - full[:, -1].float()).abs().max().item()
     assert diff < 2e-2, diff
+
+
+def test_causal_gains_without_16_byte_alignment(cuda_lib):
+    """Gains that are 4- but not 16-byte aligned take the CUDA-core kernels (the
+    tensor-core path reads them as 16-byte vectors); the result is the same."""
+    w = WORKLOADS["1024px-b1"].scaled(N=300, seed=99)
+    x = make_inputs(w)
+    d = to_dev(x)
+    gq = torch.empty(w.C + 1, dtype=torch.float32, device="cuda")[1:]
+    gk = torch.empty(w.C + 1, dtype=torch.float32, device="cuda")[1:]
+    gq.copy_(d["gq"])
+    gk.copy_(d["gk"])
+    assert gq.data_ptr() % 16 != 0
+    out = cuda_lib.forward_causal(d["q"], d["k"], d["v"], gq, gk, w.H, w.eps)
+    torch.cuda.synchronize()
+    ref = O.causal_forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps)
+    assert_close(out, ref, w.dtype, "causal, unaligned gains")

@@ -293,3 +293,20 @@ def test_independent_problems_on_concurrent_streams(cuda_lib):
     torch.cuda.synchronize()
     for w, a, o in zip(cases, alone, outs):
         assert torch.equal(a, o), w.name
+
+
+@pytest.mark.parametrize("B,N", [(2, 3000), (3, 777), (1, 16384)])
+def test_forward_passes_called_separately_equal_forward(cuda_lib, B, N):
+    """sana_linattn_forward_pass1 then _pass2 on one stream are the forward: the
+    same kernels and plan, so the output is bit-identical, also with unrelated work
+    enqueued between the two calls."""
+    w = WORKLOADS["4096px-b2-overflow"].scaled(B=B, N=N, seed=120 + N)
+    d = to_dev(make_inputs(w))
+    ref = run_forward(cuda_lib, d, w)
+    ws = torch.empty(cuda_lib.workspace_bytes(B, N, w.C, w.H), dtype=torch.uint8, device="cuda")
+    cuda_lib.forward_pass1(d["k"], d["v"], d["gk"], w.H, w.eps, ws)
+    scratch = torch.randn(1 << 20, device="cuda").sum()        # unrelated work in between
+    out = cuda_lib.forward_pass2(d["q"], d["gq"], w.H, w.eps, ws)
+    torch.cuda.synchronize()
+    assert torch.isfinite(scratch)
+    assert torch.equal(out, ref)
