@@ -517,6 +517,7 @@ constexpr int kStoresInFlight = 2;                 // TMA stores the store warp 
 constexpr int kN = 80;                             // B rows per head (see the file comment)
 constexpr int kLoRow = 48;                         // first row of the value columns' lo parts
 constexpr int kDenHi = 32, kDenLo = 33;            // rows of the normaliser's hi / lo parts
+static_assert(kDenHi == kD, "the normaliser column sits in B row e = D");
 constexpr int kBopBytes = kN * 128;                // both heads side by side in each row
 constexpr int kBopRing = 2;
 constexpr int kBufCols = kPairHeads * kN;          // 160 TMEM columns per tile
@@ -568,7 +569,8 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
     uint64_t* bempty = bfull + kBopRing;
     uint64_t* drain = bempty + kBopRing;
     uint64_t* sready = drain + 1;
-    uint32_t* tmem_slot = (uint32_t*)(sready + 1);
+    uint64_t* bfirst = sready + 1;                // the first segment's B, built by the workers
+    uint32_t* tmem_slot = (uint32_t*)(bfirst + 1);
 
     // The next grid may launch now; it waits for this one before touching memory.
     pdl_launch_dependents();
@@ -592,6 +594,7 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(&bempty[i], 1);
         }
         mbar_init(drain, 1);
+        mbar_init(bfirst, kWorkerWarps * 32);
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
@@ -657,7 +660,9 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
                 const bool lastt = (li + 1 == n) || (t == a.R - 1);
                 const int rb = seg & 1;
                 if (lane == 0) {
-                    if (first) ok = mbar_wait(&bfull[rb], (uint32_t)(seg >> 1) & 1, 403);
+                    if (first)
+                        ok = seg == 0 ? mbar_wait(bfirst, 0, 403)
+                                      : mbar_wait(&bfull[rb], (uint32_t)((seg - 1) >> 1) & 1, 403);
                     if (ok) ok = mbar_wait(&aready[st], fpar, 404);
                     if (ok && li >= kTmemBufs) ok = mbar_wait(&tfree[tb], tpar ^ 1, 405);
                 }
@@ -686,7 +691,8 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
         }
     } else if (warp == 2) {
         // ------------------------------------------------ B operand builder
-        // Per row segment: the pair's state S_j[d][e] (j = head of the pair) lands in
+        // Every row segment after the first (the workers build the first one): the
+        // pair's state S_j[d][e] (j = head of the pair) lands in
         // registers, lane = d: either the sum of the pass-1 partials of the row, slot
         // by slot in slot order (bulk copies of up to kSlotsPerRound slots at a time),
         // or the given state.  Lane pairs (d, d + 1) then write one bf16x2 each: even
@@ -697,9 +703,13 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
             const int64_t i = i0 + li;
             if (!(li == 0 || i % a.R == 0)) continue;              // not a segment start
             const int rb = seg & 1;
+            if (seg == 0) {
+                ++seg;
+                continue;
+            }
             if (seg >= 2) ok = mbar_wait(&bempty[rb], (uint32_t)((seg >> 1) - 1) & 1, 407);
             if (!ok) break;
-            if (seg == 0) pdl_wait_primary();                     // the states come from pass 1
+            if (seg == 1) pdl_wait_primary();                     // the states come from pass 1
             const int64_t r = i / a.R;
             const int b = (int)(r / a.Pp), p = (int)(r % a.Pp);
             const int h0 = p * kPairHeads;
@@ -851,11 +861,76 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
             return true;
         };
 
-        int64_t prev = -1;
+        // The first segment's B operand, built by all worker threads at once with plain
+        // loads: one round trip to L2 instead of the builder's rounds of bulk copies,
+        // which would otherwise stand between pass 1's end and the first UMMA.  Slots
+        // are summed in the builder's order, so the state is the same bit for bit.
+        // Thread item (j, e, dp): S_j[e][2dp], S_j[e][2dp + 1], consecutive threads
+        // along d (coalesced in the partials' [e][d] layout).
+        auto build_first = [&]() {
+            pdl_wait_primary();                                  // the states come from pass 1
+            const int64_t r = i0 / a.R;
+            const int b = (int)(r / a.Pp), p = (int)(r % a.Pp);
+            const int h0 = p * kPairHeads, nh = min(kPairHeads, a.H - h0);
+            const int ns = a.kv == nullptr
+                               ? p1_row_slots((int64_t)b * a.G1 + h0 / p1::kGroupHeads, a.R1, a.T1, a.P1)
+                               : 1;
+            for (int it = threadIdx.x - 128; it < kPairHeads * kDP * (kD / 2); it += kWorkerWarps * 32) {
+                const int dp = it % (kD / 2), e = (it / (kD / 2)) % kDP, jj = it / (kD / 2 * kDP);
+                const int d0 = 2 * dp;
+                float x0 = 0.f, x1 = 0.f;
+                if (jj < nh) {
+                    const size_t bh = (size_t)b * a.H + h0 + jj;
+                    if (a.kv == nullptr) {
+                        const float* src = a.part + bh * a.Smax1 * kStateFloats + e * kD + d0;
+                        int s = 0;
+                        for (; s + 4 <= ns; s += 4) {
+                            float2 v[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                v[u] = __ldcg(reinterpret_cast<const float2*>(src + (size_t)(s + u) * kStateFloats));
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                x0 += v[u].x;
+                                x1 += v[u].y;
+                            }
+                        }
+                        for (; s < ns; ++s) {
+                            const float2 v = __ldcg(reinterpret_cast<const float2*>(src + (size_t)s * kStateFloats));
+                            x0 += v.x;
+                            x1 += v.y;
+                        }
+                    } else {
+                        const float* src = a.kv + bh * kStateFloats;
+                        x0 = __ldcg(src + d0 * kDP + e);
+                        x1 = __ldcg(src + (d0 + 1) * kDP + e);
+                    }
+                }
+                const float hx0 = __bfloat162float(__float2bfloat16_rn(x0));
+                const float hx1 = __bfloat162float(__float2bfloat16_rn(x1));
+                const int chunk = jj * 4 + d0 / 8, off = (d0 % 8) * 2;
+                const int lorow = e < kD ? kLoRow + e : kDenLo;   // hi row is e (kDenHi for e = kD)
+                *reinterpret_cast<uint32_t*>(bop + sw128_offset(e, chunk) + off) = pack_bf16x2(hx0, hx1);
+                *reinterpret_cast<uint32_t*>(bop + sw128_offset(lorow, chunk) + off) =
+                    pack_bf16x2(x0 - hx0, x1 - hx1);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bfirst);
+        };
+
+        // Each group transforms its first tile (Q is not written by pass 1, so it may
+        // already have landed), then helps build the first B operand.
+        int64_t prev = -1, li = grp;
         float r_prev = 1.f, r_cur = 1.f;
-        for (int64_t li = grp; i0 + li < i1 && ok; li += 2) {
+        if (ok && i0 + li < i1) {
+            ok = transform(li, r_prev);
+            prev = li;
+            li += 2;
+        }
+        if (ok) build_first();
+        for (; i0 + li < i1 && ok; li += 2) {
             ok = transform(li, r_cur);
-            if (ok && prev >= 0) ok = epilogue(prev, r_prev);
+            if (ok) ok = epilogue(prev, r_prev);
             prev = li;
             r_prev = r_cur;
         }
