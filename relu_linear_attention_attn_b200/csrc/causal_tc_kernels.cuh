@@ -13,13 +13,13 @@
 //   2. causal_prefix_states: per (b, h) the exclusive prefix over chunks, summing
 //      each chunk's slots in slot order and the chunks in chunk order
 //      (reproducible);
-//   3. causal_apply_tc: per (b, head pair, chunk), on the tensor cores:
+//   3. causal_apply_tc: per (b, head pair, chunk), head by head, on the tensor cores:
 //        U1  P_h = phi(Q_h) phi(K_h)^T            (M = N = 128, K = 32)
-//            D_h = phi(Q_h) [P_c hi | lo]          (N = 80, pass 2's operand)
-//        the epilogue zeroes P_h[n][j] for j > n and writes it as bf16 (K-major A)
-//        U2  D_h[:, 0:48] += P_h [V_h^T ; 1 ; 0]   (N = 48, K = 128)
-//            the row of ones adds sum_{j <= n} P_h[n][j] to the normaliser column
-//        O = (D[e] + D[48 + e]) / (D[32] + D[33] + eps).
+//        the epilogue zeroes P_h[n][j] for j > n, writes it as bf16 (K-major A) and
+//        sums each masked row in fp32 (the chunk's own normaliser share)
+//        U2  D_h = phi(Q_h) [P_c hi | lo]          (N = 80, pass 2's operand)
+//            D_h[:, 0:32] += P_h V_h                (N = 32, K = 128, V MN-major)
+//        O = (D[e] + D[48 + e]) / (D[32] + D[33] + row sum + eps).
 #pragma once
 
 #include "sana_common.cuh"
@@ -33,7 +33,8 @@ constexpr int kCausalTcChunk = 128;        // tokens per chunk (UMMA M of the ap
 // Exclusive prefix over the chunks of each (b, h): pre[b][h][c] = sum_{c' < c}
 // sum_s part[b][h][c'][s] (both [e][d], column e major).  Grid B * H, 264 threads:
 // thread t owns the 16 bytes t of a state and walks the chunks in order, loading
-// eight chunks ahead.  ns_of(row) gives the slot count of a pass-1 chunk row.
+// eight chunks ahead; each chunk's slots are summed in slot order and the chunks in
+// chunk order, so the result is reproducible.
 struct PrefixArgs {
     const float* part;   // [B][H][Cc][Smax][D+1][D]
     float* pre;          // [B][H][Cc][D+1][D]
@@ -41,24 +42,45 @@ struct PrefixArgs {
     int64_t R1, T1, P1;  // pass-1 plan (stages per chunk row, items, CTAs)
 };
 
-__global__ void __launch_bounds__(kStateFloats / 4)
+constexpr int kPrefixThreads = kStateFloats / 4;
+
+__global__ void __launch_bounds__(kPrefixThreads)
 causal_prefix_states(const PrefixArgs a)
 {
+    constexpr int kBatch = 8;                      // chunks whose loads are in flight at once
+    constexpr int kSplitWords = 1024;              // chunks whose slot counts fit the bit table
+    __shared__ uint32_t split[kSplitWords];        // bit c: chunk c has two pass-1 slots
+    pdl_launch_dependents();                       // the apply reads `pre` only after its own wait
     const int64_t bh = blockIdx.x;
     const int b = (int)(bh / a.H), h = (int)(bh % a.H);
     const int i4 = threadIdx.x;
     const float4* src = reinterpret_cast<const float4*>(a.part) + bh * a.Cc * a.Smax * (kStateFloats / 4);
     float4* dst = reinterpret_cast<float4*>(a.pre) + bh * a.Cc * (kStateFloats / 4);
     const int64_t row0 = ((int64_t)b * a.G + h / p1::kGroupHeads) * a.Cc;    // pass-1 row of chunk 0
+    // With two pass-1 items per chunk, a chunk has two slots exactly when a pass-1 CTA's
+    // range starts at its second item: one division per CTA boundary instead of two per
+    // chunk and thread.
+    const bool table = a.R1 == 2 && a.Cc <= kSplitWords * 32;
+    if (table) {
+        for (int w = threadIdx.x; w < (a.Cc + 31) / 32; w += blockDim.x) split[w] = 0u;
+        __syncthreads();
+        for (int64_t c = 1 + threadIdx.x; c < a.P1; c += blockDim.x) {
+            const int64_t bnd = range_begin(c, a.T1, a.P1);
+            const int64_t cr = (bnd >> 1) - row0;
+            if ((bnd & 1) && cr >= 0 && cr < a.Cc) atomicOr(&split[cr >> 5], 1u << (cr & 31));
+        }
+        __syncthreads();
+    }
     float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c0 = 0; c0 < a.Cc; c0 += 8) {
-        float4 x[8];
+    for (int c0 = 0; c0 < a.Cc; c0 += kBatch) {
+        float4 x[kBatch];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < kBatch; ++k) {
             x[k] = make_float4(0.f, 0.f, 0.f, 0.f);
             const int c = c0 + k;
             if (c < a.Cc) {
-                const int ns = p1_row_slots(row0 + c, a.R1, a.T1, a.P1);
+                const int ns = table ? 1 + (int)((split[c >> 5] >> (c & 31)) & 1u)
+                                     : p1_row_slots(row0 + c, a.R1, a.T1, a.P1);
                 for (int s = 0; s < ns; ++s) {
                     const float4 v = __ldcg(src + ((int64_t)c * a.Smax + s) * (kStateFloats / 4) + i4);
                     x[k].x += v.x; x[k].y += v.y; x[k].z += v.z; x[k].w += v.w;
@@ -66,7 +88,7 @@ causal_prefix_states(const PrefixArgs a)
             }
         }
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < kBatch; ++k) {
             const int c = c0 + k;
             if (c < a.Cc) {
                 dst[(int64_t)c * (kStateFloats / 4) + i4] = run;
@@ -79,23 +101,23 @@ causal_prefix_states(const PrefixArgs a)
 namespace ca {
 constexpr int kTok = kCausalTcChunk;
 constexpr int kTile = kTok * 128;                  // 128 tokens x 64 channels (a head pair)
-constexpr int kStageBytes = 3 * kTile;             // [Q | K | V]
-constexpr int kStages = 2;
-constexpr int kVtRows = 48;                        // V^T rows: 32 values, ones, zeros
-constexpr int kVtAtom = kVtRows * 128;             // 64 keys of every row
-constexpr int kVtHead = 2 * kVtAtom;
+constexpr int kQSlots = 3;                         // Q tiles (phi(Q) in place, then O over it)
+constexpr int kKSlots = 2;                         // K tiles (phi(K) in place)
+constexpr int kVSlots = 3;                         // V tiles (the MN-major B operand of U2)
 constexpr int kPsAtom = kTok * 128;                // 64 keys of every query row
-constexpr int kPsHead = 2 * kPsAtom;
+constexpr int kPsBuf = 2 * kPsAtom;                // one head's masked P, bf16
 constexpr int kBopBytes = p2::kBopBytes;
-constexpr int kStagingBytes = 2 * kStateFloats * 4;
-constexpr int kPCol = 0;                           // P of head j at 128 j
-constexpr int kDCol = 256;                         // D of head j at 256 + 80 j
-constexpr int kTmemCols = 512;
-constexpr int kGroupThreads = 256;                 // a transform or epilogue group: 8 warps
+constexpr int kBufCols = 128;                      // TMEM per sub-item: P, then D over it
+constexpr int kTmemBufs = 4;
+constexpr int kTmemCols = kTmemBufs * kBufCols;
+constexpr int kGroupThreads = 256;                 // the transform or the epilogue warps
 constexpr int kThreads = 32 * (4 + 16);
-constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 2 * kVtHead + 2 * kPsHead + 2 * kBopBytes +
-                           kStagingBytes + 512;
+constexpr int kRowSumBytes = kTmemBufs * 2 * kTok * 4;   // [sub-item % 4][key half][query row]
+constexpr int kPrePer = (2 * kDP * (kD / 2) + kGroupThreads - 1) / kGroupThreads;   // B items per thread
+constexpr int kSmemBytes = 1024 + (kQSlots + kKSlots + kVSlots) * kTile + 2 * kPsBuf + 2 * kBopBytes +
+                           kRowSumBytes + 512;
 static_assert(kSmemBytes <= 232448, "shared memory");
+static_assert(kTmemCols <= 512, "TMEM");
 }  // namespace ca
 
 struct CaArgs {
@@ -108,6 +130,22 @@ struct CaArgs {
     int norm;
 };
 
+// Work item li = (b, head pair p, chunk c); sub-item u = 2 li + j is head j of the
+// pair.  Per sub-item, on the tensor cores:
+//   U1(u)  P = phi(Q_j) phi(K_j)^T                      -> TMEM buffer u % 4
+//   A(u)   epilogue: P masked to keys j <= n, bf16      -> P_s[u % 2] (K-major A);
+//          the row sums of the masked values (the chunk's own share of the
+//          normaliser, summed before the bf16 rounding) go to shared memory
+//   U2(u)  D = phi(Q_j) [P_c hi | lo] + P_s V_j          -> the same TMEM buffer
+//          (V_j straight from its landing tile, as an MN-major B operand)
+//   B(u)   epilogue: O = (D[e] + D[48 + e]) / (D[32] + D[33] + row sum + eps), over
+//          the Q tile
+// The issuer runs U1(u + 1) before U2(u) and the epilogue warps run A(u) before
+// B(u - 1), so the tensor cores work on one sub-item while the epilogue warps work
+// on its neighbours.  K tiles leave their ring once both heads' P are formed, V
+// tiles once both heads' U2 are done, Q tiles (then O) once their store has read
+// them.  The transform warps also build each item's prefix operand, its loads
+// issued one item ahead.
 __global__ void __launch_bounds__(ca::kThreads, 1)
 causal_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                 const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_o,
@@ -116,24 +154,28 @@ causal_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     using namespace ca;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_1024(smem_raw);
-    uint8_t* stages = smem;
-    uint8_t* vt = stages + kStages * kStageBytes;
-    uint8_t* ps = vt + 2 * kVtHead;
-    uint8_t* bop = ps + 2 * kPsHead;
-    float* staging = (float*)(bop + 2 * kBopBytes);
-    uint64_t* full = (uint64_t*)(staging + kStagingBytes / 4);
-    uint64_t* sempty = full + kStages;
-    uint64_t* aready = sempty + kStages;
-    uint64_t* bfull = aready + kStages;
-    uint64_t* bempty = bfull + 2;
-    uint64_t* pdone = bempty + 2;
-    uint64_t* psready = pdone + 1;
-    uint64_t* mmadone = psready + 1;
-    uint64_t* u2done = mmadone + 1;
-    uint64_t* tfree = u2done + 1;
-    uint64_t* ofull = tfree + 1;
-    uint64_t* sready = ofull + 1;
-    uint64_t* drain = sready + 1;
+    uint8_t* qring = smem;
+    uint8_t* kring = qring + kQSlots * kTile;
+    uint8_t* vring = kring + kKSlots * kTile;
+    uint8_t* ps = vring + kVSlots * kTile;
+    uint8_t* bop = ps + 2 * kPsBuf;
+    float* rowsum = (float*)(bop + 2 * kBopBytes);
+    uint64_t* qfull = (uint64_t*)((uint8_t*)rowsum + kRowSumBytes);
+    uint64_t* qempty = qfull + kQSlots;
+    uint64_t* ofull = qempty + kQSlots;
+    uint64_t* vfull = ofull + kQSlots;
+    uint64_t* vempty = vfull + kVSlots;
+    uint64_t* kfull = vempty + kVSlots;
+    uint64_t* kempty = kfull + kKSlots;
+    uint64_t* qkready = kempty + kKSlots;          // 2
+    uint64_t* bfull = qkready + 2;                 // 2
+    uint64_t* bempty = bfull + 2;                  // 2
+    uint64_t* pdone = bempty + 2;                  // kTmemBufs
+    uint64_t* mmadone = pdone + kTmemBufs;         // kTmemBufs
+    uint64_t* tfree = mmadone + kTmemBufs;         // kTmemBufs
+    uint64_t* psready = tfree + kTmemBufs;         // 2
+    uint64_t* u2done = psready + 2;                // 2
+    uint64_t* drain = u2done + 2;
     uint32_t* tmem_slot = (uint32_t*)(drain + 1);
 
     const int64_t cta = blockIdx.x;
@@ -142,22 +184,31 @@ causal_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&sempty[i], 1);
-            mbar_init(&aready[i], kGroupThreads);
+        for (int i = 0; i < kQSlots; ++i) {
+            mbar_init(&qfull[i], 1);
+            mbar_init(&qempty[i], 1);
+            mbar_init(&ofull[i], 2 * kGroupThreads);
+        }
+        for (int i = 0; i < kVSlots; ++i) {
+            mbar_init(&vfull[i], 1);
+            mbar_init(&vempty[i], 1);
+        }
+        for (int i = 0; i < kKSlots; ++i) {
+            mbar_init(&kfull[i], 1);
+            mbar_init(&kempty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bfull[i], 32);
+            mbar_init(&qkready[i], kGroupThreads);
+            mbar_init(&bfull[i], kGroupThreads);
             mbar_init(&bempty[i], 1);
+            mbar_init(&psready[i], kGroupThreads);
+            mbar_init(&u2done[i], 1);
         }
-        mbar_init(pdone, 1);
-        mbar_init(psready, kGroupThreads);
-        mbar_init(mmadone, 1);
-        mbar_init(u2done, 1);
-        mbar_init(tfree, kGroupThreads);
-        mbar_init(ofull, kGroupThreads);
-        mbar_init(sready, 1);
+        for (int i = 0; i < kTmemBufs; ++i) {
+            mbar_init(&pdone[i], 1);
+            mbar_init(&mmadone[i], 1);
+            mbar_init(&tfree[i], kGroupThreads);
+        }
         mbar_init(drain, 1);
         fence_barrier_init();
     }
@@ -167,20 +218,15 @@ causal_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         prefetch_tmap(&tmap_v);
         prefetch_tmap(&tmap_o);
     }
-    // constant parts of the operands: rows 34..47 of both B-operand buffers, and
-    // rows 32 (ones: the normaliser's intra-chunk sum) and 33..47 (zeros) of V^T
+    // Constant parts of the operands: rows 34..47 of both B-operand buffers, and all
+    // of P_s (the blocks of keys after a query's 32-row quadrant are never written).
     for (int i = threadIdx.x; i < 2 * (p2::kLoRow - p2::kDenLo - 1) * 8; i += blockDim.x) {
         const int rb = i / ((p2::kLoRow - p2::kDenLo - 1) * 8), rem = i % ((p2::kLoRow - p2::kDenLo - 1) * 8);
         *reinterpret_cast<uint4*>(bop + rb * kBopBytes + (p2::kDenLo + 1 + rem / 8) * 128 +
                                   (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
     }
-    for (int i = threadIdx.x; i < 2 * 2 * 16 * 8; i += blockDim.x) {   // [head][atom][row 32..47][chunk]
-        const int hh = i / (2 * 16 * 8), at = (i / (16 * 8)) % 2, rw = 32 + (i / 8) % 16, ch = i % 8;
-        const uint32_t one2 = 0x3F803F80u;                             // two bf16 ones
-        const uint32_t w = rw == 32 ? one2 : 0u;
-        *reinterpret_cast<uint4*>(vt + hh * kVtHead + at * kVtAtom + sw128_offset(rw, ch)) =
-            make_uint4(w, w, w, w);
-    }
+    for (int i = threadIdx.x; i < 2 * kPsBuf / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(ps)[i] = make_uint4(0, 0, 0, 0);
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
@@ -193,207 +239,212 @@ causal_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     bool ok = n > 0;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer: Q, K, V tiles
+        // ------------------------------------------------ TMA producer: Q, K, V of each item
         if (lane == 0 && ok) {
             int64_t last = -1;
             for (int64_t li = 0; li < n; ++li) {
-                const int s = (int)(li & 1);
-                if (li >= kStages) ok = mbar_wait(&sempty[s], (uint32_t)((li >> 1) - 1) & 1, 901);
-                if (!ok) break;
+                const int qs = (int)(li % kQSlots), ks = (int)(li % kKSlots), vs = (int)(li % kVSlots);
                 const int64_t i = i0 + li, r = i / a.Cc;
                 const int c = (int)(i % a.Cc), b = (int)(r / a.Pp), p = (int)(r % a.Pp);
-                uint8_t* sb = stages + s * kStageBytes;
-                mbar_arrive_expect_tx(&full[s], kStageBytes);
-                tma_load_3d(sb, &tmap_q, &full[s], p * 64, c * kTok, b);
-                tma_load_3d(sb + kTile, &tmap_k, &full[s], p * 64, c * kTok, b);
-                tma_load_3d(sb + 2 * kTile, &tmap_v, &full[s], p * 64, c * kTok, b);
+                if (li >= kQSlots) ok = mbar_wait(&qempty[qs], (uint32_t)((li / kQSlots) - 1) & 1, 901);
+                if (ok && li >= kKSlots) ok = mbar_wait(&kempty[ks], (uint32_t)((li / kKSlots) - 1) & 1, 902);
+                if (ok && li >= kVSlots) ok = mbar_wait(&vempty[vs], (uint32_t)((li / kVSlots) - 1) & 1, 903);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&qfull[qs], kTile);
+                tma_load_3d(qring + qs * kTile, &tmap_q, &qfull[qs], p * 64, c * kTok, b);
+                mbar_arrive_expect_tx(&kfull[ks], kTile);
+                tma_load_3d(kring + ks * kTile, &tmap_k, &kfull[ks], p * 64, c * kTok, b);
+                mbar_arrive_expect_tx(&vfull[vs], kTile);
+                tma_load_3d(vring + vs * kTile, &tmap_v, &vfull[vs], p * 64, c * kTok, b);
                 last = li;
             }
-            if (!ok) {
-                for (int s = 0; s < kStages; ++s) {
-                    const int64_t lj = last - ((last - s) % kStages + kStages) % kStages;
-                    if (last >= 0 && lj >= 0)
-                        mbar_wait(&full[s], (uint32_t)(lj >> 1) & 1, 902);
-                }
+            if (!ok) {   // let every issued copy land before the CTA can exit
+                for (int64_t lj = last - (kQSlots - 1) > 0 ? last - (kQSlots - 1) : 0; lj <= last; ++lj)
+                    mbar_wait(&qfull[lj % kQSlots], (uint32_t)(lj / kQSlots) & 1, 904);
+                for (int64_t lj = last - (kKSlots - 1) > 0 ? last - (kKSlots - 1) : 0; lj <= last; ++lj)
+                    mbar_wait(&kfull[lj % kKSlots], (uint32_t)(lj / kKSlots) & 1, 904);
+                for (int64_t lj = last - (kVSlots - 1) > 0 ? last - (kVSlots - 1) : 0; lj <= last; ++lj)
+                    mbar_wait(&vfull[lj % kVSlots], (uint32_t)(lj / kVSlots) & 1, 904);
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ UMMA issuer (one elected lane)
-        if (ok) {
+        // ------------------------------------------------ UMMA issuer (lane 0 alone, no
+        // warp-collective steps between the UMMAs); order U1(0), then per sub-item u:
+        // U1(u + 1), U2(u)
+        if (ok && lane == 0) {
             const uint32_t idesc_p = make_idesc_bf16(128, 128, false, false);
             const uint32_t idesc_d = make_idesc_bf16(128, p2::kN, false, false);
-            const uint32_t idesc_v = make_idesc_bf16(128, kVtRows, false, false);
-            const uint64_t st0 = make_smem_desc(smem_u32(stages), 16, 1024, kSwizzle128B);
+            const uint32_t idesc_v = make_idesc_bf16(128, kD, false, true);     // V MN-major
+            const uint64_t q0 = make_smem_desc(smem_u32(qring), 16, 1024, kSwizzle128B);
+            const uint64_t k0 = make_smem_desc(smem_u32(kring), 16, 1024, kSwizzle128B);
+            const uint64_t v0 = make_smem_desc(smem_u32(vring), kTile, 1024, kSwizzle128B);
             const uint64_t bo0 = make_smem_desc(smem_u32(bop), 16, 1024, kSwizzle128B);
             const uint64_t ps0 = make_smem_desc(smem_u32(ps), 16, 1024, kSwizzle128B);
-            const uint64_t vt0 = make_smem_desc(smem_u32(vt), 16, 1024, kSwizzle128B);
-            for (int64_t li = 0; li < n; ++li) {
-                const int s = (int)(li & 1), rb = (int)(li & 1);
-                if (lane == 0) {
-                    ok = mbar_wait(&aready[s], (uint32_t)(li >> 1) & 1, 903);
-                    if (ok) ok = mbar_wait(&bfull[rb], (uint32_t)(li >> 1) & 1, 904);
-                    if (ok && li >= 1) ok = mbar_wait(tfree, (uint32_t)(li - 1) & 1, 905);
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
+            const int64_t nsub = 2 * n;
+            auto u1 = [&](int64_t u) -> bool {
+                const int64_t li = u >> 1;
+                const int j = (int)(u & 1), tb = (int)(u % kTmemBufs);
+                if (j == 0 && !mbar_wait(&qkready[li & 1], (uint32_t)(li >> 1) & 1, 905)) return false;
+                if (u >= kTmemBufs && !mbar_wait(&tfree[tb], (uint32_t)((u / kTmemBufs) - 1) & 1, 906))
+                    return false;
                 tc_fence_after_sync();
-                const uint64_t qd = st0 + (uint64_t)((s * kStageBytes) >> 4);
-                const uint64_t kd = qd + (uint64_t)(kTile >> 4);
-                const uint64_t bd = bo0 + (uint64_t)((rb * kBopBytes) >> 4);
-#pragma unroll
-                for (int jh = 0; jh < 2; ++jh) {
-                    const uint32_t dp = tmem + kPCol + 128 * jh, dd = tmem + kDCol + p2::kN * jh;
-                    umma_bf16_elect(dp, qd + 4 * jh, kd + 4 * jh, idesc_p, false);
-                    umma_bf16_elect(dp, qd + 4 * jh + 2, kd + 4 * jh + 2, idesc_p, true);
-                    umma_bf16_elect(dd, qd + 4 * jh, bd + 4 * jh, idesc_d, false);
-                    umma_bf16_elect(dd, qd + 4 * jh + 2, bd + 4 * jh + 2, idesc_d, true);
-                }
-                umma_commit_elect(pdone);
-                umma_commit_elect(&bempty[rb]);
-                if (lane == 0) ok = mbar_wait(psready, (uint32_t)li & 1, 906);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
+                const uint64_t qd = q0 + (uint64_t)(((li % kQSlots) * kTile) >> 4) + 4 * j;
+                const uint64_t kd = k0 + (uint64_t)(((li % kKSlots) * kTile) >> 4) + 4 * j;
+                const uint32_t dp = tmem + tb * kBufCols;
+                umma_bf16(dp, qd, kd, idesc_p, false);
+                umma_bf16(dp, qd + 2, kd + 2, idesc_p, true);
+                umma_commit(&pdone[tb]);
+                if (j == 1) umma_commit(&kempty[li % kKSlots]);         // phi(K) read by both heads
+                return true;
+            };
+            auto u2 = [&](int64_t u) -> bool {
+                const int64_t li = u >> 1;
+                const int j = (int)(u & 1), tb = (int)(u % kTmemBufs), pb = (int)(u & 1);
+                const int vs = (int)(li % kVSlots);
+                if (!mbar_wait(&psready[pb], (uint32_t)(u >> 1) & 1, 907)) return false;
+                if (j == 0 && !mbar_wait(&vfull[vs], (uint32_t)(li / kVSlots) & 1, 908)) return false;
+                if (j == 0 && !mbar_wait(&bfull[li & 1], (uint32_t)(li >> 1) & 1, 909)) return false;
                 tc_fence_after_sync();
+                const uint64_t qd = q0 + (uint64_t)(((li % kQSlots) * kTile) >> 4) + 4 * j;
+                const uint64_t bd = bo0 + (uint64_t)(((li & 1) * kBopBytes) >> 4) + 4 * j;
+                const uint32_t dd = tmem + tb * kBufCols;
+                umma_bf16(dd, qd, bd, idesc_d, false);
+                umma_bf16(dd, qd + 2, bd + 2, idesc_d, true);
+                // intra-chunk part: A = P_s (K-major, 64 keys per atom), B = V_j (MN-major:
+                // head j's 32 channels of each key row; 16 keys = 2048 bytes a step)
+                const uint64_t pa = ps0 + (uint64_t)((pb * kPsBuf) >> 4);
+                const uint64_t vb = v0 + (uint64_t)((vs * kTile) >> 4) + 4 * j;
 #pragma unroll
-                for (int jh = 0; jh < 2; ++jh) {
-                    const uint32_t dd = tmem + kDCol + p2::kN * jh;
-#pragma unroll
-                    for (int k = 0; k < kTok / 16; ++k) {
-                        const uint64_t off_p = (uint64_t)((jh * kPsHead + (k >> 2) * kPsAtom) >> 4) + 2 * (k & 3);
-                        const uint64_t off_v = (uint64_t)((jh * kVtHead + (k >> 2) * kVtAtom) >> 4) + 2 * (k & 3);
-                        umma_bf16_elect(dd, ps0 + off_p, vt0 + off_v, idesc_v, true);
-                    }
+                for (int k = 0; k < kTok / 16; ++k) {
+                    const uint64_t atp = (uint64_t)(((k >> 2) * kPsAtom) >> 4) + 2 * (k & 3);
+                    umma_bf16(dd, pa + atp, vb + (uint64_t)k * 128, idesc_v, true);
                 }
-                umma_commit_elect(mmadone);
-                umma_commit_elect(u2done);
-            }
-            umma_commit_elect(drain);
-            if (lane == 0) mbar_wait(drain, 0, 907);
-            __syncwarp();
-        }
-    } else if (warp == 2) {
-        // ------------------------------------------------ B operand of each chunk's
-        // prefix state (the pair's two heads), as pass 2 builds it from a state
-        int64_t li = 0;
-        for (; li < n && ok; ++li) {
-            const int rb = (int)(li & 1);
-            if (li >= 2) ok = mbar_wait(&bempty[rb], (uint32_t)((li >> 1) - 1) & 1, 908);
-            if (!ok) break;
-            const int64_t i = i0 + li, r = i / a.Cc;
-            const int c = (int)(i % a.Cc), b = (int)(r / a.Pp), p = (int)(r % a.Pp);
-            const int h0 = 2 * p, nh = min(2, a.H - h0);
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive_expect_tx(sready, (uint32_t)(nh * kStateFloats * 4));
-                for (int j = 0; j < nh; ++j)
-                    bulk_load(staging + j * kStateFloats,
-                              a.pre + (((size_t)b * a.H + h0 + j) * a.Cc + c) * kStateFloats,
-                              kStateFloats * 4, sready);
-            }
-            ok = mbar_wait(sready, (uint32_t)li & 1, 909);
-            if (!ok) break;
-            uint8_t* dst = bop + rb * kBopBytes;
-            const int d0 = lane & ~1;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int chunk = j * 4 + d0 / 8, off = (d0 % 8) * 2;
-#pragma unroll
-                for (int e = 0; e < kDP; ++e) {
-                    const float x = j < nh ? staging[j * kStateFloats + e * kD + lane] : 0.f;
-                    const float xp = __shfl_xor_sync(0xffffffffu, x, 1);
-                    const float xe = (lane & 1) ? xp : x, xo = (lane & 1) ? x : xp;
-                    const float he = __bfloat162float(__float2bfloat16_rn(xe));
-                    const float ho = __bfloat162float(__float2bfloat16_rn(xo));
-                    const int row = (lane & 1) ? (e < kD ? p2::kLoRow + e : p2::kDenLo) : e;
-                    const uint32_t w = (lane & 1) ? pack_bf16x2(xe - he, xo - ho) : pack_bf16x2(he, ho);
-                    *reinterpret_cast<uint32_t*>(dst + sw128_offset(row, chunk) + off) = w;
+                umma_commit(&mmadone[tb]);
+                umma_commit(&u2done[pb]);
+                if (j == 1) {
+                    umma_commit(&vempty[vs]);
+                    umma_commit(&bempty[li & 1]);
                 }
+                return true;
+            };
+            ok = u1(0);
+            for (int64_t u = 0; u < nsub && ok; ++u) {
+                if (u + 1 < nsub) ok = u1(u + 1);
+                if (ok) ok = u2(u);
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            mbar_arrive(&bfull[rb]);
+            umma_commit(drain);
+            mbar_wait(drain, 0, 910);
         }
+        __syncwarp();
     } else if (warp == 3) {
         // ------------------------------------------------ O stores (over the Q tile)
         if (lane == 0 && ok) {
             for (int64_t li = 0; li < n && ok; ++li) {
-                const int s = (int)(li & 1);
-                ok = mbar_wait(ofull, (uint32_t)li & 1, 910);
+                const int qs = (int)(li % kQSlots);
+                ok = mbar_wait(&ofull[qs], (uint32_t)(li / kQSlots) & 1, 912);
                 if (!ok) break;
                 const int64_t i = i0 + li, r = i / a.Cc;
                 const int c = (int)(i % a.Cc), b = (int)(r / a.Pp), p = (int)(r % a.Pp);
-                tma_store_3d(&tmap_o, stages + s * kStageBytes, p * 64, c * kTok, b);
+                tma_store_3d(&tmap_o, qring + qs * kTile, p * 64, c * kTok, b);
                 bulk_commit_group();
                 bulk_wait_group_read<0>();
-                mbar_arrive(&sempty[s]);
+                mbar_arrive(&qempty[qs]);
             }
             bulk_wait_group<0>();
         }
-    } else if (warp < 12) {
-        // ------------------------------------------------ phi(Q), phi(K) in place, V^T:
-        // warp w takes token row 32 (w % 4) + lane of the chunk, head (w - 4) / 4 of
-        // the pair
-        // (the gains are read from global memory, 16-byte aligned: checked on the host)
-        const int tw = warp - 4, jh = tw >> 2, row = 32 * (tw & 3) + lane;
+    } else if (warp >= 4 && warp < 12) {
+        // ------------------------------------------------ phi(Q), phi(K) in place; then the
+        // item's prefix operand.  Warp w takes token row 32 (w % 4) + lane of the chunk,
+        // head (w - 4) / 4 of the pair (the gains are read from global memory, 16-byte
+        // aligned: checked on the host).  For the operand, thread t takes the items
+        // (j, e, dp) = t + 256 k: S_j[e][2dp], S_j[e][2dp + 1] of the chunk's prefix.
+        const int t = threadIdx.x - 128, tw = warp - 4, jh = tw >> 2, row = 32 * (tw & 3) + lane;
+        float2 pv[kPrePer];
+        auto load_pre = [&](int64_t li) {
+            const int64_t i = i0 + li, r = i / a.Cc;
+            const int c = (int)(i % a.Cc), b = (int)(r / a.Pp), p = (int)(r % a.Pp);
+            const int nh = min(2, a.H - 2 * p);
+#pragma unroll
+            for (int k = 0; k < kPrePer; ++k) {
+                const int it = t + k * kGroupThreads;
+                const int dp = it % (kD / 2), e = (it / (kD / 2)) % kDP, jj = it / (kD / 2 * kDP);
+                pv[k] = make_float2(0.f, 0.f);
+                if (it < 2 * kDP * (kD / 2) && jj < nh)
+                    pv[k] = __ldcg(reinterpret_cast<const float2*>(
+                        a.pre + (((size_t)b * a.H + 2 * p + jj) * a.Cc + c) * kStateFloats + e * kD + 2 * dp));
+            }
+        };
         for (int64_t li = 0; li < n && ok; ++li) {
-            const int s = (int)(li & 1);
+            const int qs = (int)(li % kQSlots), ks = (int)(li % kKSlots);
             const int64_t i = i0 + li, r = i / a.Cc;
             const int c = (int)(i % a.Cc), p = (int)(r % a.Pp);
-            ok = mbar_wait(&full[s], (uint32_t)(li >> 1) & 1, 911);
+            ok = mbar_wait(&qfull[qs], (uint32_t)(li / kQSlots) & 1, 913);
+            if (ok) ok = mbar_wait(&kfull[ks], (uint32_t)(li / kKSlots) & 1, 914);
             if (!ok) break;
             const int h = 2 * p + jh;
             const bool live = (c * kTok + row < a.N) && h < a.H;
             const int hg = live ? h : 0;
-            uint8_t* sb = stages + s * kStageBytes;
-            phi_inplace_sw128<true>(sb, row, jh * 4, a.norm ? a.gq + hg * kD : nullptr, a.eps,
-                                    a.norm != 0, !live);
-            phi_inplace_sw128<true>(sb + kTile, row, jh * 4, a.norm ? a.gk + hg * kD : nullptr, a.eps,
-                                    a.norm != 0, !live);
-            // V^T of this head: column `row` (key j = row) of rows e = 0..31
-            if (li >= 1) ok = mbar_wait(u2done, (uint32_t)(li - 1) & 1, 912);
+            phi_inplace_sw128<true>(qring + qs * kTile, row, jh * 4, a.norm ? a.gq + hg * kD : nullptr,
+                                    a.eps, a.norm != 0, !live);
+            phi_inplace_sw128<true>(kring + ks * kTile, row, jh * 4, a.norm ? a.gk + hg * kD : nullptr,
+                                    a.eps, a.norm != 0, !live);
+            fence_proxy_async_smem();
+            mbar_arrive(&qkready[li & 1]);
+            // the prefix operand, hi / lo bf16 as pass 2 builds it
+            if (li == 0) {
+                pdl_wait_primary();                               // the states come from the prefix kernel
+                load_pre(0);
+            }
+            if (li >= 2) ok = mbar_wait(&bempty[li & 1], (uint32_t)((li >> 1) - 1) & 1, 915);
             if (!ok) break;
-            uint4 u[4];
+            uint8_t* dst = bop + (li & 1) * kBopBytes;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc)
-                u[cc] = *reinterpret_cast<const uint4*>(sb + 2 * kTile + sw128_offset(row, jh * 4 + cc));
-            uint8_t* vh = vt + jh * kVtHead + (row >> 6) * kVtAtom;
-            const int kch = (row & 63) >> 3, kb = (row & 7) * 2;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const uint32_t wds[4] = {u[cc].x, u[cc].y, u[cc].z, u[cc].w};
-#pragma unroll
-                for (int k2 = 0; k2 < 4; ++k2) {
-                    const int e = cc * 8 + k2 * 2;
-                    *reinterpret_cast<uint16_t*>(vh + sw128_offset(e, kch) + kb) = (uint16_t)(wds[k2] & 0xffffu);
-                    *reinterpret_cast<uint16_t*>(vh + sw128_offset(e + 1, kch) + kb) = (uint16_t)(wds[k2] >> 16);
-                }
+            for (int k = 0; k < kPrePer; ++k) {
+                const int it = t + k * kGroupThreads;
+                if (it >= 2 * kDP * (kD / 2)) continue;
+                const int dp = it % (kD / 2), e = (it / (kD / 2)) % kDP, jj = it / (kD / 2 * kDP);
+                const int d0 = 2 * dp;
+                const float h0 = __bfloat162float(__float2bfloat16_rn(pv[k].x));
+                const float h1 = __bfloat162float(__float2bfloat16_rn(pv[k].y));
+                const int chunk = jj * 4 + d0 / 8, boff = (d0 % 8) * 2;
+                const int lorow = e < kD ? p2::kLoRow + e : p2::kDenLo;   // hi row is e (kDenHi for e = D)
+                *reinterpret_cast<uint32_t*>(dst + sw128_offset(e, chunk) + boff) = pack_bf16x2(h0, h1);
+                *reinterpret_cast<uint32_t*>(dst + sw128_offset(lorow, chunk) + boff) =
+                    pack_bf16x2(pv[k].x - h0, pv[k].y - h1);
             }
             fence_proxy_async_smem();
-            mbar_arrive(&aready[s]);
+            mbar_arrive(&bfull[li & 1]);
+            if (li + 1 < n) load_pre(li + 1);
         }
-    } else {
+    } else if (warp >= 12) {
         // ------------------------------------------------ epilogues: warp w reads TMEM lane
-        // quadrant w % 4 (query row n = 32 (w % 4) + lane), head (w - 12) / 4 of the pair
-        const int ew = warp - 12, jh = ew >> 2, q = warp & 3, nrow = 32 * q + lane;
+        // quadrant q = w % 4 (query row n = 32 q + lane); its half hh = (w - 12) / 4 takes
+        // key blocks {hh, hh + 2} of P (blocks after the quadrant are masked whole and
+        // stay zero in P_s) and value columns 16 hh .. 16 hh + 15 of D.
+        const int hh = (warp - 12) >> 2, q = warp & 3, nrow = 32 * q + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-        for (int64_t li = 0; li < n && ok; ++li) {
-            const int s = (int)(li & 1);
-            ok = mbar_wait(pdone, (uint32_t)li & 1, 913);
-            if (ok && li >= 1) ok = mbar_wait(u2done, (uint32_t)(li - 1) & 1, 914);
-            if (!ok) break;
+        const int64_t nsub = 2 * n;
+        auto epi_a = [&](int64_t u) -> bool {
+            const int tb = (int)(u % kTmemBufs), pb = (int)(u & 1);
+            if (!mbar_wait(&pdone[tb], (uint32_t)(u / kTmemBufs) & 1, 916)) return false;
+            if (u >= 2 && !mbar_wait(&u2done[pb], (uint32_t)((u >> 1) - 1) & 1, 917)) return false;
             tc_fence_after_sync();
-            // P_h[n][j] for j <= n, as bf16 into the K-major A operand of U2
-            uint8_t* ph = ps + jh * kPsHead;
+            uint8_t* pbuf = ps + pb * kPsBuf;
+            float rs = 0.f;
 #pragma unroll 1
-            for (int kc = 0; kc < kTok / 32; ++kc) {
+            for (int kk = 0; kk < 2; ++kk) {
+                const int kc = hh + 2 * kk;                       // block of 32 keys
+                if (kc > q) continue;
                 float v[32];
-                tmem_ld16(lane_base + kPCol + 128 * jh + 32 * kc, v);
-                tmem_ld16(lane_base + kPCol + 128 * jh + 32 * kc + 16, v + 16);
+                tmem_ld16(lane_base + tb * kBufCols + 32 * kc, v);
+                tmem_ld16(lane_base + tb * kBufCols + 32 * kc + 16, v + 16);
                 tmem_wait_ld();
+                if (kc == q) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (32 * kc + i > nrow) v[i] = 0.f;
-                uint8_t* at = ph + (kc >> 1) * kPsAtom;
+                    for (int i = 0; i < 32; ++i)
+                        if (i > lane) v[i] = 0.f;
+                }
+                uint8_t* at = pbuf + (kc >> 1) * kPsAtom;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     uint4 w;
@@ -403,41 +454,57 @@ causal_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
                     w.w = pack_bf16x2(v[8 * cc + 6], v[8 * cc + 7]);
                     *reinterpret_cast<uint4*>(at + sw128_offset(nrow, (kc & 1) * 4 + cc)) = w;
                 }
+                float r4[4] = {0.f, 0.f, 0.f, 0.f};                // four chains
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r4[i & 3] += v[i];
+                rs += (r4[0] + r4[1]) + (r4[2] + r4[3]);
             }
+            rowsum[((u % kTmemBufs) * 2 + hh) * kTok + nrow] = rs;
             tc_fence_before_sync();
             fence_proxy_async_smem();
-            mbar_arrive(psready);
-            // O = (hi + lo) / (den_hi + den_lo + eps), over the Q tile of the stage
-            ok = mbar_wait(mmadone, (uint32_t)li & 1, 915);
-            if (!ok) break;
+            mbar_arrive(&psready[pb]);
+            return true;
+        };
+        auto epi_b = [&](int64_t u) -> bool {
+            const int64_t li = u >> 1;
+            const int j = (int)(u & 1), tb = (int)(u % kTmemBufs);
+            if (!mbar_wait(&mmadone[tb], (uint32_t)(u / kTmemBufs) & 1, 918)) return false;
             tc_fence_after_sync();
-            const uint32_t ta = lane_base + kDCol + p2::kN * jh;
-            float hi[kD + 2], lo[kD];
-            tmem_ld16(ta, hi);
-            tmem_ld16(ta + 16, hi + 16);
-            tmem_ld2(ta + p2::kDenHi, hi + kD);
-            tmem_ld16(ta + p2::kLoRow, lo);
-            tmem_ld16(ta + p2::kLoRow + 16, lo + 16);
+            const uint32_t ta = lane_base + tb * kBufCols;
+            float hi[16], lo[16], den[2];
+            tmem_ld16(ta + 16 * hh, hi);
+            tmem_ld2(ta + p2::kDenHi, den);
+            tmem_ld16(ta + p2::kLoRow + 16 * hh, lo);
             tmem_wait_ld();
-            const float inv = __frcp_rn((hi[kD] + hi[kD + 1]) + a.eps);
-            uint8_t* ot = stages + s * kStageBytes;
+            // the row sums of A(u) (this thread's and its partner warp's), read before the
+            // buffer is handed back: A(u + 4) rewrites them once every thread has arrived
+            if (!mbar_wait(&psready[u & 1], (uint32_t)(u >> 1) & 1, 919)) return false;
+            const float intra = rowsum[(tb * 2 + 0) * kTok + nrow] + rowsum[(tb * 2 + 1) * kTok + nrow];
+            tc_fence_before_sync();
+            mbar_arrive(&tfree[tb]);
+            const float inv = __frcp_rn(((den[0] + den[1]) + intra) + a.eps);
+            uint8_t* ot = qring + (li % kQSlots) * kTile;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < 2; ++cc) {
                 float o[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) o[u] = (hi[8 * cc + u] + lo[8 * cc + u]) * inv;
+                for (int x = 0; x < 8; ++x) o[x] = (hi[8 * cc + x] + lo[8 * cc + x]) * inv;
                 uint4 w;
                 w.x = pack_bf16x2(o[0], o[1]);
                 w.y = pack_bf16x2(o[2], o[3]);
                 w.z = pack_bf16x2(o[4], o[5]);
                 w.w = pack_bf16x2(o[6], o[7]);
-                *reinterpret_cast<uint4*>(ot + sw128_offset(nrow, jh * 4 + cc)) = w;
+                *reinterpret_cast<uint4*>(ot + sw128_offset(nrow, j * 4 + 2 * hh + cc)) = w;
             }
-            tc_fence_before_sync();
             fence_proxy_async_smem();
-            mbar_arrive(tfree);
-            mbar_arrive(ofull);
+            mbar_arrive(&ofull[li % kQSlots]);
+            return true;
+        };
+        for (int64_t u = 0; u < nsub && ok; ++u) {
+            ok = epi_a(u);
+            if (ok && u >= 1) ok = epi_b(u - 1);
         }
+        if (ok && nsub > 0) ok = epi_b(nsub - 1);
     }
     tc_fence_before_sync();
     __syncthreads();

@@ -54,7 +54,10 @@ Plan make_plan(int64_t B, int64_t N, int H) {
 // every smaller count.
 constexpr int kMaxPersistentCtas = 160;
 constexpr int kP1StageTok = p1::kStageTok;
-constexpr int kMinItemsPerCta = 4;
+#ifndef SANA_MIN_ITEMS
+#define SANA_MIN_ITEMS 4
+#endif
+constexpr int kMinItemsPerCta = SANA_MIN_ITEMS;
 
 struct PersistPlan1 {
     int G, R, Smax, P;   // head groups, stages per row, partial slots per row, CTAs
@@ -404,7 +407,9 @@ int launch_causal_tc(const void* q, const void* k, const void* v, const float* g
     PrefixArgs ap{};
     ap.part = part; ap.pre = pre; ap.H = H; ap.G = G; ap.Cc = (int)Cc; ap.Smax = 2;
     ap.R1 = kR; ap.T1 = T1; ap.P1 = P1;
-    causal_prefix_states<<<(unsigned)(B * H), kStateFloats / 4, 0, st>>>(ap);
+    causal_prefix_states<<<(unsigned)(B * H), kPrefixThreads, 0, st>>>(ap);
+    rc = launch_status();
+    if (rc != SANA_OK) return rc;
     CUtensorMap tq, tk2, tv2, to;
     if (!make_tmap_bnc(&tq, q, B, N, C, ca::kTok) || !make_tmap_bnc(&tk2, k, B, N, C, ca::kTok) ||
         !make_tmap_bnc(&tv2, v, B, N, C, ca::kTok) || !make_tmap_bnc(&to, out, B, N, C, ca::kTok))
@@ -413,8 +418,8 @@ int launch_causal_tc(const void* q, const void* k, const void* v, const float* g
     a3.pre = pre; a3.gq = gq; a3.gk = gk; a3.N = (int)N; a3.H = H;
     a3.Pp = (H + 1) / 2; a3.Cc = (int)Cc; a3.T = B * a3.Pp * Cc;
     a3.P = (int)(a3.T < P ? a3.T : P); a3.eps = eps; a3.norm = gq != nullptr;
-    causal_apply_tc<<<a3.P, ca::kThreads, ca::kSmemBytes, st>>>(tq, tk2, tv2, to, a3);
-    return launch_status();
+    return launch_pdl(causal_apply_tc, dim3(a3.P), ca::kThreads, ca::kSmemBytes, st, true, tq, tk2, tv2,
+                      to, a3);
 }
 
 // The fused variant: F1 (K, V projection + state), then F2 (Q projection + apply)

@@ -862,12 +862,17 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
         };
 
         // The first segment's B operand, built by all worker threads at once with plain
-        // loads: one round trip to L2 instead of the builder's rounds of bulk copies,
-        // which would otherwise stand between pass 1's end and the first UMMA.  Slots
-        // are summed in the builder's order, so the state is the same bit for bit.
+        // loads: one round trip to memory instead of the builder's rounds of bulk
+        // copies, which would otherwise stand between pass 1's end and the first UMMA.
         // Thread item (j, e, dp): S_j[e][2dp], S_j[e][2dp + 1], consecutive threads
-        // along d (coalesced in the partials' [e][d] layout).
+        // along d (coalesced in the partials' [e][d] layout); a thread's items and up
+        // to kBatch slots of each are loaded before any is summed.  Slots are summed
+        // in the builder's order, so the state is the same bit for bit.
         auto build_first = [&]() {
+            constexpr int kItems = kPairHeads * kDP * (kD / 2);
+            constexpr int kWorkers = kWorkerWarps * 32;
+            constexpr int kPer = (kItems + kWorkers - 1) / kWorkers;
+            constexpr int kBatch = 8;
             pdl_wait_primary();                                  // the states come from pass 1
             const int64_t r = i0 / a.R;
             const int b = (int)(r / a.Pp), p = (int)(r % a.Pp);
@@ -875,44 +880,62 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
             const int ns = a.kv == nullptr
                                ? p1_row_slots((int64_t)b * a.G1 + h0 / p1::kGroupHeads, a.R1, a.T1, a.P1)
                                : 1;
-            for (int it = threadIdx.x - 128; it < kPairHeads * kDP * (kD / 2); it += kWorkerWarps * 32) {
+            const int tid = threadIdx.x - 128;
+            float x0[kPer], x1[kPer];
+            size_t off[kPer];
+            bool live[kPer];
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int it = tid + u * kWorkers;
+                const int dp = it % (kD / 2), e = (it / (kD / 2)) % kDP, jj = it / (kD / 2 * kDP);
+                live[u] = it < kItems && jj < nh;
+                const size_t bh = (size_t)b * a.H + h0 + jj;
+                off[u] = a.kv == nullptr ? bh * a.Smax1 * kStateFloats + e * kD + 2 * dp
+                                         : bh * kStateFloats + 2 * dp * kDP + e;
+                x0[u] = 0.f;
+                x1[u] = 0.f;
+            }
+            if (a.kv == nullptr) {
+                for (int s0 = 0; s0 < ns; s0 += kBatch) {
+                    float2 v[kBatch][kPer];
+#pragma unroll
+                    for (int ss = 0; ss < kBatch; ++ss)
+#pragma unroll
+                        for (int u = 0; u < kPer; ++u)
+                            v[ss][u] = live[u] && s0 + ss < ns
+                                           ? __ldcg(reinterpret_cast<const float2*>(
+                                                 a.part + off[u] + (size_t)(s0 + ss) * kStateFloats))
+                                           : make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int ss = 0; ss < kBatch; ++ss)
+#pragma unroll
+                        for (int u = 0; u < kPer; ++u)
+                            if (s0 + ss < ns) {
+                                x0[u] += v[ss][u].x;
+                                x1[u] += v[ss][u].y;
+                            }
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < kPer; ++u)
+                    if (live[u]) {
+                        x0[u] = __ldcg(a.kv + off[u]);
+                        x1[u] = __ldcg(a.kv + off[u] + kDP);
+                    }
+            }
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int it = tid + u * kWorkers;
+                if (it >= kItems) continue;
                 const int dp = it % (kD / 2), e = (it / (kD / 2)) % kDP, jj = it / (kD / 2 * kDP);
                 const int d0 = 2 * dp;
-                float x0 = 0.f, x1 = 0.f;
-                if (jj < nh) {
-                    const size_t bh = (size_t)b * a.H + h0 + jj;
-                    if (a.kv == nullptr) {
-                        const float* src = a.part + bh * a.Smax1 * kStateFloats + e * kD + d0;
-                        int s = 0;
-                        for (; s + 4 <= ns; s += 4) {
-                            float2 v[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                v[u] = __ldcg(reinterpret_cast<const float2*>(src + (size_t)(s + u) * kStateFloats));
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                x0 += v[u].x;
-                                x1 += v[u].y;
-                            }
-                        }
-                        for (; s < ns; ++s) {
-                            const float2 v = __ldcg(reinterpret_cast<const float2*>(src + (size_t)s * kStateFloats));
-                            x0 += v.x;
-                            x1 += v.y;
-                        }
-                    } else {
-                        const float* src = a.kv + bh * kStateFloats;
-                        x0 = __ldcg(src + d0 * kDP + e);
-                        x1 = __ldcg(src + (d0 + 1) * kDP + e);
-                    }
-                }
-                const float hx0 = __bfloat162float(__float2bfloat16_rn(x0));
-                const float hx1 = __bfloat162float(__float2bfloat16_rn(x1));
-                const int chunk = jj * 4 + d0 / 8, off = (d0 % 8) * 2;
+                const float hx0 = __bfloat162float(__float2bfloat16_rn(x0[u]));
+                const float hx1 = __bfloat162float(__float2bfloat16_rn(x1[u]));
+                const int chunk = jj * 4 + d0 / 8, boff = (d0 % 8) * 2;
                 const int lorow = e < kD ? kLoRow + e : kDenLo;   // hi row is e (kDenHi for e = kD)
-                *reinterpret_cast<uint32_t*>(bop + sw128_offset(e, chunk) + off) = pack_bf16x2(hx0, hx1);
-                *reinterpret_cast<uint32_t*>(bop + sw128_offset(lorow, chunk) + off) =
-                    pack_bf16x2(x0 - hx0, x1 - hx1);
+                *reinterpret_cast<uint32_t*>(bop + sw128_offset(e, chunk) + boff) = pack_bf16x2(hx0, hx1);
+                *reinterpret_cast<uint32_t*>(bop + sw128_offset(lorow, chunk) + boff) =
+                    pack_bf16x2(x0[u] - hx0, x1[u] - hx1);
             }
             fence_proxy_async_smem();
             mbar_arrive(bfirst);
