@@ -994,12 +994,16 @@ def causal_measure(args, sla, sets, stream, world, hbm_gbs):
     achieved = wb.tokens * 2 * PASS_BYTES_PER_TOKEN / (parts[big]["ms"] * 1e-3) / 1e9
     return {"value": tot_tok * world / (tot_ms * 1e-3) / 1e6, "unit": "Mtokens/s",
             "ms_per_step": tot_ms, "steps": steps, "parts": parts,
-            "chunk_tokens": 64,
+            "chunk_tokens": 128,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
                          "frac": achieved / hbm_gbs, "traffic": None,
-                         "kernel": "kv_partial_simt + causal_scan + causal_apply_simt (CUDA cores)",
+                         "kernel": "kv_partials_persistent<chunked> + causal_prefix_states + causal_apply_tc "
+                                   "(tensor cores; bf16 with gains 16-byte aligned)",
                          "workload": wb.name,
-                         "algorithmic_bytes_per_launch": wb.tokens * 2 * PASS_BYTES_PER_TOKEN},
+                         "algorithmic_bytes_per_launch": wb.tokens * 2 * PASS_BYTES_PER_TOKEN,
+                         # the two-pass design reads K and V twice (chunk states, then the apply)
+                         "design_bytes_per_launch": wb.tokens * 3 * PASS_BYTES_PER_TOKEN,
+                         "frac_of_design_bytes": achieved * 1.5 / hbm_gbs},
             "gpu_launches": steps * len(sets) * 3}
 
 
@@ -1200,8 +1204,9 @@ def mixffn_measure(args, sla, rank, dev, stream, world, bf16_tf, hbm_gbs, peak_k
 
 
 def profile_case(args):
-    """--warmup calls of sana_linattn_forward (two kernel launches each) on one
-    workload, optionally with another batch size; prints a checksum."""
+    """--warmup calls of sana_linattn_forward (two kernel launches each; with --causal
+    sana_linattn_forward_causal, three) on one workload, optionally with another batch
+    size; prints a checksum."""
     import torch
 
     import relu_linear_attention_attn_b200 as sla
@@ -1212,8 +1217,12 @@ def profile_case(args):
     if args.batch:
         w = w.scaled(B=args.batch)
     x = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in make_inputs(w).items()}
-    ws = torch.empty(sla.workspace_bytes(w.B, w.N, w.C, w.H, fused=fused),
-                     dtype=torch.uint8, device="cuda")
+    if args.causal:
+        ws = torch.empty(int(sla.load().sana_linattn_workspace_bytes(w.B, w.N, w.C, w.H, 2)),
+                         dtype=torch.uint8, device="cuda")
+    else:
+        ws = torch.empty(sla.workspace_bytes(w.B, w.N, w.C, w.H, fused=fused),
+                         dtype=torch.uint8, device="cuda")
     if args.workload == "w8a8":
         Wq, sw = sla.quantize_cols_i8(x["W"])
     for _ in range(args.warmup):
@@ -1222,6 +1231,8 @@ def profile_case(args):
         elif args.workload == "w8a8":
             xq, sx = sla.quantize_rows_i8(x["x"])
             out = sla.qkv_fused_w8a8(xq, sx, Wq, sw, x["gq"], x["gk"], w.H, w.eps, workspace=ws)
+        elif args.causal:
+            out = sla.forward_causal(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps, workspace=ws)
         else:
             out = sla.forward(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps, workspace=ws)
     torch.cuda.synchronize()
@@ -1244,6 +1255,8 @@ def main():
     ap.add_argument("--profile-case", action="store_true",
                     help="no timing: run --warmup forward calls of --workload and exit (a small, "
                          "fixed launch sequence for ncu captures)")
+    ap.add_argument("--causal", action="store_true",
+                    help="with --profile-case: the prefix (causal) form")
     ap.add_argument("--batch", type=int, default=0,
                     help="with --profile-case: batch size override for the workload")
     ap.add_argument("--concurrency", choices=["streams", "serial"], default="streams",
