@@ -71,29 +71,39 @@ causal_prefix_states(const PrefixArgs a)
         }
         __syncthreads();
     }
+    // Slot 0 of every chunk and slot 1 where it exists are loaded for a whole batch of
+    // chunks before any is summed (straight-line predicated loads: a run-time slot
+    // loop would leave one round trip per chunk); chunks with more than two slots
+    // (never produced by the chunked pass 1) take the general loop.
     float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int c0 = 0; c0 < a.Cc; c0 += kBatch) {
-        float4 x[kBatch];
+        float4 v0[kBatch], v1[kBatch];
+        int nsk[kBatch];
 #pragma unroll
         for (int k = 0; k < kBatch; ++k) {
-            x[k] = make_float4(0.f, 0.f, 0.f, 0.f);
             const int c = c0 + k;
-            if (c < a.Cc) {
-                const int ns = table ? 1 + (int)((split[c >> 5] >> (c & 31)) & 1u)
-                                     : p1_row_slots(row0 + c, a.R1, a.T1, a.P1);
-                for (int s = 0; s < ns; ++s) {
-                    const float4 v = __ldcg(src + ((int64_t)c * a.Smax + s) * (kStateFloats / 4) + i4);
-                    x[k].x += v.x; x[k].y += v.y; x[k].z += v.z; x[k].w += v.w;
-                }
-            }
+            nsk[k] = c < a.Cc ? (table ? 1 + (int)((split[c >> 5] >> (c & 31)) & 1u)
+                                       : p1_row_slots(row0 + c, a.R1, a.T1, a.P1))
+                              : 0;
         }
 #pragma unroll
         for (int k = 0; k < kBatch; ++k) {
+            const float4* sc = src + (int64_t)(c0 + k) * a.Smax * (kStateFloats / 4) + i4;
+            v0[k] = nsk[k] > 0 ? __ldcg(sc) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v1[k] = nsk[k] > 1 ? __ldcg(sc + kStateFloats / 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            if (nsk[k] == 0) continue;
             const int c = c0 + k;
-            if (c < a.Cc) {
-                dst[(int64_t)c * (kStateFloats / 4) + i4] = run;
-                run.x += x[k].x; run.y += x[k].y; run.z += x[k].z; run.w += x[k].w;
+            float4 x = v0[k];                              // slot order: 0, 1, then the rest
+            if (nsk[k] > 1) { x.x += v1[k].x; x.y += v1[k].y; x.z += v1[k].z; x.w += v1[k].w; }
+            for (int s = 2; s < nsk[k]; ++s) {
+                const float4 v = __ldcg(src + ((int64_t)c * a.Smax + s) * (kStateFloats / 4) + i4);
+                x.x += v.x; x.y += v.y; x.z += v.z; x.w += v.w;
             }
+            dst[(int64_t)c * (kStateFloats / 4) + i4] = run;
+            run.x += x.x; run.y += x.y; run.z += x.z; run.w += x.w;
         }
     }
 }
