@@ -27,7 +27,14 @@ def run(lib, d, w):
                                WORKLOADS["2048px-b8-lognormal"].scaled(B=1, N=1000, seed=94),
                                WORKLOADS["1024px-b1"].scaled(N=129, C=160, H=5, seed=96),
                                WORKLOADS["4096px-b2-overflow"].scaled(B=3, N=640, seed=97),
-                               WORKLOADS["1024px-b1"].scaled(B=2, N=2049, seed=98)],
+                               WORKLOADS["1024px-b1"].scaled(B=2, N=2049, seed=98),
+                               # chunk edges of the tensor-core form (128-token chunks):
+                               # one chunk exactly, one short of it, two and a token,
+                               # one head, and more rows than CTAs
+                               WORKLOADS["1024px-b1"].scaled(N=128, C=64, H=2, seed=100),
+                               WORKLOADS["1024px-b1"].scaled(N=127, C=96, H=3, seed=101),
+                               WORKLOADS["1024px-b1"].scaled(B=2, N=257, C=32, H=1, seed=102),
+                               WORKLOADS["1024px-b1"].scaled(B=5, N=512, C=448, H=14, seed=103)],
                          ids=lambda w: f"{w.dtype}-B{w.B}-N{w.N}-{w.gains}")
 def test_causal_small_full_parity(cuda_lib, w):
     x = make_inputs(w)

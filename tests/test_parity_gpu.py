@@ -77,7 +77,8 @@ def test_ragged_shapes_full_parity(cuda_lib, recipe, gains, B, N):
     (1, 1, 70, "gaussian", "random"), (1, 64, 70, "lognormal", "ones"),
     (1, 129, 70, "overflow", "off"), (1, 1000, 70, "gaussian", "random"),
     (1, 1024, 70, "overflow", "off"), (2, 384, 6, "gaussian", "random"),
-    (1, 500, 5, "lognormal", "random"), (3, 256, 70, "gaussian", "ones")])
+    (1, 500, 5, "lognormal", "random"), (3, 256, 70, "gaussian", "ones"),
+    (2, 300, 1, "gaussian", "random")])
 def test_short_sequences_full_parity(cuda_lib, B, N, H, recipe, gains):
     """Short sequences (N <= 1024, few work items per CTA, many partial slots per
     row): ragged token counts and head counts that leave a head group or a head
