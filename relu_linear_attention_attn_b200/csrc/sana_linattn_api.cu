@@ -270,6 +270,8 @@ int persistent_ctas() {
                              cudaFuncAttributeMaxDynamicSharedMemorySize, p1::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(kv_partials_persistent<true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, p1::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(kv_partials_persistent<false, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, p1::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(apply_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              p2::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(fused_kv<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -328,7 +330,7 @@ int launch_pdl(void (*kernel)(Args...), dim3 grid, int threads, int smem, cudaSt
 // ([B][H][Smax][D+1][D]); nothing else is written.
 int launch_partials_tc(const void* k, const void* v, const float* gk, float* part, int64_t B,
                        int64_t N, int C, int H, float eps, cudaStream_t st,
-                       PersistPlan1* plan_out) {
+                       PersistPlan1* plan_out, const float* w = nullptr) {
     const int P = persistent_ctas();
     if (P == 0) return SANA_ECUDA;
     CUtensorMap tk, tv;
@@ -339,8 +341,11 @@ int launch_partials_tc(const void* k, const void* v, const float* gk, float* par
     P1Args a{};
     a.gk = gk; a.part = part; a.T = pl.T; a.Cc = 1;
     a.N = (int)N; a.H = H; a.G = pl.G; a.R = pl.R; a.Smax = pl.Smax; a.P = pl.P;
-    a.eps = eps; a.norm = gk != nullptr;
+    a.eps = eps; a.norm = gk != nullptr; a.w = w;
     if (plan_out) *plan_out = pl;
+    if (w)
+        return launch_pdl(kv_partials_persistent<false, true>, dim3(pl.P), p1::kThreads,
+                          p1::kSmemBytes, st, true, tk, tv, a);
     return launch_pdl(kv_partials_persistent<false>, dim3(pl.P), p1::kThreads, p1::kSmemBytes, st,
                       true, tk, tv, a);
 }
@@ -549,6 +554,13 @@ size_t sana_linattn_backward_workspace_bytes(int64_t B, int64_t N, int C, int H)
     return off;
 }
 
+// The backward forms [dS | dz] on the tensor cores (bf16 phi(Q) and dnum) from this
+// many tokens on.  For very short sequences the key gradients are a small difference
+// of O(1) terms (one token: dphi(K) = phi(Q) (dnum . V + dden) = O(eps)), which the
+// bf16 rounding of the operands would dominate; there the fp32 CUDA-core reduction
+// runs instead.
+constexpr int64_t kBwdTcMinTokens = 128;
+
 int sana_linattn_backward(const void* q, const void* k, const void* v, const float* gq,
                           const float* gk, const void* dout, void* dq, void* dk, void* dv,
                           float* dgq, float* dgk, int64_t B, int64_t N, int C, int H, float eps,
@@ -609,11 +621,29 @@ int sana_linattn_backward(const void* q, const void* k, const void* v, const flo
             launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, Sz, B, N, H, C, C, eps, p,
                                stream);
         }
-        bwd_query_simt<bf16><<<gt, kBwdTile, 0, stream>>>((const bf16*)q, (const bf16*)dout, gq, Sz,
-                                                          (bf16*)dq, G, gpq, N, H, eps, nrm);
-        outer_partial_simt<bf16><<<gs, 128, 0, stream>>>((const bf16*)q, gq, G, part, N, H, p.S,
-                                                         p.tps, eps, nrm);
-        kv_combine<<<(unsigned)(B * H), 256, 0, stream>>>(part, dSz, p.S);
+        if (tc_path(dtype, C) && N >= kBwdTcMinTokens) {
+            // [dS | dz] = sum_t phi(Q)_t^T [dnum_t | dden_t] on the tensor cores: pass 1 with
+            // q in K's place (its gains gq), dnum in V's, the normaliser column weighted
+            // by dden.  dnum (bf16, (B, N, C)) and dden (fp32, (B, N, H)) use the space of
+            // the [dnum | dden] rows: B N H (64 + 4) bytes + 16 of padding <= B N H 132.
+            bf16* dnum = (bf16*)G;
+            float* dden = (float*)((char*)G + align_up((size_t)B * N * C * sizeof(bf16), 16));
+            bwd_query_simt<bf16><<<gt, kBwdTile, 0, stream>>>((const bf16*)q, (const bf16*)dout, gq,
+                                                              Sz, (bf16*)dq, nullptr, gpq, N, H,
+                                                              eps, nrm, dnum, dden);
+            PersistPlan1 pl{};
+            if ((rc = launch_status()) != SANA_OK ||
+                (rc = launch_partials_tc(q, dnum, gq, part, B, N, C, H, eps, stream, &pl, dden)) !=
+                    SANA_OK ||
+                (rc = launch_combine_tc(part, dSz, B, H, pl, stream)) != SANA_OK)
+                return rc;
+        } else {
+            bwd_query_simt<bf16><<<gt, kBwdTile, 0, stream>>>((const bf16*)q, (const bf16*)dout, gq,
+                                                              Sz, (bf16*)dq, G, gpq, N, H, eps, nrm);
+            outer_partial_simt<bf16><<<gs, 128, 0, stream>>>((const bf16*)q, gq, G, part, N, H,
+                                                             p.S, p.tps, eps, nrm);
+            kv_combine<<<(unsigned)(B * H), 256, 0, stream>>>(part, dSz, p.S);
+        }
         bwd_key_simt<bf16><<<gt, kBwdTile, 0, stream>>>((const bf16*)k, (const bf16*)v, gk, dSz,
                                                         (bf16*)dk, (bf16*)dv, gpk, N, H, eps, nrm);
     } else {

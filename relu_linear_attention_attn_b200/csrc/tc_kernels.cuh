@@ -133,7 +133,8 @@ template <bool kScaleByRms>
 __device__ __forceinline__ void phi2_inplace_sw128(uint8_t* const tile[2], const int row[2],
                                                    const int chunk0[2], const float* const g[2],
                                                    float eps, bool norm, const bool zero[2],
-                                                   float r_out[2], float* sum) {
+                                                   float r_out[2], float* sum,
+                                                   const float* wsum = nullptr) {
     uint4 u[2][4];
 #pragma unroll
     for (int it = 0; it < 2; ++it)
@@ -173,7 +174,17 @@ __device__ __forceinline__ void phi2_inplace_sw128(uint8_t* const tile[2], const
             u[it][c].y = pack_bf16x2(x[8 * c + 2], x[8 * c + 3]);
             u[it][c].z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
             u[it][c].w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
-            if (sum) {
+            if (sum && wsum) {                      // column sums weighted per item
+                const float wv = wsum[it];
+                sum[8 * c + 0] = fmaf(bf16lo(u[it][c].x), wv, sum[8 * c + 0]);
+                sum[8 * c + 1] = fmaf(bf16hi(u[it][c].x), wv, sum[8 * c + 1]);
+                sum[8 * c + 2] = fmaf(bf16lo(u[it][c].y), wv, sum[8 * c + 2]);
+                sum[8 * c + 3] = fmaf(bf16hi(u[it][c].y), wv, sum[8 * c + 3]);
+                sum[8 * c + 4] = fmaf(bf16lo(u[it][c].z), wv, sum[8 * c + 4]);
+                sum[8 * c + 5] = fmaf(bf16hi(u[it][c].z), wv, sum[8 * c + 5]);
+                sum[8 * c + 6] = fmaf(bf16lo(u[it][c].w), wv, sum[8 * c + 6]);
+                sum[8 * c + 7] = fmaf(bf16hi(u[it][c].w), wv, sum[8 * c + 7]);
+            } else if (sum) {
                 sum[8 * c + 0] += bf16lo(u[it][c].x); sum[8 * c + 1] += bf16hi(u[it][c].x);
                 sum[8 * c + 2] += bf16lo(u[it][c].y); sum[8 * c + 3] += bf16hi(u[it][c].y);
                 sum[8 * c + 4] += bf16lo(u[it][c].z); sum[8 * c + 5] += bf16hi(u[it][c].z);
@@ -236,6 +247,8 @@ static_assert(kStages >= 2 && kStages % 2 == 0, "ring slots must be even");
 
 struct P1Args {
     const float* gk;     // gains [C], or nullptr with the norm off
+    const float* w;      // kWeighted: per token-head weights [B][N][H] of the normaliser
+                         // column (sum_t phi(K)[t] w[t] in place of sum_t phi(K)[t])
     float* part;         // partial states [B][H][Smax][D+1][D]  (column e major);
                          // chunked: [B][H][Cc][Smax][D+1][D]
     int64_t T;           // work items: B * G rows x R stages (chunked: B * G * Cc rows)
@@ -247,8 +260,10 @@ struct P1Args {
 
 // One row per (b, g) over the whole sequence (the forward's state), or, with
 // kChunked, one row per (b, g, chunk of R stages): the states of the sequence's
-// chunks, which the prefix (causal) form scans.
-template <bool kChunked>
+// chunks, which the prefix (causal) form scans.  kWeighted (the backward's
+// [dS | dz] = sum_t phi(Q)_t^T [dnum_t | dden_t]): the normaliser column is
+// sum_t phi(K)[t] w[t] with w per token and head.
+template <bool kChunked, bool kWeighted = false>
 __global__ void __launch_bounds__(p1::kThreads, 1)
 kv_partials_persistent(const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v, const P1Args a)
@@ -418,7 +433,16 @@ kv_partials_persistent(const __grid_constant__ CUtensorMap tmap_k,
                                       !((tbase + t * kStageTok + lane + 32 < a.N) && (h < a.H))};
                 const float* gg[2] = {sgain + (h < a.H ? h : 0) * kD, sgain + (h < a.H ? h : 0) * kD};
                 float rr[2];
-                phi2_inplace_sw128<true>(tl, rows, ch, gg, a.eps, a.norm != 0, dead, rr, ks);
+                float wv[2] = {1.f, 1.f};
+                if (kWeighted) {
+                    const int64_t bb = (kChunked ? r / a.Cc : r) / a.G;
+                    for (int it = 0; it < 2; ++it) {
+                        const int64_t tok = tbase + (int64_t)t * kStageTok + rows[it];
+                        wv[it] = dead[it] ? 0.f : __ldg(a.w + (bb * a.N + tok) * a.H + h);
+                    }
+                }
+                phi2_inplace_sw128<true>(tl, rows, ch, gg, a.eps, a.norm != 0, dead, rr, ks,
+                                         kWeighted ? wv : nullptr);
                 fence_proxy_async_smem();
                 mbar_arrive(&aready[st]);
             }
