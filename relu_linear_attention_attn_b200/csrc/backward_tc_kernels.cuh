@@ -1,0 +1,433 @@
+// The key side of the backward of Eq. (1) ("Sana: Efficient High-Resolution Image
+// Synthesis with Linear Diffusion Transformers", section 2.1) with the per-head
+// QK-RMSNorm feature map of "SANA 1.5 ...", section "Model architecture", on the
+// tensor cores (bf16 inputs and outputs, fp32 accumulation).  With the gradient
+// state [dS | dz] of every (b, h) (dS[d][e] = sum_t phi(Q)_t[d] dnum_t[e],
+// dz[d] = sum_t phi(Q)_t[d] dden_t), per key token t and head h:
+//     dV_t[e]      = sum_d phi(K)_t[d] dS[d][e]
+//     dphi(K)_t[d] = sum_e dS[d][e] V_t[e] + dz[d]
+// then the feature map's backward gives dK and the per-channel gain gradient.
+//
+// bwd_key_tc: work item = one 128-token tile of one row (b, head pair), persistent
+// CTAs over a balanced flat list as in the forward's pass 2.  Per row segment a
+// builder warp writes two B operands per head from [dS | dz] (fp32, read from
+// global memory), K-major, 64 rows each: rows 0..31 the bf16 "hi" parts, rows
+// 32..63 the "lo" parts (x - bf16(x)), so one UMMA covers both:
+//     Bop1[n = e][k = d] = dS[d][e]        (for dV)
+//     Bop2[n = d][k = e] = dS[d][e]        (for dphi(K))
+// The workers rewrite the K tile in place as ReLU(g k) (r = 1/rms kept in a
+// register); per head two UMMAs each (M = 128, N = 64, K = 16)
+//     D1 = ReLU(g k) Bop1,   D2 = V Bop2        (V straight from its tile, K-major)
+// and the epilogue forms dV = r (D1[e] + D1[32 + e]) over the V tile, dphi(K) =
+// D2[d] + D2[32 + d] + dz[d], the feature map's backward with the raw k row (read
+// again from global memory) over the K tile, and a store warp TMA-stores both.
+// Gain gradients: each warp's 32 rows are summed per channel (butterfly) and
+// written per (tile, quadrant, head); `gain_combine_tiles` sums them in a fixed
+// order, so the result is reproducible.
+//
+// TMEM: warp w reads lanes 32 * (w % 4) .. + 31; D row i is lane i.
+#pragma once
+
+#include "sana_common.cuh"
+#include "sm100_primitives.cuh"
+#include "tc_kernels.cuh"
+
+namespace sana {
+
+namespace bk {
+constexpr int kTileTok = 128;                      // UMMA M
+constexpr int kTileBytes = kTileTok * 128;         // 128 tokens x 64 channels (a head pair)
+constexpr int kStageBytes = 2 * kTileBytes;        // [K | V]
+constexpr int kStages = 4;
+constexpr int kN = 64;                             // B rows per head: 32 hi, 32 lo
+constexpr int kBopBytes = kN * 128;                // both heads side by side in each row
+constexpr int kBopSet = 2 * kBopBytes;             // Bop1, Bop2 of a row segment
+constexpr int kBopRing = 2;
+constexpr int kBufCols = 4 * kN;                   // [D1 head 0 | D1 head 1 | D2 head 0 | D2 head 1]
+constexpr int kTmemCols = 2 * kBufCols;            // one buffer per tile group
+constexpr int kWorkerWarps = 16;                   // two tile groups of 8
+constexpr int kGroupThreads = 32 * kWorkerWarps / 2;
+constexpr int kThreads = 32 * (4 + kWorkerWarps);  // TMA, UMMA, builder, store, workers
+constexpr int kGainCache = 4096;
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBopRing * kBopSet + kGainCache * 4 + 1024;
+static_assert(kStages % 2 == 0, "each ring slot must belong to one worker group");
+static_assert(kTmemCols <= 512, "TMEM");
+static_assert(kSmemBytes <= 232448, "shared memory");
+}  // namespace bk
+
+struct BkArgs {
+    const float* dsz;    // [dS | dz]: [B][H][D][D+1]
+    const float* gk;     // gains [C] or nullptr (norm off)
+    const bf16* k;       // raw keys (B, N, C), for the feature map's backward
+    float* gpart;        // gain partials [T][4 quadrants][2 heads][D] (norm on)
+    int64_t T;           // work items: B * Pp rows x R tiles
+    int N, H, Pp, R, P;
+    float eps;
+    int norm;
+};
+
+__global__ void __launch_bounds__(bk::kThreads, 1)   // 640 threads: at most 96 registers
+bwd_key_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+           const __grid_constant__ CUtensorMap tmap_dk, const __grid_constant__ CUtensorMap tmap_dv,
+           const BkArgs a)
+{
+    using namespace bk;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align_1024(smem_raw);
+    uint8_t* stages = smem;
+    uint8_t* bop = stages + kStages * kStageBytes;
+    float* sgain = (float*)(bop + kBopRing * kBopSet);
+    uint64_t* full = (uint64_t*)(sgain + kGainCache);
+    uint64_t* aready = full + kStages;
+    uint64_t* mmadone = aready + kStages;
+    uint64_t* tready = mmadone + kStages;
+    uint64_t* empty = tready + kStages;
+    uint64_t* tfree = empty + kStages;                  // 2: one per tile group
+    uint64_t* bfull = tfree + 2;
+    uint64_t* bempty = bfull + kBopRing;
+    uint64_t* drain = bempty + kBopRing;
+    uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+
+    const int64_t c = blockIdx.x;
+    const int64_t i0 = range_begin(c, a.T, a.P), i1 = range_begin(c + 1, a.T, a.P);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int C = a.H * kD;                      // at most kGainCache (checked on the host)
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&aready[i], kGroupThreads);
+            mbar_init(&mmadone[i], 1);
+            mbar_init(&tready[i], kGroupThreads);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) mbar_init(&tfree[i], kGroupThreads);
+        for (int i = 0; i < kBopRing; ++i) {
+            mbar_init(&bfull[i], 32);
+            mbar_init(&bempty[i], 1);
+        }
+        mbar_init(drain, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmap_k);
+        prefetch_tmap(&tmap_v);
+        prefetch_tmap(&tmap_dk);
+        prefetch_tmap(&tmap_dv);
+    }
+    if (a.norm)
+        for (int i = threadIdx.x; i < C; i += blockDim.x) sgain[i] = a.gk[i];
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    // [dS | dz] and the keys' gradients come from earlier launches on this stream
+    pdl_wait_primary();
+    bool ok = i1 > i0;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (K and V tiles)
+        if (lane == 0 && ok) {
+            int64_t last = -1;
+            for (int64_t li = 0; i0 + li < i1; ++li) {
+                const int st = (int)(li % kStages);
+                if (li >= kStages) ok = mbar_wait(&empty[st], (uint32_t)((li / kStages) - 1) & 1, 601);
+                if (!ok) break;
+                const int64_t i = i0 + li, r = i / a.R;
+                const int t = (int)(i % a.R), b = (int)(r / a.Pp), p = (int)(r % a.Pp);
+                uint8_t* sb = stages + st * kStageBytes;
+                mbar_arrive_expect_tx(&full[st], kStageBytes);
+                tma_load_3d(sb, &tmap_k, &full[st], p * 64, t * kTileTok, b);
+                tma_load_3d(sb + kTileBytes, &tmap_v, &full[st], p * 64, t * kTileTok, b);
+                last = li;
+            }
+            if (!ok) {   // let every issued copy land before the CTA can exit
+                for (int64_t lj = last - (kStages - 1) > 0 ? last - (kStages - 1) : 0; lj <= last; ++lj)
+                    mbar_wait(&full[lj % kStages], (uint32_t)(lj / kStages) & 1, 602);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ UMMA issuer (lane 0 alone)
+        if (ok && lane == 0) {
+            const uint32_t idesc = make_idesc_bf16(128, kN, false, false);
+            const uint64_t s0 = make_smem_desc(smem_u32(stages), 16, 1024, kSwizzle128B);
+            const uint64_t b0 = make_smem_desc(smem_u32(bop), 16, 1024, kSwizzle128B);
+            const int64_t n = i1 - i0;
+            int seg = 0;
+            int64_t t = i0 % a.R;
+            for (int64_t li = 0; li < n && ok; ++li) {
+                const bool first = (li == 0) || (t == 0);
+                const bool lastt = (li + 1 == n) || (t == a.R - 1);
+                const int st = (int)(li % kStages), tb = (int)(li & 1), rb = seg & 1;
+                if (first) ok = mbar_wait(&bfull[rb], (uint32_t)(seg >> 1) & 1, 603);
+                if (ok) ok = mbar_wait(&aready[st], (uint32_t)(li / kStages) & 1, 604);
+                if (ok && li >= 2) ok = mbar_wait(&tfree[tb], (uint32_t)((li >> 1) - 1) & 1, 605);
+                if (!ok) break;
+                tc_fence_after_sync();
+                const uint64_t kd = s0 + (uint64_t)((st * kStageBytes) >> 4);
+                const uint64_t vd = kd + (uint64_t)(kTileBytes >> 4);
+                const uint64_t b1 = b0 + (uint64_t)((rb * kBopSet) >> 4);
+                const uint64_t b2 = b1 + (uint64_t)(kBopBytes >> 4);
+                const uint32_t d = tmem + tb * kBufCols;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    umma_bf16(d + j * kN, kd + 4 * j, b1 + 4 * j, idesc, false);
+                    umma_bf16(d + j * kN, kd + 4 * j + 2, b1 + 4 * j + 2, idesc, true);
+                    umma_bf16(d + (2 + j) * kN, vd + 4 * j, b2 + 4 * j, idesc, false);
+                    umma_bf16(d + (2 + j) * kN, vd + 4 * j + 2, b2 + 4 * j + 2, idesc, true);
+                }
+                umma_commit(&mmadone[st]);
+                if (lastt) {
+                    umma_commit(&bempty[rb]);
+                    ++seg;
+                }
+                if (++t == a.R) t = 0;
+            }
+            umma_commit(drain);
+            mbar_wait(drain, 0, 606);
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ------------------------------------------------ B operands of each row segment
+        // lane = d: the row dS[d][0..31] and dz[d] of each head of the pair
+        int seg = 0;
+        for (int64_t li = 0; i0 + li < i1 && ok; ++li) {
+            const int64_t i = i0 + li;
+            if (!(li == 0 || i % a.R == 0)) continue;              // not a segment start
+            const int rb = seg & 1;
+            if (seg >= 2) ok = mbar_wait(&bempty[rb], (uint32_t)((seg >> 1) - 1) & 1, 607);
+            if (!ok) break;
+            const int64_t r = i / a.R;
+            const int b = (int)(r / a.Pp), p = (int)(r % a.Pp);
+            const int h0 = 2 * p, nh = min(2, a.H - h0);
+            uint8_t* b1 = bop + rb * kBopSet;
+            uint8_t* b2 = b1 + kBopBytes;
+            const int d0 = lane & ~1;
+#pragma unroll 1
+            for (int j = 0; j < 2; ++j) {
+                float x[kD];
+                const float* src = a.dsz + ((size_t)b * a.H + h0 + j) * kStateFloats + lane * kDP;
+#pragma unroll
+                for (int e = 0; e < kD; ++e) x[e] = j < nh ? __ldg(src + e) : 0.f;
+                // Bop2: row n = d (this lane), K = e: lanes write their own rows, pairs of e
+#pragma unroll
+                for (int e = 0; e < kD; e += 2) {
+                    const float h_0 = __bfloat162float(__float2bfloat16_rn(x[e]));
+                    const float h_1 = __bfloat162float(__float2bfloat16_rn(x[e + 1]));
+                    const int chunk = j * 4 + e / 8, off = (e % 8) * 2;
+                    *reinterpret_cast<uint32_t*>(b2 + sw128_offset(lane, chunk) + off) = pack_bf16x2(h_0, h_1);
+                    *reinterpret_cast<uint32_t*>(b2 + sw128_offset(kD + lane, chunk) + off) =
+                        pack_bf16x2(x[e] - h_0, x[e + 1] - h_1);
+                }
+                // Bop1: row n = e, K = d: lane pairs (d, d + 1) write one bf16x2 each, even
+                // lanes the hi part, odd lanes the lo part
+                const int chunk = j * 4 + d0 / 8, off = (d0 % 8) * 2;
+#pragma unroll
+                for (int e = 0; e < kD; ++e) {
+                    const float xv = x[e];
+                    const float xp = __shfl_xor_sync(0xffffffffu, xv, 1);
+                    const float xe = (lane & 1) ? xp : xv, xo = (lane & 1) ? xv : xp;
+                    const float he = __bfloat162float(__float2bfloat16_rn(xe));
+                    const float ho = __bfloat162float(__float2bfloat16_rn(xo));
+                    const int row = (lane & 1) ? kD + e : e;
+                    const uint32_t w = (lane & 1) ? pack_bf16x2(xe - he, xo - ho) : pack_bf16x2(he, ho);
+                    *reinterpret_cast<uint32_t*>(b1 + sw128_offset(row, chunk) + off) = w;
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            mbar_arrive(&bfull[rb]);
+            ++seg;
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------ dK, dV stores (over the K, V tiles)
+        if (lane == 0 && ok) {
+            int64_t li = 0;
+            for (; i0 + li < i1 && ok; ++li) {
+                const int st = (int)(li % kStages);
+                ok = mbar_wait(&tready[st], (uint32_t)(li / kStages) & 1, 608);
+                if (!ok) break;
+                const int64_t i = i0 + li, r = i / a.R;
+                const int t = (int)(i % a.R), b = (int)(r / a.Pp), p = (int)(r % a.Pp);
+                uint8_t* sb = stages + st * kStageBytes;
+                tma_store_3d(&tmap_dk, sb, p * 64, t * kTileTok, b);
+                tma_store_3d(&tmap_dv, sb + kTileBytes, p * 64, t * kTileTok, b);
+                bulk_commit_group();
+                bulk_wait_group_read<0>();
+                mbar_arrive(&empty[st]);
+            }
+            bulk_wait_group<0>();
+        }
+    } else {
+        // ------------------------------------------------ ReLU(g k), then the epilogue
+        // Two tile groups of 8 warps take alternate tiles; in a group, warp w takes TMEM
+        // quadrant w % 4 (token rows 32 (w % 4) ..) and head (w / 4) % 2 of the pair.
+        const int wi = warp - 4;                          // 0..15
+        const int grp = wi >> 3;                          // tiles with li % 2 == grp
+        const int j = (wi >> 2) & 1;                      // head of the pair
+        const int q = warp & 3;                           // TMEM lane quadrant
+        const int row = 32 * q + lane;                    // token row of the tile
+        auto transform = [&](int64_t li, float& rk) -> bool {
+            const int st = (int)(li % kStages);
+            if (!mbar_wait(&full[st], (uint32_t)(li / kStages) & 1, 609)) return false;
+            const int64_t i = i0 + li, r = i / a.R;
+            const int t = (int)(i % a.R), p = (int)(r % a.Pp);
+            const int h = p * 2 + j;
+            const bool live = (t * kTileTok + row < a.N) && h < a.H;
+            rk = phi_inplace_sw128<false>(stages + st * kStageBytes, row, j * 4,
+                                          sgain + (live ? h : 0) * kD, a.eps, a.norm != 0, !live);
+            fence_proxy_async_smem();
+            mbar_arrive(&aready[st]);
+            return true;
+        };
+        auto epilogue = [&](int64_t li, float rk) -> bool {
+            const int st = (int)(li % kStages), tb = (int)(li & 1);
+            if (!mbar_wait(&mmadone[st], (uint32_t)(li / kStages) & 1, 610)) return false;
+            tc_fence_after_sync();
+            const int64_t i = i0 + li, r = i / a.R;
+            const int t = (int)(i % a.R), b = (int)(r / a.Pp), p = (int)(r % a.Pp);
+            const int h = p * 2 + j;
+            const int64_t tok = (int64_t)t * kTileTok + row;
+            const bool live = tok < a.N && h < a.H;
+            uint8_t* ktile = stages + st * kStageBytes;
+            uint8_t* vtile = ktile + kTileBytes;
+            const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * kBufCols;
+            // dV = r (D1 hi + lo), over this head's columns of the V tile (V was read by
+            // the UMMA that completed mmadone)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float hi[16], lo[16];
+                tmem_ld16(ta + j * kN + 16 * hf, hi);
+                tmem_ld16(ta + j * kN + kD + 16 * hf, lo);
+                tmem_wait_ld();
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    float o[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) o[u] = (hi[8 * cc + u] + lo[8 * cc + u]) * rk;
+                    uint4 w;
+                    w.x = pack_bf16x2(o[0], o[1]);
+                    w.y = pack_bf16x2(o[2], o[3]);
+                    w.z = pack_bf16x2(o[4], o[5]);
+                    w.w = pack_bf16x2(o[6], o[7]);
+                    *reinterpret_cast<uint4*>(vtile + sw128_offset(row, j * 4 + 2 * hf + cc)) = w;
+                }
+            }
+            // dphi(K) = D2 hi + lo + dz (dz from global memory: the builder's ring slot may
+            // already hold a later segment's operands)
+            float dp[kD];
+            const float* dz = a.dsz + ((size_t)b * a.H + (h < a.H ? h : 0)) * kStateFloats + kD;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float hi[16], lo[16];
+                tmem_ld16(ta + (2 + j) * kN + 16 * hf, hi);
+                tmem_ld16(ta + (2 + j) * kN + kD + 16 * hf, lo);
+                tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 16; ++u) dp[16 * hf + u] = (hi[u] + lo[u]) + __ldg(dz + (16 * hf + u) * kDP);
+            }
+            tc_fence_before_sync();
+            mbar_arrive(&tfree[tb]);
+            // the feature map's backward with the raw k row: du = dphi where g k r > 0;
+            // dk = g r du - r^3 (sum du g k / D) k; the gain term du k r
+            float x[kD];
+            if (live) {
+                const bf16* kr = a.k + ((size_t)b * a.N + tok) * (size_t)(a.H * kD) + (size_t)h * kD;
+#pragma unroll
+                for (int u = 0; u < kD; u += 8) load8(kr + u, x + u);
+            } else {
+#pragma unroll
+                for (int u = 0; u < kD; ++u) x[u] = 0.f;
+            }
+            const float* g = sgain + (h < a.H ? h : 0) * kD;
+            if (a.norm) {
+                float tsum = 0.f;
+#pragma unroll
+                for (int u = 0; u < kD; ++u) {
+                    const float gu = g[u];
+                    dp[u] = gu * x[u] > 0.f ? dp[u] : 0.f;            // du (r > 0)
+                    tsum = fmaf(dp[u] * gu, x[u], tsum);
+                }
+                const float cf = rk * rk * rk * tsum * (1.f / kD);
+#pragma unroll
+                for (int u = 0; u < kD; ++u) {
+                    const float gterm = dp[u] * x[u] * rk;             // gain gradient share
+                    dp[u] = g[u] * rk * dp[u] - cf * x[u];             // dk
+                    x[u] = gterm;
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < kD; ++u) dp[u] = x[u] > 0.f ? dp[u] : 0.f;
+            }
+            if (!live) {
+#pragma unroll
+                for (int u = 0; u < kD; ++u) { dp[u] = 0.f; x[u] = 0.f; }
+            }
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint4 w;
+                w.x = pack_bf16x2(dp[8 * cc + 0], dp[8 * cc + 1]);
+                w.y = pack_bf16x2(dp[8 * cc + 2], dp[8 * cc + 3]);
+                w.z = pack_bf16x2(dp[8 * cc + 4], dp[8 * cc + 5]);
+                w.w = pack_bf16x2(dp[8 * cc + 6], dp[8 * cc + 7]);
+                *reinterpret_cast<uint4*>(ktile + sw128_offset(row, j * 4 + cc)) = w;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&tready[st]);
+            if (a.norm) {                                 // the warp's 32 rows, per channel
+                warp_reduce_scatter32(x, lane);
+                a.gpart[((size_t)i * 4 + q) * (2 * kD) + j * kD + lane] = x[0];
+            }
+            return true;
+        };
+
+        int64_t prev = -1;
+        float r_prev = 1.f, r_cur = 1.f;
+        for (int64_t li = grp; i0 + li < i1 && ok; li += 2) {
+            ok = transform(li, r_cur);
+            if (ok && prev >= 0) ok = epilogue(prev, r_prev);
+            prev = li;
+            r_prev = r_cur;
+        }
+        if (ok && prev >= 0) ok = epilogue(prev, r_prev);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// dg[c] for c = h D + d (head pair p = h / 2, j = h % 2) = the sum over batch items,
+// the row's tiles and the 4 quadrants of gpart[(b Pp + p) R + t][quadrant][j][d], in
+// that order within each of 4 interleaved streams, the streams then added in order.
+// Grid Pp, 256 threads (stream s = thread / 64, channel j D + d = thread % 64).
+__global__ void __launch_bounds__(256)
+gain_combine_tiles(const float* __restrict__ gpart, float* __restrict__ dg, int B, int Pp, int R,
+                   int H)
+{
+    __shared__ float part[4][2 * kD];
+    const int p = blockIdx.x, s = threadIdx.x >> 6, ch = threadIdx.x & 63;
+    const int64_t per_b = (int64_t)R * 4;                  // entries per batch item
+    const int64_t total = (int64_t)B * per_b;
+    float acc = 0.f;
+    for (int64_t k = s; k < total; k += 4) {
+        const int64_t b = k / per_b, rem = k % per_b;      // rem = t * 4 + quadrant
+        acc += gpart[(((b * Pp + p) * R) * 4 + rem) * (2 * kD) + ch];
+    }
+    part[s][ch] = acc;
+    __syncthreads();
+    if (threadIdx.x < 2 * kD) {
+        const float v = ((part[0][ch] + part[1][ch]) + part[2][ch]) + part[3][ch];
+        const int h = 2 * p + ch / kD;
+        if (h < H) dg[h * kD + ch % kD] = v;
+    }
+}
+
+}  // namespace sana

@@ -13,6 +13,7 @@
 #include "sm100_primitives.cuh"
 #include "tc_kernels.cuh"
 #include "fused_kernels.cuh"
+#include "backward_tc_kernels.cuh"
 #include "quant_kernels.cuh"
 #include "causal_kernels.cuh"
 #include "backward_kernels.cuh"
@@ -283,7 +284,9 @@ int persistent_ctas() {
         cudaFuncSetAttribute(fused_qo<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              f2::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(causal_apply_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             ca::kSmemBytes) != cudaSuccess)
+                             ca::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(bwd_key_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bk::kSmemBytes) != cudaSuccess)
         return 0;
     // each persistent kernel must fit one CTA on an SM (registers, threads, smem)
     int n1 = 0, n2 = 0, n3 = 0, n4 = 0;
@@ -551,7 +554,32 @@ size_t sana_linattn_backward_workspace_bytes(int64_t B, int64_t N, int C, int H)
     off = align_up(off + (size_t)B * H * kStateFloats * 4, 256);         // [dS | dz]
     off = align_up(off + (size_t)B * N * H * kGrow * 4, 256);            // [dnum | dden] rows
     off = align_up(off + (size_t)2 * B * tiles * C * 4, 256);            // gain partials
+    // the key side on the tensor cores: gain partials per (tile, quadrant, head pair)
+    const int64_t Tk = B * ((H + 1) / 2) * tiles;
+    off = align_up(off + (size_t)Tk * 4 * 2 * kD * 4, 256);
     return off;
+}
+
+// The key side of the backward on the tensor cores (bwd_key_tc): dK, dV and the
+// per-tile gain partials from [dS | dz].
+int launch_bwd_key_tc(const void* k, const void* v, const float* gk, const float* dsz, void* dk,
+                      void* dv, float* gpart, int64_t B, int64_t N, int C, int H, float eps,
+                      cudaStream_t st) {
+    const int P = persistent_ctas();
+    if (P == 0) return SANA_ECUDA;
+    CUtensorMap tk, tv, tdk, tdv;
+    if (!make_tmap_bnc(&tk, k, B, N, C, bk::kTileTok) || !make_tmap_bnc(&tv, v, B, N, C, bk::kTileTok) ||
+        !make_tmap_bnc(&tdk, dk, B, N, C, bk::kTileTok) ||
+        !make_tmap_bnc(&tdv, dv, B, N, C, bk::kTileTok))
+        return SANA_ECUDA;
+    BkArgs a{};
+    a.dsz = dsz; a.gk = gk; a.k = (const bf16*)k; a.gpart = gpart;
+    a.N = (int)N; a.H = H; a.Pp = (H + 1) / 2; a.R = (int)((N + bk::kTileTok - 1) / bk::kTileTok);
+    a.T = B * a.Pp * (int64_t)a.R;
+    a.P = (int)(a.T < P ? a.T : P);
+    a.eps = eps; a.norm = gk != nullptr;
+    return launch_pdl(bwd_key_tc, dim3(a.P), bk::kThreads, bk::kSmemBytes, st, true, tk, tv, tdk,
+                      tdv, a);
 }
 
 // The backward forms [dS | dz] on the tensor cores (bf16 phi(Q) and dnum) from this
@@ -608,6 +636,8 @@ int sana_linattn_backward(const void* q, const void* k, const void* v, const flo
     off = align_up(off + (size_t)B * N * H * kGrow * 4, 256);
     float* gpq = (float*)(w + off);
     float* gpk = gpq + (size_t)B * tiles * C;
+    off = align_up(off + (size_t)2 * B * tiles * C * 4, 256);
+    float* gpk_tc = (float*)(w + off);
     const dim3 gs(p.S, H, (unsigned)B), gt((unsigned)tiles, H, (unsigned)B);
     const int nrm = norm ? 1 : 0;
     if (dtype == SANA_BF16) {
@@ -643,6 +673,18 @@ int sana_linattn_backward(const void* q, const void* k, const void* v, const flo
             outer_partial_simt<bf16><<<gs, 128, 0, stream>>>((const bf16*)q, gq, G, part, N, H,
                                                              p.S, p.tps, eps, nrm);
             kv_combine<<<(unsigned)(B * H), 256, 0, stream>>>(part, dSz, p.S);
+        }
+        if (tc_path(dtype, C) && N >= kBwdTcMinTokens) {
+            if ((rc = launch_status()) != SANA_OK ||
+                (rc = launch_bwd_key_tc(k, v, gk, dSz, dk, dv, gpk_tc, B, N, C, H, eps, stream)) !=
+                    SANA_OK)
+                return rc;
+            if (norm) {
+                gain_combine<<<(C + 255) / 256, 256, 0, stream>>>(gpq, dgq, B * tiles, C);
+                gain_combine_tiles<<<(unsigned)((H + 1) / 2), 256, 0, stream>>>(
+                    gpk_tc, dgk, (int)B, (H + 1) / 2, (int)tiles, H);
+            }
+            return launch_status();
         }
         bwd_key_simt<bf16><<<gt, kBwdTile, 0, stream>>>((const bf16*)k, (const bf16*)v, gk, dSz,
                                                         (bf16*)dk, (bf16*)dv, gpk, N, H, eps, nrm);
