@@ -286,7 +286,9 @@ int persistent_ctas() {
         cudaFuncSetAttribute(causal_apply_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              ca::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(bwd_key_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bk::kSmemBytes) != cudaSuccess)
+                             bk::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(bwd_query_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bq::kSmemBytes) != cudaSuccess)
         return 0;
     // each persistent kernel must fit one CTA on an SM (registers, threads, smem)
     int n1 = 0, n2 = 0, n3 = 0, n4 = 0;
@@ -557,6 +559,8 @@ size_t sana_linattn_backward_workspace_bytes(int64_t B, int64_t N, int C, int H)
     // the key side on the tensor cores: gain partials per (tile, quadrant, head pair)
     const int64_t Tk = B * ((H + 1) / 2) * tiles;
     off = align_up(off + (size_t)Tk * 4 * 2 * kD * 4, 256);
+    off = align_up(off + (size_t)((H + 1) / 2) * kGainSlices * 2 * kD * 4, 256);   // their slices
+    off = align_up(off + (size_t)Tk * 4 * 2 * kD * 4, 256);                         // query side
     return off;
 }
 
@@ -580,6 +584,29 @@ int launch_bwd_key_tc(const void* k, const void* v, const float* gk, const float
     a.eps = eps; a.norm = gk != nullptr;
     return launch_pdl(bwd_key_tc, dim3(a.P), bk::kThreads, bk::kSmemBytes, st, true, tk, tv, tdk,
                       tdv, a);
+}
+
+// The query side of the backward on the tensor cores (bwd_query_tc): dQ, dnum (bf16,
+// (B, N, C)), dden ((B, N, H) fp32) and the per-tile gain partials from the states S.
+int launch_bwd_query_tc(const void* q, const void* dout, const float* gq, const float* s, void* dq,
+                        void* dnum, float* dden, float* gpart, int64_t B, int64_t N, int C, int H,
+                        float eps, cudaStream_t st) {
+    const int P = persistent_ctas();
+    if (P == 0) return SANA_ECUDA;
+    CUtensorMap tq, tg, tdq, tdn;
+    if (!make_tmap_bnc(&tq, q, B, N, C, bq::kTileTok) ||
+        !make_tmap_bnc(&tg, dout, B, N, C, bq::kTileTok) ||
+        !make_tmap_bnc(&tdq, dq, B, N, C, bq::kTileTok) ||
+        !make_tmap_bnc(&tdn, dnum, B, N, C, bq::kTileTok))
+        return SANA_ECUDA;
+    BqArgs a{};
+    a.s = s; a.gq = gq; a.q = (const bf16*)q; a.dden = dden; a.gpart = gpart;
+    a.N = (int)N; a.H = H; a.Pp = (H + 1) / 2; a.R = (int)((N + bq::kTileTok - 1) / bq::kTileTok);
+    a.T = B * a.Pp * (int64_t)a.R;
+    a.P = (int)(a.T < P ? a.T : P);
+    a.eps = eps; a.norm = gq != nullptr;
+    return launch_pdl(bwd_query_tc, dim3(a.P), bq::kThreads, bq::kSmemBytes, st, true, tq, tg, tdq,
+                      tdn, a);
 }
 
 // The backward forms [dS | dz] on the tensor cores (bf16 phi(Q) and dnum) from this
@@ -638,6 +665,10 @@ int sana_linattn_backward(const void* q, const void* k, const void* v, const flo
     float* gpk = gpq + (size_t)B * tiles * C;
     off = align_up(off + (size_t)2 * B * tiles * C * 4, 256);
     float* gpk_tc = (float*)(w + off);
+    off = align_up(off + (size_t)B * ((H + 1) / 2) * tiles * 4 * 2 * kD * 4, 256);
+    float* gslices = (float*)(w + off);
+    off = align_up(off + (size_t)((H + 1) / 2) * kGainSlices * 2 * kD * 4, 256);
+    float* gpq_tc = (float*)(w + off);
     const dim3 gs(p.S, H, (unsigned)B), gt((unsigned)tiles, H, (unsigned)B);
     const int nrm = norm ? 1 : 0;
     if (dtype == SANA_BF16) {
@@ -652,39 +683,40 @@ int sana_linattn_backward(const void* q, const void* k, const void* v, const flo
                                stream);
         }
         if (tc_path(dtype, C) && N >= kBwdTcMinTokens) {
-            // [dS | dz] = sum_t phi(Q)_t^T [dnum_t | dden_t] on the tensor cores: pass 1 with
-            // q in K's place (its gains gq), dnum in V's, the normaliser column weighted
-            // by dden.  dnum (bf16, (B, N, C)) and dden (fp32, (B, N, H)) use the space of
-            // the [dnum | dden] rows: B N H (64 + 4) bytes + 16 of padding <= B N H 132.
+            // Query side on the tensor cores: dQ, dnum (bf16, (B, N, C)) and dden (fp32,
+            // (B, N, H)) in the space of the [dnum | dden] rows (B N H (64 + 4) bytes + 16
+            // of padding <= B N H 132).  Then [dS | dz] = sum_t phi(Q)_t^T [dnum_t | dden_t]
+            // by pass 1 with q in K's place (its gains gq), dnum in V's and the normaliser
+            // column weighted by dden; then the key side, and the gain partials' sums.
             bf16* dnum = (bf16*)G;
             float* dden = (float*)((char*)G + align_up((size_t)B * N * C * sizeof(bf16), 16));
-            bwd_query_simt<bf16><<<gt, kBwdTile, 0, stream>>>((const bf16*)q, (const bf16*)dout, gq,
-                                                              Sz, (bf16*)dq, nullptr, gpq, N, H,
-                                                              eps, nrm, dnum, dden);
             PersistPlan1 pl{};
             if ((rc = launch_status()) != SANA_OK ||
+                (rc = launch_bwd_query_tc(q, dout, gq, Sz, dq, dnum, dden, gpq_tc, B, N, C, H, eps,
+                                          stream)) != SANA_OK ||
                 (rc = launch_partials_tc(q, dnum, gq, part, B, N, C, H, eps, stream, &pl, dden)) !=
                     SANA_OK ||
-                (rc = launch_combine_tc(part, dSz, B, H, pl, stream)) != SANA_OK)
+                (rc = launch_combine_tc(part, dSz, B, H, pl, stream)) != SANA_OK ||
+                (rc = launch_bwd_key_tc(k, v, gk, dSz, dk, dv, gpk_tc, B, N, C, H, eps, stream)) !=
+                    SANA_OK)
                 return rc;
+            if (norm) {
+                const int Pp = (H + 1) / 2;
+                const float* gp[2] = {gpq_tc, gpk_tc};
+                float* dg[2] = {dgq, dgk};
+                for (int x = 0; x < 2; ++x) {
+                    gain_combine_tiles<<<dim3((unsigned)Pp, kGainSlices), 256, 0, stream>>>(
+                        gp[x], gslices, (int)B, Pp, (int)tiles);
+                    gain_combine_slices<<<(C + 255) / 256, 256, 0, stream>>>(gslices, dg[x], Pp, H);
+                }
+            }
+            return launch_status();
         } else {
             bwd_query_simt<bf16><<<gt, kBwdTile, 0, stream>>>((const bf16*)q, (const bf16*)dout, gq,
                                                               Sz, (bf16*)dq, G, gpq, N, H, eps, nrm);
             outer_partial_simt<bf16><<<gs, 128, 0, stream>>>((const bf16*)q, gq, G, part, N, H,
                                                              p.S, p.tps, eps, nrm);
             kv_combine<<<(unsigned)(B * H), 256, 0, stream>>>(part, dSz, p.S);
-        }
-        if (tc_path(dtype, C) && N >= kBwdTcMinTokens) {
-            if ((rc = launch_status()) != SANA_OK ||
-                (rc = launch_bwd_key_tc(k, v, gk, dSz, dk, dv, gpk_tc, B, N, C, H, eps, stream)) !=
-                    SANA_OK)
-                return rc;
-            if (norm) {
-                gain_combine<<<(C + 255) / 256, 256, 0, stream>>>(gpq, dgq, B * tiles, C);
-                gain_combine_tiles<<<(unsigned)((H + 1) / 2), 256, 0, stream>>>(
-                    gpk_tc, dgk, (int)B, (H + 1) / 2, (int)tiles, H);
-            }
-            return launch_status();
         }
         bwd_key_simt<bf16><<<gt, kBwdTile, 0, stream>>>((const bf16*)k, (const bf16*)v, gk, dSz,
                                                         (bf16*)dk, (bf16*)dv, gpk, N, H, eps, nrm);
