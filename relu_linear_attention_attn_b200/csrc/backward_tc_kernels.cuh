@@ -297,6 +297,16 @@ bwd_key_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ C
             uint8_t* ktile = stages + st * kStageBytes;
             uint8_t* vtile = ktile + kTileBytes;
             const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * kBufCols;
+            // the raw k row for the feature map's backward, requested first so that its
+            // latency overlaps the TMEM work below
+            uint4 kraw[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                             make_uint4(0, 0, 0, 0)};
+            if (live) {
+                const uint4* kr = reinterpret_cast<const uint4*>(
+                    a.k + ((size_t)b * a.N + tok) * (size_t)(a.H * kD) + (size_t)h * kD);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) kraw[u] = __ldg(kr + u);
+            }
             // dV = r (D1 hi + lo), over this head's columns of the V tile (V was read by
             // the UMMA that completed mmadone)
 #pragma unroll
@@ -336,13 +346,14 @@ bwd_key_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ C
             // the feature map's backward with the raw k row: du = dphi where g k r > 0;
             // dk = g r du - r^3 (sum du g k / D) k; the gain term du k r
             float x[kD];
-            if (live) {
-                const bf16* kr = a.k + ((size_t)b * a.N + tok) * (size_t)(a.H * kD) + (size_t)h * kD;
 #pragma unroll
-                for (int u = 0; u < kD; u += 8) load8(kr + u, x + u);
-            } else {
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t kw[4] = {kraw[u].x, kraw[u].y, kraw[u].z, kraw[u].w};
 #pragma unroll
-                for (int u = 0; u < kD; ++u) x[u] = 0.f;
+                for (int v2 = 0; v2 < 4; ++v2) {
+                    x[8 * u + 2 * v2] = bf16lo(kw[v2]);
+                    x[8 * u + 2 * v2 + 1] = bf16hi(kw[v2]);
+                }
             }
             const float* g = sgain + (h < a.H ? h : 0) * kD;
             if (a.norm) {
@@ -771,6 +782,14 @@ bwd_query_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             const int64_t tok = (int64_t)t * kTileTok + row;
             const bool live = tok < a.N && h < a.H;
             const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + tb * kBufCols + j * kNS;
+            uint4 qraw[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                             make_uint4(0, 0, 0, 0)};
+            if (live) {                                   // requested before the TMEM work
+                const uint4* qr = reinterpret_cast<const uint4*>(
+                    a.q + ((size_t)b * a.N + tok) * (size_t)(a.H * kD) + (size_t)h * kD);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) qraw[u] = __ldg(qr + u);
+            }
             float dp[kD];
             const float* z = a.s + ((size_t)b * a.H + (h < a.H ? h : 0)) * kStateFloats + kD;
 #pragma unroll
@@ -786,13 +805,14 @@ bwd_query_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             tc_fence_before_sync();
             mbar_arrive(&tfree[tb]);
             float x[kD];
-            if (live) {
-                const bf16* qr = a.q + ((size_t)b * a.N + tok) * (size_t)(a.H * kD) + (size_t)h * kD;
 #pragma unroll
-                for (int u = 0; u < kD; u += 8) load8(qr + u, x + u);
-            } else {
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t qw[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
 #pragma unroll
-                for (int u = 0; u < kD; ++u) x[u] = 0.f;
+                for (int v2 = 0; v2 < 4; ++v2) {
+                    x[8 * u + 2 * v2] = bf16lo(qw[v2]);
+                    x[8 * u + 2 * v2 + 1] = bf16hi(qw[v2]);
+                }
             }
             const float* g = sgain + (h < a.H ? h : 0) * kD;
             if (a.norm) {
@@ -857,11 +877,11 @@ bwd_query_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
 
 // dg[c] for c = h D + d (head pair p = h / 2, j = h % 2) = the sum over batch items,
 // the row's tiles and the 4 quadrants of gpart[(b Pp + p) R + t][quadrant][j][d]:
-// grid (Pp, 8 slices of the tile list), 256 threads = 4 interleaved streams x 64
+// grid (Pp, 32 slices of the tile list), 256 threads = 4 interleaved streams x 64
 // channels; each stream adds its entries in order, the streams are added in order
 // into slice partials part[p][slice][64], and gain_combine_slices adds the slices in
 // order, so the result is reproducible.
-constexpr int kGainSlices = 8;
+constexpr int kGainSlices = 32;
 
 __global__ void __launch_bounds__(256)
 gain_combine_tiles(const float* __restrict__ gpart, float* __restrict__ part, int B, int Pp, int R)
