@@ -55,6 +55,58 @@ static_assert(kTmemCols <= 512, "TMEM");
 static_assert(kSmemBytes <= 232448, "shared memory");
 }  // namespace bk
 
+// The feature map's backward for one row of one head, in place: dp holds dphi on
+// entry (fp32), raw the row's 32 bf16 inputs (packed pairs), g its gains (norm on), r
+// its 1/rms.  du = dphi where g x r > 0 (x > 0 with the norm off);
+//   dx = g r du - r^3 (sum_u du g x / D) x        (norm on; dx = du with the norm off)
+// dx goes out as bf16 to the swizzled row `dst` (4 chunks from chunk0), and dp
+// returns the gain gradient's share du x r (zeros with the norm off or a dead row).
+__device__ __forceinline__ void phi_bwd_row(float* dp, const uint4 raw[4], const float* g, float r,
+                                            bool norm, bool live, uint8_t* tile, int row, int chunk0) {
+    auto xr = [&](int u) -> float {
+        const uint4 w4 = raw[u >> 3];
+        const int k = (u >> 1) & 3;
+        const uint32_t w = k == 0 ? w4.x : k == 1 ? w4.y : k == 2 ? w4.z : w4.w;
+        return (u & 1) ? bf16hi(w) : bf16lo(w);
+    };
+    float cf = 0.f;
+    if (norm) {
+        float tsum = 0.f;
+#pragma unroll
+        for (int u = 0; u < kD; ++u) {
+            const float x = xr(u), gu = g[u];
+            dp[u] = gu * x > 0.f ? dp[u] : 0.f;                   // du
+            tsum = fmaf(dp[u] * gu, x, tsum);
+        }
+        cf = r * r * r * tsum * (1.f / kD);
+    } else {
+#pragma unroll
+        for (int u = 0; u < kD; ++u) dp[u] = xr(u) > 0.f ? dp[u] : 0.f;
+    }
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+        float o[8];
+#pragma unroll
+        for (int u8 = 0; u8 < 8; ++u8) {
+            const int u = 8 * cc + u8;
+            const float x = xr(u), du = dp[u];
+            o[u8] = norm ? g[u] * r * du - cf * x : du;
+            dp[u] = norm ? du * x * r : 0.f;                       // gain share
+        }
+        uint4 w;
+        w.x = pack_bf16x2(o[0], o[1]);
+        w.y = pack_bf16x2(o[2], o[3]);
+        w.z = pack_bf16x2(o[4], o[5]);
+        w.w = pack_bf16x2(o[6], o[7]);
+        if (!live) w = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(tile + sw128_offset(row, chunk0 + cc)) = w;
+    }
+    if (!live) {
+#pragma unroll
+        for (int u = 0; u < kD; ++u) dp[u] = 0.f;
+    }
+}
+
 struct BkArgs {
     const float* dsz;    // [dS | dz]: [B][H][D][D+1]
     const float* gk;     // gains [C] or nullptr (norm off)
@@ -343,56 +395,14 @@ bwd_key_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ C
             }
             tc_fence_before_sync();
             mbar_arrive(&tfree[tb]);
-            // the feature map's backward with the raw k row: du = dphi where g k r > 0;
-            // dk = g r du - r^3 (sum du g k / D) k; the gain term du k r
-            float x[kD];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint32_t kw[4] = {kraw[u].x, kraw[u].y, kraw[u].z, kraw[u].w};
-#pragma unroll
-                for (int v2 = 0; v2 < 4; ++v2) {
-                    x[8 * u + 2 * v2] = bf16lo(kw[v2]);
-                    x[8 * u + 2 * v2 + 1] = bf16hi(kw[v2]);
-                }
-            }
-            const float* g = sgain + (h < a.H ? h : 0) * kD;
-            if (a.norm) {
-                float tsum = 0.f;
-#pragma unroll
-                for (int u = 0; u < kD; ++u) {
-                    const float gu = g[u];
-                    dp[u] = gu * x[u] > 0.f ? dp[u] : 0.f;            // du (r > 0)
-                    tsum = fmaf(dp[u] * gu, x[u], tsum);
-                }
-                const float cf = rk * rk * rk * tsum * (1.f / kD);
-#pragma unroll
-                for (int u = 0; u < kD; ++u) {
-                    const float gterm = dp[u] * x[u] * rk;             // gain gradient share
-                    dp[u] = g[u] * rk * dp[u] - cf * x[u];             // dk
-                    x[u] = gterm;
-                }
-            } else {
-#pragma unroll
-                for (int u = 0; u < kD; ++u) dp[u] = x[u] > 0.f ? dp[u] : 0.f;
-            }
-            if (!live) {
-#pragma unroll
-                for (int u = 0; u < kD; ++u) { dp[u] = 0.f; x[u] = 0.f; }
-            }
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint4 w;
-                w.x = pack_bf16x2(dp[8 * cc + 0], dp[8 * cc + 1]);
-                w.y = pack_bf16x2(dp[8 * cc + 2], dp[8 * cc + 3]);
-                w.z = pack_bf16x2(dp[8 * cc + 4], dp[8 * cc + 5]);
-                w.w = pack_bf16x2(dp[8 * cc + 6], dp[8 * cc + 7]);
-                *reinterpret_cast<uint4*>(ktile + sw128_offset(row, j * 4 + cc)) = w;
-            }
+            // the feature map's backward with the raw k row -> dK over the K tile
+            phi_bwd_row(dp, kraw, sgain + (h < a.H ? h : 0) * kD, rk, a.norm != 0, live, ktile, row,
+                        j * 4);
             fence_proxy_async_smem();
             mbar_arrive(&tready[st]);
             if (a.norm) {                                 // the warp's 32 rows, per channel
-                warp_reduce_scatter32(x, lane);
-                a.gpart[((size_t)i * 4 + q) * (2 * kD) + j * kD + lane] = x[0];
+                warp_reduce_scatter32(dp, lane);
+                a.gpart[((size_t)i * 4 + q) * (2 * kD) + j * kD + lane] = dp[0];
             }
             return true;
         };
@@ -804,55 +814,13 @@ bwd_query_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             }
             tc_fence_before_sync();
             mbar_arrive(&tfree[tb]);
-            float x[kD];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint32_t qw[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
-#pragma unroll
-                for (int v2 = 0; v2 < 4; ++v2) {
-                    x[8 * u + 2 * v2] = bf16lo(qw[v2]);
-                    x[8 * u + 2 * v2 + 1] = bf16hi(qw[v2]);
-                }
-            }
-            const float* g = sgain + (h < a.H ? h : 0) * kD;
-            if (a.norm) {
-                float tsum = 0.f;
-#pragma unroll
-                for (int u = 0; u < kD; ++u) {
-                    const float gu = g[u];
-                    dp[u] = gu * x[u] > 0.f ? dp[u] : 0.f;
-                    tsum = fmaf(dp[u] * gu, x[u], tsum);
-                }
-                const float cf = rq * rq * rq * tsum * (1.f / kD);
-#pragma unroll
-                for (int u = 0; u < kD; ++u) {
-                    const float gterm = dp[u] * x[u] * rq;
-                    dp[u] = g[u] * rq * dp[u] - cf * x[u];
-                    x[u] = gterm;
-                }
-            } else {
-#pragma unroll
-                for (int u = 0; u < kD; ++u) dp[u] = x[u] > 0.f ? dp[u] : 0.f;
-            }
-            if (!live) {
-#pragma unroll
-                for (int u = 0; u < kD; ++u) { dp[u] = 0.f; x[u] = 0.f; }
-            }
-            uint8_t* qtile = stages + st * kStageBytes;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint4 w;
-                w.x = pack_bf16x2(dp[8 * cc + 0], dp[8 * cc + 1]);
-                w.y = pack_bf16x2(dp[8 * cc + 2], dp[8 * cc + 3]);
-                w.z = pack_bf16x2(dp[8 * cc + 4], dp[8 * cc + 5]);
-                w.w = pack_bf16x2(dp[8 * cc + 6], dp[8 * cc + 7]);
-                *reinterpret_cast<uint4*>(qtile + sw128_offset(row, j * 4 + cc)) = w;
-            }
+            phi_bwd_row(dp, qraw, sgain + (h < a.H ? h : 0) * kD, rq, a.norm != 0, live,
+                        stages + st * kStageBytes, row, j * 4);
             fence_proxy_async_smem();
             mbar_arrive(&tready[st]);
             if (a.norm) {
-                warp_reduce_scatter32(x, lane);
-                a.gpart[((size_t)i * 4 + q) * (2 * kD) + j * kD + lane] = x[0];
+                warp_reduce_scatter32(dp, lane);
+                a.gpart[((size_t)i * 4 + q) * (2 * kD) + j * kD + lane] = dp[0];
             }
             return true;
         };
