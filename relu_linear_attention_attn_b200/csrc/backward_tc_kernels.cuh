@@ -38,7 +38,7 @@ namespace bk {
 constexpr int kTileTok = 128;                      // UMMA M
 constexpr int kTileBytes = kTileTok * 128;         // 128 tokens x 64 channels (a head pair)
 constexpr int kStageBytes = 2 * kTileBytes;        // [K | V]
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr int kN = 64;                             // B rows per head: 32 hi, 32 lo
 constexpr int kBopBytes = kN * 128;                // both heads side by side in each row
 constexpr int kBopSet = 2 * kBopBytes;             // Bop1, Bop2 of a row segment
@@ -50,7 +50,9 @@ constexpr int kGroupThreads = 32 * kWorkerWarps / 2;
 constexpr int kThreads = 32 * (4 + kWorkerWarps);  // TMA, UMMA, builder, store, workers
 constexpr int kGainCache = 4096;
 constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBopRing * kBopSet + kGainCache * 4 + 1024;
-static_assert(kStages % 2 == 0, "each ring slot must belong to one worker group");
+// (A slot may serve the two worker groups in turn: a group's use of slot s for tile
+// li + kStages starts after the tile in it before, li, has been stored, so the
+// per-slot barriers never see two tiles' arrivals at once.)
 static_assert(kTmemCols <= 512, "TMEM");
 static_assert(kSmemBytes <= 232448, "shared memory");
 }  // namespace bk
@@ -449,7 +451,7 @@ namespace bq {
 constexpr int kTileTok = 128;
 constexpr int kTileBytes = kTileTok * 128;
 constexpr int kStageBytes = 2 * kTileBytes;        // [Q | dO]
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr int kNS = p2::kN;                        // 80: pass 2's operand of S
 constexpr int kNT = 64;                            // S_v^T: 32 hi, 32 lo
 constexpr int kBopSBytes = kNS * 128;
@@ -463,7 +465,6 @@ constexpr int kGroupThreads = 32 * kWorkerWarps / 2;
 constexpr int kThreads = 32 * (4 + kWorkerWarps);
 constexpr int kGainCache = 4096;
 constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBopRing * kBopSet + kGainCache * 4 + 1024;
-static_assert(kStages % 2 == 0, "each ring slot must belong to one worker group");
 static_assert(kBopSBytes % 1024 == 0 && kBopSet % 1024 == 0, "operand alignment");
 static_assert(kSmemBytes <= 232448, "shared memory");
 }  // namespace bq
