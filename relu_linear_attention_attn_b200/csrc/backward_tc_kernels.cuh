@@ -16,7 +16,8 @@
 //     Bop1[n = e][k = d] = dS[d][e]        (for dV)
 //     Bop2[n = d][k = e] = dS[d][e]        (for dphi(K))
 // The workers rewrite the K tile in place as ReLU(g k) (r = 1/rms kept in a
-// register); per head two UMMAs each (M = 128, N = 64, K = 16)
+// register; the gains read from global memory, 16-byte aligned, so that shared
+// memory holds six stages); per head two UMMAs each (M = 128, N = 64, K = 16)
 //     D1 = ReLU(g k) Bop1,   D2 = V Bop2        (V straight from its tile, K-major)
 // and the epilogue forms dV = r (D1[e] + D1[32 + e]) over the V tile, dphi(K) =
 // D2[d] + D2[32 + d] + dz[d], the feature map's backward with the raw k row (read
@@ -38,7 +39,7 @@ namespace bk {
 constexpr int kTileTok = 128;                      // UMMA M
 constexpr int kTileBytes = kTileTok * 128;         // 128 tokens x 64 channels (a head pair)
 constexpr int kStageBytes = 2 * kTileBytes;        // [K | V]
-constexpr int kStages = 5;
+constexpr int kStages = 6;
 constexpr int kN = 64;                             // B rows per head: 32 hi, 32 lo
 constexpr int kBopBytes = kN * 128;                // both heads side by side in each row
 constexpr int kBopSet = 2 * kBopBytes;             // Bop1, Bop2 of a row segment
@@ -48,8 +49,7 @@ constexpr int kTmemCols = 2 * kBufCols;            // one buffer per tile group
 constexpr int kWorkerWarps = 16;                   // two tile groups of 8
 constexpr int kGroupThreads = 32 * kWorkerWarps / 2;
 constexpr int kThreads = 32 * (4 + kWorkerWarps);  // TMA, UMMA, builder, store, workers
-constexpr int kGainCache = 4096;
-constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBopRing * kBopSet + kGainCache * 4 + 1024;
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBopRing * kBopSet + 1024;
 // (A slot may serve the two worker groups in turn: a group's use of slot s for tile
 // li + kStages starts after the tile in it before, li, has been stored, so the
 // per-slot barriers never see two tiles' arrivals at once.)
@@ -130,8 +130,7 @@ bwd_key_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ C
     uint8_t* smem = align_1024(smem_raw);
     uint8_t* stages = smem;
     uint8_t* bop = stages + kStages * kStageBytes;
-    float* sgain = (float*)(bop + kBopRing * kBopSet);
-    uint64_t* full = (uint64_t*)(sgain + kGainCache);
+    uint64_t* full = (uint64_t*)(bop + kBopRing * kBopSet);
     uint64_t* aready = full + kStages;
     uint64_t* mmadone = aready + kStages;
     uint64_t* tready = mmadone + kStages;
@@ -145,7 +144,6 @@ bwd_key_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ C
     const int64_t c = blockIdx.x;
     const int64_t i0 = range_begin(c, a.T, a.P), i1 = range_begin(c + 1, a.T, a.P);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int C = a.H * kD;                      // at most kGainCache (checked on the host)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -169,8 +167,6 @@ bwd_key_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ C
         prefetch_tmap(&tmap_dk);
         prefetch_tmap(&tmap_dv);
     }
-    if (a.norm)
-        for (int i = threadIdx.x; i < C; i += blockDim.x) sgain[i] = a.gk[i];
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
@@ -334,7 +330,8 @@ bwd_key_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ C
             const int h = p * 2 + j;
             const bool live = (t * kTileTok + row < a.N) && h < a.H;
             rk = phi_inplace_sw128<false>(stages + st * kStageBytes, row, j * 4,
-                                          sgain + (live ? h : 0) * kD, a.eps, a.norm != 0, !live);
+                                          a.norm ? a.gk + (live ? h : 0) * kD : nullptr, a.eps,
+                                          a.norm != 0, !live);
             fence_proxy_async_smem();
             mbar_arrive(&aready[st]);
             return true;
@@ -398,8 +395,8 @@ bwd_key_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ C
             tc_fence_before_sync();
             mbar_arrive(&tfree[tb]);
             // the feature map's backward with the raw k row -> dK over the K tile
-            phi_bwd_row(dp, kraw, sgain + (h < a.H ? h : 0) * kD, rk, a.norm != 0, live, ktile, row,
-                        j * 4);
+            phi_bwd_row(dp, kraw, a.norm ? a.gk + (h < a.H ? h : 0) * kD : nullptr, rk, a.norm != 0,
+                        live, ktile, row, j * 4);
             fence_proxy_async_smem();
             mbar_arrive(&tready[st]);
             if (a.norm) {                                 // the warp's 32 rows, per channel

@@ -613,7 +613,9 @@ int launch_bwd_query_tc(const void* q, const void* dout, const float* gq, const 
 // many tokens on.  For very short sequences the key gradients are a small difference
 // of O(1) terms (one token: dphi(K) = phi(Q) (dnum . V + dden) = O(eps)), which the
 // bf16 rounding of the operands would dominate; there the fp32 CUDA-core reduction
-// runs instead.
+// runs instead.  The tensor-core backward also wants 16-byte aligned gains (its
+// kernels read them from global memory as 16-byte vectors); others take the CUDA-core
+// path.
 constexpr int64_t kBwdTcMinTokens = 128;
 
 int sana_linattn_backward(const void* q, const void* k, const void* v, const float* gq,
@@ -682,7 +684,8 @@ int sana_linattn_backward(const void* q, const void* k, const void* v, const flo
             launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, Sz, B, N, H, C, C, eps, p,
                                stream);
         }
-        if (tc_path(dtype, C) && N >= kBwdTcMinTokens) {
+        if (tc_path(dtype, C) && N >= kBwdTcMinTokens &&
+            (!norm || (aligned(gq, 16) && aligned(gk, 16)))) {
             // Query side on the tensor cores: dQ, dnum (bf16, (B, N, C)) and dden (fp32,
             // (B, N, H)) in the space of the [dnum | dden] rows (B N H (64 + 4) bytes + 16
             // of padding <= B N H 132).  Then [dS | dz] = sum_t phi(Q)_t^T [dnum_t | dden_t]

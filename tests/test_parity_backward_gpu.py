@@ -80,3 +80,24 @@ def test_backward_is_deterministic(cuda_lib):
     torch.cuda.synchronize()
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+def test_backward_gains_without_16_byte_alignment(cuda_lib):
+    """Gains 4-byte but not 16-byte aligned: the backward takes its CUDA-core path
+    and still matches the oracle (the tensor-core kernels read gains as 16-byte
+    vectors)."""
+    w = WORKLOADS["1024px-b1"].scaled(N=300, seed=88)
+    x = make_inputs(w)
+    do = make_output_grad(w)
+    d = to_dev(x)
+    gq = torch.empty(w.C + 1, dtype=torch.float32, device="cuda")[1:]
+    gk = torch.empty(w.C + 1, dtype=torch.float32, device="cuda")[1:]
+    gq.copy_(d["gq"])
+    gk.copy_(d["gk"])
+    assert gq.data_ptr() % 16 != 0 and gk.data_ptr() % 16 != 0
+    got = cuda_lib.backward(d["q"], d["k"], d["v"], gq, gk, do.cuda(), w.H, w.eps)
+    torch.cuda.synchronize()
+    ref = O.backward(x["q"], x["k"], x["v"], x["gq"], x["gk"], do, w.H, w.eps)
+    dv_scale = float(np.abs(ref[2]).max())
+    for name, g, r in zip(("dq", "dk", "dv", "dgq", "dgk"), got, ref):
+        _close(g, r, w.dtype, f"unaligned gains {name}", dv_scale, own_l2=True)
