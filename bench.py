@@ -1047,7 +1047,7 @@ def backward_measure(args, sla, sets, stream, world, hbm_gbs):
                       "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / hbm_gbs})
         tot_tok += w.tokens
         tot_ms += ms
-        launches += steps * (8 if d["gq"] is not None else 6)
+        launches += steps * (10 if d["gq"] is not None else 6)
         del do, grads, ws
     big = max(range(len(sets)), key=lambda i: sets[i][0].tokens * 1e9 + sets[i][0].N)
     wb = sets[big][0]
@@ -1057,8 +1057,9 @@ def backward_measure(args, sla, sets, stream, world, hbm_gbs):
             "ms_per_step": tot_ms, "steps": steps, "parts": parts,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
                          "frac": achieved / hbm_gbs, "traffic": None,
-                         "kernel": "kv state + bwd_query_simt + outer_partial_simt + "
-                                   "bwd_key_simt + gain_combine (CUDA cores)",
+                         "kernel": "forward state (pass 1 + combine) + bwd_query_tc + pass 1 "
+                                   "(q, dnum; dden-weighted) + combine + bwd_key_tc + gain "
+                                   "sums (tensor cores; bf16, N >= 128, gains 16-byte aligned)",
                          "workload": wb.name, "algorithmic_bytes_per_launch": by_big},
             "gpu_launches": launches}
 

@@ -93,9 +93,11 @@ SANA_API int sana_linattn_forward(const void* q, const void* k, const void* v,
  *   O_n = phi(Q_n) S_n[:, :D] / (phi(Q_n) S_n[:, D] + eps),
  *   S_n = sum_{j <= n} phi(K_j)^T [V_j | 1].
  * Arguments, dtypes, layouts and errors as for sana_linattn_forward; workspace:
- * at least sana_linattn_workspace_bytes(B, N, C, H, 2) bytes (one fp32 state per
- * 64-token chunk of every (b, h)).  Chunk states are combined in chunk order, so
- * results are reproducible. */
+ * at least sana_linattn_workspace_bytes(B, N, C, H, 2) bytes (the states of
+ * every 128-token chunk of every (b, h) and their prefixes on the tensor-core path
+ * (bf16, C <= 4096, gains 16-byte aligned); one fp32 state per 64-token chunk on
+ * the CUDA-core path).  Chunk states are combined in chunk order, so results are
+ * reproducible. */
 SANA_API int sana_linattn_forward_causal(const void* q, const void* k, const void* v,
                                          const float* gq, const float* gk, void* out,
                                          int64_t B, int64_t N, int C, int H, float eps,
@@ -108,7 +110,12 @@ SANA_API int sana_linattn_forward_causal(const void* q, const void* k, const voi
  * the norm on, dgq, dgk = dL/dgq, dL/dgk (fp32 [C]; both NULL with the norm off,
  * when gq = gk = NULL).  Recomputes the forward state itself, the way
  * sana_linattn_forward forms it (for bf16 with C <= 4096 on the tensor cores,
- * phi(K) and V as bf16 operands, fp32 sums).  All tensors
+ * phi(K) and V as bf16 operands, fp32 sums).  For bf16 with C <= 4096, N >= 128 and
+ * gains 16-byte aligned (or none) the whole backward runs on the tensor cores:
+ * dnum = dO / (den + eps) is rounded to bf16 as the operand of dphi(Q) and of the
+ * gradient state [dS | dz], which pass 1 of the forward forms; otherwise (fp32,
+ * shorter sequences, whose key gradients are small differences of O(1) terms, or
+ * other gains) CUDA-core kernels with fp32 intermediates run.  All tensors
  * 16-byte aligned (gains and their gradients 4-byte); outputs must not overlap
  * inputs or each other.  workspace: at least
  * sana_linattn_backward_workspace_bytes(B, N, C, H) bytes.  Sums are formed in a
