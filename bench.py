@@ -1206,8 +1206,8 @@ def mixffn_measure(args, sla, rank, dev, stream, world, bf16_tf, hbm_gbs, peak_k
 
 def profile_case(args):
     """--warmup calls of sana_linattn_forward (two kernel launches each; with --causal
-    sana_linattn_forward_causal, three) on one workload, optionally with another batch
-    size; prints a checksum."""
+    sana_linattn_forward_causal, three; with --backward sana_linattn_backward) on one
+    workload, optionally with another batch size; prints a checksum."""
     import torch
 
     import relu_linear_attention_attn_b200 as sla
@@ -1218,7 +1218,11 @@ def profile_case(args):
     if args.batch:
         w = w.scaled(B=args.batch)
     x = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in make_inputs(w).items()}
-    if args.causal:
+    if args.backward:
+        from relu_linear_attention_attn_b200.synthetic import make_output_grad
+        dout = make_output_grad(w).cuda()
+        ws = None
+    elif args.causal:
         ws = torch.empty(int(sla.load().sana_linattn_workspace_bytes(w.B, w.N, w.C, w.H, 2)),
                          dtype=torch.uint8, device="cuda")
     else:
@@ -1232,6 +1236,8 @@ def profile_case(args):
         elif args.workload == "w8a8":
             xq, sx = sla.quantize_rows_i8(x["x"])
             out = sla.qkv_fused_w8a8(xq, sx, Wq, sw, x["gq"], x["gk"], w.H, w.eps, workspace=ws)
+        elif args.backward:
+            out = sla.backward(x["q"], x["k"], x["v"], x["gq"], x["gk"], dout, w.H, w.eps)[0]
         elif args.causal:
             out = sla.forward_causal(x["q"], x["k"], x["v"], x["gq"], x["gk"], w.H, w.eps, workspace=ws)
         else:
@@ -1258,6 +1264,8 @@ def main():
                          "fixed launch sequence for ncu captures)")
     ap.add_argument("--causal", action="store_true",
                     help="with --profile-case: the prefix (causal) form")
+    ap.add_argument("--backward", action="store_true",
+                    help="with --profile-case: the backward (dO drawn as in the bench)")
     ap.add_argument("--batch", type=int, default=0,
                     help="with --profile-case: batch size override for the workload")
     ap.add_argument("--concurrency", choices=["streams", "serial"], default="streams",
