@@ -12,10 +12,8 @@
 //   dg[d] += du[d] x[d] r,  dx[c] = g[c] r du[c] - (r^3 x[c] / D) sum_d du[d] g[d] x[d].
 //
 // CUDA-core kernels (first version), all sums in fp32 and in a fixed order:
-//   bwd_query_simt   one thread per (query token, head): dQ, [dnum | dden] rows (or,
-//                    for bf16, dnum as a (B, N, C) tensor and dden per token-head,
-//                    from which pass 1 of the forward forms [dS | dz] on the tensor
-//                    cores, its column sums weighted by dden), the CTA's gain partial
+//   bwd_query_simt   one thread per (query token, head): dQ, [dnum | dden] rows,
+//                    the CTA's gain partial
 //   outer_partial_simt  split-N partials of phi(Q)^T [dnum | dden] (dS, dz),
 //                    combined by kv_combine
 //   bwd_key_simt     one thread per (key token, head): dK, dV, gain partial
@@ -158,8 +156,7 @@ __global__ void __launch_bounds__(kBwdTile)
 bwd_query_simt(const T* __restrict__ q, const T* __restrict__ dout,
                const float* __restrict__ gq, const float* __restrict__ Sz,
                T* __restrict__ dq, float* __restrict__ G, float* __restrict__ gpart,
-               int64_t N, int H, float eps, int norm, T* __restrict__ dnum_out = nullptr,
-               float* __restrict__ dden_out = nullptr)
+               int64_t N, int H, float eps, int norm)
 {
     __shared__ __align__(16) float sS[kD][kSPitch];
     __shared__ float red[kBwdTile];
@@ -186,20 +183,13 @@ bwd_query_simt(const T* __restrict__ q, const T* __restrict__ dout,
 #pragma unroll
         for (int e = 0; e < kD; ++e) dot = fmaf(go[e], num[e] / den, dot);
         const float dden = -dot / den;
+        float* gr = G + (((int64_t)b * N + n) * H + h) * kGrow;
 #pragma unroll
-        for (int e = 0; e < kD; ++e) go[e] = go[e] / den;   // dnum
-        if (dnum_out) {
-            // dnum as a (B, N, C) tensor of the input type and dden per token-head: the
-            // operands of the tensor-core pass that forms [dS | dz]
-#pragma unroll
-            for (int i = 0; i < kD; i += 8) store8(dnum_out + row + i, go + i);
-            dden_out[((int64_t)b * N + n) * H + h] = dden;
-        } else {
-            float* gr = G + (((int64_t)b * N + n) * H + h) * kGrow;
-#pragma unroll
-            for (int e = 0; e < kD; ++e) gr[e] = go[e];
-            gr[kD] = dden;
+        for (int e = 0; e < kD; ++e) {
+            go[e] = go[e] / den;                  // dnum
+            gr[e] = go[e];
         }
+        gr[kD] = dden;
         float dp[kD];
         state_vec(sS, go, dp);                    // dnum S^T
 #pragma unroll

@@ -470,7 +470,7 @@ struct BqArgs {
     const float* s;      // forward states [B][H][D][D+1]
     const float* gq;     // gains [C] or nullptr (norm off)
     const bf16* q;       // raw queries, for the feature map's backward
-    float* dden;         // [B][N][H] output
+    float* dden;         // [B][H][N] output
     float* gpart;        // gain partials [T][4 quadrants][2 heads][D] (norm on)
     int64_t T;
     int N, H, Pp, R, P;
@@ -773,7 +773,7 @@ bwd_query_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                 }
             }
             dden = live ? -dot * inv : 0.f;
-            if (live) a.dden[((size_t)b * a.N + tok) * a.H + h] = dden;
+            if (live) a.dden[((size_t)b * a.H + h) * a.N + tok] = dden;   // (B, H, N): coalesced
             tc_fence_before_sync();
             fence_proxy_async_smem();
             mbar_arrive(&pready[st]);

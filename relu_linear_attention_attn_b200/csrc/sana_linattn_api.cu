@@ -587,7 +587,7 @@ int launch_bwd_key_tc(const void* k, const void* v, const float* gk, const float
 }
 
 // The query side of the backward on the tensor cores (bwd_query_tc): dQ, dnum (bf16,
-// (B, N, C)), dden ((B, N, H) fp32) and the per-tile gain partials from the states S.
+// (B, N, C)), dden ((B, H, N) fp32) and the per-tile gain partials from the states S.
 int launch_bwd_query_tc(const void* q, const void* dout, const float* gq, const float* s, void* dq,
                         void* dnum, float* dden, float* gpart, int64_t B, int64_t N, int C, int H,
                         float eps, cudaStream_t st) {
@@ -687,7 +687,7 @@ int sana_linattn_backward(const void* q, const void* k, const void* v, const flo
         if (tc_path(dtype, C) && N >= kBwdTcMinTokens &&
             (!norm || (aligned(gq, 16) && aligned(gk, 16)))) {
             // Query side on the tensor cores: dQ, dnum (bf16, (B, N, C)) and dden (fp32,
-            // (B, N, H)) in the space of the [dnum | dden] rows (B N H (64 + 4) bytes + 16
+            // (B, H, N)) in the space of the [dnum | dden] rows (B N H (64 + 4) bytes + 16
             // of padding <= B N H 132).  Then [dS | dz] = sum_t phi(Q)_t^T [dnum_t | dden_t]
             // by pass 1 with q in K's place (its gains gq), dnum in V's and the normaliser
             // column weighted by dden; then the key side, and the gain partials' sums.

@@ -247,7 +247,7 @@ static_assert(kStages >= 2 && kStages % 2 == 0, "ring slots must be even");
 
 struct P1Args {
     const float* gk;     // gains [C], or nullptr with the norm off
-    const float* w;      // kWeighted: per token-head weights [B][N][H] of the normaliser
+    const float* w;      // kWeighted: per token-head weights [B][H][N] of the normaliser
                          // column (sum_t phi(K)[t] w[t] in place of sum_t phi(K)[t])
     float* part;         // partial states [B][H][Smax][D+1][D]  (column e major);
                          // chunked: [B][H][Cc][Smax][D+1][D]
@@ -438,7 +438,7 @@ kv_partials_persistent(const __grid_constant__ CUtensorMap tmap_k,
                     const int64_t bb = (kChunked ? r / a.Cc : r) / a.G;
                     for (int it = 0; it < 2; ++it) {
                         const int64_t tok = tbase + (int64_t)t * kStageTok + rows[it];
-                        wv[it] = dead[it] ? 0.f : __ldg(a.w + (bb * a.N + tok) * a.H + h);
+                        wv[it] = dead[it] ? 0.f : __ldg(a.w + (bb * a.H + h) * a.N + tok);
                     }
                 }
                 phi2_inplace_sw128<true>(tl, rows, ch, gg, a.eps, a.norm != 0, dead, rr, ks,
