@@ -656,7 +656,8 @@ def run_ours(args, rank, world, local):
                                                                (2 * PASS_BYTES_PER_TOKEN) / 1e6 *
                                                                world)}},
                      "parts": parts,
-                     "gpu_launches": args.steps * len(sets) * 2,
+                     "gpu_launches": args.steps * sum(sla.forward_kernels(w.B, w.N, w.C, w.H)
+                                                      for w, _, _ in sets),
                      "per_pass_timing": "a second K-step loop of the forward's two kernels as "
                                         "separate calls (sana_linattn_forward_pass1, _pass2), "
                                         "each after a 512 MB L2-evicting read, CUDA events "

@@ -79,13 +79,24 @@ SANA_API size_t sana_linattn_workspace_bytes(int64_t B, int64_t N, int C, int H,
  * q, k, v, out: (B, N, C) in `dtype`.  gq, gk: fp32 [C] or both NULL.
  * workspace: at least sana_linattn_workspace_bytes(B, N, C, H, 0) bytes; its
  * contents on entry do not matter and are garbage on exit.
- * bf16 with C <= 4096 runs on the tensor cores as two persistent passes (the
- * state, then its application); fp32 and wider problems run CUDA-core kernels. */
+ * bf16 with C <= 4096 runs on the tensor cores: short problems (N <= 1024 and at
+ * most 400 CTAs of 128 tokens x 4 heads, e.g. the 1024px latent at batch 1 to 3)
+ * as ONE launch of thread-block clusters that reduce the state among their CTAs
+ * through distributed shared memory; everything else as two persistent passes
+ * (the state, then its application).  fp32 and wider problems run CUDA-core
+ * kernels.  Either way the result is a fixed function of the inputs (reductions
+ * in a fixed order: bitwise reproducible). */
 SANA_API int sana_linattn_forward(const void* q, const void* k, const void* v,
                          const float* gq, const float* gk, void* out,
                          int64_t B, int64_t N, int C, int H, float eps,
                          sana_dtype dtype, void* workspace, size_t ws_bytes,
                          cudaStream_t stream);
+
+/* How many kernels sana_linattn_forward (and sana_linattn_forward_noalloc) launch
+ * for this shape and dtype: 1 (one cluster launch, short problems on the tensor
+ * cores), 2 (the two persistent passes) or 3 (the CUDA-core path); 0 for an empty
+ * shape (B or N zero); a negative sana_status for an invalid one.  Host only. */
+SANA_API int sana_linattn_forward_kernels(int64_t B, int64_t N, int C, int H, sana_dtype dtype);
 
 /* The prefix (causal) form of Eq. (1): the explainer page of the Sana notes
  * describes linear attention as a cumulative prefix sum; here token n sees keys
@@ -140,9 +151,13 @@ SANA_API int sana_linattn_kv_state(const void* k, const void* v, const float* gk
                           sana_dtype dtype, void* workspace, size_t ws_bytes,
                           cudaStream_t stream);
 
-/* The two passes of sana_linattn_forward as separate calls; issued one after
- * the other on the same stream they are exactly the forward (same kernels, same
- * plan, bit-identical output), and other work may be enqueued between them.
+/* The two persistent passes of sana_linattn_forward as separate calls; issued
+ * one after the other on the same stream they are exactly the forward wherever
+ * the forward runs the two passes (same kernels, same plan, bit-identical
+ * output), and other work may be enqueued between them.  For the short problems
+ * that the forward runs as one cluster launch they still run the two passes; the
+ * results then agree with the forward's to rounding (the state's partial sums
+ * are added in another order).
  *   sana_linattn_forward_pass1: the split-N partial states of phi(K)^T [V | 1]
  *     (one per contiguous token range of every (b, h), a fixed function of B, N, H
  *     and the device) into `workspace`.

@@ -98,6 +98,8 @@ def _declare(lib):
     lib.sana_mixffn_forward.argtypes = [vp, vp, fp, fp, fp, vp, fp, vp, i64, ci, ci, ci, ci, ci,
                                         vp, sz, vp]
     lib.sana_mixffn_forward.restype = ctypes.c_int
+    lib.sana_linattn_forward_kernels.argtypes = [i64, i64, ci, ci, ci]
+    lib.sana_linattn_forward_kernels.restype = ctypes.c_int
     lib.sana_linattn_strerror.argtypes = [ci]
     lib.sana_linattn_strerror.restype = ctypes.c_char_p
     return lib
@@ -127,6 +129,14 @@ def workspace_bytes(B: int, N: int, C: int, H: int, fused: bool = False) -> int:
 
 
 # --------------------------------------------------------------------------- torch marshalling
+def forward_kernels(B: int, N: int, C: int, H: int, dtype: str = "bf16") -> int:
+    """How many kernels forward() launches for this shape: 1 (one cluster launch),
+    2 (the two persistent passes), 3 (the CUDA-core path), 0 when empty."""
+    rc = load().sana_linattn_forward_kernels(B, N, C, H, {"bf16": 0, "f32": 1}[dtype])
+    _check("sana_linattn_forward_kernels", min(rc, 0))
+    return rc
+
+
 def _torch():
     import torch
     return torch

@@ -19,6 +19,7 @@
 #include "backward_kernels.cuh"
 #include "mixffn_kernels.cuh"
 #include "causal_tc_kernels.cuh"
+#include "short_tc_kernels.cuh"
 
 namespace sana {
 namespace {
@@ -288,7 +289,9 @@ int persistent_ctas() {
         cudaFuncSetAttribute(bwd_key_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              bk::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(bwd_query_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bq::kSmemBytes) != cudaSuccess)
+                             bq::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(forward_short_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sc::kSmemBytes) != cudaSuccess)
         return 0;
     // each persistent kernel must fit one CTA on an SM (registers, threads, smem)
     int n1 = 0, n2 = 0, n3 = 0, n4 = 0;
@@ -385,6 +388,52 @@ int launch_apply_tc(const void* q, const float* gq, const float* kv, const float
     }
     return launch_pdl(apply_persistent, dim3(pl.P), p2::kThreads, p2::kSmemBytes, st,
                       kv == nullptr, tq, to, a);
+}
+
+// Short sequences (bf16, N <= 128 * 8): the whole forward as one launch of
+// clusters of S = ceil(N / 128) CTAs, one cluster per (b, group of 4 heads).
+constexpr int64_t kShortMaxN = (int64_t)sc::kTok * sc::kMaxCluster;
+// Beyond this many CTAs (about 2.7 per SM) the persistent passes, which stream
+// tiles through deep rings, are faster than one tile per CTA (measured on B200 at
+// N = 777 and 1024: B = 3 and below favour the clusters, B = 4 and above the passes).
+constexpr int64_t kShortMaxCtas = 400;
+
+bool short_path(int64_t B, int64_t N, int H) {
+    const int64_t S = (N + sc::kTok - 1) / sc::kTok, G = (H + sc::kHeads - 1) / sc::kHeads;
+    return N <= kShortMaxN && B <= 65535 && B * G * S <= kShortMaxCtas;
+}
+
+int launch_short_tc(const void* q, const void* k, const void* v, const float* gq,
+                    const float* gk, void* out, int64_t B, int64_t N, int C, int H, float eps,
+                    cudaStream_t st) {
+    if (persistent_ctas() == 0) return SANA_ECUDA;           // the kernel attributes
+    const int S = (int)((N + sc::kTok - 1) / sc::kTok);
+    const int G = (H + sc::kHeads - 1) / sc::kHeads;
+    CUtensorMap tq, tk, tv, to;
+    if (!make_tmap_bnc(&tq, q, B, N, C, sc::kTok) || !make_tmap_bnc(&to, out, B, N, C, sc::kTok) ||
+        !make_tmap_bnc(&tk, k, B, N, C, sc::kStageTok) ||
+        !make_tmap_bnc(&tv, v, B, N, C, sc::kStageTok))
+        return SANA_ECUDA;
+    ScArgs a{};
+    a.gq = gq; a.gk = gk; a.N = (int)N; a.H = H; a.S = S; a.eps = eps;
+    a.norm = gq != nullptr && gk != nullptr;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)S, (unsigned)G, (unsigned)B);
+    cfg.blockDim = dim3(sc::kThreads);
+    cfg.dynamicSmemBytes = sc::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, forward_short_cluster, tq, tk, tv, to, a) == cudaSuccess
+               ? SANA_OK
+               : SANA_ECUDA;
 }
 
 // The prefix (causal) form on the tensor cores (bf16): pass 1 with one row per
@@ -887,7 +936,10 @@ int sana_linattn_forward(const void* q, const void* k, const void* v, const floa
     const Plan p = make_plan(B, N, H);
     float* part = (float*)((char*)workspace + L.part_off);
     float* kv = (float*)((char*)workspace + L.kv_off);
-    if (tc_path(dtype, C)) {
+    if (tc_path(dtype, C) && short_path(B, N, H)) {
+        if ((rc = launch_short_tc(q, k, v, gq, gk, out, B, N, C, H, eps, stream)) != SANA_OK)
+            return rc;
+    } else if (tc_path(dtype, C)) {
         PersistPlan1 pl{};
         if ((rc = launch_partials_tc(k, v, gk, part, B, N, C, H, eps, stream, &pl)) != SANA_OK ||
             (rc = launch_apply_tc(q, gq, nullptr, part, &pl, out, B, N, C, H, eps, stream)) !=
@@ -904,6 +956,15 @@ int sana_linattn_forward(const void* q, const void* k, const void* v, const floa
                                    stream);
     }
     return launch_status();
+}
+
+int sana_linattn_forward_kernels(int64_t B, int64_t N, int C, int H, sana_dtype dtype) {
+    int rc;
+    if ((rc = check_dims(B, N, C, H)) != SANA_OK) return rc;
+    if (dtype != SANA_BF16 && dtype != SANA_F32) return SANA_EINVAL;
+    if (B == 0 || N == 0) return 0;
+    if (!tc_path(dtype, C)) return 3;
+    return short_path(B, N, H) ? 1 : 2;
 }
 
 int sana_linattn_forward_pass1(const void* k, const void* v, const float* gk, int64_t B,

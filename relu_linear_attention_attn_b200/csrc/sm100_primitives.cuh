@@ -310,6 +310,34 @@ __device__ __forceinline__ void tmem_ld1(uint32_t taddr, float* v) {
     v[0] = __uint_as_float(r);
 }
 
+// ------------------------------------------------------------------ clusters
+// The cluster-wide barrier in its two halves.  arrive.release publishes this
+// thread's earlier shared-memory writes to the cluster; wait.acquire returns once
+// every thread of every CTA in the cluster has arrived.  All threads must take
+// part, whatever path they took.
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Address, in the cluster's shared window, of the same byte in CTA `rank`'s
+// shared memory (rank < cluster size).
+__device__ __forceinline__ uint32_t map_shared_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+// 8-byte load from another CTA's shared memory (8-byte aligned address).
+__device__ __forceinline__ float2 ld_cluster_f32x2(uint32_t addr) {
+    float2 v;
+    asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
 // ------------------------------------------------------------------ descriptors
 // Shared-memory matrix descriptor for tcgen05.mma (sm_100 format):
 //   [0,14) start address >> 4, [16,30) leading byte offset >> 4,

@@ -64,6 +64,26 @@ def test_workspace_bytes():
     assert a >= 2 * 1 * 70 * 32 * 33 * 4
 
 
+def test_forward_kernel_count_follows_the_dispatch():
+    """Short problems on the tensor cores are one cluster launch (clusters of
+    ceil(N / 128) <= 8 CTAs per batch item and group of 4 heads, at most 400 CTAs);
+    longer or larger ones the two persistent passes; fp32 or C > 4096 the CUDA-core
+    path (3 launches)."""
+    fk = sla.forward_kernels
+    assert fk(1, 1024, 2240, 70) == 1              # the 1024px latent, batch 1: 8 x 18 CTAs
+    assert fk(2, 1024, 2240, 70) == 1              # 288 CTAs
+    assert fk(3, 777, 2240, 70) == 1               # 3 x 18 x 7 = 378
+    assert fk(3, 1024, 2240, 70) == 2              # 432 > 400
+    assert fk(1, 1025, 2240, 70) == 2              # longer than 8 x 128 tokens
+    assert fk(8, 4096, 2240, 70) == 2
+    assert fk(1, 1, 32, 1) == 1
+    assert fk(1, 1024, 2240, 70, "f32") == 3
+    assert fk(1, 256, 4128, 129) == 3              # gains of more than 4096 channels
+    assert fk(0, 1024, 2240, 70) == 0 and fk(1, 0, 2240, 70) == 0
+    with pytest.raises(sla.SanaError):
+        fk(1, 1024, 2240, 71)                      # C % H != 0
+
+
 FAKE = 1 << 36   # a 256-byte-aligned address that is never dereferenced
 
 

@@ -78,12 +78,15 @@ def test_ragged_shapes_full_parity(cuda_lib, recipe, gains, B, N):
     (1, 129, 70, "overflow", "off"), (1, 1000, 70, "gaussian", "random"),
     (1, 1024, 70, "overflow", "off"), (2, 384, 6, "gaussian", "random"),
     (1, 500, 5, "lognormal", "random"), (3, 256, 70, "gaussian", "ones"),
-    (2, 300, 1, "gaussian", "random")])
+    (2, 300, 1, "gaussian", "random"), (2, 1024, 70, "lognormal", "random"),
+    (1, 896, 3, "overflow", "off"), (4, 128, 70, "gaussian", "random"),
+    (1, 1023, 70, "lognormal", "ones"), (1, 640, 4, "gaussian", "random")])
 def test_short_sequences_full_parity(cuda_lib, B, N, H, recipe, gains):
-    """Short sequences (N <= 1024, few work items per CTA, many partial slots per
-    row): ragged token counts and head counts that leave a head group or a head
-    pair partly or wholly empty; the one-call forward and the split kv_state +
-    apply both match the oracle, and the forward is reproducible bit for bit."""
+    """Short sequences: ragged token counts (clusters of 1 to 8 CTAs, a partly
+    empty last CTA) and head counts that leave a head group or a head pair partly
+    or wholly empty; the one-call forward (one cluster launch at these sizes) and
+    the split kv_state + apply (the persistent passes) both match the oracle, and
+    the forward is reproducible bit for bit."""
     w = Workload(f"short-{B}x{N}-h{H}", B=B, N=N, C=32 * H, H=H, dtype="bf16", recipe=recipe,
                  gains=gains, eps=1e-6, seed=300 + 7 * B + N + H)
     x = make_inputs(w)
@@ -296,11 +299,12 @@ def test_independent_problems_on_concurrent_streams(cuda_lib):
         assert torch.equal(a, o), w.name
 
 
-@pytest.mark.parametrize("B,N", [(2, 3000), (3, 777), (1, 16384)])
+@pytest.mark.parametrize("B,N", [(2, 3000), (3, 1500), (1, 16384)])
 def test_forward_passes_called_separately_equal_forward(cuda_lib, B, N):
-    """sana_linattn_forward_pass1 then _pass2 on one stream are the forward: the
-    same kernels and plan, so the output is bit-identical, also with unrelated work
-    enqueued between the two calls."""
+    """sana_linattn_forward_pass1 then _pass2 on one stream are the forward (for
+    sequences the forward runs as the two persistent passes): the same kernels and
+    plan, so the output is bit-identical, also with unrelated work enqueued between
+    the two calls."""
     w = WORKLOADS["4096px-b2-overflow"].scaled(B=B, N=N, seed=120 + N)
     d = to_dev(make_inputs(w))
     ref = run_forward(cuda_lib, d, w)
