@@ -16,22 +16,23 @@
 //      the normaliser column sums on the CUDA cores, and one UMMA chain
 //          D[(h,d), (h',e)] = sum_t phi(K)[t,(h,d)] V[t,(h',e)]   (M=N=128, K=128)
 //      whose diagonal blocks are this CTA's partial states (as in pass 1).
-//   2. The partial state (4 heads x (D+1) x D fp32) goes to shared memory.
-//      Cluster barrier.  CTA s sums its share of the state's 132 rows (head, e)
-//      over the S partials, read from the peers' shared memory in rank order
-//      (fixed order: the result is bitwise reproducible and the same in every
-//      CTA).  Cluster barrier.
+//   2. The partial state (4 heads x (D+1) x D fp32) goes to shared memory; the
+//      CTA transforms its Q tile while the cluster barrier completes.  CTA s then
+//      sums its share of the state's 132 rows (head, e) over the S partials, read
+//      from the peers' shared memory in rank order (fixed order: the result is
+//      bitwise reproducible and the same in every CTA).  Cluster barrier.
 //   3. Every CTA reads the summed rows back from their owners and writes its own
-//      copy of pass 2's B operand (hi / lo bf16 parts, rows 0..31 hi, 32 / 33 the
-//      normaliser's hi / lo, 48..79 lo), then per head two UMMAs (M=128, N=80,
-//      K=16 each) against phi(Q), and the epilogue O = r num / (r den + eps)
-//      written over the Q tile and TMA-stored.
+//      B operands (per head 64 rows: the bf16 "hi" parts of the value columns,
+//      then their "lo" parts x - bf16(x), so the state keeps ~16 mantissa bits),
+//      then per head two UMMAs (M=128, N=64, K=16 each) against phi(Q).  The
+//      normaliser phi(Q) . ksum is a 32-term fp32 dot product on the CUDA cores,
+//      which frees the TMEM columns it would take: all four heads fit at once.
+//      Epilogue O = r num / (r den + eps) written over the Q tile and TMA-stored.
 //
 // Shared memory (about 99 KB, two CTAs per SM): the K / V tiles (64 KB) become,
 // once the state UMMAs have read them, the partial-state export, the summed rows
 // and the B operands; the Q tile (32 KB) becomes O.  TMEM: 256 columns, the state
-// accumulator in 0..127, then heads (pair, j) = (0,0), (0,1), (1,0) at 0, 80, 160
-// and (1,1) at 0 again once head (0,0) has been read out.
+// accumulator in 0..127, then head (pair p, j) in 64 (2 p + j) .. + 63.
 //
 // TMEM: warp w reads lanes 32 * (w % 4) .. + 31; D row i is lane i.
 #pragma once
@@ -58,13 +59,14 @@ constexpr int kStateBytes = kRows * kD * 4;        // 16,896
 constexpr int kExportOff = 0;                      // this CTA's partial state   (in K / V)
 constexpr int kRedOff = 17 * 1024;                 // the rows this CTA summed   (in K / V)
 constexpr int kBopOff = 34 * 1024;                 // B operands of the 2 pairs  (in K / V)
-constexpr int kN = 80;                             // B rows per head (pass 2's layout)
-constexpr int kLoRow = 48, kDenHi = 32, kDenLo = 33;
-constexpr int kBopBytes = kN * 128;                // one pair, 10 KB
+constexpr int kN = 64;                             // B rows per head: D hi, then D lo parts
+constexpr int kBopBytes = kN * 128;                // one pair, 8 KB
 constexpr int kQOff = kKVBytes;
 constexpr int kGainOff = kQOff + kQBytes;          // gk[128], gq[128]
 constexpr int kKsOff = kGainOff + 2 * kHeads * kD * 4;   // column sums [2 stages][4 heads][32]
-constexpr int kBarOff = kKsOff + 2 * kHeads * kD * 4;
+constexpr int kOwnOff = kKsOff + 2 * kHeads * kD * 4;    // owning CTA of each state row
+constexpr int kKsumOff = kOwnOff + 256;                  // the summed normaliser rows [4][32]
+constexpr int kBarOff = kKsumOff + kHeads * kD * 4;
 constexpr int kSmemBytes = 1024 + kBarOff + 64;
 constexpr int kTmemCols = 256;
 static_assert(kExportOff + kStateBytes <= kRedOff && kRedOff + kStateBytes <= kBopOff, "layout");
@@ -99,16 +101,16 @@ forward_short_cluster(const __grid_constant__ CUtensorMap tmap_q,
     float* sgk = (float*)(smem + kGainOff);
     float* sgq = sgk + kHeads * kD;
     float* kspart = (float*)(smem + kKsOff);
+    uint8_t* sown = smem + kOwnOff;
+    float* sksum = (float*)(smem + kKsumOff);
     float* expo = (float*)(smem + kExportOff);
     float* red = (float*)(smem + kRedOff);
     uint8_t* bop = smem + kBopOff;
     uint64_t* bar_kv = (uint64_t*)(smem + kBarOff);
     uint64_t* bar_q = bar_kv + 1;
     uint64_t* bar_acc = bar_kv + 2;
-    uint64_t* bar_mma_a = bar_kv + 3;
-    uint64_t* bar_mma_b = bar_kv + 4;
-    uint64_t* bar_tfree = bar_kv + 5;
-    uint32_t* tmem_slot = (uint32_t*)(bar_kv + 6);
+    uint64_t* bar_mma = bar_kv + 3;
+    uint32_t* tmem_slot = (uint32_t*)(bar_kv + 4);
 
     const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int S = a.S;
@@ -121,9 +123,7 @@ forward_short_cluster(const __grid_constant__ CUtensorMap tmap_q,
         mbar_init(bar_kv, 1);
         mbar_init(bar_q, 1);
         mbar_init(bar_acc, 1);
-        mbar_init(bar_mma_a, 1);
-        mbar_init(bar_mma_b, 1);
-        mbar_init(bar_tfree, 4 * 32);
+        mbar_init(bar_mma, 1);
         fence_barrier_init();
         prefetch_tmap(&tmap_k);
         prefetch_tmap(&tmap_v);
@@ -155,6 +155,9 @@ forward_short_cluster(const __grid_constant__ CUtensorMap tmap_q,
         const int c = g * 128 + (tid & 127);
         (tid < 128 ? sgk : sgq)[tid & 127] = c < C ? (tid < 128 ? a.gk : a.gq)[c] : 0.f;
     }
+    // state rows (head, e) are split over the cluster's CTAs in contiguous ranges
+    if (tid < kRows) sown[tid] = (uint8_t)owner_cta(tid, kRows, S);
+    const int r0 = s * kRows / S, r1 = (s + 1) * kRows / S;
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -197,12 +200,28 @@ forward_short_cluster(const __grid_constant__ CUtensorMap tmap_q,
         umma_commit_elect(bar_acc);
     }
 
-    // ---------------------------------------------------------------- phi(Q) meanwhile
-    // warp w: token row 32 (w % 4) + lane (its TMEM lane), heads (pair 0, w / 4) and
-    // (pair 1, w / 4).  The positive per-token factor r of phi(Q) is applied in the
-    // epilogue (O = r num' / (r den' + eps)), so the operand holds ReLU(g q).
+    // ---------------------------------------------------------------- 2. export, reduce
+    // warp w: token row 32 (w % 4) + lane (its TMEM lane quadrant) in the apply;
+    // here head w % 4's diagonal block, columns e in [16 (w / 4), + 16)
     const int q4 = warp & 3, jj = warp >> 2;
     const int row = 32 * q4 + lane;
+    ok = mbar_wait(bar_acc, 0, 503) && ok;
+    tc_fence_after_sync();
+    {
+        float v[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * q4) << 16) + 32 * q4 + 16 * jj, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) expo[(q4 * kDP + 16 * jj + i) * kD + lane] = v[i];
+        if (jj == 0)
+            expo[(q4 * kDP + kD) * kD + lane] =
+                kspart[q4 * kD + lane] + kspart[(kHeads + q4) * kD + lane];
+    }
+    tc_fence_before_sync();
+    cluster_arrive();
+    // phi(Q) while the cluster catches up: heads (pair 0, w / 4) and (pair 1, w / 4)
+    // of token row `row`.  The positive per-token factor r of phi(Q) is applied in
+    // the epilogue (O = r num' / (r den' + eps)), so the operand holds ReLU(g q).
     float rq[2];
     {
         ok = mbar_wait(bar_q, 0, 502) && ok;
@@ -214,49 +233,29 @@ forward_short_cluster(const __grid_constant__ CUtensorMap tmap_q,
         phi2_inplace_sw128<false>(tl, rows, ch, gg, a.eps, a.norm != 0, dead, rq, nullptr);
         fence_proxy_async_smem();
     }
-
-    // ---------------------------------------------------------------- 2. export, reduce
-    ok = mbar_wait(bar_acc, 0, 503) && ok;
-    tc_fence_after_sync();
-    {
-        // warp w: head q4's diagonal block, lanes d, columns e in [16 (w / 4), + 16)
-        float v[16];
-        tmem_ld16(tmem + ((uint32_t)(32 * q4) << 16) + 32 * q4 + 16 * jj, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) expo[(q4 * kDP + 16 * jj + i) * kD + lane] = v[i];
-        if (jj == 0)
-            expo[(q4 * kDP + kD) * kD + lane] =
-                kspart[q4 * kD + lane] + kspart[(kHeads + q4) * kD + lane];
-        // B operand rows that never carry data stay zero
-        for (int i = tid; i < 2 * (kLoRow - kDenLo - 1) * 8; i += kThreads) {
-            const int p = i / ((kLoRow - kDenLo - 1) * 8), rem = i % ((kLoRow - kDenLo - 1) * 8);
-            *reinterpret_cast<uint4*>(bop + p * kBopBytes + (kDenLo + 1 + rem / 8) * 128 +
-                                      (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
-        }
-    }
-    tc_fence_before_sync();
-    cluster_arrive();
     cluster_wait();                                               // every partial is out
     {
-        const int r0 = (int)range_begin(s, kRows, S), r1 = (int)range_begin(s + 1, kRows, S);
+        // items: 4 consecutive d of one row this CTA owns; its S partials are summed
+        // in rank order
         const uint32_t ex = smem_u32(expo);
-        for (int it = tid; it < (r1 - r0) * (kD / 2); it += kThreads) {
-            const int r = r0 + it / (kD / 2), dp = it % (kD / 2);
-            const uint32_t off = (uint32_t)(r * kD + 2 * dp) * 4;
-            float2 v[kMaxCluster];
+        for (int it = tid; it < (r1 - r0) * (kD / 4); it += kThreads) {
+            const int r = r0 + (it >> 3), dq = it & 7;
+            const uint32_t off = (uint32_t)(r * kD + 4 * dq) * 4;
+            float4 v[kMaxCluster];
 #pragma unroll
             for (int src = 0; src < kMaxCluster; ++src)
-                v[src] = src < S ? ld_cluster_f32x2(map_shared_rank(ex + off, src))
-                                 : make_float2(0.f, 0.f);
-            float2 acc = v[0];
+                v[src] = src < S ? ld_cluster_f32x4(map_shared_rank(ex + off, src))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 acc = v[0];
 #pragma unroll
             for (int src = 1; src < kMaxCluster; ++src)
                 if (src < S) {
                     acc.x += v[src].x;
                     acc.y += v[src].y;
+                    acc.z += v[src].z;
+                    acc.w += v[src].w;
                 }
-            *reinterpret_cast<float2*>(red + r * kD + 2 * dp) = acc;
+            *reinterpret_cast<float4*>(red + r * kD + 4 * dq) = acc;
         }
     }
     cluster_arrive();
@@ -264,34 +263,43 @@ forward_short_cluster(const __grid_constant__ CUtensorMap tmap_q,
 
     // ---------------------------------------------------------------- 3. B operands
     {
-        constexpr int kItems = kRows * (kD / 2);
+        // items: 4 consecutive d of one row, read from the row's owner.  Value rows
+        // (e < D) go to the B operand as bf16 hi / lo parts (rows e and D + e); the
+        // normaliser row stays fp32 for the epilogue's CUDA-core dot product.
+        constexpr int kItems = kRows * (kD / 4);
         constexpr int kPer = (kItems + kThreads - 1) / kThreads;
         const uint32_t rd = smem_u32(red);
-        float2 v[kPer];
+        float4 v[kPer];
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
             const int it = tid + u * kThreads;
-            const int r = it / (kD / 2), dp = it % (kD / 2);
-            v[u] = it < kItems ? ld_cluster_f32x2(map_shared_rank(
-                                     rd + (uint32_t)(r * kD + 2 * dp) * 4,
-                                     (uint32_t)owner_cta(r, kRows, S)))
-                               : make_float2(0.f, 0.f);
+            const int r = it >> 3, dq = it & 7;
+            v[u] = it < kItems ? ld_cluster_f32x4(map_shared_rank(
+                                     rd + (uint32_t)(r * kD + 4 * dq) * 4, sown[r]))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
             const int it = tid + u * kThreads;
             if (it >= kItems) continue;
-            const int r = it / (kD / 2), dp = it % (kD / 2);
+            const int r = it >> 3, dq = it & 7;
             const int j = r / kDP, e = r % kDP;
-            const int d0 = 2 * dp;
+            const int d0 = 4 * dq;
+            if (e == kD) {
+                *reinterpret_cast<float4*>(sksum + j * kD + d0) = v[u];
+                continue;
+            }
             const int chunk = (j & 1) * 4 + d0 / 8, boff = (d0 % 8) * 2;
             uint8_t* dst = bop + (j >> 1) * kBopBytes;
             const float h0 = __bfloat162float(__float2bfloat16_rn(v[u].x));
             const float h1 = __bfloat162float(__float2bfloat16_rn(v[u].y));
-            const int lorow = e < kD ? kLoRow + e : kDenLo;      // hi row is e (kDenHi for e = D)
-            *reinterpret_cast<uint32_t*>(dst + sw128_offset(e, chunk) + boff) = pack_bf16x2(h0, h1);
-            *reinterpret_cast<uint32_t*>(dst + sw128_offset(lorow, chunk) + boff) =
-                pack_bf16x2(v[u].x - h0, v[u].y - h1);
+            const float h2 = __bfloat162float(__float2bfloat16_rn(v[u].z));
+            const float h3 = __bfloat162float(__float2bfloat16_rn(v[u].w));
+            *reinterpret_cast<uint2*>(dst + sw128_offset(e, chunk) + boff) =
+                make_uint2(pack_bf16x2(h0, h1), pack_bf16x2(h2, h3));
+            *reinterpret_cast<uint2*>(dst + sw128_offset(kD + e, chunk) + boff) =
+                make_uint2(pack_bf16x2(v[u].x - h0, v[u].y - h1),
+                           pack_bf16x2(v[u].z - h2, v[u].w - h3));
         }
         fence_proxy_async_smem();
     }
@@ -300,83 +308,77 @@ forward_short_cluster(const __grid_constant__ CUtensorMap tmap_q,
     __syncthreads();
     tc_fence_after_sync();
 
-    if (warp == 4) {
+    if (warp == 0) {
+        // head (p, j) of the row: D[t, n] = sum_d phi(Q)[t, d] Bop_(p,j)[n, d] in
+        // columns 64 (2 p + j) .. + 63 (n < D: hi parts of the value columns, n >= D: lo)
         const uint32_t idesc = make_idesc_bf16(128, kN, false, false);
         const uint64_t a0 = make_smem_desc(smem_u32(sq), 16, 1024, kSwizzle128B);
-        const uint64_t a1 = a0 + (uint64_t)(kQBoxBytes >> 4);
         const uint64_t b0 = make_smem_desc(smem_u32(bop), 16, 1024, kSwizzle128B);
-        const uint64_t b1 = b0 + (uint64_t)(kBopBytes >> 4);
-        umma_bf16_elect(tmem, a0, b0, idesc, false);
-        umma_bf16_elect(tmem, a0 + 2, b0 + 2, idesc, true);
-        umma_bf16_elect(tmem + kN, a0 + 4, b0 + 4, idesc, false);
-        umma_bf16_elect(tmem + kN, a0 + 6, b0 + 6, idesc, true);
-        umma_bf16_elect(tmem + 2 * kN, a1, b1, idesc, false);
-        umma_bf16_elect(tmem + 2 * kN, a1 + 2, b1 + 2, idesc, true);
-        umma_commit_elect(bar_mma_a);
-        bool freed = true;
-        if (lane == 0) freed = mbar_wait(bar_tfree, 0, 504);
-        ok = __shfl_sync(0xffffffffu, freed, 0) && ok;
-        tc_fence_after_sync();
-        umma_bf16_elect(tmem, a1 + 4, b1 + 4, idesc, false);      // head (1, 1) over (0, 0)
-        umma_bf16_elect(tmem, a1 + 6, b1 + 6, idesc, true);
-        umma_commit_elect(bar_mma_b);
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const uint64_t ad = a0 + (uint64_t)((p * kQBoxBytes) >> 4) + 4 * j;
+                const uint64_t bd = b0 + (uint64_t)((p * kBopBytes) >> 4) + 4 * j;
+                umma_bf16_elect(tmem + kN * (2 * p + j), ad, bd, idesc, false);
+                umma_bf16_elect(tmem + kN * (2 * p + j), ad + 2, bd + 2, idesc, true);
+            }
+        umma_commit_elect(bar_mma);
     }
 
     // ---------------------------------------------------------------- epilogue
-    // head (pair p, jj) of token row `row`: O = (hi + lo) r / (r (den_hi + den_lo) + eps)
-    auto load_out = [&](uint32_t col, float r, uint4* w) {
-        const uint32_t ta = tmem + ((uint32_t)(32 * q4) << 16) + col;
-        float hi[kD + 2], lo[kD];
+    // head (p, jj) of token row `row`:
+    //   O = (hi + lo) r / (r den' + eps),  den' = phi(Q)' . ksum (fp32, CUDA cores)
+    ok = mbar_wait(bar_mma, 0, 505) && ok;
+    tc_fence_after_sync();
+#pragma unroll 1
+    for (int p = 0; p < 2; ++p) {
+        uint8_t* box = sq + p * kQBoxBytes;
+        const float* ksj = sksum + (2 * p + jj) * kD;
+        float den = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint4 u = *reinterpret_cast<const uint4*>(box + sw128_offset(row, jj * 4 + c));
+            const float4 k0 = *reinterpret_cast<const float4*>(ksj + 8 * c);
+            const float4 k1 = *reinterpret_cast<const float4*>(ksj + 8 * c + 4);
+            den = fmaf(bf16lo(u.x), k0.x, den); den = fmaf(bf16hi(u.x), k0.y, den);
+            den = fmaf(bf16lo(u.y), k0.z, den); den = fmaf(bf16hi(u.y), k0.w, den);
+            den = fmaf(bf16lo(u.z), k1.x, den); den = fmaf(bf16hi(u.z), k1.y, den);
+            den = fmaf(bf16lo(u.w), k1.z, den); den = fmaf(bf16hi(u.w), k1.w, den);
+        }
+        const uint32_t ta = tmem + ((uint32_t)(32 * q4) << 16) + kN * (2 * p + jj);
+        float hi[kD], lo[kD];
         tmem_ld16(ta, hi);
         tmem_ld16(ta + 16, hi + 16);
-        tmem_ld2(ta + kDenHi, hi + kD);
-        tmem_ld16(ta + kLoRow, lo);
-        tmem_ld16(ta + kLoRow + 16, lo + 16);
+        tmem_ld16(ta + kD, lo);
+        tmem_ld16(ta + kD + 16, lo + 16);
         tmem_wait_ld();
-        const float den = hi[kD] + hi[kD + 1];
+        const float r = p == 0 ? rq[0] : rq[1];
         const float scale = r * __frcp_rn(fmaf(r, den, a.eps));
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
             float o[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) o[u] = (hi[8 * cc + u] + lo[8 * cc + u]) * scale;
-            w[cc].x = pack_bf16x2(o[0], o[1]);
-            w[cc].y = pack_bf16x2(o[2], o[3]);
-            w[cc].z = pack_bf16x2(o[4], o[5]);
-            w[cc].w = pack_bf16x2(o[6], o[7]);
+            uint4 w;
+            w.x = pack_bf16x2(o[0], o[1]);
+            w.y = pack_bf16x2(o[2], o[3]);
+            w.z = pack_bf16x2(o[4], o[5]);
+            w.w = pack_bf16x2(o[6], o[7]);
+            *reinterpret_cast<uint4*>(box + sw128_offset(row, jj * 4 + cc)) = w;
         }
-    };
-    auto store_out = [&](uint8_t* box, const uint4* w) {
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-            *reinterpret_cast<uint4*>(box + sw128_offset(row, jj * 4 + cc)) = w[cc];
-    };
-    {
-        uint4 w[4];
-        ok = mbar_wait(bar_mma_a, 0, 505) && ok;
-        tc_fence_after_sync();
-        load_out(jj == 0 ? 0 : kN, rq[0], w);                       // head (0, jj)
-        if (jj == 0) {
-            tc_fence_before_sync();
-            mbar_arrive(bar_tfree);                               // columns 0..79 are free
-        }
-        store_out(sq, w);
-        if (jj == 0) load_out(2 * kN, rq[1], w);                   // head (1, 0)
-        ok = mbar_wait(bar_mma_b, 0, 506) && ok;                  // pair 1's operand is read
-        tc_fence_after_sync();
-        if (jj == 1) load_out(0, rq[1], w);                        // head (1, 1)
-        store_out(sq + kQBoxBytes, w);
-        fence_proxy_async_smem();
     }
+    fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
     if (tid == 0) {
         tma_store_3d(&tmap_o, sq, g * 128, tok0, b);
         if (g * 128 + 64 < C) tma_store_3d(&tmap_o, sq + kQBoxBytes, g * 128 + 64, tok0, b);
         bulk_commit_group();
-        bulk_wait_group<0>();
+        bulk_wait_group_read<0>();         // the tile may go; the writes finish on their own
     }
     cluster_wait();                // no peer still reads this CTA's shared memory
+    __syncwarp();
     if (warp == 0) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, kTmemCols);

@@ -338,6 +338,16 @@ __device__ __forceinline__ float2 ld_cluster_f32x2(uint32_t addr) {
     return v;
 }
 
+// 16-byte load from another CTA's shared memory (16-byte aligned address).
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
 // ------------------------------------------------------------------ descriptors
 // Shared-memory matrix descriptor for tcgen05.mma (sm_100 format):
 //   [0,14) start address >> 4, [16,30) leading byte offset >> 4,
