@@ -1016,7 +1016,7 @@ def backward_measure(args, sla, sets, stream, world, hbm_gbs):
     import torch
     from relu_linear_attention_attn_b200.synthetic import make_output_grad
     steps = max(3, min(args.steps, 10))
-    parts, tot_tok, tot_ms = [], 0, 0.0
+    parts, tot_tok, tot_ms, tot_ms_st = [], 0, 0.0, 0.0
     launches = 0
     for w, d, _ in sets:
         dev = d["q"].device
@@ -1027,35 +1027,53 @@ def backward_measure(args, sla, sets, stream, world, hbm_gbs):
         ws = torch.empty(int(sla.load().sana_linattn_backward_workspace_bytes(w.B, w.N, w.C, w.H)),
                          dtype=torch.uint8, device=dev)
 
+        # the forward's state, as a training step holds it from its forward (untimed)
+        kv = sla.kv_state(d["k"], d["v"], d["gk"], w.H, w.eps)
+
         def call():
             sla.backward(d["q"], d["k"], d["v"], d["gq"], d["gk"], do, w.H, w.eps, grads=grads,
                          workspace=ws)
-        for _ in range(max(args.warmup, 3)):
-            call()
-        torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(steps)]
-        barrier(world)
-        torch.cuda.synchronize()
-        for a, b in evs:
-            a.record(stream)
-            call()
-            b.record(stream)
-        torch.cuda.synchronize()
-        ms = max_over_ranks(statistics.fmean(a.elapsed_time(b) for a, b in evs), world)
+
+        def call_with_state():
+            sla.backward(d["q"], d["k"], d["v"], d["gq"], d["gk"], do, w.H, w.eps, grads=grads,
+                         workspace=ws, kv=kv)
+
+        def timed(fn):
+            for _ in range(max(args.warmup, 3)):
+                fn()
+            torch.cuda.synchronize()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(steps)]
+            barrier(world)
+            torch.cuda.synchronize()
+            for a, b in evs:
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+            return max_over_ranks(statistics.fmean(a.elapsed_time(b) for a, b in evs), world)
+        ms = timed(call)
+        ms_st = timed(call_with_state)
         by = w.tokens * 7 * PASS_BYTES_PER_TOKEN // 2
         parts.append({"workload": w.name, "ms": ms, "Mtokens_per_s": w.tokens / (ms * 1e-3) / 1e6,
-                      "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / hbm_gbs})
+                      "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / hbm_gbs,
+                      "ms_with_forward_state": ms_st,
+                      "hbm_frac_with_forward_state": by / (ms_st * 1e-3) / 1e9 / hbm_gbs})
         tot_tok += w.tokens
         tot_ms += ms
+        tot_ms_st += ms_st
         launches += steps * (10 if d["gq"] is not None else 6)
-        del do, grads, ws
+        launches += steps * (8 if d["gq"] is not None else 4)
+        del do, grads, ws, kv
     big = max(range(len(sets)), key=lambda i: sets[i][0].tokens * 1e9 + sets[i][0].N)
     wb = sets[big][0]
     by_big = wb.tokens * 7 * PASS_BYTES_PER_TOKEN // 2
     achieved = by_big / (parts[big]["ms"] * 1e-3) / 1e9
     return {"value": tot_tok * world / (tot_ms * 1e-3) / 1e6, "unit": "Mtokens/s",
             "ms_per_step": tot_ms, "steps": steps, "parts": parts,
+            # sana_linattn_backward_with_state: the forward's state passed in, as a
+            # training step holds it (no second pass over k and v for it)
+            "value_with_forward_state": tot_tok * world / (tot_ms_st * 1e-3) / 1e6,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
                          "frac": achieved / hbm_gbs, "traffic": None,
                          "kernel": "forward state (pass 1 + combine) + bwd_query_tc + pass 1 "

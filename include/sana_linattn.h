@@ -140,6 +140,20 @@ SANA_API int sana_linattn_backward(const void* q, const void* k, const void* v,
                                    sana_dtype dtype, void* workspace, size_t ws_bytes,
                                    cudaStream_t stream);
 
+/* sana_linattn_backward with the forward's state passed in, as a training step
+ * holds it (sana_linattn_kv_state's output for the same k, v, gk, eps: kv (B, H, D,
+ * D+1) fp32, 16-byte aligned, read only; it must not overlap the outputs or the
+ * workspace).  The state is then not formed again: the same gradients, bit for bit,
+ * one pass over k and v fewer.  kv NULL is SANA_EINVAL (for B, N > 0); everything
+ * else as for sana_linattn_backward, whose workspace size applies. */
+SANA_API int sana_linattn_backward_with_state(const void* q, const void* k, const void* v,
+                                              const float* gq, const float* gk,
+                                              const float* kv, const void* dout, void* dq,
+                                              void* dk, void* dv, float* dgq, float* dgk,
+                                              int64_t B, int64_t N, int C, int H, float eps,
+                                              sana_dtype dtype, void* workspace,
+                                              size_t ws_bytes, cudaStream_t stream);
+
 /* The state half of Eq. (1) (the sums formed once and reused by every query,
  * section 2.1 of the Sana notes): kv (B, H, D, D+1) fp32 receives
  * S_{b,h}[d][e] = sum_n phi(K)[d] V[e] for e < D and S_{b,h}[d][D] =

@@ -70,6 +70,9 @@ def _declare(lib):
     lib.sana_linattn_backward.argtypes = [vp, vp, vp, fp, fp, vp, vp, vp, vp, fp, fp, i64, i64,
                                           ci, ci, cf, ci, vp, sz, vp]
     lib.sana_linattn_backward.restype = ctypes.c_int
+    lib.sana_linattn_backward_with_state.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, vp, vp, fp,
+                                                     fp, i64, i64, ci, ci, cf, ci, vp, sz, vp]
+    lib.sana_linattn_backward_with_state.restype = ctypes.c_int
     lib.sana_linattn_forward_causal.argtypes = [vp, vp, vp, fp, fp, vp, i64, i64, ci, ci, cf, ci,
                                                 vp, sz, vp]
     lib.sana_linattn_forward_causal.restype = ctypes.c_int
@@ -209,10 +212,12 @@ def forward(q, k, v, gq, gk, H: int, eps: float, out=None, workspace=None, strea
 
 
 def backward(q, k, v, gq, gk, dout, H: int, eps: float, grads=None, workspace=None,
-             stream=None):
+             stream=None, kv=None):
     """Gradients of forward()'s output: returns (dq, dk, dv, dgq, dgk); dgq, dgk
     (float32 [C]) are None with the norm off.  `grads`, when given, is that tuple
-    preallocated (the results are written into it)."""
+    preallocated (the results are written into it).  `kv`, when given, is the
+    forward's state (kv_state() of the same k, v, gk, eps): it is used instead of
+    being formed again (sana_linattn_backward_with_state)."""
     torch = _torch()
     B, N, C = q.shape
     for t, n in ((k, "k"), (v, "v"), (dout, "dout")):
@@ -236,12 +241,23 @@ def backward(q, k, v, gq, gk, dout, H: int, eps: float, grads=None, workspace=No
             dgk = torch.empty(C, dtype=torch.float32, device=q.device)
     ws, wsb = _workspace(int(load().sana_linattn_backward_workspace_bytes(B, N, C, H)), q.device,
                          workspace, stream)
-    rc = load().sana_linattn_backward(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _gain(gq, "gq"),
-                                      _gain(gk, "gk"), _dev(dout, "dout"), _dev(dq, "dq"),
-                                      _dev(dk, "dk"), _dev(dv, "dv"), _dev(dgq, "dgq"),
-                                      _dev(dgk, "dgk"), B, N, C, H, float(eps), dt,
-                                      None if ws is None else ws.data_ptr(), wsb, _stream(stream))
-    _check("sana_linattn_backward", rc)
+    wsp = None if ws is None else ws.data_ptr()
+    if kv is None:
+        rc = load().sana_linattn_backward(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
+                                          _gain(gq, "gq"), _gain(gk, "gk"), _dev(dout, "dout"),
+                                          _dev(dq, "dq"), _dev(dk, "dk"), _dev(dv, "dv"),
+                                          _dev(dgq, "dgq"), _dev(dgk, "dgk"), B, N, C, H,
+                                          float(eps), dt, wsp, wsb, _stream(stream))
+        _check("sana_linattn_backward", rc)
+    else:
+        if kv.dtype != torch.float32 or kv.shape != (B, H, C // H, C // H + 1):
+            raise ValueError("kv must be float32 (B, H, D, D+1), as kv_state() returns")
+        rc = load().sana_linattn_backward_with_state(
+            _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _gain(gq, "gq"), _gain(gk, "gk"),
+            _dev(kv, "kv"), _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"), _dev(dv, "dv"),
+            _dev(dgq, "dgq"), _dev(dgk, "dgk"), B, N, C, H, float(eps), dt, wsp, wsb,
+            _stream(stream))
+        _check("sana_linattn_backward_with_state", rc)
     return dq, dk, dv, dgq, dgk
 
 

@@ -667,11 +667,19 @@ int launch_bwd_query_tc(const void* q, const void* dout, const float* gq, const 
 // path.
 constexpr int64_t kBwdTcMinTokens = 128;
 
-int sana_linattn_backward(const void* q, const void* k, const void* v, const float* gq,
-                          const float* gk, const void* dout, void* dq, void* dk, void* dv,
-                          float* dgq, float* dgk, int64_t B, int64_t N, int C, int H, float eps,
-                          sana_dtype dtype, void* workspace, size_t ws_bytes,
-                          cudaStream_t stream) {
+}  // extern "C"
+
+namespace sana {
+namespace {
+
+// The backward; `state` is the forward's (B, H, D, D+1) state when the caller has
+// it (sana_linattn_backward_with_state), else nullptr and it is formed here exactly
+// as sana_linattn_kv_state forms it.
+int backward_impl(const void* q, const void* k, const void* v, const float* gq,
+                  const float* gk, const void* dout, void* dq, void* dk, void* dv,
+                  float* dgq, float* dgk, int64_t B, int64_t N, int C, int H, float eps,
+                  sana_dtype dtype, void* workspace, size_t ws_bytes, cudaStream_t stream,
+                  const float* state) {
     int rc;
     if ((rc = check_dims(B, N, C, H)) != SANA_OK) return rc;
     if ((rc = check_eps(eps)) != SANA_OK) return rc;
@@ -700,13 +708,20 @@ int sana_linattn_backward(const void* q, const void* k, const void* v, const flo
     if ((rc = validate_ws(workspace, ws_bytes, need)) != SANA_OK) return rc;
     for (const void* i : ins) if (overlaps(workspace, need, i, bytes)) return SANA_EINVAL;
     for (void* o : outs) if (overlaps(workspace, need, o, bytes)) return SANA_EINVAL;
+    const size_t state_bytes = (size_t)B * H * kStateFloats * sizeof(float);
+    if (state) {
+        if (!aligned(state, 16)) return SANA_EALIGN;
+        if (overlaps(workspace, need, state, state_bytes)) return SANA_EINVAL;
+        for (void* o : outs) if (overlaps(o, bytes, state, state_bytes)) return SANA_EINVAL;
+    }
     const Plan p = make_plan(B, N, H);
     const int64_t tiles = (N + kBwdTile - 1) / kBwdTile;
     char* w = (char*)workspace;
     size_t off = 0;
     float* part = (float*)(w + off);
     off = align_up(off + (size_t)B * H * max_splits(B, N, H) * kStateFloats * 4, 256);
-    float* Sz = (float*)(w + off);
+    float* Sz_ws = (float*)(w + off);
+    const float* Sz = state ? state : Sz_ws;
     off = align_up(off + (size_t)B * H * kStateFloats * 4, 256);
     float* dSz = (float*)(w + off);
     off = align_up(off + (size_t)B * H * kStateFloats * 4, 256);
@@ -723,15 +738,17 @@ int sana_linattn_backward(const void* q, const void* k, const void* v, const flo
     const dim3 gs(p.S, H, (unsigned)B), gt((unsigned)tiles, H, (unsigned)B);
     const int nrm = norm ? 1 : 0;
     if (dtype == SANA_BF16) {
-        // the forward state as the bf16 forward forms it (tensor-core pass 1 + combine)
-        if (tc_path(dtype, C)) {
+        // the forward state as sana_linattn_kv_state forms it (tensor-core pass 1 +
+        // combine), unless the caller passed it in
+        if (state) {
+        } else if (tc_path(dtype, C)) {
             PersistPlan1 pl{};
             if ((rc = launch_partials_tc(k, v, gk, part, B, N, C, H, eps, stream, &pl)) != SANA_OK ||
-                (rc = launch_combine_tc(part, Sz, B, H, pl, stream)) != SANA_OK)
+                (rc = launch_combine_tc(part, Sz_ws, B, H, pl, stream)) != SANA_OK)
                 return rc;
         } else {
-            launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, Sz, B, N, H, C, C, eps, p,
-                               stream);
+            launch_state<bf16>((const bf16*)k, (const bf16*)v, gk, part, Sz_ws, B, N, H, C, C, eps,
+                               p, stream);
         }
         if (tc_path(dtype, C) && N >= kBwdTcMinTokens &&
             (!norm || (aligned(gq, 16) && aligned(gk, 16)))) {
@@ -773,8 +790,9 @@ int sana_linattn_backward(const void* q, const void* k, const void* v, const flo
         bwd_key_simt<bf16><<<gt, kBwdTile, 0, stream>>>((const bf16*)k, (const bf16*)v, gk, dSz,
                                                         (bf16*)dk, (bf16*)dv, gpk, N, H, eps, nrm);
     } else {
-        launch_state<float>((const float*)k, (const float*)v, gk, part, Sz, B, N, H, C, C, eps, p,
-                            stream);
+        if (!state)
+            launch_state<float>((const float*)k, (const float*)v, gk, part, Sz_ws, B, N, H, C, C,
+                                eps, p, stream);
         bwd_query_simt<float><<<gt, kBwdTile, 0, stream>>>((const float*)q, (const float*)dout, gq,
                                                            Sz, (float*)dq, G, gpq, N, H, eps, nrm);
         outer_partial_simt<float><<<gs, 128, 0, stream>>>((const float*)q, gq, G, part, N, H, p.S,
@@ -789,6 +807,33 @@ int sana_linattn_backward(const void* q, const void* k, const void* v, const flo
         gain_combine<<<(C + 255) / 256, 256, 0, stream>>>(gpk, dgk, B * tiles, C);
     }
     return launch_status();
+}
+
+}  // namespace
+}  // namespace sana
+
+using namespace sana;
+
+extern "C" {
+
+int sana_linattn_backward(const void* q, const void* k, const void* v, const float* gq,
+                          const float* gk, const void* dout, void* dq, void* dk, void* dv,
+                          float* dgq, float* dgk, int64_t B, int64_t N, int C, int H, float eps,
+                          sana_dtype dtype, void* workspace, size_t ws_bytes,
+                          cudaStream_t stream) {
+    return backward_impl(q, k, v, gq, gk, dout, dq, dk, dv, dgq, dgk, B, N, C, H, eps, dtype,
+                         workspace, ws_bytes, stream, nullptr);
+}
+
+int sana_linattn_backward_with_state(const void* q, const void* k, const void* v,
+                                     const float* gq, const float* gk, const float* kv,
+                                     const void* dout, void* dq, void* dk, void* dv, float* dgq,
+                                     float* dgk, int64_t B, int64_t N, int C, int H, float eps,
+                                     sana_dtype dtype, void* workspace, size_t ws_bytes,
+                                     cudaStream_t stream) {
+    if (!kv && B > 0 && N > 0) return SANA_EINVAL;
+    return backward_impl(q, k, v, gq, gk, dout, dq, dk, dv, dgq, dgk, B, N, C, H, eps, dtype,
+                         workspace, ws_bytes, stream, kv);
 }
 
 int sana_linattn_forward_causal(const void* q, const void* k, const void* v, const float* gq,

@@ -242,6 +242,21 @@ def test_backward_entry_point_rejects_bad_arguments(lib):
     a = list(base)
     a[14] = 35
     assert lib.sana_linattn_backward(*a) == EUNSUP
+    # with the forward's state: (q, k, v, gq, gk, kv, dout, ...)
+    kv = FAKE + (10 << 30)
+    w = base[:5] + [kv] + base[5:]
+    a = list(w)
+    a[5] = None                                  # the state is required
+    assert lib.sana_linattn_backward_with_state(*a) == EINVAL
+    a = list(w)
+    a[5] = kv + 4                                # misaligned state
+    assert lib.sana_linattn_backward_with_state(*a) == EALIGN
+    a = list(w)
+    a[5] = base[18 - 1] + 256                    # the state inside the workspace
+    assert lib.sana_linattn_backward_with_state(*a) == EINVAL
+    a = list(w)
+    a[5] = base[6]                               # the state overlaps dq
+    assert lib.sana_linattn_backward_with_state(*a) == EINVAL
 
 
 

@@ -82,6 +82,26 @@ def test_backward_is_deterministic(cuda_lib):
         assert torch.equal(x, y)
 
 
+@pytest.mark.parametrize("w", [WORKLOADS["1024px-b1"].scaled(B=2, N=1000, seed=90),
+                               WORKLOADS["1024px-b1"].scaled(N=64, seed=91),
+                               WORKLOADS["4096px-b2-overflow"].scaled(B=1, N=700, seed=92),
+                               WORKLOADS["tiny-512px-f32"].scaled(N=300, gains="random", seed=93)],
+                         ids=lambda w: f"{w.dtype}-B{w.B}-N{w.N}-{w.gains}")
+def test_backward_with_the_forward_state_equals_backward(cuda_lib, w):
+    """sana_linattn_backward_with_state given kv_state()'s state: the same gradients
+    bit for bit (the backward forms its state exactly as kv_state does), on the
+    tensor-core path, the short-sequence and fp32 CUDA-core paths and with the norm
+    off."""
+    d = to_dev(make_inputs(w))
+    do = make_output_grad(w).cuda()
+    kv = cuda_lib.kv_state(d["k"], d["v"], d["gk"], w.H, w.eps)
+    a = cuda_lib.backward(d["q"], d["k"], d["v"], d["gq"], d["gk"], do, w.H, w.eps)
+    b = cuda_lib.backward(d["q"], d["k"], d["v"], d["gq"], d["gk"], do, w.H, w.eps, kv=kv)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert (x is None and y is None) or torch.equal(x, y)
+
+
 def test_backward_gains_without_16_byte_alignment(cuda_lib):
     """Gains 4-byte but not 16-byte aligned: the backward takes its CUDA-core path
     and still matches the oracle (the tensor-core kernels read gains as 16-byte
