@@ -20,7 +20,7 @@ import ctypes
 import os
 import threading
 
-__all__ = ["load", "lib_path", "workspace_bytes", "forward", "forward_noalloc", "forward_pass1", "forward_pass2", "kv_state", "apply", "qkv_fused",
+__all__ = ["load", "lib_path", "workspace_bytes", "forward", "forward_noalloc", "forward_pass1", "forward_pass2", "forward_kernels", "kv_state", "apply", "qkv_fused",
            "qkv_fused_w8a8", "quantize_rows_i8", "quantize_cols_i8", "forward_causal",
            "backward", "gemm_bias", "mixffn_dwconv_glu", "mixffn_workspace_bytes",
            "mixffn_forward", "GATES",

@@ -12,7 +12,7 @@
 // tiles at once.  The hardware schedules a cluster's CTAs together, so they can
 // wait for one another at cluster barriers without any spin on global memory.
 //
-//   1. phi(K) in place (the feature map of the pages' Eq. (1) after the QK norm),
+//   1. phi(K) in place (the feature map of Eq. (1) after the QK norm),
 //      the normaliser column sums on the CUDA cores, and one UMMA chain
 //          D[(h,d), (h',e)] = sum_t phi(K)[t,(h,d)] V[t,(h',e)]   (M=N=128, K=128)
 //      whose diagonal blocks are this CTA's partial states (as in pass 1).
