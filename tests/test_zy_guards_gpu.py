@@ -28,6 +28,8 @@ def _ok(*guards):
 
 @pytest.mark.parametrize("name,kw", [("1024px-b1", dict(B=2, N=333, seed=61)),
                                      ("1024px-b1", dict(N=1, seed=62)),
+                                     ("1024px-b1", dict(N=1500, seed=65)),
+                                     ("4096px-b2-overflow", dict(B=1, N=1024, seed=66)),
                                      ("tiny-512px-f32", dict(N=77, seed=63))])
 def test_forward_and_causal_stay_in_bounds(cuda_lib, name, kw):
     w = WORKLOADS[name].scaled(**kw)
