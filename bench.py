@@ -1214,8 +1214,8 @@ def mixffn_measure(args, sla, rank, dev, stream, world, bf16_tf, hbm_gbs, peak_k
             "step_tflops": (fl_expand + fl_project) / (sum(ms) * 1e-3) / 1e12,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16_tf, "unit": "TFLOP/s",
                          "frac": tf / bf16_tf,
-                         "traffic": ncu_traffic("gemm_bias_bf16", w.name, MIXFFN_SOURCES),
-                         "kernel": "gemm_bias_bf16 (expand, 16384 x 2240 x 11200)",
+                         "traffic": ncu_traffic("gemm_bias_bf16_2sm", w.name, MIXFFN_SOURCES),
+                         "kernel": "gemm_bias_bf16_2sm (expand, 16384 x 2240 x 11200; UMMA over SM pairs)",
                          "flop_per_launch": fl_expand,
                          "peak_kind": f"{peak_kind} bf16 burst (bf16_tflops)"},
             "e2e": {"value": M * world / (e2e_ms * 1e-3) / 1e6, "unit": "Mtokens/s",

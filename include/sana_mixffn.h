@@ -38,7 +38,8 @@ extern "C" {
 typedef enum { SANA_GATE_SIGMOID = 0, SANA_GATE_SILU = 1 } sana_gate;
 
 /* D[M][Nc] = A[M][K] W[K][Nc] (+ bias[Nc]) with bf16 A, W, D and fp32
- * accumulation on the tensor cores (tcgen05 UMMA, TMA-fed).  Both 1x1
+ * accumulation on the tensor cores (tcgen05 UMMA, TMA-fed, each UMMA spread over a
+ * pair of SMs: clusters of two CTAs with 256 x 256 tiles).  Both 1x1
  * convolutions of the Mix-FFN are this call.  K and Nc must be positive
  * multiples of 8 (TMA row pitch), M >= 0 (0: nothing launched), M < 2^31;
  * A, W, D 16-byte aligned, bias 4-byte aligned or NULL; D must not overlap A, W

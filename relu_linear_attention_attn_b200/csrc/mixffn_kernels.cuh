@@ -4,20 +4,21 @@
 // 2.3: the convolution's zero padding carries position; "SANA 1.5", section
 // "Model architecture": C = 2240, FFN width F = 5600).  Tokens n = y * Ws + x of a
 // row-major (Hs, Ws) grid:
-//   U  = X W1 + b1                    gemm_bias_bf16     (1x1 expand, C -> 2F)
+//   U  = X W1 + b1                    gemm_bias_bf16_2sm (1x1 expand, C -> 2F)
 //   Hg = Cv[:, :F] * gate(Cv[:, F:]), dwconv3x3_glu      (depthwise 3x3 with zero
 //        Cv = dwconv3x3(U) + bdw                          padding, then the GLU)
-//   Y  = Hg W2 + b2                   gemm_bias_bf16     (1x1 project, F -> C)
+//   Y  = Hg W2 + b2                   gemm_bias_bf16_2sm (1x1 project, F -> C)
 // U and Hg are stored in bf16; every sum accumulates in fp32.
 //
-// gemm_bias_bf16: D[M][Nc] = A[M][K] W[K][Nc] (+ bias) on the sm_100a tensor cores.
-//   Persistent: CTA c takes tiles c, c + grid, ... of 128 rows x 256 columns, in
-//   groups of 8 row blocks with the row block fastest inside a group, so concurrent
-//   CTAs share A rows and a band of W columns through L2.  Warp 0 is
-//   the TMA producer (4-stage ring of A 128 x 64 k, K-major, and W 64 k x 256 n,
-//   MN-major, both 128-byte swizzled), warp 1 issues 128x256x16 UMMAs into one
-//   of two TMEM accumulators, warps 2-9 drain the other (bias, bf16, stores), so
-//   a tile's epilogue overlaps the next tile's main loop.
+// gemm_bias_bf16_2sm: D[M][Nc] = A[M][K] W[K][Nc] (+ bias) on the sm_100a tensor
+//   cores, each UMMA spread over a pair of SMs (256 x 256 tiles; see below).
+//   Persistent: pair p takes tiles p, p + pairs, ... in groups of 4 row-pair blocks
+//   with the row block fastest inside a group, so concurrent pairs share A rows and
+//   a band of W columns through L2.  Warp 0 is the TMA producer (7-stage ring of
+//   the CTA's A 128 x 64 k, K-major, and its W 64 k x 128 n, MN-major, both
+//   128-byte swizzled), warp 1 of the leader CTA issues the UMMAs into one of two
+//   TMEM accumulators, warps 2-9 of both CTAs drain the other (bias, bf16,
+//   stores), so a tile's epilogue overlaps the next tile's main loop.
 // dwconv3x3_glu: CTA (channel chunk, column strip, batch) marches down the grid
 //   rows of a 32-token strip for 32 value channels and the 32 matching gate
 //   channels.  An 8-row TMA ring brings in each input row once, with one halo
@@ -46,60 +47,140 @@ __device__ __forceinline__ void tma_load_4d_u(void* dst, const CUtensorMap* m, u
 }
 
 // ============================================================================ GEMM
-namespace gm {
-constexpr int kBM = 128;                        // UMMA M: rows per tile
-constexpr int kBN = 256;                        // UMMA N: columns per tile
-constexpr int kBK = 64;                         // k per stage: 128 bytes of an A row
-constexpr int kABytes = kBM * 128;              // 16 KB
-constexpr int kWBox = kBK * 128;                // 8 KB: 64 k rows x 64 n
-constexpr int kWBoxes = kBN / 64;
-constexpr int kStageBytes = kABytes + kWBoxes * kWBox;   // 48 KB
-constexpr int kStages = 4;
-constexpr int kTmemCols = 2 * kBN;              // two accumulators
-constexpr int kEpiWarps = 8;                    // two per TMEM lane quadrant
-constexpr int kThreads = 32 * (2 + kEpiWarps);
-constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
-}  // namespace gm
-
 struct GemmArgs {
     const float* bias;   // [Nc] or nullptr
     bf16* d;             // [M][Nc] row-major
     int64_t M;
     int Nc, K;
-    int mb, nb;          // tiles along M and along Nc
+    int mb, nb;          // 128-row blocks along M, 256-column blocks along Nc
 };
 
-// Tile t -> (row block, column block).  Tiles go in groups of kGroupRows row blocks;
-// within a group the row block is fastest, so the CTAs running at once share a few
-// A row blocks and a band of W columns, and each W column block is used by the
-// group's row blocks back to back (it stays in L2 across the group even while the
-// output stream passes through, instead of being re-read from DRAM per row block).
-constexpr int kGroupRows = 8;
-__device__ __forceinline__ void gemm_tile(int64_t t, const GemmArgs& a, int& mblk, int& nblk) {
-    const int64_t per_group = (int64_t)kGroupRows * a.nb;
+// ============================================================================ GEMM, 2 SMs
+// The same D = A W (+ bias) with the UMMA spread over a pair of SMs (a cluster of
+// two CTAs, tcgen05 cta_group::2): one instruction computes a 256 x 256 x 16 tile
+// step, CTA r of the pair supplying rows [128 r, 128 r + 128) of the A tile and
+// columns [128 r, 128 r + 128) of the W tile from its own shared memory, and
+// receiving rows [128 r, + 128) x all 256 columns of the product in its own TMEM.
+// Each SM thus streams 32 KB of operands per 64-deep k step instead of 48 KB for
+// the same tensor work: the single-SM kernel is bound by that stream from L2.
+//
+// Hand-offs: both CTAs' TMA loads (unicast, each into its own shared memory)
+// complete on the leader CTA's `full` barrier (the cta_group::2 form of the load),
+// which the leader's producer arms with the bytes of both halves; only the leader
+// issues UMMAs, and its commits arrive on `empty` and `accfull` in both CTAs at
+// once (the commit's CTA mask); both CTAs' epilogue warps arrive on the leader's
+// `accempty`.  (Passing the leader's phases on to the peer by remote arrives
+// instead, with no mask on the commit, measured half the speed: a stage's round
+// trip then carries two more hand-offs.)
+namespace g2 {
+constexpr int kBM = 128;                        // rows per CTA (the pair: 256)
+constexpr int kBN = 256;                        // columns per tile (128 per CTA's W half)
+constexpr int kBK = 64;
+constexpr int kABytes = kBM * 128;              // 16 KB
+constexpr int kWBox = kBK * 128;                // 8 KB: 64 k rows x 64 n
+constexpr int kWBoxes = 2;                      // this CTA's 128 columns
+constexpr int kStageBytes = kABytes + kWBoxes * kWBox;   // 32 KB
+constexpr int kStages = 7;
+constexpr int kTmemCols = 2 * kBN;              // two accumulators
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+static_assert(kSmemBytes <= 232448, "shared memory");
+constexpr int kGroupPairs = 4;                  // row-pair blocks per raster group
+}  // namespace g2
+
+// Tile t -> (row-pair block, column block), grouped as gemm_tile does.
+__device__ __forceinline__ void gemm_tile2(int64_t t, int mb2, int nb, int& mblk, int& nblk) {
+    const int64_t per_group = (int64_t)g2::kGroupPairs * nb;
     const int64_t grp = t / per_group, local = t % per_group;
-    const int rows = (int)min((int64_t)kGroupRows, a.mb - grp * kGroupRows);
+    const int rows = (int)min((int64_t)g2::kGroupPairs, mb2 - grp * g2::kGroupPairs);
     nblk = (int)(local / rows);
-    mblk = (int)(grp * kGroupRows + local % rows);
+    mblk = (int)(grp * g2::kGroupPairs + local % rows);
 }
 
-__global__ void __launch_bounds__(gm::kThreads, 1)
-gemm_bias_bf16(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
-               const GemmArgs a)
+// TMA load into this CTA's shared memory whose bytes complete on the pair leader's
+// mbarrier (a shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m,
+                                                 uint32_t leader_bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(m), "r"(leader_bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+// D[tmem] (+)= A * B^T over the pair (M = 256), issued by the leader alone.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(0u)
+        : "memory");
+}
+
+// Arrive once on the leader's own mbarrier when its pair UMMAs so far are complete.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// The same, arriving on the barrier at this offset in both CTAs of the pair (CTA
+// mask 0b11).  This is the commit's own signal, not a data copy.
+__device__ __forceinline__ void umma_commit_both(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"((uint16_t)3)
+        : "memory");
+}
+
+// Wait for a phase by polling (no suspension, so a hand-off on the critical path
+// costs no wake-up), giving up after `limit_ns` as mbar_wait does.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, int site,
+                                               uint64_t limit_ns = 2000000000ull) {
+    if (mbar_test(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_test(bar, parity)) return true;
+        if (global_timer_ns() - t0 > limit_ns) {
+            record_error(kErrWaitTimeout, site);
+            return false;
+        }
+    }
+}
+
+// Arrive on an mbarrier of another CTA of the cluster (release at cluster scope).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+__global__ void __launch_bounds__(g2::kThreads, 1)
+gemm_bias_bf16_2sm(const __grid_constant__ CUtensorMap tmap_a,
+                   const __grid_constant__ CUtensorMap tmap_w, const GemmArgs a)
 {
-    using namespace gm;
+    using namespace g2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_1024(smem_raw);
     uint8_t* stages = smem;
-    uint64_t* full = (uint64_t*)(stages + kStages * kStageBytes);
+    uint64_t* full = (uint64_t*)(stages + kStages * kStageBytes);   // used in the leader
     uint64_t* empty = full + kStages;
     uint64_t* accfull = empty + kStages;         // [2]
-    uint64_t* accempty = accfull + 2;            // [2]
+    uint64_t* accempty = accfull + 2;            // [2], used in the leader
     uint64_t* drained = accempty + 2;
     uint32_t* tmem_slot = (uint32_t*)(drained + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t tiles = (int64_t)a.mb * a.nb;
+    const uint32_t rank = blockIdx.x & 1;        // rank in the cluster of two
+    const bool leader = rank == 0;
+    const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int mb2 = (int)((a.M + 2 * kBM - 1) / (2 * kBM));
+    const int64_t tiles = (int64_t)mb2 * a.nb;
     const int ksteps = (a.K + kBK - 1) / kBK;
 
     if (threadIdx.x == 0) {
@@ -109,7 +190,7 @@ gemm_bias_bf16(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&accfull[i], 1);
-            mbar_init(&accempty[i], 32 * kEpiWarps);
+            mbar_init(&accempty[i], 2 * kEpiWarps);
         }
         mbar_init(drained, 1);
         fence_barrier_init();
@@ -119,62 +200,65 @@ gemm_bias_bf16(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
         prefetch_tmap(&tmap_w);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, kTmemCols);
-        tmem_relinquish();
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     tc_fence_before_sync();
     __syncthreads();
+    cluster_arrive();                            // both CTAs' barriers are initialised
+    cluster_wait();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
-            int64_t step = 0, last = -1;
-            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            int64_t step = 0;
+            for (int64_t t = pair; t < tiles && ok; t += npairs) {
                 int mblk, nblk;
-                gemm_tile(t, a, mblk, nblk);
-                const int m0 = mblk * kBM;
-                const int n0 = nblk * kBN;
+                gemm_tile2(t, mb2, a.nb, mblk, nblk);
+                const int m0 = mblk * 2 * kBM + (int)rank * kBM;
+                const int n0 = nblk * kBN + (int)rank * (kBN / 2);
                 for (int kk = 0; kk < ksteps; ++kk, ++step) {
                     const int st = (int)(step % kStages);
-                    if (step >= kStages)
-                        ok = mbar_wait(&empty[st], (uint32_t)((step / kStages) - 1) & 1, 601);
-                    if (!ok) break;
+                    if (step >= kStages) {
+                        ok = mbar_wait_spin(&empty[st], (uint32_t)((step / kStages) - 1) & 1, 621);
+                        if (!ok) break;
+                    }
                     uint8_t* sb = stages + st * kStageBytes;
-                    mbar_arrive_expect_tx(&full[st], kStageBytes);
-                    tma_load_2d(sb, &tmap_a, &full[st], kk * kBK, m0);
+                    const uint32_t fb = map_shared_rank(smem_u32(&full[st]), 0);
+                    if (leader) mbar_arrive_expect_tx(&full[st], 2 * kStageBytes);
+                    tma_load_2d_pair(sb, &tmap_a, fb, kk * kBK, m0);
 #pragma unroll
                     for (int j = 0; j < kWBoxes; ++j)
-                        tma_load_2d(sb + kABytes + j * kWBox, &tmap_w, &full[st], n0 + 64 * j,
-                                    kk * kBK);
-                    last = step;
+                        tma_load_2d_pair(sb + kABytes + j * kWBox, &tmap_w, fb, n0 + 64 * j,
+                                         kk * kBK);
                 }
             }
-            if (!ok) {        // let every copy already issued land before the CTA exits
-                for (int st = 0; st < kStages; ++st) {
-                    const int64_t li = last - ((last - st) % kStages + kStages) % kStages;
-                    if (last >= 0 && li >= 0)
-                        mbar_wait(&full[st], (uint32_t)(li / kStages) & 1, 602);
-                }
-            }
+            // Before the CTA may exit, every slot's last load must have been consumed.
+            const int64_t n = step;
+            for (int64_t s2 = n - kStages > 0 ? n - kStages : 0; s2 < n && ok; ++s2)
+                ok = mbar_wait(&empty[s2 % kStages], (uint32_t)(s2 / kStages) & 1, 622);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ UMMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = make_idesc_bf16(kBM, kBN, false, true);   // A K-, W MN-major
+        // ------------------------------------------------ UMMA issuer (the leader's lane 0)
+        if (leader && lane == 0) {
+            const uint32_t idesc = make_idesc_bf16(2 * kBM, kBN, false, true);
             int64_t step = 0;
             int lt = 0;
-            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++lt) {
+            for (int64_t t = pair; t < tiles && ok; t += npairs, ++lt) {
                 const int buf = lt & 1;
-                if (lt >= 2) ok = mbar_wait(&accempty[buf], (uint32_t)((lt >> 1) - 1) & 1, 603);
+                if (lt >= 2) ok = mbar_wait(&accempty[buf], (uint32_t)((lt >> 1) - 1) & 1, 624);
                 if (!ok) break;
                 tc_fence_after_sync();
                 const uint32_t acc = tmem + buf * kBN;
                 for (int kk = 0; kk < ksteps; ++kk, ++step) {
                     const int st = (int)(step % kStages);
-                    ok = mbar_wait(&full[st], (uint32_t)(step / kStages) & 1, 604);
+                    ok = mbar_wait_spin(&full[st], (uint32_t)(step / kStages) & 1, 625);
                     if (!ok) break;
                     tc_fence_after_sync();
                     const uint32_t ab = smem_u32(stages + st * kStageBytes);
@@ -184,30 +268,29 @@ gemm_bias_bf16(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
                         const uint64_t ad = make_smem_desc(ab + k4 * 32, 16, 1024, kSwizzle128B);
                         const uint64_t bd = make_smem_desc(wb + k4 * 16 * 128, kWBox, 1024,
                                                            kSwizzle128B);
-                        umma_bf16(acc, ad, bd, idesc, kk > 0 || k4 > 0);
+                        umma_bf16_pair(acc, ad, bd, idesc, kk > 0 || k4 > 0);
                     }
-                    umma_commit(&empty[st]);
+                    umma_commit_both(&empty[st]);
                 }
                 if (!ok) break;
-                umma_commit(&accfull[buf]);
+                umma_commit_both(&accfull[buf]);
             }
-            // every UMMA issued has completed before the TMEM is released
-            umma_commit(drained);
-            mbar_wait(drained, 0, 605);
+            umma_commit_pair(drained);
+            mbar_wait(drained, 0, 626);
         }
     } else {
-        // ------------------------------------------------ epilogue
-        const int q = warp & 3;                        // TMEM lane quadrant
-        const int half = (warp - 2) >> 2;              // columns [128 half, 128 half + 128)
+        // ------------------------------------------------ epilogue (both CTAs: own rows)
+        const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
         int lt = 0;
-        for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++lt) {
+        for (int64_t t = pair; t < tiles && ok; t += npairs, ++lt) {
             const int buf = lt & 1;
-            ok = mbar_wait(&accfull[buf], (uint32_t)(lt >> 1) & 1, 606);
+            ok = mbar_wait(&accfull[buf], (uint32_t)(lt >> 1) & 1, 627);
             if (!ok) break;
             tc_fence_after_sync();
             int mblk, nblk;
-            gemm_tile(t, a, mblk, nblk);
-            const int64_t row = (int64_t)mblk * kBM + 32 * q + lane;
+            gemm_tile2(t, mb2, a.nb, mblk, nblk);
+            const int64_t row = (int64_t)mblk * 2 * kBM + (int)rank * kBM + 32 * q + lane;
             const int n0 = nblk * kBN;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
@@ -232,14 +315,19 @@ gemm_bias_bf16(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
                 }
             }
             tc_fence_before_sync();
-            mbar_arrive(&accempty[buf]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(map_shared_rank(smem_u32(&accempty[buf]), 0));
         }
     }
     tc_fence_before_sync();
     __syncthreads();
+    cluster_arrive();                            // both CTAs are done with the TMEM
+    cluster_wait();
     if (warp == 1) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem, kTmemCols);
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(kTmemCols)
+                     : "memory");
     }
 }
 

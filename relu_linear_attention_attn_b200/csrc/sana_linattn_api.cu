@@ -1255,12 +1255,12 @@ int gemm_ctas() {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         sms <= 0)
         return 0;
-    if (cudaFuncSetAttribute(gemm_bias_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             gm::kSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_bias_bf16_2sm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             g2::kSmemBytes) != cudaSuccess)
         return 0;
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemm_bias_bf16, gm::kThreads,
-                                                      gm::kSmemBytes) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemm_bias_bf16_2sm, g2::kThreads,
+                                                      g2::kSmemBytes) != cudaSuccess ||
         per_sm < 1)
         return 0;
     ctas[dev] = sms;
@@ -1288,7 +1288,7 @@ int launch_gemm(const void* A, const void* W, const float* bias, void* D, int64_
     const int P = gemm_ctas();
     if (!P) return SANA_EUNSUPPORTED;
     CUtensorMap ta, tw;
-    if (!make_tmap_rowmajor(&ta, A, M, K, gm::kBM) || !make_tmap_rowmajor(&tw, W, K, Nc, gm::kBK))
+    if (!make_tmap_rowmajor(&ta, A, M, K, g2::kBM) || !make_tmap_rowmajor(&tw, W, K, Nc, g2::kBK))
         return SANA_ECUDA;
     GemmArgs a{};
     a.bias = bias;
@@ -1296,11 +1296,24 @@ int launch_gemm(const void* A, const void* W, const float* bias, void* D, int64_
     a.M = M;
     a.Nc = Nc;
     a.K = K;
-    a.mb = (int)((M + gm::kBM - 1) / gm::kBM);
-    a.nb = (Nc + gm::kBN - 1) / gm::kBN;
-    const int64_t tiles = (int64_t)a.mb * a.nb;
-    const unsigned grid = (unsigned)(tiles < P ? tiles : P);
-    gemm_bias_bf16<<<grid, gm::kThreads, gm::kSmemBytes, st>>>(ta, tw, a);
+    a.mb = (int)((M + g2::kBM - 1) / g2::kBM);
+    a.nb = (Nc + g2::kBN - 1) / g2::kBN;
+    // pairs of SMs (clusters of two CTAs), one 256 x 256 tile at a time
+    const int64_t tiles2 = (int64_t)((M + 2 * g2::kBM - 1) / (2 * g2::kBM)) * a.nb;
+    const int64_t pairs = tiles2 < P / 2 ? tiles2 : P / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(g2::kThreads);
+    cfg.dynamicSmemBytes = g2::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gemm_bias_bf16_2sm, ta, tw, a) != cudaSuccess) return SANA_ECUDA;
     return launch_status();
 }
 
