@@ -32,13 +32,15 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row(cuda_lib):
     """Calls in a row on different shapes, so each one meets the one before's
     leftovers in the shared scratch: the bf16 tensor-core path twice, then the
     fp32 CUDA-core path (which also uses the scratch's state region and a
-    different split plan).  The no-allocation call runs the same kernels with the
-    same fixed plan as sana_linattn_forward, so the two agree bit for bit; each
-    is also checked against the fp64 oracle."""
+    different split plan), then the one-launch short-sequence path (which needs
+    no scratch).  The no-allocation call runs the same kernels with the same fixed
+    plan as sana_linattn_forward, so the two agree bit for bit; each is also
+    checked against the fp64 oracle."""
     lib = cuda_lib.load()
     cases = (WORKLOADS["2048px-b8-lognormal"].scaled(B=2, N=3000, seed=61),
              WORKLOADS["4096px-b2-overflow"].scaled(B=1, N=5000, seed=62),
-             WORKLOADS["tiny-512px-f32"].scaled(seed=63))
+             WORKLOADS["tiny-512px-f32"].scaled(seed=63),
+             WORKLOADS["1024px-b1"].scaled(seed=64))
     for w in cases:
         x = make_inputs(w)
         d = to_dev(x)
