@@ -12,7 +12,7 @@
 //
 // gemm_bias_bf16_2sm: D[M][Nc] = A[M][K] W[K][Nc] (+ bias) on the sm_100a tensor
 //   cores, each UMMA spread over a pair of SMs (256 x 256 tiles; see below).
-//   Persistent: pair p takes tiles p, p + pairs, ... in groups of 4 row-pair blocks
+//   Persistent: pair p takes tiles p, p + pairs, ... in groups of 2 row-pair blocks
 //   with the row block fastest inside a group, so concurrent pairs share A rows and
 //   a band of W columns through L2.  Warp 0 is the TMA producer (7-stage ring of
 //   the CTA's A 128 x 64 k, K-major, and its W 64 k x 128 n, MN-major, both
@@ -86,7 +86,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
 static_assert(kSmemBytes <= 232448, "shared memory");
-constexpr int kGroupPairs = 4;                  // row-pair blocks per raster group
+constexpr int kGroupPairs = 2;                  // row-pair blocks per raster group
 }  // namespace g2
 
 // Tile t -> (row-pair block, column block), grouped as gemm_tile does.
