@@ -190,6 +190,7 @@ KERNEL_SOURCES = ("relu_linear_attention_attn_b200/csrc/tc_kernels.cuh",
 
 # the sources the Mix-FFN kernels compile from
 MIXFFN_SOURCES = ("relu_linear_attention_attn_b200/csrc/mixffn_kernels.cuh",
+                  "relu_linear_attention_attn_b200/csrc/sm100_pair.cuh",
                   "relu_linear_attention_attn_b200/csrc/f32x2.cuh",
                   "relu_linear_attention_attn_b200/csrc/tc_kernels.cuh",
                   "relu_linear_attention_attn_b200/csrc/sana_common.cuh",

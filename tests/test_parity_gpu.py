@@ -126,8 +126,11 @@ def test_fused_full_size_sampled_parity(cuda_lib):
 
 
 @pytest.mark.parametrize("B,N,gains", [(1, 1, "random"), (1, 300, "random"), (2, 129, "off"),
-                                       (1, 1000, "ones")])
+                                       (1, 1000, "ones"), (2, 800, "random"), (3, 333, "off")])
 def test_fused_small_full_parity(cuda_lib, B, N, gains):
+    """Small shapes: one to eight token splits per head group, a last split with
+    fewer tiles than the others (2 x 800: 7 tiles in splits of 2), the norm on and
+    off."""
     w = WORKLOADS["fused-2048px-b4"].scaled(B=B, N=N, gains=gains, seed=40 + N)
     x = make_inputs(w)
     d = to_dev(x)
