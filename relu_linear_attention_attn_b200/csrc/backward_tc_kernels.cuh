@@ -537,8 +537,7 @@ bwd_query_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
         *reinterpret_cast<uint4*>(bop + rb * kBopSet + (p2::kDenLo + 1 + rem / 8) * 128 + (rem % 8) * 16) =
             make_uint4(0, 0, 0, 0);
     }
-    if (a.norm)
-        for (int i = threadIdx.x; i < C; i += blockDim.x) sgain[i] = a.gq[i];
+    if (a.norm) load_gains<bq::kGainCache, bq::kThreads>(sgain, a.gq, C, threadIdx.x);
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();

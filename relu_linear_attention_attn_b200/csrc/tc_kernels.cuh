@@ -199,6 +199,31 @@ __device__ __forceinline__ void phi2_inplace_sw128(uint8_t* const tile[2], const
             *reinterpret_cast<uint4*>(tile[it] + sw128_offset(row[it], chunk0[it] + c)) = u[it][c];
 }
 
+// Copy n <= kMax floats (a gain vector) from global to shared memory as thread
+// `tid` of kThreadsT: each thread issues up to kBatch of its loads before any
+// store, so the copy costs ceil(kMax / (kThreadsT kBatch)) memory round trips
+// instead of one per strided loop iteration.
+template <int kMax, int kThreadsT, int kBatch = 8>
+__device__ __forceinline__ void load_gains(float* dst, const float* __restrict__ src, int n,
+                                           int tid) {
+    constexpr int kPer = (kMax + kThreadsT - 1) / kThreadsT;
+#pragma unroll 1
+    for (int u0 = 0; u0 < kPer; u0 += kBatch) {
+        if (tid + u0 * kThreadsT >= n) break;
+        float v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int i = tid + (u0 + u) * kThreadsT;
+            v[u] = (u0 + u < kPer && i < n) ? __ldg(src + i) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int i = tid + (u0 + u) * kThreadsT;
+            if (u0 + u < kPer && i < n) dst[i] = v[u];
+        }
+    }
+}
+
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
     return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
 }
@@ -405,8 +430,7 @@ kv_partials_persistent(const __grid_constant__ CUtensorMap tmap_k,
         const int wi = wt >> 5;                          // transform warp 0..7
         const int grp = wt >> 7;                         // stages with li % 2 == grp
         const int hl = wi & 3;                           // head within the row
-        if (a.norm)
-            for (int i = wt; i < C; i += 32 * kTransformWarps) sgain[i] = a.gk[i];
+        if (a.norm) load_gains<kGainCache, 32 * kTransformWarps>(sgain, a.gk, C, wt);
         named_barrier_sync(2, 32 * kTransformWarps);
         int seg = 0;
         for (int64_t sb = i0; sb < i1 && ok; ++seg) {
@@ -631,8 +655,7 @@ apply_persistent(const __grid_constant__ CUtensorMap tmap_q,
         *reinterpret_cast<uint4*>(bop + rb * kBopBytes + (kDenLo + 1 + rem / 8) * 128 +
                                   (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
     }
-    if (a.norm)
-        for (int i = threadIdx.x; i < C; i += blockDim.x) sgain[i] = a.gq[i];
+    if (a.norm) load_gains<kGainCache, kThreads>(sgain, a.gq, C, threadIdx.x);
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
