@@ -15,7 +15,8 @@ timed in the same run and reported under "fused".
 value: tokens of all ranks / device time of the K timed steps (max over ranks).
 e2e: the same metric through sana_linattn_forward with host (pinned) buffers,
 host->device copies of q, k, v and the device->host copy of the output inside the
-timed region.  cpu_baseline: the fp64 CPU oracle, as it stands, on a bounded
+timed region; the fused and Mix-FFN legs carry their own e2e (x uploaded, the
+output downloaded each step).  cpu_baseline: the fp64 CPU oracle, as it stands, on a bounded
 sample of the same workload (rank 0, N=1 only).
 """
 from __future__ import annotations
@@ -948,6 +949,26 @@ def fused_measure(args, sla, w, rank, dev, stream, world, bf16_tf, peak_kind):
         torch.cuda.synchronize()
         barrier(world)
     ms = max_over_ranks(statistics.fmean(a.elapsed_time(b) for a, b in evs), world)
+    # e2e: the public call with host buffers (pinned x uploaded, O downloaded each step)
+    hx = x["x"].pin_memory()
+    ho = torch.empty_like(hx).pin_memory()
+    dx = torch.empty_like(d["x"])
+
+    def e2e_step():
+        dx.copy_(hx, non_blocking=True)
+        sla.qkv_fused(dx, d["W"], d["gq"], d["gk"], w.H, w.eps, out=out, workspace=ws)
+        ho.copy_(out, non_blocking=True)
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / steps, world)
     flops = 2.0 * w.tokens * w.C * 3 * w.C
     tf = flops / (ms * 1e-3) / 1e12
     return {"workload": w.name, "value": w.tokens * world / (ms * 1e-3) / 1e6,
@@ -957,6 +978,9 @@ def fused_measure(args, sla, w, rank, dev, stream, world, bf16_tf, peak_kind):
                          "kernel": "fused_kv + fused_qo (the whole fused op)",
                          "flop_per_launch": flops,
                          "peak_kind": f"{peak_kind} bf16 burst (bf16_tflops)"},
+            "e2e": {"value": w.tokens * world / (e2e_ms * 1e-3) / 1e6, "unit": "Mtokens/s",
+                    "h2d_bytes_per_step": hx.numel() * hx.element_size(),
+                    "d2h_bytes_per_step": ho.numel() * ho.element_size()},
             "gpu_launches": steps * 2, "clocks": clk.summary()}
 
 
